@@ -1,0 +1,370 @@
+"""Benchmark of the ThinK decode-time path on B200.
+
+One step = one pass of the whole path over one layer of the long-context
+workload (Mistral-7B-shaped GQA layer: B=1, 32 query / 8 KV heads, d=128,
+N=131072, S_obs=64, lambda=0.6 -> T=51): score the key channels, select the
+top T per KV head, compact K, then 256 decode steps of pruned-K attention, each
+with a fresh query. Inputs are resident in HBM before the timed region and are
+larger than L2 (K 268 MB; K'+V 375 MB read per decode step).
+
+value = algorithmic bytes of the step (one read of K + K' written + Q_win +
+idx, plus 256 x (K' + V + q + out + idx)) / device time of the step, in GB/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+With N > 1 (torchrun, one process per GPU) every rank runs an independent
+replica on its own data: the path has no exchange step, so there is no
+collective on the data path; the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "pruned-K decode attention HBM GB/s (% of 8 TB/s); prune pass µs/layer"
+WORKLOAD = "mistral_7b_long"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", default="native", choices=["native", "reference"])
+    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------ clocks ---
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, cuda_index: int, period_s: float = 0.02):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        self.error = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = self._handle(cuda_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: clocks stay unreported
+            self.nv, self.error = None, repr(e)
+
+    def _handle(self, idx):
+        import torch
+        nv = self.nv
+        try:
+            pr = torch.cuda.get_device_properties(idx)
+            bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+            return nv.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(idx)
+
+    def _run(self):
+        nv = self.nv
+        get_r = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = get_r(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception as e:
+                self.error = repr(e)
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [],
+                    "note": self.error or "no samples"}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------- workload ---
+
+def workload():
+    from query_driven_key_b200 import workloads as W
+    return W.WORKLOADS[WORKLOAD]
+
+
+def step_bytes(w, T):
+    from query_driven_key_b200 import workloads as W
+    return W.prune_bytes(w, T) + w.decode_steps * W.decode_bytes(w, T)
+
+
+def cpu_baseline(w, T, seed_layer=0):
+    """The fp64 oracle as it stands, on this host's cores, on a bounded sample
+    of the workload: the whole prune pass plus 4 of the 256 decode steps."""
+    import torch
+    import oracle
+    from query_driven_key_b200 import workloads as W
+
+    q_win, k, v = W.gen_layer(w, seed_layer)
+    f64 = lambda t: t.to(torch.float64).numpy()
+    qw, kk, vv = f64(q_win), f64(k), f64(v)
+    qs = [f64(W.gen_decode_q(w, s, seed_layer)) for s in range(4)]
+    o = oracle.default_oracle()
+    t0 = time.perf_counter()
+    _, idx, kp = o.prune(qw, kk, T)
+    for q in qs:
+        o.decode(q, kp, vv, idx)
+    dt = time.perf_counter() - t0
+    nbytes = W.prune_bytes(w, T) + len(qs) * W.decode_bytes(w, T)
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": o.num_threads(), "kind": "oracle",
+            "sample": f"prune of all {w.B * w.Hkv} KV heads + {len(qs)} of {w.decode_steps} decode "
+                      f"steps, fp64 C loops (OpenMP over heads), {dt:.2f} s"}
+
+
+# ----------------------------------------------------- reference arm ---
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import torch
+    import oracle
+    from query_driven_key_b200 import workloads as W
+
+    w = workload()
+    T = oracle.t_from_lambda(w.d, w.lam)
+    q_win, k, v = W.gen_layer(w)
+    f64 = lambda t: t.to(torch.float64).numpy()
+    qw, kk, vv = f64(q_win), f64(k), f64(v)
+    o = oracle.default_oracle()
+    times = []
+    for i in range(args.warmup + args.steps):
+        q = f64(W.gen_decode_q(w, i))
+        t0 = time.perf_counter()
+        _, idx, kp = o.prune(qw, kk, T)
+        o.decode(q, kp, vv, idx)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+    nbytes = W.prune_bytes(w, T) + W.decode_bytes(w, T)
+    sec = sum(times) / len(times)
+    value = nbytes / sec / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, bf16-rounded inputs)",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
+                   "S_obs": w.S_obs, "lambda": w.lam, "T": T,
+                   "sample": "each step: prune pass + 1 of the 256 decode steps"},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": o.num_threads(), "kind": "oracle",
+                         "sample": "prune of all KV heads + 1 decode step per timed step"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# -------------------------------------------------------- native arm ---
+
+def run_native(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world and world > 1:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    import query_driven_key_b200 as qdk
+    from query_driven_key_b200 import workloads as W
+
+    w = workload()
+    T = qdk.think_t_from_lambda(w.d, w.lam)
+    # each rank: an independent replica on its own data
+    q_win, k, v = W.gen_layer(w, layer=rank)
+    qs = torch.stack([W.gen_decode_q(w, s, layer=rank) for s in range(w.decode_steps)])
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        qw_d, k_d, v_d, qs_d = (t.to(dev) for t in (q_win, k, v, qs))
+        cache = qdk.PrunedCache(w.B, w.Hq, w.Hkv, w.N, T, w.d, dtype=w.dtype, device=dev)
+        outs = torch.empty((w.decode_steps, w.B, w.Hq, w.d), dtype=torch.float32, device=dev)
+    stream.synchronize()
+
+    launches_per_step = 4 + 2 * w.decode_steps  # score x2, select, compact, decode x2 per step
+
+    def one_step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        cache.prune(qw_d, k_d, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        for s in range(w.decode_steps):
+            cache.decode(qs_d[s], v_d, outs[s], stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        one_step()
+    stream.synchronize()
+    assert qdk.think_read_device_status(cache.decode_ws, stream) == 0
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        t_start.record(stream)
+        for i in range(args.steps):
+            one_step(evs[i])
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    prune_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    decode_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    if world > 1:
+        t = torch.tensor([total_ms, sum(prune_ms), sum(decode_ms)], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, prune_sum, decode_sum = t.tolist()
+    else:
+        prune_sum, decode_sum = sum(prune_ms), sum(decode_ms)
+    assert qdk.think_read_device_status(cache.decode_ws, stream) == 0
+
+    ms_per_step = total_ms / args.steps
+    nbytes = step_bytes(w, T)
+    value = world * nbytes / (ms_per_step * 1e-3) / 1e9
+    dec_bytes = W.decode_bytes(w, T)
+    dec_us = decode_sum / args.steps / w.decode_steps * 1e3
+    prune_us = prune_sum / args.steps * 1e3
+    achieved = dec_bytes / (dec_us * 1e-6) / 1e9
+    peak, peak_kind = measured_peaks()
+
+    # ---------------------------------------------- end to end (host buffers)
+    e2e = None
+    if args.e2e_steps > 0:
+        pin = lambda t: t.pin_memory()
+        h_qw, h_k, h_v, h_qs = pin(q_win), pin(k), pin(v), pin(qs)
+        h_out = torch.empty(outs.shape, dtype=torch.float32).pin_memory()
+        h_idx = torch.empty(cache.idx.shape, dtype=torch.int32).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in (h_qw, h_k, h_v, h_qs))
+        d2h = h_out.numel() * 4 + h_idx.numel() * 4
+
+        def e2e_step():
+            qw_d.copy_(h_qw, non_blocking=True)
+            k_d.copy_(h_k, non_blocking=True)
+            v_d.copy_(h_v, non_blocking=True)
+            qs_d.copy_(h_qs, non_blocking=True)
+            one_step()
+            h_out.copy_(outs, non_blocking=True)
+            h_idx.copy_(cache.idx, non_blocking=True)
+
+        with torch.cuda.stream(stream):
+            e2e_step()
+            stream.synchronize()
+            if world > 1:
+                dist.barrier()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(args.e2e_steps):
+                e2e_step()
+            e1.record(stream)
+            stream.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = t.item()
+        e2e = {"value": world * nbytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+               "steps": args.e2e_steps}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded LogNormal(0,1.5) channel-scaled N(0,1) keys, N(0,1) values/queries)",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
+                   "S_obs": w.S_obs, "lambda": w.lam, "T": T, "decode_steps_per_step": w.decode_steps,
+                   "parallelism": f"{world} independent replica(s), no collective",
+                   "l2": "inputs larger than L2 (K 268 MB, K'+V 375 MB per decode step), no flush"},
+        "pct_of_8tbs": value / world / NOMINAL_HBM_GBS * 100.0,
+        "decode_gbs": achieved,
+        "decode_pct_of_8tbs": achieved / NOMINAL_HBM_GBS * 100.0,
+        "decode_us_per_step": dec_us,
+        "prune_us_per_layer": prune_us,
+        "prune_gbs_1read": W.prune_bytes(w, T) / (prune_us * 1e-6) / 1e9,
+        "roofline": {"kernel": "think_pruned_decode_attn (split kernel + combine kernel), "
+                               "CUDA events around each step's 256 decode calls",
+                     "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": f"{peak_kind} hbm_gbs",
+                     "algorithmic_bytes_per_launch": dec_bytes, "traffic": None},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+        "e2e": e2e,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, T)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_native(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

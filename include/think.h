@@ -1,0 +1,165 @@
+/*
+ * think.h -- C ABI of the ThinK decode-time hot path on NVIDIA B200 (sm_100a).
+ *
+ * Method: "ThinK: Thinner Key Cache by Query-Driven Pruning" (Xu et al., ICLR
+ * 2025).  Its method section gives the flow (technical framework): compute
+ * every key channel's relevance to the query, sort the channels, prune the
+ * least relevant ones, then run inference with the pruned ("thinner") key
+ * cache; its abstract states the aim of the ranking (lose as little of the
+ * attention weights as possible).  The library implements that flow as four
+ * calls, each one or two hand-written CUDA kernels:
+ *
+ *   think_score_channels      s[c] = sum_g ||Qwin_g[:,c]||_2 * ||K[:,c]||_2
+ *   think_select_channels     keep the T largest s[c] (ties: lower index)
+ *   think_compact_keys        K'[n,t] = K[n, idx[t]]   (V is not touched)
+ *   think_pruned_decode_attn  out = softmax((q[idx] . K'^T) / sqrt(d)) V
+ *
+ * Conventions shared by every call
+ *   - Shapes: B batch, Hq query heads, Hkv KV heads (G = Hq/Hkv query heads
+ *     share one KV head; query head h reads KV head h / G), N cached tokens,
+ *     d head width (only d = 128 is built), S_obs window queries, T kept
+ *     channels (1 <= T <= d).
+ *   - dtype: THINK_BF16 (bfloat16) or THINK_F32 (float32) for every input
+ *     tensor of a call; accumulation is fp32 (decode) and fp64 (scores).
+ *   - All tensor pointers are DEVICE pointers, 16-byte aligned.  Strides are
+ *     in ELEMENTS and must be multiples of 16 bytes / element size; the last
+ *     dimension (channels) is always contiguous.
+ *   - Ownership: the caller owns every buffer, including workspaces.  No call
+ *     allocates, frees or synchronises.  Every call validates its arguments
+ *     on the host before any CUDA call, then enqueues its kernels on `stream`
+ *     (a cudaStream_t passed as void*; NULL = the legacy default stream) and
+ *     returns.  Kernel faults surface at the caller's next synchronisation.
+ *   - Errors: a call that returns anything but THINK_OK launched nothing
+ *     (except THINK_ERR_CUDA, returned when a launch itself failed).
+ *   - Empty batches (B == 0 or Hkv == 0) return THINK_OK and launch nothing.
+ *   - Inputs must be finite; selection on NaN/Inf keys is unspecified.
+ *   - Calls on different streams with disjoint buffers may run concurrently;
+ *     calls that share a workspace must be stream-ordered.
+ */
+#ifndef THINK_H_
+#define THINK_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    THINK_OK = 0,
+    THINK_ERR_INVALID_ARG = 1,   /* null pointer, bad shape, T out of range, ... */
+    THINK_ERR_UNSUPPORTED = 2,   /* d != 128, group size not in {1,2,4,8}, ... */
+    THINK_ERR_WORKSPACE = 3,     /* workspace missing or too small */
+    THINK_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed */
+    THINK_ERR_ALIGNMENT = 5      /* pointer or stride not 16-byte aligned */
+} think_status_t;
+
+typedef enum { THINK_F32 = 0, THINK_BF16 = 1 } think_dtype_t;
+
+/* Device-side status bits written into the first 4 bytes of a decode
+ * workspace when a bounded wait inside the decode kernel gives up (the kernel
+ * then returns early and its output is invalid).  Read them with
+ * think_read_device_status; clear them with think_workspace_init. */
+#define THINK_DEVICE_TIMEOUT_FULL  0x1u   /* a tile load never arrived */
+#define THINK_DEVICE_TIMEOUT_EMPTY 0x2u   /* a stage was never released */
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *think_status_string(think_status_t status);
+
+/* Kept channels for pruning ratio lambda (ThinK abstract: prune the least
+ * significant channels): T = floor((1 - lambda) * d + 0.5), clamped to
+ * [1, d].  Returns 0 if d < 1 or lambda is not finite. */
+int think_t_from_lambda(int d, double lambda);
+
+/* Smallest valid token pitch of the thinner key cache for N tokens and the
+ * given dtype: N rounded up to a multiple of 16 bytes.  Returns -1 if N < 0. */
+int64_t think_pruned_ld(int64_t N, think_dtype_t dtype);
+
+/* ---------------------------------------------------------------- score --
+ * Channel relevance of the key cache to the observation window (ThinK,
+ * method section: "compute each channel's relevance to the query"; abstract:
+ * keep the attention weights Qwin K^T).  For each batch item b and KV head
+ * h_kv, with the group's query heads g = h_kv*G .. h_kv*G+G-1:
+ *     kn2[c]  = sum_n K[b,h_kv,n,c]^2                 (fp64)
+ *     s[c]    = sum_g sqrt(sum_s Qwin[b,g,s,c]^2) * sqrt(kn2[c])
+ * which is the Frobenius norm of channel c's rank-one share Qwin_g[:,c]K[:,c]^T
+ * of the window's attention logits, summed over the group.
+ *
+ *   q_win     [B][Hq][S_obs][d] contiguous, dtype.  May be NULL if S_obs == 0.
+ *   k         key cache; element (b,h,n,c) at k[b*k_strides[0] + h*k_strides[1]
+ *             + n*k_strides[2] + c].
+ *   scores    [B][Hkv][d] fp64 output, contiguous.
+ *   workspace device scratch of at least think_score_workspace_size() bytes,
+ *             16-byte aligned; contents on entry do not matter.
+ * Bit-for-bit deterministic for a given shape (fixed summation order).
+ * N == 0 or S_obs == 0 gives all-zero scores. */
+size_t think_score_workspace_size(int B, int Hkv, int64_t N, int d);
+think_status_t think_score_channels(const void *q_win, const void *k, const int64_t k_strides[3],
+                                    int B, int Hq, int Hkv, int64_t N, int S_obs, int d,
+                                    think_dtype_t dtype, double *scores,
+                                    void *workspace, size_t workspace_bytes, void *stream);
+
+/* --------------------------------------------------------------- select --
+ * Top-T channels per (b, h_kv) (ThinK, method section: sort the channels by
+ * relevance and prune the low ones).  Order: larger score first, equal
+ * scores by lower channel index.  The kept channels are written in ascending
+ * channel order, so T = d gives idx = 0..d-1.
+ *   scores  [B][Hkv][d] fp64 (as written by think_score_channels; >= 0).
+ *   idx     [B][Hkv][T] int32 output, contiguous, 4-byte aligned. */
+think_status_t think_select_channels(const double *scores, int B, int Hkv, int d, int T,
+                                     int32_t *idx, void *stream);
+
+/* -------------------------------------------------------------- compact --
+ * Thinner key cache (ThinK title and method section: the key cache keeps only
+ * the selected channels; V is left as it is).  K'[n,t] = K[n, idx[t]], a pure
+ * copy (bit-exact).  K' is stored channel-major so that decode reads each kept
+ * channel as one contiguous run of tokens:
+ *     element (b, h, t, n) of K' at k_pruned[((b*Hkv + h)*T + t)*ldk + n]
+ * with ldk >= N and ldk*sizeof(dtype) a multiple of 16 (see think_pruned_ld).
+ * Columns n in [N, ldk) are not written.
+ *   k, k_strides as for think_score_channels; idx [B][Hkv][T] int32, each in
+ *   [0, d) (checked on the device: an out-of-range index copies zeros). */
+think_status_t think_compact_keys(const void *k, const int64_t k_strides[3], int B, int Hkv,
+                                  int64_t N, int d, think_dtype_t dtype, const int32_t *idx,
+                                  int T, void *k_pruned, int64_t ldk, void *stream);
+
+/* --------------------------------------------------------------- decode --
+ * Decode attention with the thinner key cache (ThinK, method section: run
+ * inference with the pruned cache).  For every query head h (KV head
+ * h_kv = h / G):
+ *     z[n]   = scale * sum_t q[b,h,idx[b,h_kv,t]] * K'[b,h_kv,t,n]
+ *     out    = sum_n softmax(z)[n] * V[b,h_kv,n,:]
+ * Pass scale = 1/sqrt(d) (the full head width, not T) for the unpruned
+ * model's temperature.  Split-N flash decoding: tiles of K' and V are staged
+ * in shared memory by TMA, partial (max, sum, weighted V) per split go to the
+ * workspace, and a second kernel merges them.
+ *   q         [B][Hq][d] contiguous, dtype.
+ *   k_pruned  thinner key cache with pitch ldk, as written by think_compact_keys.
+ *   v         element (b,h,n,c) at v[b*v_strides[0] + h*v_strides[1] + n*v_strides[2] + c].
+ *   idx       [B][Hkv][T] int32 kept channels, each in [0, d).
+ *   out       [B][Hq][d] fp32 output, contiguous.
+ *   workspace at least think_decode_workspace_size() bytes, 16-byte aligned,
+ *             zeroed once by think_workspace_init before its first use (its
+ *             first 4 bytes hold the device status bits; the rest is scratch).
+ * Requires N >= 1 and G in {1, 2, 4, 8}. */
+size_t think_decode_workspace_size(int B, int Hq, int Hkv, int64_t N, int d, think_dtype_t dtype);
+think_status_t think_pruned_decode_attn(const void *q, const void *k_pruned, int64_t ldk,
+                                        const void *v, const int64_t v_strides[3],
+                                        const int32_t *idx, int B, int Hq, int Hkv, int64_t N,
+                                        int d, int T, think_dtype_t dtype, float scale,
+                                        float *out, void *workspace, size_t workspace_bytes,
+                                        void *stream);
+
+/* Zero a decode workspace (stream-ordered memset). */
+think_status_t think_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
+
+/* Copy the device status bits of a decode workspace to *status after the
+ * stream's queued work has finished (synchronises `stream`). */
+think_status_t think_read_device_status(const void *workspace, uint32_t *status, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* THINK_H_ */

@@ -1,0 +1,224 @@
+"""Python binding of libthink.so, the C-ABI CUDA library of the ThinK decode path.
+
+"ThinK: Thinner Key Cache by Query-Driven Pruning": score every key channel
+against the observation-window queries, keep the top-T channels per KV head,
+compact K into a thinner cache, and run decode attention with it.
+
+Argument marshalling only: every function passes device pointers, sizes and
+strides of torch tensors to the C entry point of the same name; every step of
+the computation runs in the library's CUDA kernels. There is no CPU fallback:
+importing this package raises if ``libthink.so`` cannot be loaded.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libthink.so")
+
+THINK_OK = 0
+THINK_ERR_INVALID_ARG = 1
+THINK_ERR_UNSUPPORTED = 2
+THINK_ERR_WORKSPACE = 3
+THINK_ERR_CUDA = 4
+THINK_ERR_ALIGNMENT = 5
+THINK_F32 = 0
+THINK_BF16 = 1
+THINK_DEVICE_TIMEOUT_FULL = 0x1
+THINK_DEVICE_TIMEOUT_EMPTY = 0x2
+
+EXPORTED = (
+    "think_status_string", "think_t_from_lambda", "think_pruned_ld",
+    "think_score_workspace_size", "think_score_channels", "think_select_channels",
+    "think_compact_keys", "think_decode_workspace_size", "think_pruned_decode_attn",
+    "think_workspace_init", "think_read_device_status",
+)
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"libthink.so not found at {LIB_PATH}; build it with "
+            "`python query_driven_key_b200/build.py` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, I64, SZ, D, F = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t,
+                           ctypes.c_double, ctypes.c_float)
+    I64P = ctypes.POINTER(ctypes.c_int64)
+    lib.think_status_string.argtypes = [I]
+    lib.think_status_string.restype = ctypes.c_char_p
+    lib.think_t_from_lambda.argtypes = [I, D]
+    lib.think_t_from_lambda.restype = I
+    lib.think_pruned_ld.argtypes = [I64, I]
+    lib.think_pruned_ld.restype = I64
+    lib.think_score_workspace_size.argtypes = [I, I, I64, I]
+    lib.think_score_workspace_size.restype = SZ
+    lib.think_score_channels.argtypes = [P, P, I64P, I, I, I, I64, I, I, I, P, P, SZ, P]
+    lib.think_score_channels.restype = I
+    lib.think_select_channels.argtypes = [P, I, I, I, I, P, P]
+    lib.think_select_channels.restype = I
+    lib.think_compact_keys.argtypes = [P, I64P, I, I, I64, I, I, P, I, P, I64, P]
+    lib.think_compact_keys.restype = I
+    lib.think_decode_workspace_size.argtypes = [I, I, I, I64, I, I]
+    lib.think_decode_workspace_size.restype = SZ
+    lib.think_pruned_decode_attn.argtypes = [P, P, I64, P, I64P, P, I, I, I, I64, I, I, I, F, P,
+                                             P, SZ, P]
+    lib.think_pruned_decode_attn.restype = I
+    lib.think_workspace_init.argtypes = [P, SZ, P]
+    lib.think_workspace_init.restype = I
+    lib.think_read_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint32), P]
+    lib.think_read_device_status.restype = I
+    return lib
+
+
+lib = _load()
+
+
+class ThinkError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {lib.think_status_string(code).decode()}")
+
+
+def _check(code: int, where: str) -> None:
+    if code != THINK_OK:
+        raise ThinkError(code, where)
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return THINK_BF16
+    if t.dtype == torch.float32:
+        return THINK_F32
+    raise ThinkError(THINK_ERR_INVALID_ARG, f"dtype {t.dtype}")
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr()) if t.numel() > 0 else ctypes.c_void_p(t.data_ptr() or 0)
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _strides3(t: torch.Tensor):
+    if t.dim() != 4 or t.stride(3) != 1:
+        raise ThinkError(THINK_ERR_INVALID_ARG, "expected a [B,H,N,d] tensor with contiguous channels")
+    return (ctypes.c_int64 * 3)(t.stride(0), t.stride(1), t.stride(2))
+
+
+def think_t_from_lambda(d: int, lam: float) -> int:
+    return lib.think_t_from_lambda(int(d), float(lam))
+
+
+def think_pruned_ld(N: int, dtype: torch.dtype = torch.bfloat16) -> int:
+    return lib.think_pruned_ld(int(N), THINK_BF16 if dtype == torch.bfloat16 else THINK_F32)
+
+
+def think_score_workspace_size(B: int, Hkv: int, N: int, d: int = 128) -> int:
+    return lib.think_score_workspace_size(B, Hkv, N, d)
+
+
+def think_decode_workspace_size(B: int, Hq: int, Hkv: int, N: int, d: int = 128,
+                                dtype: torch.dtype = torch.bfloat16) -> int:
+    return lib.think_decode_workspace_size(B, Hq, Hkv, N, d,
+                                           THINK_BF16 if dtype == torch.bfloat16 else THINK_F32)
+
+
+def think_score_channels(q_win: torch.Tensor, k: torch.Tensor, scores: torch.Tensor,
+                         workspace: torch.Tensor, stream=None) -> None:
+    """q_win [B,Hq,S_obs,d] (contiguous), k [B,Hkv,N,d] -> scores [B,Hkv,d] fp64."""
+    B, Hq, S, d = q_win.shape
+    _, Hkv, N, _ = k.shape
+    if not q_win.is_contiguous() or scores.dtype != torch.float64:
+        raise ThinkError(THINK_ERR_INVALID_ARG, "think_score_channels")
+    _check(lib.think_score_channels(_ptr(q_win), _ptr(k), _strides3(k), B, Hq, Hkv, N, S, d,
+                                    _dtype(k), _ptr(scores), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(stream)),
+           "think_score_channels")
+
+
+def think_select_channels(scores: torch.Tensor, T: int, idx: torch.Tensor, stream=None) -> None:
+    """scores [B,Hkv,d] fp64 -> idx [B,Hkv,T] int32 (ascending kept channels)."""
+    B, Hkv, d = scores.shape
+    if scores.dtype != torch.float64 or idx.dtype != torch.int32 or not idx.is_contiguous():
+        raise ThinkError(THINK_ERR_INVALID_ARG, "think_select_channels")
+    _check(lib.think_select_channels(_ptr(scores), B, Hkv, d, int(T), _ptr(idx), _stream(stream)),
+           "think_select_channels")
+
+
+def think_compact_keys(k: torch.Tensor, idx: torch.Tensor, k_pruned: torch.Tensor, ldk: int,
+                       stream=None) -> None:
+    """k [B,Hkv,N,d], idx [B,Hkv,T] -> k_pruned, element (b,h,t,n) at ((b*Hkv+h)*T+t)*ldk+n."""
+    B, Hkv, N, d = k.shape
+    T = idx.shape[-1]
+    if idx.dtype != torch.int32 or k_pruned.dtype != k.dtype:
+        raise ThinkError(THINK_ERR_INVALID_ARG, "think_compact_keys")
+    _check(lib.think_compact_keys(_ptr(k), _strides3(k), B, Hkv, N, d, _dtype(k), _ptr(idx), T,
+                                  _ptr(k_pruned), int(ldk), _stream(stream)), "think_compact_keys")
+
+
+def think_pruned_decode_attn(q: torch.Tensor, k_pruned: torch.Tensor, ldk: int, v: torch.Tensor,
+                             idx: torch.Tensor, out: torch.Tensor, workspace: torch.Tensor,
+                             scale: float | None = None, N: int | None = None,
+                             stream=None) -> None:
+    """q [B,Hq,d], thinner K (pitch ldk), v [B,Hkv,N,d], idx [B,Hkv,T] -> out [B,Hq,d] fp32."""
+    B, Hq, d = q.shape
+    _, Hkv, Nv, _ = v.shape
+    N = Nv if N is None else N
+    T = idx.shape[-1]
+    if scale is None:
+        scale = 1.0 / float(d) ** 0.5
+    if not q.is_contiguous() or out.dtype != torch.float32 or idx.dtype != torch.int32:
+        raise ThinkError(THINK_ERR_INVALID_ARG, "think_pruned_decode_attn")
+    _check(lib.think_pruned_decode_attn(_ptr(q), _ptr(k_pruned), int(ldk), _ptr(v), _strides3(v),
+                                        _ptr(idx), B, Hq, Hkv, N, d, T, _dtype(q), float(scale),
+                                        _ptr(out), _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(),
+                                        _stream(stream)), "think_pruned_decode_attn")
+
+
+def think_workspace_init(workspace: torch.Tensor, stream=None) -> None:
+    _check(lib.think_workspace_init(_ptr(workspace), workspace.numel() * workspace.element_size(),
+                                    _stream(stream)), "think_workspace_init")
+
+
+def think_read_device_status(workspace: torch.Tensor, stream=None) -> int:
+    st = ctypes.c_uint32(0)
+    _check(lib.think_read_device_status(_ptr(workspace), ctypes.byref(st), _stream(stream)),
+           "think_read_device_status")
+    return st.value
+
+
+class PrunedCache:
+    """Device buffers of one pruned layer: kept channels, thinner K, V, workspaces.
+
+    A convenience holder for callers of the functions above; it allocates with
+    torch on construction and then only calls the C entry points."""
+
+    def __init__(self, B: int, Hq: int, Hkv: int, N: int, T: int, d: int = 128,
+                 dtype: torch.dtype = torch.bfloat16, device="cuda"):
+        self.B, self.Hq, self.Hkv, self.N, self.T, self.d, self.dtype = B, Hq, Hkv, N, T, d, dtype
+        self.ldk = think_pruned_ld(N, dtype)
+        self.scores = torch.empty((B, Hkv, d), dtype=torch.float64, device=device)
+        self.idx = torch.empty((B, Hkv, T), dtype=torch.int32, device=device)
+        self.k_pruned = torch.empty((B, Hkv, T, self.ldk), dtype=dtype, device=device)
+        self.score_ws = torch.empty(max(16, think_score_workspace_size(B, Hkv, N, d)),
+                                    dtype=torch.uint8, device=device)
+        self.decode_ws = torch.zeros(max(256, think_decode_workspace_size(B, Hq, Hkv, N, d, dtype)),
+                                     dtype=torch.uint8, device=device)
+
+    def prune(self, q_win, k, stream=None):
+        think_score_channels(q_win, k, self.scores, self.score_ws, stream)
+        think_select_channels(self.scores, self.T, self.idx, stream)
+        think_compact_keys(k, self.idx, self.k_pruned, self.ldk, stream)
+
+    def decode(self, q, v, out, scale=None, stream=None):
+        think_pruned_decode_attn(q, self.k_pruned, self.ldk, v, self.idx, out, self.decode_ws,
+                                 scale=scale, N=self.N, stream=stream)

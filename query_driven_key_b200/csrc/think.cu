@@ -1,0 +1,417 @@
+// think.cu -- host side of the C ABI declared in include/think.h: argument
+// validation, launch planning, TMA descriptors and kernel launches.
+//
+// Method: "ThinK: Thinner Key Cache by Query-Driven Pruning" (method section:
+// score channels against the query, sort, prune, infer with the pruned cache).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "decode_kernels.cuh"
+#include "prune_kernels.cuh"
+#include "think.h"
+
+namespace think {
+namespace {
+
+constexpr int kTargetSMs = 148;             // B200
+constexpr int kScoreBlocksPerSM = 4;        // 256-thread score blocks resident per SM
+constexpr int kDecodeBlocksPerSM = 2;       // decode blocks the plan aims to keep per SM
+constexpr size_t kDecodeHeader = 256;       // status word + reserved, start of the workspace
+constexpr size_t kSmemPerSM = 233472;       // 228 KB
+constexpr size_t kSmemPerBlockMax = 232448; // 227 KB opt-in
+constexpr size_t kSmemReservedPerBlock = 1024;
+
+inline size_t esize(think_dtype_t t) { return t == THINK_BF16 ? 2 : 4; }
+inline bool dtype_ok(int t) { return t == THINK_F32 || t == THINK_BF16; }
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+inline think_status_t launch_status()
+{
+    return cudaGetLastError() == cudaSuccess ? THINK_OK : THINK_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- plans --
+
+struct ScorePlan {
+    int splits;
+    int64_t rows_per_split;
+};
+
+ScorePlan plan_score(int64_t heads, int64_t N)
+{
+    ScorePlan p;
+    const int64_t target = (int64_t)kTargetSMs * kScoreBlocksPerSM;
+    int64_t s = heads >= target ? 1 : target / heads;
+    s = std::max<int64_t>(1, std::min<int64_t>(s, ceil_div(std::max<int64_t>(N, 1), 256)));
+    p.rows_per_split = ceil_div(std::max<int64_t>(N, 1), s);
+    p.splits = (int)ceil_div(std::max<int64_t>(N, 1), p.rows_per_split);
+    return p;
+}
+
+struct DecodeSplit {
+    int splits;
+    int tiles_per_split;
+};
+
+// Split the token axis so that heads*splits fills kDecodeBlocksPerSM blocks on
+// every SM in one wave; each split is a whole number of 128-token tiles.
+DecodeSplit plan_decode_split(int64_t heads, int64_t N)
+{
+    const int64_t tiles = ceil_div(N, kBN);
+    const int64_t target = (int64_t)kTargetSMs * kDecodeBlocksPerSM;
+    int64_t s = std::max<int64_t>(1, target / std::max<int64_t>(heads, 1));
+    s = std::min(s, tiles);
+    const int64_t tps = ceil_div(tiles, s);
+    DecodeSplit d;
+    d.tiles_per_split = (int)tps;
+    d.splits = (int)ceil_div(tiles, tps);
+    return d;
+}
+
+struct DecodeSmem {
+    uint32_t stage_bytes, v_off, tx_bytes;
+    int stages;
+    size_t bytes;
+};
+
+DecodeSmem plan_decode_smem(int T, int G, size_t es)
+{
+    DecodeSmem s;
+    const size_t kt = (size_t)T * kBN * es;
+    const size_t vb = (size_t)kBN * kD * es;
+    s.v_off = (uint32_t)align_up(kt, 1024);
+    s.stage_bytes = (uint32_t)align_up(s.v_off + vb, 1024);
+    s.tx_bytes = (uint32_t)(kt + vb);
+    const size_t extra = align_up((size_t)T * G, 4) * 4 + (size_t)kConsumerWarps * 32 * G * 4 +
+                         2 * 8 * 8 /* up to 8 stages of full+empty barriers */ + 1024 /* alignment slack */;
+    const size_t per_block_2 = kSmemPerSM / kDecodeBlocksPerSM - kSmemReservedPerBlock;
+    int st = (int)((per_block_2 - extra) / s.stage_bytes);
+    if (st >= 2) {
+        s.stages = std::min(st, 4);
+    } else {
+        st = (int)((kSmemPerBlockMax - extra) / s.stage_bytes);
+        s.stages = std::min(std::max(st, 1), 4);
+    }
+    s.bytes = (size_t)s.stages * s.stage_bytes + extra;
+    // the block-merge scratch reuses stage memory: [warps][G][D] + [warps][G][2] floats
+    return s;
+}
+
+// ------------------------------------------------------------ TMA maps --
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 4-D map over (x, y, z, w) with element strides sy, sz, sw for y, z, w; box (bx, by, 1, 1).
+bool make_map_4d(CUtensorMap *m, think_dtype_t dt, const void *base, uint64_t dx, uint64_t dy,
+                 uint64_t dz, uint64_t dw, int64_t sy, int64_t sz, int64_t sw, uint32_t bx,
+                 uint32_t by)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const size_t es = esize(dt);
+    cuuint64_t dims[4] = {dx, dy, dz, dw};
+    cuuint64_t strides[3] = {(cuuint64_t)sy * es, (cuuint64_t)sz * es, (cuuint64_t)sw * es};
+    cuuint32_t box[4] = {bx, by, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUresult r = fn(m, dt == THINK_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                              : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                          4, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------- validation --
+
+bool strides_ok(const int64_t s[3], size_t es)
+{
+    const int64_t q = (int64_t)(16 / es);
+    for (int i = 0; i < 3; ++i)
+        if (s[i] < 0 || s[i] % q != 0) return false;
+    return true;
+}
+
+template <typename TIn, int G>
+think_status_t launch_decode_g(const CUtensorMap &mk, const CUtensorMap &mv, const DecodeArgs &a,
+                               const DecodeSmem &sm, int heads, cudaStream_t st)
+{
+    auto kern = pruned_decode_split_kernel<TIn, G>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm.bytes) !=
+        cudaSuccess)
+        return THINK_ERR_CUDA;
+    dim3 grid(a.splits, heads);
+    kern<<<grid, kDecodeThreads, sm.bytes, st>>>(mk, mv, a);
+    return launch_status();
+}
+
+template <typename TIn>
+think_status_t launch_decode(int G, const CUtensorMap &mk, const CUtensorMap &mv,
+                             const DecodeArgs &a, const DecodeSmem &sm, int heads, cudaStream_t st)
+{
+    switch (G) {
+    case 1: return launch_decode_g<TIn, 1>(mk, mv, a, sm, heads, st);
+    case 2: return launch_decode_g<TIn, 2>(mk, mv, a, sm, heads, st);
+    case 4: return launch_decode_g<TIn, 4>(mk, mv, a, sm, heads, st);
+    case 8: return launch_decode_g<TIn, 8>(mk, mv, a, sm, heads, st);
+    default: return THINK_ERR_UNSUPPORTED;
+    }
+}
+
+}  // namespace
+}  // namespace think
+
+using namespace think;
+
+extern "C" {
+
+const char *think_status_string(think_status_t s)
+{
+    switch (s) {
+    case THINK_OK: return "THINK_OK";
+    case THINK_ERR_INVALID_ARG: return "THINK_ERR_INVALID_ARG: invalid argument";
+    case THINK_ERR_UNSUPPORTED: return "THINK_ERR_UNSUPPORTED: shape or dtype not built";
+    case THINK_ERR_WORKSPACE: return "THINK_ERR_WORKSPACE: workspace missing or too small";
+    case THINK_ERR_CUDA: return "THINK_ERR_CUDA: a CUDA call failed";
+    case THINK_ERR_ALIGNMENT: return "THINK_ERR_ALIGNMENT: pointer or stride not 16-byte aligned";
+    }
+    return "THINK_ERR_UNKNOWN";
+}
+
+int think_t_from_lambda(int d, double lambda)
+{
+    if (d < 1 || !std::isfinite(lambda)) return 0;
+    const double t = std::floor((1.0 - lambda) * (double)d + 0.5);
+    if (t < 1.0) return 1;
+    if (t > (double)d) return d;
+    return (int)t;
+}
+
+int64_t think_pruned_ld(int64_t N, think_dtype_t dtype)
+{
+    if (N < 0 || !dtype_ok(dtype)) return -1;
+    const int64_t q = (int64_t)(16 / esize(dtype));
+    return ceil_div(N, q) * q;
+}
+
+size_t think_score_workspace_size(int B, int Hkv, int64_t N, int d)
+{
+    if (B <= 0 || Hkv <= 0 || N < 0 || d != kD) return 0;
+    const int64_t heads = (int64_t)B * Hkv;
+    const ScorePlan p = plan_score(heads, N);
+    return (size_t)heads * p.splits * kD * sizeof(double);
+}
+
+think_status_t think_score_channels(const void *q_win, const void *k, const int64_t k_strides[3],
+                                    int B, int Hq, int Hkv, int64_t N, int S_obs, int d,
+                                    think_dtype_t dtype, double *scores, void *workspace,
+                                    size_t workspace_bytes, void *stream)
+{
+    if (B < 0 || Hq < 0 || Hkv < 0 || N < 0 || S_obs < 0) return THINK_ERR_INVALID_ARG;
+    if (!dtype_ok(dtype)) return THINK_ERR_INVALID_ARG;
+    if (d != kD) return THINK_ERR_UNSUPPORTED;
+    if (B == 0 || Hkv == 0) return THINK_OK;
+    if (Hq < Hkv || Hq % Hkv != 0) return THINK_ERR_INVALID_ARG;
+    if (!k || !k_strides || !scores || !workspace || (S_obs > 0 && !q_win))
+        return THINK_ERR_INVALID_ARG;
+    const int64_t heads = (int64_t)B * Hkv;
+    if (heads > 65535) return THINK_ERR_UNSUPPORTED;
+    const size_t es = esize(dtype);
+    if (!aligned16(k) || !aligned16(workspace) || (q_win && !aligned16(q_win)) ||
+        !strides_ok(k_strides, es) || (reinterpret_cast<uintptr_t>(scores) & 7u))
+        return THINK_ERR_ALIGNMENT;
+    const ScorePlan p = plan_score(heads, N);
+    if (workspace_bytes < (size_t)heads * p.splits * kD * sizeof(double)) return THINK_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    double *part = static_cast<double *>(workspace);
+    dim3 g1(p.splits, (unsigned)heads);
+    if (dtype == THINK_BF16) {
+        score_partial_kernel<__nv_bfloat16><<<g1, 256, 0, st>>>(
+            static_cast<const __nv_bfloat16 *>(k), k_strides[0], k_strides[1], k_strides[2], Hkv,
+            N, p.rows_per_split, p.splits, part);
+        score_finalize_kernel<__nv_bfloat16><<<(unsigned)heads, kD, 0, st>>>(
+            part, p.splits, static_cast<const __nv_bfloat16 *>(q_win), Hq, Hkv, S_obs, scores);
+    } else {
+        score_partial_kernel<float><<<g1, 256, 0, st>>>(static_cast<const float *>(k), k_strides[0],
+                                                        k_strides[1], k_strides[2], Hkv, N,
+                                                        p.rows_per_split, p.splits, part);
+        score_finalize_kernel<float><<<(unsigned)heads, kD, 0, st>>>(
+            part, p.splits, static_cast<const float *>(q_win), Hq, Hkv, S_obs, scores);
+    }
+    return launch_status();
+}
+
+think_status_t think_select_channels(const double *scores, int B, int Hkv, int d, int T,
+                                     int32_t *idx, void *stream)
+{
+    if (B < 0 || Hkv < 0) return THINK_ERR_INVALID_ARG;
+    if (d != kD) return THINK_ERR_UNSUPPORTED;
+    if (T < 1 || T > d) return THINK_ERR_INVALID_ARG;
+    if (B == 0 || Hkv == 0) return THINK_OK;
+    if (!scores || !idx) return THINK_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(scores) & 7u) || (reinterpret_cast<uintptr_t>(idx) & 3u))
+        return THINK_ERR_ALIGNMENT;
+    const int64_t heads = (int64_t)B * Hkv;
+    if (heads > (int64_t)INT32_MAX / 2) return THINK_ERR_UNSUPPORTED;
+    select_kernel<<<(unsigned)ceil_div(heads, 4), 128, 0, static_cast<cudaStream_t>(stream)>>>(
+        scores, (int)heads, T, idx);
+    return launch_status();
+}
+
+think_status_t think_compact_keys(const void *k, const int64_t k_strides[3], int B, int Hkv,
+                                  int64_t N, int d, think_dtype_t dtype, const int32_t *idx,
+                                  int T, void *k_pruned, int64_t ldk, void *stream)
+{
+    if (B < 0 || Hkv < 0 || N < 0) return THINK_ERR_INVALID_ARG;
+    if (!dtype_ok(dtype)) return THINK_ERR_INVALID_ARG;
+    if (d != kD) return THINK_ERR_UNSUPPORTED;
+    if (T < 1 || T > d) return THINK_ERR_INVALID_ARG;
+    if (ldk < N) return THINK_ERR_INVALID_ARG;
+    if (B == 0 || Hkv == 0 || N == 0) return THINK_OK;
+    if (!k || !k_strides || !idx || !k_pruned) return THINK_ERR_INVALID_ARG;
+    const int64_t heads = (int64_t)B * Hkv;
+    if (heads > 65535) return THINK_ERR_UNSUPPORTED;
+    const size_t es = esize(dtype);
+    if (!aligned16(k) || !aligned16(k_pruned) || !strides_ok(k_strides, es) ||
+        (ldk * (int64_t)es) % 16 != 0 || (reinterpret_cast<uintptr_t>(idx) & 3u))
+        return THINK_ERR_ALIGNMENT;
+    if (ceil_div(N, 64) > INT32_MAX) return THINK_ERR_UNSUPPORTED;
+    dim3 grid((unsigned)ceil_div(N, 64), (unsigned)heads);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dtype == THINK_BF16)
+        compact_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+            static_cast<const __nv_bfloat16 *>(k), k_strides[0], k_strides[1], k_strides[2], Hkv, N,
+            idx, T, static_cast<__nv_bfloat16 *>(k_pruned), ldk);
+    else
+        compact_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float *>(k), k_strides[0],
+                                                    k_strides[1], k_strides[2], Hkv, N, idx, T,
+                                                    static_cast<float *>(k_pruned), ldk);
+    return launch_status();
+}
+
+size_t think_decode_workspace_size(int B, int Hq, int Hkv, int64_t N, int d, think_dtype_t dtype)
+{
+    if (B <= 0 || Hkv <= 0 || Hq < Hkv || Hq % Hkv != 0 || N <= 0 || d != kD || !dtype_ok(dtype))
+        return 0;
+    const int64_t heads = (int64_t)B * Hkv;
+    const int G = Hq / Hkv;
+    const DecodeSplit sp = plan_decode_split(heads, N);
+    const size_t slots = (size_t)heads * sp.splits * G;
+    return kDecodeHeader + slots * kD * sizeof(float) + slots * 2 * sizeof(float);
+}
+
+think_status_t think_pruned_decode_attn(const void *q, const void *k_pruned, int64_t ldk,
+                                        const void *v, const int64_t v_strides[3],
+                                        const int32_t *idx, int B, int Hq, int Hkv, int64_t N,
+                                        int d, int T, think_dtype_t dtype, float scale, float *out,
+                                        void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (B < 0 || Hq < 0 || Hkv < 0 || N < 0) return THINK_ERR_INVALID_ARG;
+    if (!dtype_ok(dtype) || !std::isfinite(scale)) return THINK_ERR_INVALID_ARG;
+    if (d != kD) return THINK_ERR_UNSUPPORTED;
+    if (T < 1 || T > d) return THINK_ERR_INVALID_ARG;
+    if (B == 0 || Hkv == 0) return THINK_OK;
+    if (Hq < Hkv || Hq % Hkv != 0) return THINK_ERR_INVALID_ARG;
+    const int G = Hq / Hkv;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return THINK_ERR_UNSUPPORTED;
+    if (N == 0 || ldk < N) return THINK_ERR_INVALID_ARG;
+    if (!q || !k_pruned || !v || !v_strides || !idx || !out || !workspace)
+        return THINK_ERR_INVALID_ARG;
+    const int64_t heads = (int64_t)B * Hkv;
+    if (heads > 65535 || N > (int64_t)INT32_MAX - kBN) return THINK_ERR_UNSUPPORTED;
+    const size_t es = esize(dtype);
+    if (!aligned16(q) || !aligned16(k_pruned) || !aligned16(v) || !aligned16(workspace) ||
+        !aligned16(out) || !strides_ok(v_strides, es) || (ldk * (int64_t)es) % 16 != 0 ||
+        (reinterpret_cast<uintptr_t>(idx) & 3u))
+        return THINK_ERR_ALIGNMENT;
+    const size_t need = think_decode_workspace_size(B, Hq, Hkv, N, d, dtype);
+    if (workspace_bytes < need) return THINK_ERR_WORKSPACE;
+
+    const DecodeSplit sp = plan_decode_split(heads, N);
+    const DecodeSmem sm = plan_decode_smem(T, G, es);
+    if (sm.bytes > kSmemPerBlockMax) return THINK_ERR_UNSUPPORTED;
+    CUtensorMap mk, mv;
+    // K'^T: x = token (pitch ldk), y = kept channel, z = KV head, w = batch
+    if (!make_map_4d(&mk, dtype, k_pruned, (uint64_t)N, (uint64_t)T, (uint64_t)Hkv, (uint64_t)B,
+                     ldk, (int64_t)T * ldk, (int64_t)Hkv * T * ldk, kBN, (uint32_t)T))
+        return THINK_ERR_CUDA;
+    // V: x = channel, y = token, z = KV head, w = batch
+    if (!make_map_4d(&mv, dtype, v, kD, (uint64_t)N, (uint64_t)Hkv, (uint64_t)B, v_strides[2],
+                     v_strides[1], v_strides[0], kD, kBN))
+        return THINK_ERR_CUDA;
+
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    const size_t slots = (size_t)heads * sp.splits * G;
+    DecodeArgs a;
+    a.q = q;
+    a.idx = idx;
+    a.status = reinterpret_cast<unsigned *>(ws);
+    a.part_o = reinterpret_cast<float *>(ws + kDecodeHeader);
+    a.part_ml = a.part_o + slots * kD;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.T = T;
+    a.N = N;
+    a.tiles_per_split = sp.tiles_per_split;
+    a.splits = sp.splits;
+    a.stages = sm.stages;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.stage_bytes = sm.stage_bytes;
+    a.v_off = sm.v_off;
+    a.tx_bytes = sm.tx_bytes;
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    think_status_t r = dtype == THINK_BF16
+                           ? launch_decode<__nv_bfloat16>(G, mk, mv, a, sm, (int)heads, st)
+                           : launch_decode<float>(G, mk, mv, a, sm, (int)heads, st);
+    if (r != THINK_OK) return r;
+    decode_combine_kernel<<<(unsigned)((int64_t)B * Hq), kD, 0, st>>>(a.part_o, a.part_ml, out, Hq,
+                                                                      Hkv, sp.splits);
+    return launch_status();
+}
+
+think_status_t think_workspace_init(void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (!workspace) return THINK_ERR_INVALID_ARG;
+    if (workspace_bytes == 0) return THINK_OK;
+    return cudaMemsetAsync(workspace, 0, workspace_bytes, static_cast<cudaStream_t>(stream)) ==
+                   cudaSuccess
+               ? THINK_OK
+               : THINK_ERR_CUDA;
+}
+
+think_status_t think_read_device_status(const void *workspace, uint32_t *status, void *stream)
+{
+    if (!workspace || !status) return THINK_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(status, workspace, sizeof(uint32_t), cudaMemcpyDeviceToHost, st) !=
+        cudaSuccess)
+        return THINK_ERR_CUDA;
+    return cudaStreamSynchronize(st) == cudaSuccess ? THINK_OK : THINK_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,66 @@
+"""Shared helpers of the GPU parity tests: run the library on a workload and
+compare with the fp64 oracle under the acceptance rules.
+
+Acceptance (bf16 inputs, fp32 accumulation): kept-channel indices and the
+thinner key cache bit-exact; decode output max-abs <= 2e-3 and relative L2
+<= 1e-3. fp32 inputs: max-abs <= 1e-5 and relative L2 <= 1e-6. Index lists may
+differ only at a near-tie: every channel in which they differ must have an
+oracle score within 1e-6 relative of the cut (the T-th largest score).
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+
+TOL = {torch.bfloat16: (2e-3, 1e-3), torch.float32: (1e-5, 1e-6)}
+NEAR_TIE_REL = 1e-6
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def check_scores(gpu_scores: torch.Tensor, ora_scores: np.ndarray, rtol: float = 1e-12):
+    g = f64(gpu_scores)
+    np.testing.assert_allclose(g, ora_scores, rtol=rtol, atol=0)
+
+
+def idx_mismatch_heads(gpu_idx: np.ndarray, ora_idx: np.ndarray, ora_scores: np.ndarray, T: int):
+    """Return the list of (b, h) whose index lists differ; assert every difference
+    is a near-tie at the cut and that the GPU list is a valid ascending set."""
+    bad = []
+    B, H, _ = ora_idx.shape
+    for b in range(B):
+        for h in range(H):
+            gi = gpu_idx[b, h]
+            assert np.all(np.diff(gi) > 0), f"idx not strictly ascending at {(b, h)}: {gi}"
+            assert gi.min() >= 0 and gi.max() < ora_scores.shape[-1]
+            if np.array_equal(gi, ora_idx[b, h]):
+                continue
+            s = ora_scores[b, h]
+            cut = np.sort(s)[::-1][T - 1]
+            diff = np.setxor1d(gi, ora_idx[b, h])
+            for c in diff:
+                assert abs(s[c] - cut) <= NEAR_TIE_REL * abs(cut), (
+                    f"head {(b, h)}: channel {c} score {s[c]!r} is not a near-tie of cut {cut!r}")
+            bad.append((b, h))
+    return bad
+
+
+def check_out(gpu_out: torch.Tensor, ora_out: np.ndarray, dtype, where: str = ""):
+    g = f64(gpu_out)
+    max_abs_tol, rel_l2_tol = TOL[dtype]
+    err = np.abs(g - ora_out)
+    max_abs = float(err.max()) if err.size else 0.0
+    rel_l2 = float(np.linalg.norm(g - ora_out) / max(np.linalg.norm(ora_out), 1e-300))
+    assert np.all(np.isfinite(g)), f"{where}: non-finite output"
+    assert max_abs <= max_abs_tol and rel_l2 <= rel_l2_tol, (
+        f"{where}: max_abs {max_abs:.3e} (tol {max_abs_tol}) rel_l2 {rel_l2:.3e} (tol {rel_l2_tol})")
+    return max_abs, rel_l2
+
+
+def kp_logical(k_pruned: torch.Tensor, N: int) -> np.ndarray:
+    """Thinner cache buffer [B,Hkv,T,ldk] -> K'[B,Hkv,N,T] values (fp64)."""
+    return f64(k_pruned[..., :N].transpose(-1, -2))

@@ -1,0 +1,127 @@
+"""CPU checks of the C ABI: the library loads, exports every entry point the
+header declares, and its host-side logic (T rule, pitch, workspace sizes,
+argument validation) behaves as documented. No kernel is launched here: every
+call below is rejected by host validation before any CUDA call, or is a pure
+host function."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+
+qdk = pytest.importorskip("query_driven_key_b200")
+lib = qdk.lib
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "think.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(think_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in think.h but not exported"
+    assert set(names) == set(qdk.EXPORTED)
+
+
+def test_library_is_built_for_sm100a_in_tree():
+    assert os.path.dirname(qdk.LIB_PATH) == os.path.dirname(qdk.__file__)
+
+
+@pytest.mark.parametrize("d", [1, 8, 10, 128])
+def test_t_from_lambda_matches_oracle_rule(d):
+    for i in range(0, 101):
+        lam = i / 100
+        assert qdk.think_t_from_lambda(d, lam) == oracle.t_from_lambda(d, lam), (d, lam)
+    assert lib.think_t_from_lambda(0, 0.5) == 0
+    assert lib.think_t_from_lambda(128, float("nan")) == 0
+
+
+def test_pruned_pitch():
+    import torch
+    assert qdk.think_pruned_ld(0) == 0
+    assert qdk.think_pruned_ld(1) == 8
+    assert qdk.think_pruned_ld(131072) == 131072
+    assert qdk.think_pruned_ld(4097) == 4104
+    assert qdk.think_pruned_ld(5, torch.float32) == 8
+    assert lib.think_pruned_ld(-1, 1) == -1
+
+
+def test_workspace_sizes():
+    assert qdk.think_score_workspace_size(1, 8, 131072) > 0
+    assert qdk.think_score_workspace_size(1, 8, 131072, d=64) == 0
+    n4 = qdk.think_decode_workspace_size(1, 32, 8, 131072)
+    assert n4 >= 256 + 8 * 4 * 130 * 4
+    assert qdk.think_decode_workspace_size(1, 32, 8, 0) == 0
+    assert qdk.think_decode_workspace_size(1, 30, 8, 100) == 0       # Hq not a multiple of Hkv
+
+
+def test_status_strings():
+    for code in range(6):
+        assert lib.think_status_string(code).startswith(b"THINK_")
+    assert lib.think_status_string(99) == b"THINK_ERR_UNKNOWN"
+
+
+I64x3 = ctypes.c_int64 * 3
+FAKE = ctypes.c_void_p(0x10000)       # never dereferenced: validation rejects first
+MISALIGNED = ctypes.c_void_p(0x10008)
+
+
+def test_score_validation():
+    st = (128 * 64, 128 * 64, 128)
+    s = I64x3(*st)
+    f = lib.think_score_channels
+    assert f(FAKE, FAKE, s, 1, 4, 2, 64, 8, 64, 1, FAKE, FAKE, 1 << 20, None) == qdk.THINK_ERR_UNSUPPORTED
+    assert f(FAKE, FAKE, s, 0, 4, 2, 64, 8, 128, 1, FAKE, FAKE, 0, None) == qdk.THINK_OK   # empty
+    assert f(FAKE, None, s, 1, 4, 2, 64, 8, 128, 1, FAKE, FAKE, 1 << 20, None) == qdk.THINK_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, s, 1, 6, 4, 64, 8, 128, 1, FAKE, FAKE, 1 << 20, None) == qdk.THINK_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, s, 1, 4, 2, 64, 8, 128, 7, FAKE, FAKE, 1 << 20, None) == qdk.THINK_ERR_INVALID_ARG
+    assert f(FAKE, MISALIGNED, s, 1, 4, 2, 64, 8, 128, 1, FAKE, FAKE, 1 << 20, None) == qdk.THINK_ERR_ALIGNMENT
+    bad = I64x3(128 * 64, 128 * 64, 130)
+    assert f(FAKE, FAKE, bad, 1, 4, 2, 64, 8, 128, 1, FAKE, FAKE, 1 << 20, None) == qdk.THINK_ERR_ALIGNMENT
+    assert f(FAKE, FAKE, s, 1, 4, 2, 64, 8, 128, 1, FAKE, FAKE, 16, None) == qdk.THINK_ERR_WORKSPACE
+
+
+def test_select_validation():
+    f = lib.think_select_channels
+    assert f(FAKE, 1, 2, 128, 0, FAKE, None) == qdk.THINK_ERR_INVALID_ARG
+    assert f(FAKE, 1, 2, 128, 129, FAKE, None) == qdk.THINK_ERR_INVALID_ARG
+    assert f(FAKE, 1, 2, 96, 10, FAKE, None) == qdk.THINK_ERR_UNSUPPORTED
+    assert f(None, 1, 2, 128, 10, FAKE, None) == qdk.THINK_ERR_INVALID_ARG
+    assert f(FAKE, 0, 2, 128, 10, FAKE, None) == qdk.THINK_OK
+
+
+def test_compact_validation():
+    s = I64x3(128 * 64, 128 * 64, 128)
+    f = lib.think_compact_keys
+    assert f(FAKE, s, 1, 2, 64, 128, 1, FAKE, 10, FAKE, 63, None) == qdk.THINK_ERR_INVALID_ARG   # ldk < N
+    assert f(FAKE, s, 1, 2, 64, 128, 1, FAKE, 10, FAKE, 68, None) == qdk.THINK_ERR_ALIGNMENT     # 136 B pitch
+    assert f(FAKE, s, 1, 2, 64, 128, 1, FAKE, 0, FAKE, 64, None) == qdk.THINK_ERR_INVALID_ARG
+    assert f(FAKE, s, 1, 2, 0, 128, 1, FAKE, 10, FAKE, 0, None) == qdk.THINK_OK                  # N == 0
+
+
+def test_decode_validation():
+    s = I64x3(128 * 64 * 2, 128 * 64, 128)
+    f = lib.think_pruned_decode_attn
+    args = lambda **kw: dict(dict(q=FAKE, kp=FAKE, ldk=64, v=FAKE, vs=s, idx=FAKE, B=1, Hq=4, Hkv=2,
+                                   N=64, d=128, T=10, dt=1, scale=0.088, out=FAKE, ws=FAKE,
+                                   wsb=1 << 20), **kw)
+    call = lambda a: f(a["q"], a["kp"], a["ldk"], a["v"], a["vs"], a["idx"], a["B"], a["Hq"], a["Hkv"],
+                       a["N"], a["d"], a["T"], a["dt"], a["scale"], a["out"], a["ws"], a["wsb"], None)
+    assert call(args(N=0, ldk=0)) == qdk.THINK_ERR_INVALID_ARG          # attention over no keys
+    assert call(args(Hq=6)) == qdk.THINK_ERR_UNSUPPORTED                 # group of 3
+    assert call(args(Hq=32, Hkv=2)) == qdk.THINK_ERR_UNSUPPORTED         # group of 16
+    assert call(args(T=0)) == qdk.THINK_ERR_INVALID_ARG
+    assert call(args(d=64)) == qdk.THINK_ERR_UNSUPPORTED
+    assert call(args(scale=float("inf"))) == qdk.THINK_ERR_INVALID_ARG
+    assert call(args(q=MISALIGNED)) == qdk.THINK_ERR_ALIGNMENT
+    assert call(args(wsb=64)) == qdk.THINK_ERR_WORKSPACE
+    assert call(args(out=None)) == qdk.THINK_ERR_INVALID_ARG
+    assert call(args(B=0)) == qdk.THINK_OK

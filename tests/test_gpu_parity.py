@@ -1,0 +1,221 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 CPU oracle.
+
+Every input comes from the seeded generators in query_driven_key_b200.workloads;
+every expected value comes from the oracle on the same (bf16-rounded) inputs.
+Kept channels and the thinner key cache must match bit for bit (near-ties at the
+cut excepted, see tests/helpers.py); decode outputs within the stated
+tolerances. The full-size workloads run in the same launch configuration as
+bench.py (the launch plan depends only on the shape).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests.helpers import TOL, check_out, check_scores, f64, idx_mismatch_heads, kp_logical
+
+pytestmark = pytest.mark.gpu
+
+qdk = pytest.importorskip("query_driven_key_b200")
+from query_driven_key_b200 import workloads as W  # noqa: E402
+
+DEV = "cuda"
+
+
+def _prune_gpu(q_win, k, T):
+    B, Hq, S, d = q_win.shape
+    _, Hkv, N, _ = k.shape
+    cache = qdk.PrunedCache(B, Hq, Hkv, N, T, d, dtype=k.dtype)
+    cache.prune(q_win, k)
+    return cache
+
+
+def _full_path_check(w, q_win, k, v, steps, T=None):
+    T = qdk.think_t_from_lambda(w.d, w.lam) if T is None else T
+    assert T == oracle.t_from_lambda(w.d, w.lam)
+    qd, kd, vd = q_win.to(DEV), k.to(DEV), v.to(DEV)
+    cache = _prune_gpu(qd, kd, T)
+    torch.cuda.synchronize()
+    ora_scores, ora_idx, ora_kp = oracle.oracle_prune(f64(q_win), f64(k), T)
+    check_scores(cache.scores, ora_scores)
+    gpu_idx = cache.idx.cpu().numpy()
+    ties = idx_mismatch_heads(gpu_idx, ora_idx, ora_scores, T)
+    if ties:
+        # Near-tie heads: compact and decode again from the oracle's kept set so
+        # both sides attend over the same channels.
+        cache.idx.copy_(torch.from_numpy(ora_idx))
+        qdk.think_compact_keys(kd, cache.idx, cache.k_pruned, cache.ldk)
+    assert np.array_equal(kp_logical(cache.k_pruned, w.N), ora_kp), "thinner key cache differs"
+    out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=DEV)
+    fv = f64(v)
+    for step in steps:
+        q = W.gen_decode_q(w, step)
+        cache.decode(q.to(DEV), vd, out)
+        torch.cuda.synchronize()
+        ora = oracle.oracle_decode(f64(q), ora_kp, fv, ora_idx)
+        check_out(out, ora, w.dtype, where=f"{w.name} step {step}")
+    assert qdk.think_read_device_status(cache.decode_ws) == 0
+    return cache
+
+
+def test_tiny_fp32():
+    w = W.WORKLOADS["tiny_fp32"]
+    q_win, k, v = W.gen_layer(w)
+    _full_path_check(w, q_win, k, v, steps=range(w.decode_steps))
+
+
+def test_llama2_mha_all_steps():
+    w = W.WORKLOADS["llama2_7b_mha"]
+    q_win, k, v = W.gen_layer(w)
+    _full_path_check(w, q_win, k, v, steps=range(w.decode_steps))
+
+
+def test_llama3_gqa_lowrank():
+    w = W.WORKLOADS["llama3_8b_gqa"]
+    q_win, k, v = W.gen_layer(w)
+    _full_path_check(w, q_win, k, v, steps=[0, 1, 2])
+
+
+def test_mistral_long_context():
+    # the bench workload, full size: prune + decode steps {0, 1, 2, last}
+    w = W.WORKLOADS["mistral_7b_long"]
+    q_win, k, v = W.gen_layer(w)
+    _full_path_check(w, q_win, k, v, steps=[0, 1, 2, w.decode_steps - 1])
+
+
+@pytest.mark.parametrize("layer", [0, 31])
+def test_sweep_32_layers(layer):
+    # Each (B, lambda) of the sweep on one layer; the GPU runs the whole batch,
+    # the oracle checks the first and last batch items.
+    base = W.WORKLOADS["sweep_32l"]
+    for B in W.SWEEP_BATCHES:
+        w = base.with_(B=B)
+        q_win, k, v = W.gen_layer(w, layer)
+        qd, kd, vd = q_win.to(DEV), k.to(DEV), v.to(DEV)
+        q = W.gen_decode_q(w, 0, layer)
+        for lam in W.SWEEP_LAMBDAS:
+            T = qdk.think_t_from_lambda(w.d, lam)
+            cache = _prune_gpu(qd, kd, T)
+            out = torch.empty((B, w.Hq, w.d), dtype=torch.float32, device=DEV)
+            cache.decode(q.to(DEV), vd, out)
+            torch.cuda.synchronize()
+            gpu_idx = cache.idx.cpu().numpy()
+            for b in sorted({0, B - 1}):
+                ora_scores, ora_idx, ora_kp = oracle.oracle_prune(f64(q_win[b:b + 1]), f64(k[b:b + 1]), T)
+                check_scores(cache.scores[b:b + 1], ora_scores)
+                assert not idx_mismatch_heads(gpu_idx[b:b + 1], ora_idx, ora_scores, T)
+                assert np.array_equal(kp_logical(cache.k_pruned[b:b + 1], w.N), ora_kp)
+                ora = oracle.oracle_decode(f64(q[b:b + 1]), ora_kp, f64(v[b:b + 1]), ora_idx)
+                check_out(out[b:b + 1], ora, w.dtype, where=f"layer {layer} B{B} lam{lam} b{b}")
+                if lam == 0.0:
+                    assert np.array_equal(ora_idx[0], np.broadcast_to(np.arange(w.d), (w.Hkv, w.d)))
+                    assert np.array_equal(kp_logical(cache.k_pruned[b:b + 1], w.N), f64(k[b:b + 1]))
+                    dense = oracle.oracle_dense_decode(f64(q[b:b + 1]), f64(k[b:b + 1]), f64(v[b:b + 1]))
+                    check_out(out[b:b + 1], dense, w.dtype, where="lambda=0 vs dense")
+
+
+# ------------------------------------------------------------ edge cases ---
+
+def _random_case(seed, B, Hq, Hkv, N, S, dtype, k_pad=0, v_pad=0):
+    g = torch.Generator().manual_seed(seed)
+    d = 128
+    q_win = torch.randn((B, Hq, S, d), generator=g).to(dtype)
+    kbig = torch.randn((B, Hkv, N + k_pad, d), generator=g) * torch.exp(torch.randn((B, Hkv, 1, d), generator=g))
+    vbig = torch.randn((B, Hkv, N + v_pad, d), generator=g)
+    q = torch.randn((B, Hq, d), generator=g).to(dtype)
+    # strided views when padded: the token axis of a bigger buffer
+    return q_win, kbig.to(dtype)[:, :, :N], vbig.to(dtype)[:, :, :N], q
+
+
+EDGE = [
+    # (B, Hq, Hkv, N, S, T)
+    (1, 1, 1, 1, 1, 1),
+    (1, 2, 1, 7, 3, 128),
+    (2, 4, 2, 100, 5, 127),
+    (1, 8, 1, 129, 4, 51),
+    (3, 8, 4, 1000, 8, 77),
+    (1, 16, 2, 4097, 16, 64),
+    (2, 32, 4, 2049, 32, 1),
+    (1, 4, 4, 257, 0, 13),     # empty window: all scores zero, channels 0..T-1 kept
+]
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("case", EDGE)
+def test_edge_shapes(case, dtype):
+    B, Hq, Hkv, N, S, T = case
+    q_win, k, v, q = _random_case(hash(case) & 0xFFFF, B, Hq, Hkv, N, S, dtype, k_pad=8, v_pad=16)
+    kd, vd = k.to(DEV), v.to(DEV)
+    # keep the strided layout on the device
+    kd = torch.empty((B, Hkv, N + 8, 128), dtype=dtype, device=DEV)[:, :, :N].copy_(k)
+    vd = torch.empty((B, Hkv, N + 16, 128), dtype=dtype, device=DEV)[:, :, :N].copy_(v)
+    cache = _prune_gpu(q_win.to(DEV), kd, T)
+    out = torch.empty((B, Hq, 128), dtype=torch.float32, device=DEV)
+    cache.decode(q.to(DEV), vd, out)
+    torch.cuda.synchronize()
+    ora_scores, ora_idx, ora_kp = oracle.oracle_prune(f64(q_win), f64(k), T)
+    check_scores(cache.scores, ora_scores)
+    assert not idx_mismatch_heads(cache.idx.cpu().numpy(), ora_idx, ora_scores, T)
+    assert np.array_equal(kp_logical(cache.k_pruned, N), ora_kp)
+    check_out(out, oracle.oracle_decode(f64(q), ora_kp, f64(v), ora_idx), dtype, where=str(case))
+    if S == 0:
+        assert np.array_equal(cache.idx.cpu().numpy()[0, 0], np.arange(T))
+
+
+def test_ldk_larger_than_needed_and_exact_ties():
+    # duplicate channels give exact score ties: lower index must win on both sides
+    B, Hq, Hkv, N, S, T = 1, 4, 2, 300, 6, 40
+    q_win, k, v, q = _random_case(5, B, Hq, Hkv, N, S, torch.bfloat16)
+    k[..., 64:96] = k[..., 0:32]
+    q_win[..., 64:96] = q_win[..., 0:32]
+    kd = k.contiguous().to(DEV)
+    ldk = 512
+    scores = torch.empty((B, Hkv, 128), dtype=torch.float64, device=DEV)
+    ws = torch.empty(qdk.think_score_workspace_size(B, Hkv, N), dtype=torch.uint8, device=DEV)
+    idx = torch.empty((B, Hkv, T), dtype=torch.int32, device=DEV)
+    kp = torch.full((B, Hkv, T, ldk), 7.0, dtype=torch.bfloat16, device=DEV)
+    qdk.think_score_channels(q_win.to(DEV), kd, scores, ws)
+    qdk.think_select_channels(scores, T, idx)
+    qdk.think_compact_keys(kd, idx, kp, ldk)
+    torch.cuda.synchronize()
+    s, oi, okp = oracle.oracle_prune(f64(q_win), f64(k), T)
+    assert np.array_equal(idx.cpu().numpy(), oi)
+    assert np.array_equal(kp_logical(kp, N), okp)
+    assert torch.all(kp[..., N:] == 7.0), "columns beyond N must not be written"
+
+
+def test_scores_are_deterministic():
+    w = W.WORKLOADS["llama2_7b_mha"]
+    q_win, k, _ = W.gen_slice(w, 0, 0)
+    qd, kd = q_win[None].to(DEV), k[None].to(DEV)
+    a = _prune_gpu(qd, kd, 77)
+    b = _prune_gpu(qd, kd, 77)
+    torch.cuda.synchronize()
+    assert torch.equal(a.scores, b.scores)
+    assert torch.equal(a.idx, b.idx)
+
+
+# ------------------------------------------------------------ validation ---
+
+def test_host_validation_errors_launch_nothing():
+    B, Hq, Hkv, N = 1, 4, 2, 64
+    q = torch.zeros((B, Hq, 128), dtype=torch.bfloat16, device=DEV)
+    v = torch.zeros((B, Hkv, N, 128), dtype=torch.bfloat16, device=DEV)
+    idx = torch.zeros((B, Hkv, 4), dtype=torch.int32, device=DEV)
+    out = torch.zeros((B, Hq, 128), dtype=torch.float32, device=DEV)
+    kp = torch.zeros((B, Hkv, 4, 64), dtype=torch.bfloat16, device=DEV)
+    ws_n = qdk.think_decode_workspace_size(B, Hq, Hkv, N)
+    ws = torch.zeros(ws_n, dtype=torch.uint8, device=DEV)
+    with pytest.raises(qdk.ThinkError) as e:
+        qdk.think_pruned_decode_attn(q, kp, 64, v, idx, out, ws[: ws_n - 16])
+    assert e.value.code == qdk.THINK_ERR_WORKSPACE
+    with pytest.raises(qdk.ThinkError) as e:
+        qdk.think_pruned_decode_attn(q, kp, 60, v, idx, out, ws)   # pitch not 16-byte multiple
+    assert e.value.code in (qdk.THINK_ERR_ALIGNMENT, qdk.THINK_ERR_INVALID_ARG)
+    q3 = torch.zeros((B, 6, 128), dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(qdk.ThinkError) as e:
+        qdk.think_pruned_decode_attn(q3, kp, 64, v, idx, torch.zeros((B, 6, 128), device=DEV),
+                                     torch.zeros(1 << 20, dtype=torch.uint8, device=DEV))
+    assert e.value.code == qdk.THINK_ERR_UNSUPPORTED          # group of 3
+    torch.cuda.synchronize()
+    assert torch.all(out == 0)
