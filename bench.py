@@ -137,9 +137,10 @@ def step_bytes(w, T):
     return W.prune_bytes(w, T) + w.decode_steps * W.decode_bytes(w, T)
 
 
-def cpu_baseline(w, T, seed_layer=0):
+def cpu_baseline(w, T, seed_layer=0, budget_s=12.0):
     """The fp64 oracle as it stands, on this host's cores, on a bounded sample
-    of the workload: the whole prune pass plus 4 of the 256 decode steps."""
+    of the workload: the whole prune pass plus as many of the 256 decode steps
+    as fit in about budget_s seconds (at least 4)."""
     import torch
     import oracle
     from query_driven_key_b200 import workloads as W
@@ -147,16 +148,17 @@ def cpu_baseline(w, T, seed_layer=0):
     q_win, k, v = W.gen_layer(w, seed_layer)
     f64 = lambda t: t.to(torch.float64).numpy()
     qw, kk, vv = f64(q_win), f64(k), f64(v)
-    qs = [f64(W.gen_decode_q(w, s, seed_layer)) for s in range(4)]
     o = oracle.default_oracle()
     t0 = time.perf_counter()
     _, idx, kp = o.prune(qw, kk, T)
-    for q in qs:
-        o.decode(q, kp, vv, idx)
+    steps = 0
+    while steps < w.decode_steps and (steps < 4 or time.perf_counter() - t0 < budget_s):
+        o.decode(f64(W.gen_decode_q(w, steps, seed_layer)), kp, vv, idx)
+        steps += 1
     dt = time.perf_counter() - t0
-    nbytes = W.prune_bytes(w, T) + len(qs) * W.decode_bytes(w, T)
+    nbytes = W.prune_bytes(w, T) + steps * W.decode_bytes(w, T)
     return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": o.num_threads(), "kind": "oracle",
-            "sample": f"prune of all {w.B * w.Hkv} KV heads + {len(qs)} of {w.decode_steps} decode "
+            "sample": f"prune of all {w.B * w.Hkv} KV heads + {steps} of {w.decode_steps} decode "
                       f"steps, fp64 C loops (OpenMP over heads), {dt:.2f} s"}
 
 
