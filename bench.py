@@ -238,7 +238,7 @@ def run_native(args):
         outs = torch.empty((w.decode_steps, w.B, w.Hq, w.d), dtype=torch.float32, device=dev)
     stream.synchronize()
 
-    launches_per_step = 4 + 2 * w.decode_steps  # score x2, select, compact, decode x2 per step
+    launches_per_step = 2 + w.decode_steps  # prune: score+select, compact; one kernel per decode
 
     def one_step(ev=None):
         if ev is not None:
@@ -343,7 +343,7 @@ def run_native(args):
         "decode_us_per_step": dec_us,
         "prune_us_per_layer": prune_us,
         "prune_gbs_1read": W.prune_bytes(w, T) / (prune_us * 1e-6) / 1e9,
-        "roofline": {"kernel": "think_pruned_decode_attn (split kernel + combine kernel), "
+        "roofline": {"kernel": "pruned_decode_kernel (think_pruned_decode_attn, one launch), "
                                "CUDA events around each step's 256 decode calls",
                      "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": f"{peak_kind} hbm_gbs",

@@ -7,12 +7,14 @@
  * least relevant ones, then run inference with the pruned ("thinner") key
  * cache; its abstract states the aim of the ranking (lose as little of the
  * attention weights as possible).  The library implements that flow as four
- * calls, each one or two hand-written CUDA kernels:
+ * calls, each one hand-written CUDA kernel:
  *
  *   think_score_channels      s[c] = sum_g ||Qwin_g[:,c]||_2 * ||K[:,c]||_2
  *   think_select_channels     keep the T largest s[c] (ties: lower index)
  *   think_compact_keys        K'[n,t] = K[n, idx[t]]   (V is not touched)
  *   think_pruned_decode_attn  out = softmax((q[idx] . K'^T) / sqrt(d)) V
+ *
+ * plus think_prune, the first three in two launches.
  *
  * Conventions shared by every call
  *   - Shapes: B batch, Hq query heads, Hkv KV heads (G = Hq/Hkv query heads
@@ -91,10 +93,12 @@ int64_t think_pruned_ld(int64_t N, think_dtype_t dtype);
  *             + n*k_strides[2] + c].
  *   scores    [B][Hkv][d] fp64 output, contiguous.
  *   workspace device scratch of at least think_score_workspace_size() bytes,
- *             16-byte aligned; contents on entry do not matter.
- * Bit-for-bit deterministic for a given shape (fixed summation order).
- * N == 0 or S_obs == 0 gives all-zero scores. */
-size_t think_score_workspace_size(int B, int Hkv, int64_t N, int d);
+ *             16-byte aligned, zeroed once by think_workspace_init before its
+ *             first use (it starts with per-head arrival counters that every
+ *             call leaves at zero; the rest is scratch).
+ * One kernel launch.  Bit-for-bit deterministic for a given shape (fixed
+ * summation order).  N == 0 or S_obs == 0 gives all-zero scores. */
+size_t think_score_workspace_size(int B, int Hq, int Hkv, int64_t N, int d);
 think_status_t think_score_channels(const void *q_win, const void *k, const int64_t k_strides[3],
                                     int B, int Hq, int Hkv, int64_t N, int S_obs, int d,
                                     think_dtype_t dtype, double *scores,
@@ -124,6 +128,17 @@ think_status_t think_compact_keys(const void *k, const int64_t k_strides[3], int
                                   int64_t N, int d, think_dtype_t dtype, const int32_t *idx,
                                   int T, void *k_pruned, int64_t ldk, void *stream);
 
+/* ---------------------------------------------------------------- prune --
+ * The whole prune step of one layer in two launches: scores and the top-T
+ * selection in one kernel (the last block of each head selects), then the
+ * compaction.  Same results as think_score_channels, think_select_channels
+ * and think_compact_keys called in a row; arguments as documented there.
+ * workspace: think_score_workspace_size() bytes, zeroed once before first use. */
+think_status_t think_prune(const void *q_win, const void *k, const int64_t k_strides[3], int B,
+                           int Hq, int Hkv, int64_t N, int S_obs, int d, think_dtype_t dtype,
+                           int T, double *scores, int32_t *idx, void *k_pruned, int64_t ldk,
+                           void *workspace, size_t workspace_bytes, void *stream);
+
 /* --------------------------------------------------------------- decode --
  * Decode attention with the thinner key cache (ThinK, method section: run
  * inference with the pruned cache).  For every query head h (KV head
@@ -131,17 +146,20 @@ think_status_t think_compact_keys(const void *k, const int64_t k_strides[3], int
  *     z[n]   = scale * sum_t q[b,h,idx[b,h_kv,t]] * K'[b,h_kv,t,n]
  *     out    = sum_n softmax(z)[n] * V[b,h_kv,n,:]
  * Pass scale = 1/sqrt(d) (the full head width, not T) for the unpruned
- * model's temperature.  Split-N flash decoding: tiles of K' and V are staged
- * in shared memory by TMA, partial (max, sum, weighted V) per split go to the
- * workspace, and a second kernel merges them.
+ * model's temperature.  Split-N flash decoding in one kernel launch: tiles of
+ * K' and V are staged in shared memory by TMA, each block writes a partial
+ * (max, sum, weighted V) for its split to the workspace, and the last block
+ * of each KV head to finish merges that head's partials into `out`.
  *   q         [B][Hq][d] contiguous, dtype.
  *   k_pruned  thinner key cache with pitch ldk, as written by think_compact_keys.
  *   v         element (b,h,n,c) at v[b*v_strides[0] + h*v_strides[1] + n*v_strides[2] + c].
  *   idx       [B][Hkv][T] int32 kept channels, each in [0, d).
  *   out       [B][Hq][d] fp32 output, contiguous.
  *   workspace at least think_decode_workspace_size() bytes, 16-byte aligned,
- *             zeroed once by think_workspace_init before its first use (its
- *             first 4 bytes hold the device status bits; the rest is scratch).
+ *             zeroed once by think_workspace_init before its first use.  Its
+ *             first 4 bytes hold the device status bits, then come per-head
+ *             arrival counters that every completed call leaves at zero; the
+ *             rest is scratch.
  * Requires N >= 1 and G in {1, 2, 4, 8}. */
 size_t think_decode_workspace_size(int B, int Hq, int Hkv, int64_t N, int d, think_dtype_t dtype);
 think_status_t think_pruned_decode_attn(const void *q, const void *k_pruned, int64_t ldk,
@@ -151,7 +169,7 @@ think_status_t think_pruned_decode_attn(const void *q, const void *k_pruned, int
                                         float *out, void *workspace, size_t workspace_bytes,
                                         void *stream);
 
-/* Zero a decode workspace (stream-ordered memset). */
+/* Zero a score or decode workspace (stream-ordered memset). */
 think_status_t think_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
 
 /* Copy the device status bits of a decode workspace to *status after the

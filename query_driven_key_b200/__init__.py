@@ -33,7 +33,7 @@ THINK_DEVICE_TIMEOUT_EMPTY = 0x2
 EXPORTED = (
     "think_status_string", "think_t_from_lambda", "think_pruned_ld",
     "think_score_workspace_size", "think_score_channels", "think_select_channels",
-    "think_compact_keys", "think_decode_workspace_size", "think_pruned_decode_attn",
+    "think_compact_keys", "think_prune", "think_decode_workspace_size", "think_pruned_decode_attn",
     "think_workspace_init", "think_read_device_status",
 )
 
@@ -53,7 +53,7 @@ def _load() -> ctypes.CDLL:
     lib.think_t_from_lambda.restype = I
     lib.think_pruned_ld.argtypes = [I64, I]
     lib.think_pruned_ld.restype = I64
-    lib.think_score_workspace_size.argtypes = [I, I, I64, I]
+    lib.think_score_workspace_size.argtypes = [I, I, I, I64, I]
     lib.think_score_workspace_size.restype = SZ
     lib.think_score_channels.argtypes = [P, P, I64P, I, I, I, I64, I, I, I, P, P, SZ, P]
     lib.think_score_channels.restype = I
@@ -61,6 +61,8 @@ def _load() -> ctypes.CDLL:
     lib.think_select_channels.restype = I
     lib.think_compact_keys.argtypes = [P, I64P, I, I, I64, I, I, P, I, P, I64, P]
     lib.think_compact_keys.restype = I
+    lib.think_prune.argtypes = [P, P, I64P, I, I, I, I64, I, I, I, I, P, P, P, I64, P, SZ, P]
+    lib.think_prune.restype = I
     lib.think_decode_workspace_size.argtypes = [I, I, I, I64, I, I]
     lib.think_decode_workspace_size.restype = SZ
     lib.think_pruned_decode_attn.argtypes = [P, P, I64, P, I64P, P, I, I, I, I64, I, I, I, F, P,
@@ -121,8 +123,8 @@ def think_pruned_ld(N: int, dtype: torch.dtype = torch.bfloat16) -> int:
     return lib.think_pruned_ld(int(N), THINK_BF16 if dtype == torch.bfloat16 else THINK_F32)
 
 
-def think_score_workspace_size(B: int, Hkv: int, N: int, d: int = 128) -> int:
-    return lib.think_score_workspace_size(B, Hkv, N, d)
+def think_score_workspace_size(B: int, Hq: int, Hkv: int, N: int, d: int = 128) -> int:
+    return lib.think_score_workspace_size(B, Hq, Hkv, N, d)
 
 
 def think_decode_workspace_size(B: int, Hq: int, Hkv: int, N: int, d: int = 128,
@@ -162,6 +164,21 @@ def think_compact_keys(k: torch.Tensor, idx: torch.Tensor, k_pruned: torch.Tenso
         raise ThinkError(THINK_ERR_INVALID_ARG, "think_compact_keys")
     _check(lib.think_compact_keys(_ptr(k), _strides3(k), B, Hkv, N, d, _dtype(k), _ptr(idx), T,
                                   _ptr(k_pruned), int(ldk), _stream(stream)), "think_compact_keys")
+
+
+def think_prune(q_win: torch.Tensor, k: torch.Tensor, T: int, scores: torch.Tensor,
+                idx: torch.Tensor, k_pruned: torch.Tensor, ldk: int, workspace: torch.Tensor,
+                stream=None) -> None:
+    """Scores + top-T selection (one launch) then compaction (one launch)."""
+    B, Hq, S, d = q_win.shape
+    _, Hkv, N, _ = k.shape
+    if (not q_win.is_contiguous() or scores.dtype != torch.float64 or idx.dtype != torch.int32
+            or k_pruned.dtype != k.dtype):
+        raise ThinkError(THINK_ERR_INVALID_ARG, "think_prune")
+    _check(lib.think_prune(_ptr(q_win), _ptr(k), _strides3(k), B, Hq, Hkv, N, S, d, _dtype(k),
+                           int(T), _ptr(scores), _ptr(idx), _ptr(k_pruned), int(ldk),
+                           _ptr(workspace), workspace.numel() * workspace.element_size(),
+                           _stream(stream)), "think_prune")
 
 
 def think_pruned_decode_attn(q: torch.Tensor, k_pruned: torch.Tensor, ldk: int, v: torch.Tensor,
@@ -209,12 +226,17 @@ class PrunedCache:
         self.scores = torch.empty((B, Hkv, d), dtype=torch.float64, device=device)
         self.idx = torch.empty((B, Hkv, T), dtype=torch.int32, device=device)
         self.k_pruned = torch.empty((B, Hkv, T, self.ldk), dtype=dtype, device=device)
-        self.score_ws = torch.empty(max(16, think_score_workspace_size(B, Hkv, N, d)),
+        self.score_ws = torch.zeros(max(256, think_score_workspace_size(B, Hq, Hkv, N, d)),
                                     dtype=torch.uint8, device=device)
         self.decode_ws = torch.zeros(max(256, think_decode_workspace_size(B, Hq, Hkv, N, d, dtype)),
                                      dtype=torch.uint8, device=device)
 
     def prune(self, q_win, k, stream=None):
+        think_prune(q_win, k, self.T, self.scores, self.idx, self.k_pruned, self.ldk,
+                    self.score_ws, stream)
+
+    def prune_stepwise(self, q_win, k, stream=None):
+        """The same prune through the three separate entry points."""
         think_score_channels(q_win, k, self.scores, self.score_ws, stream)
         think_select_channels(self.scores, self.T, self.idx, stream)
         think_compact_keys(k, self.idx, self.k_pruned, self.ldk, stream)

@@ -5,13 +5,17 @@
 // For query head h of KV head h/G:  z[n] = scale * q[idx] . K'[:,n],
 // out = softmax(z) V, with V at full width.
 //
-// Split-N flash decoding.  Block (split, head) streams its run of 128-token
-// tiles of K'^T ([T][128]) and V ([128][128]) through a ring of shared-memory
-// stages filled by TMA (one elected producer thread, mbarrier completion), and
-// four consumer warps each own 32 tokens of every tile with their own running
-// (max, sum, weighted V) per query head of the group.  The block merges its
-// four warps and writes one partial per (head, split, group member); the
-// combine kernel merges the splits.  Every mbarrier wait is bounded in time.
+// Split-N flash decoding in one kernel.  Block (split, head) streams its run
+// of 128-token tiles of K'^T ([T][128]) and V ([128][128]) through a ring of
+// shared-memory stages filled by TMA (one elected producer thread, mbarrier
+// completion).  Four consumer warps each own 32 tokens of every tile and keep
+// their own running (max, sum, weighted V) for the G query heads of the group:
+//   logits   lane = token, fp32 FFMA2 over pairs of query heads;
+//   weighted V  each half-warp takes one token at a time, each lane 8 channels,
+//            FFMA2 over channel pairs.
+// The block merges its warps and writes one partial per (head, split); the
+// last block of a head to finish (a ticket counter in the workspace) merges
+// the head's partials into the output.  Every mbarrier wait is bounded.
 #pragma once
 
 #include "ptx.cuh"
@@ -21,15 +25,18 @@ namespace think {
 
 constexpr int kBN = 128;                  // tokens per tile
 constexpr int kConsumerWarps = 4;         // kConsumerWarps * 32 == kBN
-constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
+constexpr int kConsumerThreads = kConsumerWarps * 32;
+constexpr int kDecodeThreads = kConsumerThreads + 32;
 static_assert(kConsumerWarps * 32 == kBN, "one token per consumer lane per tile");
 
 struct DecodeArgs {
     const void *q;          // [B][Hq][D]
     const int32_t *idx;     // [B][Hkv][T]
+    float *out;             // [B][Hq][D]
     float *part_o;          // [heads][splits][G][D]
-    float *part_ml;         // [heads][splits][G][2]  (running max in log2 units, sum)
+    float *part_ml;         // [heads][splits][G][2]  (max in log2 units, sum)
     unsigned *status;       // device status bits
+    unsigned *tickets;      // [heads] arrival counters, zero between calls
     int Hq, Hkv, T;
     int64_t N;
     int tiles_per_split, splits, stages;
@@ -53,14 +60,90 @@ __device__ __forceinline__ float warp_sum(float x)
     return x;
 }
 
+// Logits of one token for the G query heads: s[g] += q'[t][g] * k[t].
+template <int G> struct QK;
+template <> struct QK<1> {
+    float s;
+    __device__ __forceinline__ void zero() { s = 0.f; }
+    __device__ __forceinline__ void step(const float *q, float k) { s = fmaf(q[0], k, s); }
+    __device__ __forceinline__ float get(int) const { return s; }
+};
+template <> struct QK<2> {
+    float2 s;
+    __device__ __forceinline__ void zero() { s = make_float2(0.f, 0.f); }
+    __device__ __forceinline__ void step(const float *q, float k)
+    {
+        s = __ffma2_rn(*reinterpret_cast<const float2 *>(q), make_float2(k, k), s);
+    }
+    __device__ __forceinline__ float get(int g) const { return g ? s.y : s.x; }
+};
+template <> struct QK<4> {
+    float2 s[2];
+    __device__ __forceinline__ void zero() { s[0] = s[1] = make_float2(0.f, 0.f); }
+    __device__ __forceinline__ void step(const float *q, float k)
+    {
+        const float4 qq = *reinterpret_cast<const float4 *>(q);
+        const float2 kk = make_float2(k, k);
+        s[0] = __ffma2_rn(make_float2(qq.x, qq.y), kk, s[0]);
+        s[1] = __ffma2_rn(make_float2(qq.z, qq.w), kk, s[1]);
+    }
+    __device__ __forceinline__ float get(int g) const
+    {
+        return (g & 1) ? s[g >> 1].y : s[g >> 1].x;
+    }
+};
+template <> struct QK<8> {
+    float2 s[4];
+    __device__ __forceinline__ void zero() { s[0] = s[1] = s[2] = s[3] = make_float2(0.f, 0.f); }
+    __device__ __forceinline__ void step(const float *q, float k)
+    {
+        const float4 qa = *reinterpret_cast<const float4 *>(q);
+        const float4 qb = *reinterpret_cast<const float4 *>(q + 4);
+        const float2 kk = make_float2(k, k);
+        s[0] = __ffma2_rn(make_float2(qa.x, qa.y), kk, s[0]);
+        s[1] = __ffma2_rn(make_float2(qa.z, qa.w), kk, s[1]);
+        s[2] = __ffma2_rn(make_float2(qb.x, qb.y), kk, s[2]);
+        s[3] = __ffma2_rn(make_float2(qb.z, qb.w), kk, s[3]);
+    }
+    __device__ __forceinline__ float get(int g) const
+    {
+        return (g & 1) ? s[g >> 1].y : s[g >> 1].x;
+    }
+};
+
+// 8 consecutive channels of one V row as 4 float2 pairs.
+template <typename TIn> struct V8;
+template <> struct V8<__nv_bfloat16> {
+    static __device__ __forceinline__ void load(const __nv_bfloat16 *p, float2 v[4])
+    {
+        const uint4 w = *reinterpret_cast<const uint4 *>(p);
+        v[0] = make_float2(bf16lo(w.x), bf16hi(w.x));
+        v[1] = make_float2(bf16lo(w.y), bf16hi(w.y));
+        v[2] = make_float2(bf16lo(w.z), bf16hi(w.z));
+        v[3] = make_float2(bf16lo(w.w), bf16hi(w.w));
+    }
+};
+template <> struct V8<float> {
+    static __device__ __forceinline__ void load(const float *p, float2 v[4])
+    {
+        const float4 a = *reinterpret_cast<const float4 *>(p);
+        const float4 b = *reinterpret_cast<const float4 *>(p + 4);
+        v[0] = make_float2(a.x, a.y);
+        v[1] = make_float2(a.z, a.w);
+        v[2] = make_float2(b.x, b.y);
+        v[3] = make_float2(b.z, b.w);
+    }
+};
+
 template <typename TIn, int G>
 __global__ void __launch_bounds__(kDecodeThreads)
-    pruned_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
-                               const __grid_constant__ CUtensorMap tm_v, const DecodeArgs a)
+    pruned_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v, const DecodeArgs a)
 {
     extern __shared__ unsigned char smem_dyn[];
-    unsigned char *smem = reinterpret_cast<unsigned char *>(
-        (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned base, kept as shared-array arithmetic so that every
+    // access below compiles to shared-memory loads and stores.
+    unsigned char *smem = smem_dyn + ((1024u - (smem_addr(smem_dyn) & 1023u)) & 1023u);
 
     const int split = blockIdx.x;
     const int head = blockIdx.y;
@@ -73,8 +156,9 @@ __global__ void __launch_bounds__(kDecodeThreads)
 
     float *qs = reinterpret_cast<float *>(smem + (size_t)stages * a.stage_bytes);  // [T][G]
     const int qs_len = ((T * G + 3) / 4) * 4;
-    float *pbuf = qs + qs_len;                                                   // [warps][32][G]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(pbuf + kConsumerWarps * 32 * G);
+    float2 *pdup = reinterpret_cast<float2 *>(qs + qs_len);  // [warps][32 tokens][G] as (p, p)
+    uint64_t *bars = reinterpret_cast<uint64_t *>(pdup + kConsumerWarps * 32 * G);
+    unsigned *flag = reinterpret_cast<unsigned *>(bars + 2 * stages);
     const uint32_t full0 = smem_addr(bars);
     const uint32_t empty0 = smem_addr(bars + stages);
 
@@ -120,9 +204,9 @@ __global__ void __launch_bounds__(kDecodeThreads)
                 const uint32_t full = full0 + 8 * s;
                 mbar_arrive_expect_tx(full, a.tx_bytes);
                 const int x = (int)((tile0 + it) * kBN);
-                unsigned char *st = smem + (size_t)s * a.stage_bytes;
-                tma_load_4d(smem_addr(st), &tm_k, x, 0, kv, b, full);
-                tma_load_4d(smem_addr(st + a.v_off), &tm_v, 0, x, kv, b, full);
+                const uint32_t st = smem_addr(smem + (size_t)s * a.stage_bytes);
+                tma_load_4d(st, &tm_k, x, 0, kv, b, full);
+                tma_load_4d(st + a.v_off, &tm_v, 0, x, kv, b, full);
                 ++issued;
             }
             if (!ok) {
@@ -136,16 +220,19 @@ __global__ void __launch_bounds__(kDecodeThreads)
     }
 
     // ---------------------------------------------------------- consumers
-    float m[G], l[G], acc[G][4];
+    float m[G], l[G];
+    float2 acc[G][4];  // channels 8*(lane&15) .. +7 of the tokens of half-warp lane>>4
 #pragma unroll
     for (int g = 0; g < G; ++g) {
         m[g] = -INFINITY;
         l[g] = 0.f;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) acc[g][e] = 0.f;
+        for (int e = 0; e < 4; ++e) acc[g][e] = make_float2(0.f, 0.f);
     }
-    const int j = warp * 32 + lane;  // this lane's token inside a tile
-    float *pw = pbuf + warp * 32 * G;
+    const int j = warp * 32 + lane;  // this lane's token inside a tile (logits)
+    const int half = lane >> 4;      // token parity this lane takes in the weighted sum
+    const int dch = 8 * (lane & 15); // first of this lane's 8 channels
+    float2 *pw = pdup + warp * 32 * G;
 
     for (int it = 0; it < ntiles; ++it) {
         const int s = it % stages;
@@ -157,43 +244,38 @@ __global__ void __launch_bounds__(kDecodeThreads)
         const TIn *vt = reinterpret_cast<const TIn *>(st + a.v_off);
         const bool valid = (tile0 + it) * kBN + j < a.N;
 
-        // logits of this lane's token for the G heads of the group
-        float sc[G];
-#pragma unroll
-        for (int g = 0; g < G; ++g) sc[g] = 0.f;
+        QK<G> sc;
+        sc.zero();
 #pragma unroll 4
-        for (int t = 0; t < T; ++t) {
-            const float kvv = Elem<TIn>::to_float(kt[t * kBN + j]);
-            const float *qt = qs + t * G;
-#pragma unroll
-            for (int g = 0; g < G; ++g) sc[g] = fmaf(qt[g], kvv, sc[g]);
-        }
+        for (int t = 0; t < T; ++t) sc.step(qs + t * G, Elem<TIn>::to_float(kt[t * kBN + j]));
+
         // online softmax over this warp's 32 tokens
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-            const float x = valid ? sc[g] : -INFINITY;
+            const float x = valid ? sc.get(g) : -INFINITY;
             const float mnew = fmaxf(m[g], warp_max(x));
             const float alpha = (m[g] == mnew) ? 1.f : exp2_approx(m[g] - mnew);
             const float p = valid ? exp2_approx(x - mnew) : 0.f;
             l[g] = fmaf(l[g], alpha, p);
+            const float2 al = make_float2(alpha, alpha);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) acc[g][e] *= alpha;
+            for (int e = 0; e < 4; ++e) acc[g][e] = __fmul2_rn(acc[g][e], al);
             m[g] = mnew;
-            pw[lane * G + g] = p;
+            pw[lane * G + g] = make_float2(p, p);
         }
         __syncwarp();
-        // weighted V over the same 32 tokens; this lane owns channels 4*lane..4*lane+3
+        // weighted V: half-warp `half` takes tokens 2*jj + half of this warp's 32
+        const TIn *vrow = vt + (size_t)(warp * 32 + half) * kD + dch;
 #pragma unroll 4
-        for (int jj = 0; jj < 32; ++jj) {
-            const float4 vv = Elem<TIn>::load4(vt + (warp * 32 + jj) * kD + 4 * lane);
-            const float *pj = pw + jj * G;
+        for (int jj = 0; jj < 16; ++jj) {
+            float2 v[4];
+            V8<TIn>::load(vrow + (size_t)(2 * jj) * kD, v);
+            const float2 *pp = pw + (2 * jj + half) * G;
 #pragma unroll
             for (int g = 0; g < G; ++g) {
-                const float p = pj[g];
-                acc[g][0] = fmaf(p, vv.x, acc[g][0]);
-                acc[g][1] = fmaf(p, vv.y, acc[g][1]);
-                acc[g][2] = fmaf(p, vv.z, acc[g][2]);
-                acc[g][3] = fmaf(p, vv.w, acc[g][3]);
+                const float2 p2 = pp[g];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[g][e] = __ffma2_rn(v[e], p2, acc[g][e]);
             }
         }
         __syncwarp();
@@ -202,21 +284,32 @@ __global__ void __launch_bounds__(kDecodeThreads)
 
     // ------------------------------------------- merge the four warps
 #pragma unroll
-    for (int g = 0; g < G; ++g) l[g] = warp_sum(l[g]);
-    named_barrier(1, kConsumerWarps * 32);  // every consumer is done with the stages
+    for (int g = 0; g < G; ++g) {
+        l[g] = warp_sum(l[g]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            acc[g][e].x += __shfl_xor_sync(0xffffffffu, acc[g][e].x, 16);
+            acc[g][e].y += __shfl_xor_sync(0xffffffffu, acc[g][e].y, 16);
+        }
+    }
+    named_barrier(1, kConsumerThreads);  // every consumer is done with the stages
     float *mo = reinterpret_cast<float *>(smem);                 // [warps][G][D]
     float *mml = mo + kConsumerWarps * G * kD;                   // [warps][G][2]
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-        *reinterpret_cast<float4 *>(mo + (warp * G + g) * kD + 4 * lane) =
-            make_float4(acc[g][0], acc[g][1], acc[g][2], acc[g][3]);
+        if (half == 0) {
+            float4 *dst = reinterpret_cast<float4 *>(mo + (warp * G + g) * kD + dch);
+            dst[0] = make_float4(acc[g][0].x, acc[g][0].y, acc[g][1].x, acc[g][1].y);
+            dst[1] = make_float4(acc[g][2].x, acc[g][2].y, acc[g][3].x, acc[g][3].y);
+        }
         if (lane == 0) {
             mml[(warp * G + g) * 2] = m[g];
             mml[(warp * G + g) * 2 + 1] = l[g];
         }
     }
-    named_barrier(1, kConsumerWarps * 32);
-    const int dch = tid;  // 0..127: one output channel per consumer thread
+    named_barrier(1, kConsumerThreads);
+    const int d = tid;  // 0..127: one output channel per consumer thread
+    const int64_t slot0 = ((int64_t)head * a.splits + split) * G;
 #pragma unroll
     for (int g = 0; g < G; ++g) {
         float M = -INFINITY;
@@ -228,42 +321,71 @@ __global__ void __launch_bounds__(kDecodeThreads)
             const float mw = mml[(w * G + g) * 2];
             if (mw == -INFINITY) continue;
             const float sw = exp2_approx(mw - M);
-            O = fmaf(mo[(w * G + g) * kD + dch], sw, O);
+            O = fmaf(mo[(w * G + g) * kD + d], sw, O);
             L = fmaf(mml[(w * G + g) * 2 + 1], sw, L);
         }
-        const int64_t slot = ((int64_t)head * a.splits + split) * G + g;
-        a.part_o[slot * kD + dch] = O;
-        if (dch == 0) {
-            a.part_ml[slot * 2] = M;
-            a.part_ml[slot * 2 + 1] = L;
+        a.part_o[(slot0 + g) * kD + d] = O;
+        if (d == 0) {
+            a.part_ml[(slot0 + g) * 2] = M;
+            a.part_ml[(slot0 + g) * 2 + 1] = L;
         }
     }
-}
 
-// Merge the per-split partials of one query head: out = sum_s O_s 2^(M_s-M)
-// / sum_s L_s 2^(M_s-M).  One block per (b, h), one thread per channel.
-__global__ void __launch_bounds__(kD)
-    decode_combine_kernel(const float *__restrict__ part_o, const float *__restrict__ part_ml,
-                          float *__restrict__ out, int Hq, int Hkv, int splits)
-{
-    const int bh = blockIdx.x;
-    const int G = Hq / Hkv;
-    const int b = bh / Hq, h = bh % Hq;
-    const int head = b * Hkv + h / G, g = h % G;
-    const int dch = threadIdx.x;
-    float M = -INFINITY;
-    for (int s = 0; s < splits; ++s)
-        M = fmaxf(M, part_ml[(((int64_t)head * splits + s) * G + g) * 2]);
-    float O = 0.f, L = 0.f;
-    for (int s = 0; s < splits; ++s) {
-        const int64_t slot = ((int64_t)head * splits + s) * G + g;
-        const float ms = part_ml[slot * 2];
-        if (ms == -INFINITY) continue;
-        const float w = exp2_approx(ms - M);
-        O = fmaf(part_o[slot * kD + dch], w, O);
-        L = fmaf(part_ml[slot * 2 + 1], w, L);
+    // ------------------------------- last block of this head merges splits
+    __threadfence();
+    named_barrier(1, kConsumerThreads);
+    if (tid == 0) {
+        const unsigned ticket = atomicAdd(a.tickets + head, 1u);
+        *flag = (ticket == (unsigned)(a.splits - 1)) ? 1u : 0u;
     }
-    out[(int64_t)bh * kD + dch] = O / L;
+    named_barrier(1, kConsumerThreads);
+    if (*flag == 0u) return;
+    __threadfence();
+    // weights w[s][g] = 2^(M_s - M*) in shared memory (stage memory is free now)
+    const int nsg = a.splits * G;
+    float *sw = reinterpret_cast<float *>(smem);   // [splits][G]
+    float *sl = sw + nsg;                          // [splits][G]
+    float *smax = sl + nsg;                        // [G]
+    float *sL = smax + G;                          // [G]
+    const float *pml = a.part_ml + (int64_t)head * a.splits * G * 2;
+    for (int i = d; i < nsg; i += kConsumerThreads) {
+        sw[i] = __ldcg(pml + 2 * i);
+        sl[i] = __ldcg(pml + 2 * i + 1);
+    }
+    named_barrier(1, kConsumerThreads);
+    if (d < G) {
+        float M = -INFINITY;
+        for (int s2 = 0; s2 < a.splits; ++s2) M = fmaxf(M, sw[s2 * G + d]);
+        smax[d] = M;
+    }
+    named_barrier(1, kConsumerThreads);
+    for (int i = d; i < nsg; i += kConsumerThreads) {
+        const float ms = sw[i];
+        sw[i] = (ms == -INFINITY) ? 0.f : exp2_approx(ms - smax[i % G]);
+    }
+    named_barrier(1, kConsumerThreads);
+    if (d < G) {
+        float L = 0.f;
+        for (int s2 = 0; s2 < a.splits; ++s2) L = fmaf(sl[s2 * G + d], sw[s2 * G + d], L);
+        sL[d] = L;
+    }
+    named_barrier(1, kConsumerThreads);
+    const float *po = a.part_o + (int64_t)head * a.splits * G * kD + d;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        float O0 = 0.f, O1 = 0.f, O2 = 0.f, O3 = 0.f;
+        int s2 = 0;
+        for (; s2 + 4 <= a.splits; s2 += 4) {
+            O0 = fmaf(__ldcg(po + ((int64_t)(s2 + 0) * G + g) * kD), sw[(s2 + 0) * G + g], O0);
+            O1 = fmaf(__ldcg(po + ((int64_t)(s2 + 1) * G + g) * kD), sw[(s2 + 1) * G + g], O1);
+            O2 = fmaf(__ldcg(po + ((int64_t)(s2 + 2) * G + g) * kD), sw[(s2 + 2) * G + g], O2);
+            O3 = fmaf(__ldcg(po + ((int64_t)(s2 + 3) * G + g) * kD), sw[(s2 + 3) * G + g], O3);
+        }
+        for (; s2 < a.splits; ++s2)
+            O0 = fmaf(__ldcg(po + ((int64_t)s2 * G + g) * kD), sw[s2 * G + g], O0);
+        a.out[((int64_t)b * a.Hq + (int64_t)kv * G + g) * kD + d] = ((O0 + O1) + (O2 + O3)) / sL[g];
+    }
+    if (d == 0) a.tickets[head] = 0u;  // ready for the next call
 }
 
 }  // namespace think

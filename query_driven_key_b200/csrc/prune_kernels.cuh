@@ -9,34 +9,78 @@
 
 namespace think {
 
+// Top-T of the kD channel scores held in shared memory, by one warp:
+// rank(c) = #channels before c in the order (score descending, index
+// ascending); c is kept if rank(c) < T; kept channels are written ascending.
+// Scores are non-negative doubles, whose bit patterns order like their values.
+__device__ __forceinline__ void select_top_t_warp(const unsigned long long *sv, int T,
+                                                  int32_t *__restrict__ idx_out, int lane)
+{
+    unsigned long long mine[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) mine[j] = sv[lane + 32 * j];
+    int base = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int c = lane + 32 * j;
+        int rank = 0;
+#pragma unroll 8
+        for (int c2 = 0; c2 < kD; ++c2) {
+            const unsigned long long u = sv[c2];
+            rank += (u > mine[j]) | ((u == mine[j]) & (c2 < c));
+        }
+        const bool keep = rank < T;
+        const unsigned ball = __ballot_sync(0xffffffffu, keep);
+        if (keep) idx_out[base + __popc(ball & ((1u << lane) - 1u))] = c;
+        base += __popc(ball);
+    }
+}
+
+struct ScoreArgs {
+    const void *k;
+    int64_t sb, sh, sn;        // element strides of K (batch, head, token)
+    const void *qwin;          // [B][Hq][S][D]
+    int Hq, Hkv, S;
+    int64_t N, rows_per_split;
+    int splits;
+    double *part;              // [heads][splits][D]   partial channel energies
+    double *qn2;               // [heads][G][D]        window-query channel energies
+    unsigned *tickets;         // [heads], zero between calls
+    double *scores;            // [heads][D]
+    int T;                     // > 0: also select the top T into idx
+    int32_t *idx;              // [heads][T]
+};
+
 // ---------------------------------------------------------------------------
-// Score, stage 1: per (split of the token axis, head) partial channel energy
-//   part[head][split][c] = sum_{n in split} K[n,c]^2   (fp64)
-// 16-byte loads, 256 threads: for bf16 a row (256 B) is 16 threads x 8
-// channels and a pass covers 16 rows.  The square of a bf16 or fp32 value is
-// exact in fp64, so every product below is exact and only the order of the
+// Score.  Block (split, head) sums K[n,c]^2 (fp64) over its run of tokens with
+// 16-byte loads (bf16: 16 threads x 8 channels per row, 16 rows per pass, 8
+// passes in flight); blocks split < G also sum the window-query energies of
+// query head kv*G + split.  The last block of the head to finish (ticket
+// counter) adds the partials in split order and forms
+//     s[c] = sum_g sqrt(qn2[g][c]) * sqrt(kn2[c])
+// with each operation rounded as written, then optionally selects the top T.
+// The square of a bf16 or fp32 value is exact in fp64; only the order of the
 // additions differs from a sequential sum.
 // ---------------------------------------------------------------------------
 template <typename TIn>
-__global__ void __launch_bounds__(256)
-    score_partial_kernel(const TIn *__restrict__ k, int64_t sb, int64_t sh, int64_t sn, int Hkv,
-                         int64_t N, int64_t rows_per_split, int splits,
-                         double *__restrict__ part)
+__global__ void __launch_bounds__(256) score_kernel(const ScoreArgs a)
 {
     constexpr int VEC = 16 / sizeof(TIn);  // channels per 16-byte load
     constexpr int TPR = kD / VEC;          // threads per row
     constexpr int RPP = 256 / TPR;         // rows per pass
-    constexpr int UNROLL = 4;
+    constexpr int UNROLL = 8;
     __shared__ double red[RPP][kD];
+    __shared__ unsigned last;
 
     const int head = blockIdx.y;
     const int split = blockIdx.x;
-    const int b = head / Hkv, h = head % Hkv;
+    const int b = head / a.Hkv, kv = head % a.Hkv;
+    const int G = a.Hq / a.Hkv;
     const int cg = threadIdx.x % TPR;
     const int r = threadIdx.x / TPR;
-    const int64_t n0 = (int64_t)split * rows_per_split;
-    const int64_t n1 = min(N, n0 + rows_per_split);
-    const TIn *base = k + (int64_t)b * sb + (int64_t)h * sh + cg * VEC;
+    const int64_t n0 = (int64_t)split * a.rows_per_split;
+    const int64_t n1 = min(a.N, n0 + a.rows_per_split);
+    const TIn *base = static_cast<const TIn *>(a.k) + (int64_t)b * a.sb + (int64_t)kv * a.sh + cg * VEC;
 
     double acc[VEC];
 #pragma unroll
@@ -47,7 +91,7 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
         for (int u = 0; u < UNROLL; ++u) {
             const int64_t nn = n + (int64_t)u * RPP;
-            w[u] = (nn < n1) ? __ldg(reinterpret_cast<const uint4 *>(base + nn * sn))
+            w[u] = (nn < n1) ? __ldg(reinterpret_cast<const uint4 *>(base + nn * a.sn))
                              : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
@@ -72,52 +116,64 @@ __global__ void __launch_bounds__(256)
     }
 #pragma unroll
     for (int e = 0; e < VEC; ++e) red[r][cg * VEC + e] = acc[e];
+
+    // window-query energies of the group's query heads g = split, split + splits, ...
+    const int tid = threadIdx.x;
+    if (tid < kD) {
+        for (int g = split; g < G; g += a.splits) {
+            const int64_t h = (int64_t)kv * G + g;
+            const TIn *qh = static_cast<const TIn *>(a.qwin) + (((int64_t)b * a.Hq + h) * a.S) * kD + tid;
+            double q2 = 0.0;
+            for (int s = 0; s < a.S; ++s) {
+                const double x = (double)Elem<TIn>::to_float(qh[(int64_t)s * kD]);
+                q2 = __dadd_rn(q2, __dmul_rn(x, x));
+            }
+            a.qn2[((int64_t)head * G + g) * kD + tid] = q2;
+        }
+    }
     __syncthreads();
-    if (threadIdx.x < kD) {
+    if (tid < kD) {
         double s = 0.0;
 #pragma unroll 4
-        for (int rr = 0; rr < RPP; ++rr) s += red[rr][threadIdx.x];
-        part[((int64_t)head * splits + split) * kD + threadIdx.x] = s;
+        for (int rr = 0; rr < RPP; ++rr) s += red[rr][tid];
+        a.part[((int64_t)head * a.splits + split) * kD + tid] = s;
     }
-}
 
-// ---------------------------------------------------------------------------
-// Score, stage 2: one block per head, one thread per channel.
-//   kn2 = sum over splits (fixed order);  qn2_g = sum_s Qwin_g[s,c]^2
-//   s[c] = sum_g sqrt(qn2_g) * sqrt(kn2)     (each step rounded as written)
-// ---------------------------------------------------------------------------
-template <typename TIn>
-__global__ void __launch_bounds__(kD)
-    score_finalize_kernel(const double *__restrict__ part, int splits, const TIn *__restrict__ qwin,
-                          int Hq, int Hkv, int S, double *__restrict__ scores)
-{
-    const int head = blockIdx.x;
-    const int c = threadIdx.x;
-    const int b = head / Hkv, kv = head % Hkv;
-    const int G = Hq / Hkv;
-    double kn2 = 0.0;
-    for (int s = 0; s < splits; ++s) kn2 = __dadd_rn(kn2, part[((int64_t)head * splits + s) * kD + c]);
-    const double knorm = sqrt(kn2);
-    double sc = 0.0;
-    for (int g = 0; g < G; ++g) {
-        const int64_t h = (int64_t)kv * G + g;
-        const TIn *qh = qwin + (((int64_t)b * Hq + h) * S) * kD + c;
-        double qn2 = 0.0;
-        for (int s = 0; s < S; ++s) {
-            const double x = (double)Elem<TIn>::to_float(qh[(int64_t)s * kD]);
-            qn2 = __dadd_rn(qn2, __dmul_rn(x, x));
+    // ------------------------------------------ last block of the head
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) last = (atomicAdd(a.tickets + head, 1u) == (unsigned)(a.splits - 1)) ? 1u : 0u;
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    __shared__ unsigned long long sv[kD];
+    if (tid < kD) {
+        const double *p = a.part + (int64_t)head * a.splits * kD + tid;
+        double k0 = 0.0;
+        int s = 0;
+        for (; s + 8 <= a.splits; s += 8) {  // loads issued together, added in split order
+            double v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = __ldcg(p + (int64_t)(s + u) * kD);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) k0 = __dadd_rn(k0, v[u]);
         }
-        sc = __dadd_rn(sc, __dmul_rn(sqrt(qn2), knorm));
+        for (; s < a.splits; ++s) k0 = __dadd_rn(k0, __ldcg(p + (int64_t)s * kD));
+        const double knorm = sqrt(k0);
+        double sc = 0.0;
+        for (int g = 0; g < G; ++g)
+            sc = __dadd_rn(sc, __dmul_rn(sqrt(__ldcg(a.qn2 + ((int64_t)head * G + g) * kD + tid)), knorm));
+        a.scores[(int64_t)head * kD + tid] = sc;
+        sv[tid] = __double_as_longlong(sc);
     }
-    scores[(int64_t)head * kD + c] = sc;
+    if (tid == 0) a.tickets[head] = 0u;  // ready for the next call
+    if (a.T <= 0) return;
+    __syncthreads();
+    if (tid < 32) select_top_t_warp(sv, a.T, a.idx + (int64_t)head * a.T, tid);
 }
 
 // ---------------------------------------------------------------------------
-// Select: one warp per head.  Rank of channel c = number of channels that come
-// before it in the order (score descending, index ascending); c is kept if
-// its rank is below T.  Scores are non-negative doubles, whose bit patterns
-// order like their values, so the comparison is done on the 64-bit patterns.
-// The kept channels are written in ascending channel order.
+// Select (stand-alone): one warp per head.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(128)
     select_kernel(const double *__restrict__ scores, int heads, int T, int32_t *__restrict__ idx)
@@ -126,75 +182,89 @@ __global__ void __launch_bounds__(128)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int head = blockIdx.x * 4 + warp;
     if (head >= heads) return;
-    unsigned long long mine[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        mine[j] = __double_as_longlong(scores[(int64_t)head * kD + lane + 32 * j]);
-        sv[warp][lane + 32 * j] = mine[j];
-    }
+    for (int j = 0; j < 4; ++j)
+        sv[warp][lane + 32 * j] = __double_as_longlong(scores[(int64_t)head * kD + lane + 32 * j]);
     __syncwarp();
-    int base = 0;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const int c = lane + 32 * j;
-        int rank = 0;
-#pragma unroll 8
-        for (int c2 = 0; c2 < kD; ++c2) {
-            const unsigned long long u = sv[warp][c2];
-            rank += (u > mine[j]) | ((u == mine[j]) & (c2 < c));
-        }
-        const bool keep = rank < T;
-        const unsigned ball = __ballot_sync(0xffffffffu, keep);
-        if (keep) idx[(int64_t)head * T + base + __popc(ball & ((1u << lane) - 1u))] = c;
-        base += __popc(ball);
-    }
+    select_top_t_warp(sv[warp], T, idx + (int64_t)head * T, lane);
 }
 
 // ---------------------------------------------------------------------------
 // Compact: K'^T[t][n] = K[n][idx[t]] for a tile of 64 tokens of one head.
-// The tile is read with 16-byte loads (each lane a 32- or 64-byte run of one
-// row) and written transposed into shared memory (channel-major, padded
-// pitch), so every kept channel is then one contiguous 16-byte-vector run of
-// tokens both in shared memory and in the output.  A pure copy: bit-exact.
+// Each thread loads a 4-token x 8-channel block (four 16-byte loads, one per
+// token row), regroups it in registers into 8 channel runs of 4 tokens, and
+// stores those transposed into shared memory (channel-major, padded pitch).
+// Every kept channel is then one contiguous run of tokens, copied out with
+// 16-byte stores.  A pure copy: bit-exact.
 // ---------------------------------------------------------------------------
+template <typename TIn> struct Transpose4;
+// bf16: four 16-byte rows (tokens) of 8 channels -> 8 channel runs of 4 tokens (8 bytes)
+template <> struct Transpose4<__nv_bfloat16> {
+    static constexpr int CH = 8;
+    static __device__ __forceinline__ void run(const uint4 w[4], uint2 out[CH])
+    {
+        const uint32_t r[4][4] = {{w[0].x, w[0].y, w[0].z, w[0].w}, {w[1].x, w[1].y, w[1].z, w[1].w},
+                                  {w[2].x, w[2].y, w[2].z, w[2].w}, {w[3].x, w[3].y, w[3].z, w[3].w}};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {  // channel pair (2i, 2i+1)
+            out[2 * i] = make_uint2(__byte_perm(r[0][i], r[1][i], 0x5410), __byte_perm(r[2][i], r[3][i], 0x5410));
+            out[2 * i + 1] = make_uint2(__byte_perm(r[0][i], r[1][i], 0x7632), __byte_perm(r[2][i], r[3][i], 0x7632));
+        }
+    }
+};
+// fp32: four 16-byte rows (tokens) of 4 channels -> 4 channel runs of 4 tokens (16 bytes)
+template <> struct Transpose4<float> {
+    static constexpr int CH = 4;
+    static __device__ __forceinline__ void run(const uint4 w[4], uint4 out[CH])
+    {
+        out[0] = make_uint4(w[0].x, w[1].x, w[2].x, w[3].x);
+        out[1] = make_uint4(w[0].y, w[1].y, w[2].y, w[3].y);
+        out[2] = make_uint4(w[0].z, w[1].z, w[2].z, w[3].z);
+        out[3] = make_uint4(w[0].w, w[1].w, w[2].w, w[3].w);
+    }
+};
+
 template <typename TIn>
 __global__ void __launch_bounds__(256)
     compact_kernel(const TIn *__restrict__ k, int64_t sb, int64_t sh, int64_t sn, int Hkv, int64_t N,
                    const int32_t *__restrict__ idx, int T, TIn *__restrict__ kp, int64_t ldk)
 {
     constexpr int BNC = 64;                       // tokens per block
-    constexpr int VEC = 16 / sizeof(TIn);         // elements per 16 bytes
-    constexpr int PITCH = BNC + VEC;              // padded smem row (16-byte multiple)
-    constexpr int CPW = kD / 8;                   // channels per warp (16)
-    constexpr int LOADS = CPW / VEC;              // 16-byte loads per lane per row
+    constexpr int VEC = 16 / sizeof(TIn);         // elements per 16 bytes (channels per load)
+    constexpr int PITCH = BNC + VEC;              // padded smem row, elements (16-byte multiple)
+    constexpr int CGROUPS = kD / VEC;             // channel groups of one row: 16 (bf16), 32 (fp32)
+    constexpr int TGROUPS = 256 / CGROUPS;        // token groups of 4 per pass: 16 (bf16), 8 (fp32)
+    constexpr int PASSES = BNC / (4 * TGROUPS);   // 1 (bf16), 2 (fp32)
     constexpr int LPR = BNC / VEC;                // lanes per output row
     constexpr int RPI = 32 / LPR;                 // output rows per warp instruction
+    using Run = typename std::conditional<sizeof(TIn) == 2, uint2, uint4>::type;
     __shared__ __align__(16) TIn sT[kD][PITCH];
 
     const int head = blockIdx.y;
     const int b = head / Hkv, h = head % Hkv;
     const int64_t n0 = (int64_t)blockIdx.x * BNC;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const TIn *kh = k + (int64_t)b * sb + (int64_t)h * sh + warp * CPW;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // lane -> (token group, channel group); the 16 lanes of a half-warp cover
+    // 16 token groups of one channel group, so their shared stores form one
+    // contiguous 128-byte run per channel.
+    const int tg = (CGROUPS == 16) ? (lane & 15) : (lane & 7);
+    const int cgi = (CGROUPS == 16) ? (warp * 2 + (lane >> 4)) : (warp * 4 + (lane >> 3));
+    const TIn *kh = k + (int64_t)b * sb + (int64_t)h * sh + cgi * VEC;
 
-    uint4 w[2][LOADS];
 #pragma unroll
-    for (int rg = 0; rg < 2; ++rg) {
-        const int64_t n = n0 + rg * 32 + lane;
+    for (int pass = 0; pass < PASSES; ++pass) {
+        const int row0 = (pass * TGROUPS + tg) * 4;
+        uint4 w[4];
 #pragma unroll
-        for (int q = 0; q < LOADS; ++q)
-            w[rg][q] = (n < N) ? __ldg(reinterpret_cast<const uint4 *>(kh + n * sn + q * VEC))
-                               : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int rg = 0; rg < 2; ++rg) {
-        const int row = rg * 32 + lane;
-#pragma unroll
-        for (int q = 0; q < LOADS; ++q) {
-            const TIn *e = reinterpret_cast<const TIn *>(&w[rg][q]);
-#pragma unroll
-            for (int i = 0; i < VEC; ++i) sT[warp * CPW + q * VEC + i][row] = e[i];
+        for (int i = 0; i < 4; ++i) {
+            const int64_t n = n0 + row0 + i;
+            w[i] = (n < N) ? __ldg(reinterpret_cast<const uint4 *>(kh + n * sn)) : make_uint4(0, 0, 0, 0);
         }
+        Run runs[Transpose4<TIn>::CH];
+        Transpose4<TIn>::run(w, runs);
+#pragma unroll
+        for (int c = 0; c < Transpose4<TIn>::CH; ++c)
+            *reinterpret_cast<Run *>(&sT[cgi * VEC + c][row0]) = runs[c];
     }
     __syncthreads();
 

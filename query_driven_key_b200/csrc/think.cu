@@ -19,7 +19,7 @@ namespace think {
 namespace {
 
 constexpr int kTargetSMs = 148;             // B200
-constexpr int kScoreBlocksPerSM = 4;        // 256-thread score blocks resident per SM
+constexpr int kScoreBlocksPerSM = 8;        // 256-thread score blocks resident per SM
 constexpr int kDecodeBlocksPerSM = 2;       // decode blocks the plan aims to keep per SM
 constexpr size_t kDecodeHeader = 256;       // status word + reserved, start of the workspace
 constexpr size_t kSmemPerSM = 233472;       // 228 KB
@@ -89,8 +89,10 @@ DecodeSmem plan_decode_smem(int T, int G, size_t es)
     s.v_off = (uint32_t)align_up(kt, 1024);
     s.stage_bytes = (uint32_t)align_up(s.v_off + vb, 1024);
     s.tx_bytes = (uint32_t)(kt + vb);
-    const size_t extra = align_up((size_t)T * G, 4) * 4 + (size_t)kConsumerWarps * 32 * G * 4 +
-                         2 * 8 * 8 /* up to 8 stages of full+empty barriers */ + 1024 /* alignment slack */;
+    const size_t extra = align_up((size_t)T * G, 4) * 4          /* q' */ +
+                         (size_t)kConsumerWarps * 32 * G * 8          /* softmax weights (p, p) */ +
+                         2 * 8 * 8 + 16 /* up to 8 stages of full+empty barriers, a flag */ +
+                         1024 /* alignment slack */;
     const size_t per_block_2 = kSmemPerSM / kDecodeBlocksPerSM - kSmemReservedPerBlock;
     int st = (int)((per_block_2 - extra) / s.stage_bytes);
     if (st >= 2) {
@@ -100,7 +102,8 @@ DecodeSmem plan_decode_smem(int T, int G, size_t es)
         s.stages = std::min(std::max(st, 1), 4);
     }
     s.bytes = (size_t)s.stages * s.stage_bytes + extra;
-    // the block-merge scratch reuses stage memory: [warps][G][D] + [warps][G][2] floats
+    // The block merge ([warps][G][D] + [warps][G][2] floats) and the split merge
+    // (2 x splits x G floats, splits <= 2 x 148) reuse the stage memory.
     return s;
 }
 
@@ -160,7 +163,7 @@ template <typename TIn, int G>
 think_status_t launch_decode_g(const CUtensorMap &mk, const CUtensorMap &mv, const DecodeArgs &a,
                                const DecodeSmem &sm, int heads, cudaStream_t st)
 {
-    auto kern = pruned_decode_split_kernel<TIn, G>;
+    auto kern = pruned_decode_kernel<TIn, G>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm.bytes) !=
         cudaSuccess)
         return THINK_ERR_CUDA;
@@ -180,6 +183,117 @@ think_status_t launch_decode(int G, const CUtensorMap &mk, const CUtensorMap &mv
     case 8: return launch_decode_g<TIn, 8>(mk, mv, a, sm, heads, st);
     default: return THINK_ERR_UNSUPPORTED;
     }
+}
+
+
+// ---------------------------------------------------------------- score --
+
+struct ScoreWs {
+    size_t tickets, qn2, part, total;  // byte offsets and total size
+};
+
+ScoreWs score_ws_layout(int64_t heads, int G, const ScorePlan &p)
+{
+    ScoreWs w;
+    w.tickets = 0;
+    w.qn2 = align_up((size_t)heads * sizeof(unsigned), 256);
+    w.part = w.qn2 + align_up((size_t)heads * G * kD * sizeof(double), 256);
+    w.total = w.part + (size_t)heads * p.splits * kD * sizeof(double);
+    return w;
+}
+
+think_status_t validate_score(const void *q_win, const void *k, const int64_t k_strides[3], int B,
+                              int Hq, int Hkv, int64_t N, int S_obs, int d, think_dtype_t dtype,
+                              const double *scores, const void *workspace, size_t workspace_bytes)
+{
+    if (B < 0 || Hq < 0 || Hkv < 0 || N < 0 || S_obs < 0) return THINK_ERR_INVALID_ARG;
+    if (!dtype_ok(dtype)) return THINK_ERR_INVALID_ARG;
+    if (d != kD) return THINK_ERR_UNSUPPORTED;
+    if (B == 0 || Hkv == 0) return THINK_OK;
+    if (Hq < Hkv || Hq % Hkv != 0) return THINK_ERR_INVALID_ARG;
+    if (!k || !k_strides || !scores || !workspace || (S_obs > 0 && !q_win))
+        return THINK_ERR_INVALID_ARG;
+    const int64_t heads = (int64_t)B * Hkv;
+    if (heads > 65535) return THINK_ERR_UNSUPPORTED;
+    const size_t es = esize(dtype);
+    if (!aligned16(k) || !aligned16(workspace) || (q_win && !aligned16(q_win)) ||
+        !strides_ok(k_strides, es) || (reinterpret_cast<uintptr_t>(scores) & 7u))
+        return THINK_ERR_ALIGNMENT;
+    if (workspace_bytes < score_ws_layout(heads, Hq / Hkv, plan_score(heads, N)).total)
+        return THINK_ERR_WORKSPACE;
+    return THINK_OK;
+}
+
+think_status_t launch_score(const void *q_win, const void *k, const int64_t k_strides[3], int B,
+                            int Hq, int Hkv, int64_t N, int S_obs, think_dtype_t dtype, int T,
+                            double *scores, int32_t *idx, void *workspace, cudaStream_t st)
+{
+    const int64_t heads = (int64_t)B * Hkv;
+    const ScorePlan p = plan_score(heads, N);
+    const ScoreWs w = score_ws_layout(heads, Hq / Hkv, p);
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    ScoreArgs a;
+    a.k = k;
+    a.sb = k_strides[0];
+    a.sh = k_strides[1];
+    a.sn = k_strides[2];
+    a.qwin = q_win;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.S = S_obs;
+    a.N = N;
+    a.rows_per_split = p.rows_per_split;
+    a.splits = p.splits;
+    a.tickets = reinterpret_cast<unsigned *>(ws + w.tickets);
+    a.qn2 = reinterpret_cast<double *>(ws + w.qn2);
+    a.part = reinterpret_cast<double *>(ws + w.part);
+    a.scores = scores;
+    a.T = T;
+    a.idx = idx;
+    dim3 grid(p.splits, (unsigned)heads);
+    if (dtype == THINK_BF16)
+        score_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(a);
+    else
+        score_kernel<float><<<grid, 256, 0, st>>>(a);
+    return launch_status();
+}
+
+think_status_t validate_compact(const void *k, const int64_t k_strides[3], int B, int Hkv, int64_t N,
+                                int d, think_dtype_t dtype, const int32_t *idx, int T,
+                                const void *k_pruned, int64_t ldk)
+{
+    if (B < 0 || Hkv < 0 || N < 0) return THINK_ERR_INVALID_ARG;
+    if (!dtype_ok(dtype)) return THINK_ERR_INVALID_ARG;
+    if (d != kD) return THINK_ERR_UNSUPPORTED;
+    if (T < 1 || T > d) return THINK_ERR_INVALID_ARG;
+    if (ldk < N) return THINK_ERR_INVALID_ARG;
+    if (B == 0 || Hkv == 0 || N == 0) return THINK_OK;
+    if (!k || !k_strides || !idx || !k_pruned) return THINK_ERR_INVALID_ARG;
+    const int64_t heads = (int64_t)B * Hkv;
+    if (heads > 65535) return THINK_ERR_UNSUPPORTED;
+    const size_t es = esize(dtype);
+    if (!aligned16(k) || !aligned16(k_pruned) || !strides_ok(k_strides, es) ||
+        (ldk * (int64_t)es) % 16 != 0 || (reinterpret_cast<uintptr_t>(idx) & 3u))
+        return THINK_ERR_ALIGNMENT;
+    if (ceil_div(N, 64) > INT32_MAX) return THINK_ERR_UNSUPPORTED;
+    return THINK_OK;
+}
+
+think_status_t launch_compact(const void *k, const int64_t k_strides[3], int B, int Hkv, int64_t N,
+                              think_dtype_t dtype, const int32_t *idx, int T, void *k_pruned,
+                              int64_t ldk, cudaStream_t st)
+{
+    const int64_t heads = (int64_t)B * Hkv;
+    dim3 grid((unsigned)ceil_div(N, 64), (unsigned)heads);
+    if (dtype == THINK_BF16)
+        compact_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+            static_cast<const __nv_bfloat16 *>(k), k_strides[0], k_strides[1], k_strides[2], Hkv, N,
+            idx, T, static_cast<__nv_bfloat16 *>(k_pruned), ldk);
+    else
+        compact_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float *>(k), k_strides[0],
+                                                    k_strides[1], k_strides[2], Hkv, N, idx, T,
+                                                    static_cast<float *>(k_pruned), ldk);
+    return launch_status();
 }
 
 }  // namespace
@@ -218,12 +332,11 @@ int64_t think_pruned_ld(int64_t N, think_dtype_t dtype)
     return ceil_div(N, q) * q;
 }
 
-size_t think_score_workspace_size(int B, int Hkv, int64_t N, int d)
+size_t think_score_workspace_size(int B, int Hq, int Hkv, int64_t N, int d)
 {
-    if (B <= 0 || Hkv <= 0 || N < 0 || d != kD) return 0;
+    if (B <= 0 || Hkv <= 0 || Hq < Hkv || Hq % Hkv != 0 || N < 0 || d != kD) return 0;
     const int64_t heads = (int64_t)B * Hkv;
-    const ScorePlan p = plan_score(heads, N);
-    return (size_t)heads * p.splits * kD * sizeof(double);
+    return score_ws_layout(heads, Hq / Hkv, plan_score(heads, N)).total;
 }
 
 think_status_t think_score_channels(const void *q_win, const void *k, const int64_t k_strides[3],
@@ -231,38 +344,11 @@ think_status_t think_score_channels(const void *q_win, const void *k, const int6
                                     think_dtype_t dtype, double *scores, void *workspace,
                                     size_t workspace_bytes, void *stream)
 {
-    if (B < 0 || Hq < 0 || Hkv < 0 || N < 0 || S_obs < 0) return THINK_ERR_INVALID_ARG;
-    if (!dtype_ok(dtype)) return THINK_ERR_INVALID_ARG;
-    if (d != kD) return THINK_ERR_UNSUPPORTED;
-    if (B == 0 || Hkv == 0) return THINK_OK;
-    if (Hq < Hkv || Hq % Hkv != 0) return THINK_ERR_INVALID_ARG;
-    if (!k || !k_strides || !scores || !workspace || (S_obs > 0 && !q_win))
-        return THINK_ERR_INVALID_ARG;
-    const int64_t heads = (int64_t)B * Hkv;
-    if (heads > 65535) return THINK_ERR_UNSUPPORTED;
-    const size_t es = esize(dtype);
-    if (!aligned16(k) || !aligned16(workspace) || (q_win && !aligned16(q_win)) ||
-        !strides_ok(k_strides, es) || (reinterpret_cast<uintptr_t>(scores) & 7u))
-        return THINK_ERR_ALIGNMENT;
-    const ScorePlan p = plan_score(heads, N);
-    if (workspace_bytes < (size_t)heads * p.splits * kD * sizeof(double)) return THINK_ERR_WORKSPACE;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    double *part = static_cast<double *>(workspace);
-    dim3 g1(p.splits, (unsigned)heads);
-    if (dtype == THINK_BF16) {
-        score_partial_kernel<__nv_bfloat16><<<g1, 256, 0, st>>>(
-            static_cast<const __nv_bfloat16 *>(k), k_strides[0], k_strides[1], k_strides[2], Hkv,
-            N, p.rows_per_split, p.splits, part);
-        score_finalize_kernel<__nv_bfloat16><<<(unsigned)heads, kD, 0, st>>>(
-            part, p.splits, static_cast<const __nv_bfloat16 *>(q_win), Hq, Hkv, S_obs, scores);
-    } else {
-        score_partial_kernel<float><<<g1, 256, 0, st>>>(static_cast<const float *>(k), k_strides[0],
-                                                        k_strides[1], k_strides[2], Hkv, N,
-                                                        p.rows_per_split, p.splits, part);
-        score_finalize_kernel<float><<<(unsigned)heads, kD, 0, st>>>(
-            part, p.splits, static_cast<const float *>(q_win), Hq, Hkv, S_obs, scores);
-    }
-    return launch_status();
+    const think_status_t v = validate_score(q_win, k, k_strides, B, Hq, Hkv, N, S_obs, d, dtype,
+                                            scores, workspace, workspace_bytes);
+    if (v != THINK_OK || B == 0 || Hkv == 0) return v;
+    return launch_score(q_win, k, k_strides, B, Hq, Hkv, N, S_obs, dtype, 0, scores, nullptr,
+                        workspace, static_cast<cudaStream_t>(stream));
 }
 
 think_status_t think_select_channels(const double *scores, int B, int Hkv, int d, int T,
@@ -286,31 +372,29 @@ think_status_t think_compact_keys(const void *k, const int64_t k_strides[3], int
                                   int64_t N, int d, think_dtype_t dtype, const int32_t *idx,
                                   int T, void *k_pruned, int64_t ldk, void *stream)
 {
-    if (B < 0 || Hkv < 0 || N < 0) return THINK_ERR_INVALID_ARG;
-    if (!dtype_ok(dtype)) return THINK_ERR_INVALID_ARG;
-    if (d != kD) return THINK_ERR_UNSUPPORTED;
+    const think_status_t v = validate_compact(k, k_strides, B, Hkv, N, d, dtype, idx, T, k_pruned, ldk);
+    if (v != THINK_OK || B == 0 || Hkv == 0 || N == 0) return v;
+    return launch_compact(k, k_strides, B, Hkv, N, dtype, idx, T, k_pruned, ldk,
+                          static_cast<cudaStream_t>(stream));
+}
+
+think_status_t think_prune(const void *q_win, const void *k, const int64_t k_strides[3], int B,
+                           int Hq, int Hkv, int64_t N, int S_obs, int d, think_dtype_t dtype,
+                           int T, double *scores, int32_t *idx, void *k_pruned, int64_t ldk,
+                           void *workspace, size_t workspace_bytes, void *stream)
+{
+    think_status_t v = validate_score(q_win, k, k_strides, B, Hq, Hkv, N, S_obs, d, dtype, scores,
+                                      workspace, workspace_bytes);
+    if (v != THINK_OK) return v;
     if (T < 1 || T > d) return THINK_ERR_INVALID_ARG;
-    if (ldk < N) return THINK_ERR_INVALID_ARG;
-    if (B == 0 || Hkv == 0 || N == 0) return THINK_OK;
-    if (!k || !k_strides || !idx || !k_pruned) return THINK_ERR_INVALID_ARG;
-    const int64_t heads = (int64_t)B * Hkv;
-    if (heads > 65535) return THINK_ERR_UNSUPPORTED;
-    const size_t es = esize(dtype);
-    if (!aligned16(k) || !aligned16(k_pruned) || !strides_ok(k_strides, es) ||
-        (ldk * (int64_t)es) % 16 != 0 || (reinterpret_cast<uintptr_t>(idx) & 3u))
-        return THINK_ERR_ALIGNMENT;
-    if (ceil_div(N, 64) > INT32_MAX) return THINK_ERR_UNSUPPORTED;
-    dim3 grid((unsigned)ceil_div(N, 64), (unsigned)heads);
+    if (B > 0 && Hkv > 0 && (!idx || (reinterpret_cast<uintptr_t>(idx) & 3u)))
+        return idx ? THINK_ERR_ALIGNMENT : THINK_ERR_INVALID_ARG;
+    v = validate_compact(k, k_strides, B, Hkv, N, d, dtype, idx, T, k_pruned, ldk);
+    if (v != THINK_OK || B == 0 || Hkv == 0) return v;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (dtype == THINK_BF16)
-        compact_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
-            static_cast<const __nv_bfloat16 *>(k), k_strides[0], k_strides[1], k_strides[2], Hkv, N,
-            idx, T, static_cast<__nv_bfloat16 *>(k_pruned), ldk);
-    else
-        compact_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float *>(k), k_strides[0],
-                                                    k_strides[1], k_strides[2], Hkv, N, idx, T,
-                                                    static_cast<float *>(k_pruned), ldk);
-    return launch_status();
+    v = launch_score(q_win, k, k_strides, B, Hq, Hkv, N, S_obs, dtype, T, scores, idx, workspace, st);
+    if (v != THINK_OK || N == 0) return v;
+    return launch_compact(k, k_strides, B, Hkv, N, dtype, idx, T, k_pruned, ldk, st);
 }
 
 size_t think_decode_workspace_size(int B, int Hq, int Hkv, int64_t N, int d, think_dtype_t dtype)
@@ -321,7 +405,8 @@ size_t think_decode_workspace_size(int B, int Hq, int Hkv, int64_t N, int d, thi
     const int G = Hq / Hkv;
     const DecodeSplit sp = plan_decode_split(heads, N);
     const size_t slots = (size_t)heads * sp.splits * G;
-    return kDecodeHeader + slots * kD * sizeof(float) + slots * 2 * sizeof(float);
+    return kDecodeHeader + align_up((size_t)heads * sizeof(unsigned), 256) +
+           slots * kD * sizeof(float) + slots * 2 * sizeof(float);
 }
 
 think_status_t think_pruned_decode_attn(const void *q, const void *k_pruned, int64_t ldk,
@@ -370,7 +455,10 @@ think_status_t think_pruned_decode_attn(const void *q, const void *k_pruned, int
     a.q = q;
     a.idx = idx;
     a.status = reinterpret_cast<unsigned *>(ws);
-    a.part_o = reinterpret_cast<float *>(ws + kDecodeHeader);
+    a.tickets = reinterpret_cast<unsigned *>(ws + kDecodeHeader);
+    a.part_o = reinterpret_cast<float *>(ws + kDecodeHeader +
+                                         align_up((size_t)heads * sizeof(unsigned), 256));
+    a.out = out;
     a.part_ml = a.part_o + slots * kD;
     a.Hq = Hq;
     a.Hkv = Hkv;
@@ -388,10 +476,7 @@ think_status_t think_pruned_decode_attn(const void *q, const void *k_pruned, int
     think_status_t r = dtype == THINK_BF16
                            ? launch_decode<__nv_bfloat16>(G, mk, mv, a, sm, (int)heads, st)
                            : launch_decode<float>(G, mk, mv, a, sm, (int)heads, st);
-    if (r != THINK_OK) return r;
-    decode_combine_kernel<<<(unsigned)((int64_t)B * Hq), kD, 0, st>>>(a.part_o, a.part_ml, out, Hq,
-                                                                      Hkv, sp.splits);
-    return launch_status();
+    return r;
 }
 
 think_status_t think_workspace_init(void *workspace, size_t workspace_bytes, void *stream)

@@ -25,7 +25,7 @@ def declared_functions():
 
 def test_every_declared_symbol_is_exported():
     names = declared_functions()
-    assert len(names) >= 11
+    assert len(names) >= 12
     for n in names:
         assert hasattr(lib, n), f"{n} declared in think.h but not exported"
     assert set(names) == set(qdk.EXPORTED)
@@ -55,8 +55,9 @@ def test_pruned_pitch():
 
 
 def test_workspace_sizes():
-    assert qdk.think_score_workspace_size(1, 8, 131072) > 0
-    assert qdk.think_score_workspace_size(1, 8, 131072, d=64) == 0
+    assert qdk.think_score_workspace_size(1, 32, 8, 131072) > 0
+    assert qdk.think_score_workspace_size(1, 32, 8, 131072, d=64) == 0
+    assert qdk.think_score_workspace_size(1, 30, 8, 100) == 0
     n4 = qdk.think_decode_workspace_size(1, 32, 8, 131072)
     assert n4 >= 256 + 8 * 4 * 130 * 4
     assert qdk.think_decode_workspace_size(1, 32, 8, 0) == 0
@@ -87,6 +88,17 @@ def test_score_validation():
     bad = I64x3(128 * 64, 128 * 64, 130)
     assert f(FAKE, FAKE, bad, 1, 4, 2, 64, 8, 128, 1, FAKE, FAKE, 1 << 20, None) == qdk.THINK_ERR_ALIGNMENT
     assert f(FAKE, FAKE, s, 1, 4, 2, 64, 8, 128, 1, FAKE, FAKE, 16, None) == qdk.THINK_ERR_WORKSPACE
+
+
+def test_prune_validation():
+    st = I64x3(128 * 64, 128 * 64, 128)
+    f = lib.think_prune
+    ok_ws = qdk.think_score_workspace_size(1, 4, 2, 64)
+    assert f(FAKE, FAKE, st, 1, 4, 2, 64, 8, 128, 1, 0, FAKE, FAKE, FAKE, 64, FAKE, ok_ws, None) == qdk.THINK_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, st, 1, 4, 2, 64, 8, 128, 1, 10, FAKE, None, FAKE, 64, FAKE, ok_ws, None) == qdk.THINK_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, st, 1, 4, 2, 64, 8, 128, 1, 10, FAKE, FAKE, FAKE, 63, FAKE, ok_ws, None) == qdk.THINK_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, st, 1, 4, 2, 64, 8, 128, 1, 10, FAKE, FAKE, FAKE, 64, FAKE, ok_ws - 8, None) == qdk.THINK_ERR_WORKSPACE
+    assert f(FAKE, FAKE, st, 0, 4, 2, 64, 8, 128, 1, 10, FAKE, FAKE, FAKE, 64, FAKE, 0, None) == qdk.THINK_OK
 
 
 def test_select_validation():

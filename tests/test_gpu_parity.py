@@ -171,7 +171,7 @@ def test_ldk_larger_than_needed_and_exact_ties():
     kd = k.contiguous().to(DEV)
     ldk = 512
     scores = torch.empty((B, Hkv, 128), dtype=torch.float64, device=DEV)
-    ws = torch.empty(qdk.think_score_workspace_size(B, Hkv, N), dtype=torch.uint8, device=DEV)
+    ws = torch.zeros(qdk.think_score_workspace_size(B, Hq, Hkv, N), dtype=torch.uint8, device=DEV)
     idx = torch.empty((B, Hkv, T), dtype=torch.int32, device=DEV)
     kp = torch.full((B, Hkv, T, ldk), 7.0, dtype=torch.bfloat16, device=DEV)
     qdk.think_score_channels(q_win.to(DEV), kd, scores, ws)
@@ -182,6 +182,24 @@ def test_ldk_larger_than_needed_and_exact_ties():
     assert np.array_equal(idx.cpu().numpy(), oi)
     assert np.array_equal(kp_logical(kp, N), okp)
     assert torch.all(kp[..., N:] == 7.0), "columns beyond N must not be written"
+
+
+def test_fused_prune_equals_stepwise_calls():
+    w = W.WORKLOADS["llama3_8b_gqa"].with_(B=2, N=5000)
+    q_win, k, _ = W.gen_layer(w)
+    qd, kd = q_win.to(DEV), k.to(DEV)
+    a = qdk.PrunedCache(w.B, w.Hq, w.Hkv, w.N, 64, dtype=k.dtype)
+    b = qdk.PrunedCache(w.B, w.Hq, w.Hkv, w.N, 64, dtype=k.dtype)
+    a.prune(qd, kd)
+    b.prune_stepwise(qd, kd)
+    torch.cuda.synchronize()
+    assert torch.equal(a.scores, b.scores)
+    assert torch.equal(a.idx, b.idx)
+    assert torch.equal(a.k_pruned[..., : w.N], b.k_pruned[..., : w.N])
+    # counters are left at zero: a second call gives the same result
+    a.prune(qd, kd)
+    torch.cuda.synchronize()
+    assert torch.equal(a.idx, b.idx)
 
 
 def test_scores_are_deterministic():
