@@ -125,6 +125,23 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
+# ------------------------------------------------------- multi-rank ---
+
+def max_over_ranks(values, device=None):
+    """Element-wise max of a list of floats over all ranks (identity on one rank)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def aggregate_gbs(world: int, bytes_per_rank_step: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank moves bytes_per_rank_step per step."""
+    return world * bytes_per_rank_step / (ms_per_step * 1e-3) / 1e9
+
+
 # ----------------------------------------------------------- workload ---
 
 def workload():
@@ -272,17 +289,12 @@ def run_native(args):
     total_ms = t_start.elapsed_time(t_end)
     prune_ms = [e[0].elapsed_time(e[1]) for e in evs]
     decode_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    if world > 1:
-        t = torch.tensor([total_ms, sum(prune_ms), sum(decode_ms)], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, prune_sum, decode_sum = t.tolist()
-    else:
-        prune_sum, decode_sum = sum(prune_ms), sum(decode_ms)
+    total_ms, prune_sum, decode_sum = max_over_ranks([total_ms, sum(prune_ms), sum(decode_ms)], dev)
     assert qdk.think_read_device_status(cache.decode_ws, stream) == 0
 
     ms_per_step = total_ms / args.steps
     nbytes = step_bytes(w, T)
-    value = world * nbytes / (ms_per_step * 1e-3) / 1e9
+    value = aggregate_gbs(world, nbytes, ms_per_step)
     dec_bytes = W.decode_bytes(w, T)
     dec_us = decode_sum / args.steps / w.decode_steps * 1e3
     prune_us = prune_sum / args.steps * 1e3
@@ -319,12 +331,8 @@ def run_native(args):
                 e2e_step()
             e1.record(stream)
             stream.synchronize()
-        e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = t.item()
-        e2e = {"value": world * nbytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+        e2e_ms = max_over_ranks([e0.elapsed_time(e1) / args.e2e_steps], dev)[0]
+        e2e = {"value": aggregate_gbs(world, nbytes, e2e_ms), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                "steps": args.e2e_steps}
 
