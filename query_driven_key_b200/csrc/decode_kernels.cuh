@@ -135,6 +135,81 @@ template <> struct V8<float> {
     }
 };
 
+// Write this block's partial (O[g][d] for d = tid, max M[g] in log2 units,
+// sum L[g]) for (head, split); the last block of the head to arrive merges
+// every split of the head into `out`.  Called by the kConsumerThreads
+// consumer threads only; `scratch` is free shared memory of at least
+// (2 * splits * G + 2 * G) floats, `flag` one shared word.
+template <int G>
+__device__ __forceinline__ void finish_split(const DecodeArgs &a, int head, int split, int b, int kv,
+                                             int d, const float (&O)[G], const float (&M)[G],
+                                             const float (&L)[G], float *scratch, unsigned *flag)
+{
+    const int64_t slot0 = ((int64_t)head * a.splits + split) * G;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        a.part_o[(slot0 + g) * kD + d] = O[g];
+        if (d == 0) {
+            a.part_ml[(slot0 + g) * 2] = M[g];
+            a.part_ml[(slot0 + g) * 2 + 1] = L[g];
+        }
+    }
+    __threadfence();
+    named_barrier(1, kConsumerThreads);
+    if (d == 0) {
+        const unsigned ticket = atomicAdd(a.tickets + head, 1u);
+        *flag = (ticket == (unsigned)(a.splits - 1)) ? 1u : 0u;
+    }
+    named_barrier(1, kConsumerThreads);
+    if (*flag == 0u) return;
+    __threadfence();
+    // weights w[s][g] = 2^(M_s - M*)
+    const int nsg = a.splits * G;
+    float *sw = scratch;        // [splits][G]
+    float *sl = sw + nsg;       // [splits][G]
+    float *smax = sl + nsg;     // [G]
+    float *sL = smax + G;       // [G]
+    const float *pml = a.part_ml + (int64_t)head * a.splits * G * 2;
+    for (int i = d; i < nsg; i += kConsumerThreads) {
+        sw[i] = __ldcg(pml + 2 * i);
+        sl[i] = __ldcg(pml + 2 * i + 1);
+    }
+    named_barrier(1, kConsumerThreads);
+    if (d < G) {
+        float Mx = -INFINITY;
+        for (int s2 = 0; s2 < a.splits; ++s2) Mx = fmaxf(Mx, sw[s2 * G + d]);
+        smax[d] = Mx;
+    }
+    named_barrier(1, kConsumerThreads);
+    for (int i = d; i < nsg; i += kConsumerThreads) {
+        const float ms = sw[i];
+        sw[i] = (ms == -INFINITY) ? 0.f : exp2_approx(ms - smax[i % G]);
+    }
+    named_barrier(1, kConsumerThreads);
+    if (d < G) {
+        float Ls = 0.f;
+        for (int s2 = 0; s2 < a.splits; ++s2) Ls = fmaf(sl[s2 * G + d], sw[s2 * G + d], Ls);
+        sL[d] = Ls;
+    }
+    named_barrier(1, kConsumerThreads);
+    const float *po = a.part_o + (int64_t)head * a.splits * G * kD + d;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        float O0 = 0.f, O1 = 0.f, O2 = 0.f, O3 = 0.f;
+        int s2 = 0;
+        for (; s2 + 4 <= a.splits; s2 += 4) {
+            O0 = fmaf(__ldcg(po + ((int64_t)(s2 + 0) * G + g) * kD), sw[(s2 + 0) * G + g], O0);
+            O1 = fmaf(__ldcg(po + ((int64_t)(s2 + 1) * G + g) * kD), sw[(s2 + 1) * G + g], O1);
+            O2 = fmaf(__ldcg(po + ((int64_t)(s2 + 2) * G + g) * kD), sw[(s2 + 2) * G + g], O2);
+            O3 = fmaf(__ldcg(po + ((int64_t)(s2 + 3) * G + g) * kD), sw[(s2 + 3) * G + g], O3);
+        }
+        for (; s2 < a.splits; ++s2)
+            O0 = fmaf(__ldcg(po + ((int64_t)s2 * G + g) * kD), sw[s2 * G + g], O0);
+        a.out[((int64_t)b * a.Hq + (int64_t)kv * G + g) * kD + d] = ((O0 + O1) + (O2 + O3)) / sL[g];
+    }
+    if (d == 0) a.tickets[head] = 0u;  // ready for the next call
+}
+
 template <typename TIn, int G>
 __global__ void __launch_bounds__(kDecodeThreads)
     pruned_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
@@ -309,83 +384,25 @@ __global__ void __launch_bounds__(kDecodeThreads)
     }
     named_barrier(1, kConsumerThreads);
     const int d = tid;  // 0..127: one output channel per consumer thread
-    const int64_t slot0 = ((int64_t)head * a.splits + split) * G;
+    float O[G], M[G], L[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-        float M = -INFINITY;
+        M[g] = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, mml[(w * G + g) * 2]);
-        float O = 0.f, L = 0.f;
+        for (int w = 0; w < kConsumerWarps; ++w) M[g] = fmaxf(M[g], mml[(w * G + g) * 2]);
+        O[g] = 0.f;
+        L[g] = 0.f;
 #pragma unroll
         for (int w = 0; w < kConsumerWarps; ++w) {
             const float mw = mml[(w * G + g) * 2];
             if (mw == -INFINITY) continue;
-            const float sw = exp2_approx(mw - M);
-            O = fmaf(mo[(w * G + g) * kD + d], sw, O);
-            L = fmaf(mml[(w * G + g) * 2 + 1], sw, L);
-        }
-        a.part_o[(slot0 + g) * kD + d] = O;
-        if (d == 0) {
-            a.part_ml[(slot0 + g) * 2] = M;
-            a.part_ml[(slot0 + g) * 2 + 1] = L;
+            const float sw = exp2_approx(mw - M[g]);
+            O[g] = fmaf(mo[(w * G + g) * kD + d], sw, O[g]);
+            L[g] = fmaf(mml[(w * G + g) * 2 + 1], sw, L[g]);
         }
     }
-
-    // ------------------------------- last block of this head merges splits
-    __threadfence();
-    named_barrier(1, kConsumerThreads);
-    if (tid == 0) {
-        const unsigned ticket = atomicAdd(a.tickets + head, 1u);
-        *flag = (ticket == (unsigned)(a.splits - 1)) ? 1u : 0u;
-    }
-    named_barrier(1, kConsumerThreads);
-    if (*flag == 0u) return;
-    __threadfence();
-    // weights w[s][g] = 2^(M_s - M*) in shared memory (stage memory is free now)
-    const int nsg = a.splits * G;
-    float *sw = reinterpret_cast<float *>(smem);   // [splits][G]
-    float *sl = sw + nsg;                          // [splits][G]
-    float *smax = sl + nsg;                        // [G]
-    float *sL = smax + G;                          // [G]
-    const float *pml = a.part_ml + (int64_t)head * a.splits * G * 2;
-    for (int i = d; i < nsg; i += kConsumerThreads) {
-        sw[i] = __ldcg(pml + 2 * i);
-        sl[i] = __ldcg(pml + 2 * i + 1);
-    }
-    named_barrier(1, kConsumerThreads);
-    if (d < G) {
-        float M = -INFINITY;
-        for (int s2 = 0; s2 < a.splits; ++s2) M = fmaxf(M, sw[s2 * G + d]);
-        smax[d] = M;
-    }
-    named_barrier(1, kConsumerThreads);
-    for (int i = d; i < nsg; i += kConsumerThreads) {
-        const float ms = sw[i];
-        sw[i] = (ms == -INFINITY) ? 0.f : exp2_approx(ms - smax[i % G]);
-    }
-    named_barrier(1, kConsumerThreads);
-    if (d < G) {
-        float L = 0.f;
-        for (int s2 = 0; s2 < a.splits; ++s2) L = fmaf(sl[s2 * G + d], sw[s2 * G + d], L);
-        sL[d] = L;
-    }
-    named_barrier(1, kConsumerThreads);
-    const float *po = a.part_o + (int64_t)head * a.splits * G * kD + d;
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-        float O0 = 0.f, O1 = 0.f, O2 = 0.f, O3 = 0.f;
-        int s2 = 0;
-        for (; s2 + 4 <= a.splits; s2 += 4) {
-            O0 = fmaf(__ldcg(po + ((int64_t)(s2 + 0) * G + g) * kD), sw[(s2 + 0) * G + g], O0);
-            O1 = fmaf(__ldcg(po + ((int64_t)(s2 + 1) * G + g) * kD), sw[(s2 + 1) * G + g], O1);
-            O2 = fmaf(__ldcg(po + ((int64_t)(s2 + 2) * G + g) * kD), sw[(s2 + 2) * G + g], O2);
-            O3 = fmaf(__ldcg(po + ((int64_t)(s2 + 3) * G + g) * kD), sw[(s2 + 3) * G + g], O3);
-        }
-        for (; s2 < a.splits; ++s2)
-            O0 = fmaf(__ldcg(po + ((int64_t)s2 * G + g) * kD), sw[s2 * G + g], O0);
-        a.out[((int64_t)b * a.Hq + (int64_t)kv * G + g) * kD + d] = ((O0 + O1) + (O2 + O3)) / sL[g];
-    }
-    if (d == 0) a.tickets[head] = 0u;  // ready for the next call
+    named_barrier(1, kConsumerThreads);  // merge scratch below overwrites mo/mml
+    finish_split<G>(a, head, split, b, kv, d, O, M, L, reinterpret_cast<float *>(smem), flag);
 }
 
 }  // namespace think

@@ -63,12 +63,33 @@ struct ScoreArgs {
 // additions differs from a sequential sum.
 // ---------------------------------------------------------------------------
 template <typename TIn>
-__global__ void __launch_bounds__(256) score_kernel(const ScoreArgs a)
+__device__ __forceinline__ void add_squares(const uint4 &w, double *acc)
+{
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+    if constexpr (sizeof(TIn) == 2) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const double lo = (double)bf16lo(ww[e]);
+            const double hi = (double)bf16hi(ww[e]);
+            acc[2 * e] = fma(lo, lo, acc[2 * e]);
+            acc[2 * e + 1] = fma(hi, hi, acc[2 * e + 1]);
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const double x = (double)__uint_as_float(ww[e]);
+            acc[e] = fma(x, x, acc[e]);
+        }
+    }
+}
+
+template <typename TIn>
+__global__ void __launch_bounds__(256, sizeof(TIn) == 2 ? 4 : 2) score_kernel(const ScoreArgs a)
 {
     constexpr int VEC = 16 / sizeof(TIn);  // channels per 16-byte load
     constexpr int TPR = kD / VEC;          // threads per row
     constexpr int RPP = 256 / TPR;         // rows per pass
-    constexpr int UNROLL = 8;
+    constexpr int UNROLL = sizeof(TIn) == 2 ? 8 : 4;  // 16-byte loads in flight per thread
     __shared__ double red[RPP][kD];
     __shared__ unsigned last;
 
@@ -76,61 +97,50 @@ __global__ void __launch_bounds__(256) score_kernel(const ScoreArgs a)
     const int split = blockIdx.x;
     const int b = head / a.Hkv, kv = head % a.Hkv;
     const int G = a.Hq / a.Hkv;
-    const int cg = threadIdx.x % TPR;
-    const int r = threadIdx.x / TPR;
+    const int tid = threadIdx.x;
+    const int cg = tid % TPR;
+    const int r = tid / TPR;
     const int64_t n0 = (int64_t)split * a.rows_per_split;
     const int64_t n1 = min(a.N, n0 + a.rows_per_split);
     const TIn *base = static_cast<const TIn *>(a.k) + (int64_t)b * a.sb + (int64_t)kv * a.sh + cg * VEC;
 
-    double acc[VEC];
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) acc[e] = 0.0;
-
-    for (int64_t n = n0 + r; n < n1; n += (int64_t)RPP * UNROLL) {
-        uint4 w[UNROLL];
-#pragma unroll
-        for (int u = 0; u < UNROLL; ++u) {
-            const int64_t nn = n + (int64_t)u * RPP;
-            w[u] = (nn < n1) ? __ldg(reinterpret_cast<const uint4 *>(base + nn * a.sn))
-                             : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int u = 0; u < UNROLL; ++u) {
-            const uint32_t ww[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
-            if constexpr (sizeof(TIn) == 2) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const double lo = (double)bf16lo(ww[e]);
-                    const double hi = (double)bf16hi(ww[e]);
-                    acc[2 * e] = fma(lo, lo, acc[2 * e]);
-                    acc[2 * e + 1] = fma(hi, hi, acc[2 * e + 1]);
-                }
-            } else {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const double x = (double)__uint_as_float(ww[e]);
-                    acc[e] = fma(x, x, acc[e]);
-                }
-            }
-        }
-    }
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) red[r][cg * VEC + e] = acc[e];
-
     // window-query energies of the group's query heads g = split, split + splits, ...
-    const int tid = threadIdx.x;
     if (tid < kD) {
         for (int g = split; g < G; g += a.splits) {
             const int64_t h = (int64_t)kv * G + g;
             const TIn *qh = static_cast<const TIn *>(a.qwin) + (((int64_t)b * a.Hq + h) * a.S) * kD + tid;
             double q2 = 0.0;
-            for (int s = 0; s < a.S; ++s) {
+            int s = 0;
+            for (; s + 8 <= a.S; s += 8) {  // loads issued together, added in order
+                double x[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) x[u] = (double)Elem<TIn>::to_float(qh[(int64_t)(s + u) * kD]);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) q2 = __dadd_rn(q2, __dmul_rn(x[u], x[u]));
+            }
+            for (; s < a.S; ++s) {
                 const double x = (double)Elem<TIn>::to_float(qh[(int64_t)s * kD]);
                 q2 = __dadd_rn(q2, __dmul_rn(x, x));
             }
             a.qn2[((int64_t)head * G + g) * kD + tid] = q2;
         }
     }
+
+    double acc[VEC];
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) acc[e] = 0.0;
+    int64_t n = n0 + r;
+    for (; n + (int64_t)(UNROLL - 1) * RPP < n1; n += (int64_t)RPP * UNROLL) {
+        uint4 w[UNROLL];
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u)
+            w[u] = __ldg(reinterpret_cast<const uint4 *>(base + (n + (int64_t)u * RPP) * a.sn));
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u) add_squares<TIn>(w[u], acc);
+    }
+    for (; n < n1; n += RPP) add_squares<TIn>(__ldg(reinterpret_cast<const uint4 *>(base + n * a.sn)), acc);
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) red[r][cg * VEC + e] = acc[e];
     __syncthreads();
     if (tid < kD) {
         double s = 0.0;

@@ -7,11 +7,13 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <cstdlib>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
 
 #include "decode_kernels.cuh"
+#include "decode_tc.cuh"
 #include "prune_kernels.cuh"
 #include "think.h"
 
@@ -19,7 +21,7 @@ namespace think {
 namespace {
 
 constexpr int kTargetSMs = 148;             // B200
-constexpr int kScoreBlocksPerSM = 8;        // 256-thread score blocks resident per SM
+constexpr int kScoreBlocksPerSM = 4;        // 256-thread score blocks resident per SM
 constexpr int kDecodeBlocksPerSM = 2;       // decode blocks the plan aims to keep per SM
 constexpr size_t kDecodeHeader = 256;       // status word + reserved, start of the workspace
 constexpr size_t kSmemPerSM = 233472;       // 228 KB
@@ -31,6 +33,12 @@ inline bool dtype_ok(int t) { return t == THINK_F32 || t == THINK_BF16; }
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+inline bool env_flag(const char *name)
+{
+    const char *v = std::getenv(name);
+    return v && v[0] == '1';
+}
 
 inline think_status_t launch_status()
 {
@@ -62,10 +70,10 @@ struct DecodeSplit {
 
 // Split the token axis so that heads*splits fills kDecodeBlocksPerSM blocks on
 // every SM in one wave; each split is a whole number of 128-token tiles.
-DecodeSplit plan_decode_split(int64_t heads, int64_t N)
+DecodeSplit plan_decode_split(int64_t heads, int64_t N, int blocks_per_sm = kDecodeBlocksPerSM)
 {
     const int64_t tiles = ceil_div(N, kBN);
-    const int64_t target = (int64_t)kTargetSMs * kDecodeBlocksPerSM;
+    const int64_t target = (int64_t)kTargetSMs * blocks_per_sm;
     int64_t s = std::max<int64_t>(1, target / std::max<int64_t>(heads, 1));
     s = std::min(s, tiles);
     const int64_t tps = ceil_div(tiles, s);
@@ -132,7 +140,7 @@ EncodeTiledFn encode_fn()
 // 4-D map over (x, y, z, w) with element strides sy, sz, sw for y, z, w; box (bx, by, 1, 1).
 bool make_map_4d(CUtensorMap *m, think_dtype_t dt, const void *base, uint64_t dx, uint64_t dy,
                  uint64_t dz, uint64_t dw, int64_t sy, int64_t sz, int64_t sw, uint32_t bx,
-                 uint32_t by)
+                 uint32_t by, bool swizzle128 = false)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
@@ -144,7 +152,8 @@ bool make_map_4d(CUtensorMap *m, think_dtype_t dt, const void *base, uint64_t dx
     const CUresult r = fn(m, dt == THINK_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                               : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
                           4, const_cast<void *>(base), dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -296,6 +305,67 @@ think_status_t launch_compact(const void *k, const int64_t k_strides[3], int B, 
     return launch_status();
 }
 
+
+// --------------------------------------------------------- tcgen05 decode --
+
+struct TcPlan {
+    int stages, blocks_per_sm;
+    size_t bytes;
+};
+
+// Two blocks per SM with as many stages (2..4) as fit; otherwise one block
+// per SM with up to 4 stages.
+TcPlan plan_decode_tc(int T)
+{
+    TcPlan p;
+    const size_t per_block_2 = kSmemPerSM / 2 - kSmemReservedPerBlock;
+    for (int st = 4; st >= 2; --st) {
+        const size_t bytes = tc_layout(T, st).total + 1024;
+        if (bytes <= per_block_2) {
+            p.stages = st;
+            p.blocks_per_sm = 2;
+            p.bytes = bytes;
+            return p;
+        }
+    }
+    for (int st = 4; st >= 2; --st) {
+        const size_t bytes = tc_layout(T, st).total + 1024;
+        if (bytes <= kSmemPerBlockMax) {
+            p.stages = st;
+            p.blocks_per_sm = 1;
+            p.bytes = bytes;
+            return p;
+        }
+    }
+    p.stages = 0;
+    return p;
+}
+
+template <int G>
+think_status_t launch_decode_tc_g(const CUtensorMap &mk, const CUtensorMap &mv, const DecodeArgs &a,
+                                  size_t bytes, int heads, cudaStream_t st)
+{
+    auto kern = pruned_decode_tc_kernel<G>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+        cudaSuccess)
+        return THINK_ERR_CUDA;
+    dim3 grid(a.splits, heads);
+    kern<<<grid, kTcThreads, bytes, st>>>(mk, mv, a);
+    return launch_status();
+}
+
+think_status_t launch_decode_tc(int G, const CUtensorMap &mk, const CUtensorMap &mv,
+                                const DecodeArgs &a, size_t bytes, int heads, cudaStream_t st)
+{
+    switch (G) {
+    case 1: return launch_decode_tc_g<1>(mk, mv, a, bytes, heads, st);
+    case 2: return launch_decode_tc_g<2>(mk, mv, a, bytes, heads, st);
+    case 4: return launch_decode_tc_g<4>(mk, mv, a, bytes, heads, st);
+    case 8: return launch_decode_tc_g<8>(mk, mv, a, bytes, heads, st);
+    default: return THINK_ERR_UNSUPPORTED;
+    }
+}
+
 }  // namespace
 }  // namespace think
 
@@ -436,18 +506,34 @@ think_status_t think_pruned_decode_attn(const void *q, const void *k_pruned, int
     const size_t need = think_decode_workspace_size(B, Hq, Hkv, N, d, dtype);
     if (workspace_bytes < need) return THINK_ERR_WORKSPACE;
 
-    const DecodeSplit sp = plan_decode_split(heads, N);
+    // bf16: tcgen05 kernel; fp32 (kept exact in fp32): CUDA-core kernel.  The
+    // environment variable THINK_DECODE_CUDA_CORES=1 selects the CUDA-core
+    // kernel for bf16 too (for comparisons; same results within tolerance).
+    const bool use_tc = dtype == THINK_BF16 && !env_flag("THINK_DECODE_CUDA_CORES");
+    const TcPlan tp = plan_decode_tc(T);
     const DecodeSmem sm = plan_decode_smem(T, G, es);
-    if (sm.bytes > kSmemPerBlockMax) return THINK_ERR_UNSUPPORTED;
+    if (use_tc ? tp.stages == 0 : sm.bytes > kSmemPerBlockMax) return THINK_ERR_UNSUPPORTED;
+    const DecodeSplit sp = plan_decode_split(heads, N, use_tc ? tp.blocks_per_sm : kDecodeBlocksPerSM);
     CUtensorMap mk, mv;
-    // K'^T: x = token (pitch ldk), y = kept channel, z = KV head, w = batch
-    if (!make_map_4d(&mk, dtype, k_pruned, (uint64_t)N, (uint64_t)T, (uint64_t)Hkv, (uint64_t)B,
-                     ldk, (int64_t)T * ldk, (int64_t)Hkv * T * ldk, kBN, (uint32_t)T))
-        return THINK_ERR_CUDA;
-    // V: x = channel, y = token, z = KV head, w = batch
-    if (!make_map_4d(&mv, dtype, v, kD, (uint64_t)N, (uint64_t)Hkv, (uint64_t)B, v_strides[2],
-                     v_strides[1], v_strides[0], kD, kBN))
-        return THINK_ERR_CUDA;
+    if (use_tc) {
+        // K'^T in 64-token halves, V in 64-channel halves, 128-byte swizzle (the
+        // tensor core's MN-major canonical layout)
+        if (!make_map_4d(&mk, dtype, k_pruned, (uint64_t)N, (uint64_t)T, (uint64_t)Hkv, (uint64_t)B,
+                         ldk, (int64_t)T * ldk, (int64_t)Hkv * T * ldk, 64, (uint32_t)T, true))
+            return THINK_ERR_CUDA;
+        if (!make_map_4d(&mv, dtype, v, kD, (uint64_t)N, (uint64_t)Hkv, (uint64_t)B, v_strides[2],
+                         v_strides[1], v_strides[0], 64, kBN, true))
+            return THINK_ERR_CUDA;
+    } else {
+        // K'^T: x = token (pitch ldk), y = kept channel, z = KV head, w = batch
+        if (!make_map_4d(&mk, dtype, k_pruned, (uint64_t)N, (uint64_t)T, (uint64_t)Hkv, (uint64_t)B,
+                         ldk, (int64_t)T * ldk, (int64_t)Hkv * T * ldk, kBN, (uint32_t)T))
+            return THINK_ERR_CUDA;
+        // V: x = channel, y = token, z = KV head, w = batch
+        if (!make_map_4d(&mv, dtype, v, kD, (uint64_t)N, (uint64_t)Hkv, (uint64_t)B, v_strides[2],
+                         v_strides[1], v_strides[0], kD, kBN))
+            return THINK_ERR_CUDA;
+    }
 
     unsigned char *ws = static_cast<unsigned char *>(workspace);
     const size_t slots = (size_t)heads * sp.splits * G;
@@ -466,17 +552,16 @@ think_status_t think_pruned_decode_attn(const void *q, const void *k_pruned, int
     a.N = N;
     a.tiles_per_split = sp.tiles_per_split;
     a.splits = sp.splits;
-    a.stages = sm.stages;
+    a.stages = use_tc ? tp.stages : sm.stages;
     a.scale_log2 = scale * 1.4426950408889634f;
     a.stage_bytes = sm.stage_bytes;
     a.v_off = sm.v_off;
     a.tx_bytes = sm.tx_bytes;
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    think_status_t r = dtype == THINK_BF16
-                           ? launch_decode<__nv_bfloat16>(G, mk, mv, a, sm, (int)heads, st)
-                           : launch_decode<float>(G, mk, mv, a, sm, (int)heads, st);
-    return r;
+    if (use_tc) return launch_decode_tc(G, mk, mv, a, tp.bytes, (int)heads, st);
+    if (dtype == THINK_BF16) return launch_decode<__nv_bfloat16>(G, mk, mv, a, sm, (int)heads, st);
+    return launch_decode<float>(G, mk, mv, a, sm, (int)heads, st);
 }
 
 think_status_t think_workspace_init(void *workspace, size_t workspace_bytes, void *stream)
