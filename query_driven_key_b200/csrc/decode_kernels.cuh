@@ -40,6 +40,8 @@ struct DecodeArgs {
     int Hq, Hkv, T;
     int64_t N;
     int tiles_per_split, splits, stages;
+    int stages_v;           // tcgen05 kernel: V ring slots (stages = K' ring slots)
+    int prefetch;           // tiles prefetched into L2 ahead of the TMA loads
     float scale_log2;       // scale * log2(e)
     uint32_t stage_bytes;   // bytes per ring stage (multiple of 1024)
     uint32_t v_off;         // offset of the V tile inside a stage
@@ -135,79 +137,110 @@ template <> struct V8<float> {
     }
 };
 
-// Write this block's partial (O[g][d] for d = tid, max M[g] in log2 units,
-// sum L[g]) for (head, split); the last block of the head to arrive merges
-// every split of the head into `out`.  Called by the kConsumerThreads
-// consumer threads only; `scratch` is free shared memory of at least
-// (2 * splits * G + 2 * G) floats, `flag` one shared word.
-template <int G>
+// Write this block's partial (O[g][d] for d = tid < 128, max M[g] in log2
+// units, sum L[g]) for (head, split); the last block of the head to arrive
+// merges every split of the head into `out`.  Called by the NT threads
+// 0 .. NT-1 of the block (NT a multiple of 128), which synchronise on named
+// barrier `bar`; `scratch` is free shared memory of at least
+// (2 * splits * G + 2 * G + (NT / 128) * G * 128) floats, `flag` one shared
+// word.  The merge issues its global loads together: one round trip for the
+// (max, sum) pairs and about one per 8 * NT / 128 splits for the outputs.
+template <int G, int NT>
 __device__ __forceinline__ void finish_split(const DecodeArgs &a, int head, int split, int b, int kv,
-                                             int d, const float (&O)[G], const float (&M)[G],
-                                             const float (&L)[G], float *scratch, unsigned *flag)
+                                             int tid, const float (&O)[G], const float (&M)[G],
+                                             const float (&L)[G], float *scratch, unsigned *flag,
+                                             int bar)
 {
+    static_assert(NT % 128 == 0, "whole channel rows per thread group");
+    constexpr int P = NT / 128;            // thread groups splitting the split axis
     const int64_t slot0 = ((int64_t)head * a.splits + split) * G;
+    if (tid < 128) {
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-        a.part_o[(slot0 + g) * kD + d] = O[g];
-        if (d == 0) {
-            a.part_ml[(slot0 + g) * 2] = M[g];
-            a.part_ml[(slot0 + g) * 2 + 1] = L[g];
+        for (int g = 0; g < G; ++g) {
+            a.part_o[(slot0 + g) * kD + tid] = O[g];
+            if (tid == 0) {
+                a.part_ml[(slot0 + g) * 2] = M[g];
+                a.part_ml[(slot0 + g) * 2 + 1] = L[g];
+            }
         }
     }
     __threadfence();
-    named_barrier(1, kConsumerThreads);
-    if (d == 0) {
+    named_barrier(bar, NT);
+    if (tid == 0) {
         const unsigned ticket = atomicAdd(a.tickets + head, 1u);
         *flag = (ticket == (unsigned)(a.splits - 1)) ? 1u : 0u;
     }
-    named_barrier(1, kConsumerThreads);
+    named_barrier(bar, NT);
     if (*flag == 0u) return;
     __threadfence();
-    // weights w[s][g] = 2^(M_s - M*)
-    const int nsg = a.splits * G;
-    float *sw = scratch;        // [splits][G]
-    float *sl = sw + nsg;       // [splits][G]
-    float *smax = sl + nsg;     // [G]
-    float *sL = smax + G;       // [G]
-    const float *pml = a.part_ml + (int64_t)head * a.splits * G * 2;
-    for (int i = d; i < nsg; i += kConsumerThreads) {
-        sw[i] = __ldcg(pml + 2 * i);
-        sl[i] = __ldcg(pml + 2 * i + 1);
+    const int S = a.splits;
+    const int nsg = S * G;
+    float *sw = scratch;            // [splits][G]  max, then weight 2^(M_s - M*)
+    float *sl = sw + nsg;           // [splits][G]  sum
+    float *smax = sl + nsg;         // [G]
+    float *sL = smax + G;           // [G]
+    float *sp = sL + G;             // [P][G][128]  per-group output sums
+    const float *pml = a.part_ml + (int64_t)head * S * G * 2;
+    for (int i = tid; i < nsg; i += NT) {
+        const float2 ml = __ldcg(reinterpret_cast<const float2 *>(pml) + i);
+        sw[i] = ml.x;
+        sl[i] = ml.y;
     }
-    named_barrier(1, kConsumerThreads);
-    if (d < G) {
+    named_barrier(bar, NT);
+    if (tid < G) {
         float Mx = -INFINITY;
-        for (int s2 = 0; s2 < a.splits; ++s2) Mx = fmaxf(Mx, sw[s2 * G + d]);
-        smax[d] = Mx;
+        for (int s2 = 0; s2 < S; ++s2) Mx = fmaxf(Mx, sw[s2 * G + tid]);
+        smax[tid] = Mx;
     }
-    named_barrier(1, kConsumerThreads);
-    for (int i = d; i < nsg; i += kConsumerThreads) {
+    named_barrier(bar, NT);
+    for (int i = tid; i < nsg; i += NT) {
         const float ms = sw[i];
         sw[i] = (ms == -INFINITY) ? 0.f : exp2_approx(ms - smax[i % G]);
     }
-    named_barrier(1, kConsumerThreads);
-    if (d < G) {
+    named_barrier(bar, NT);
+    if (tid < G) {
         float Ls = 0.f;
-        for (int s2 = 0; s2 < a.splits; ++s2) Ls = fmaf(sl[s2 * G + d], sw[s2 * G + d], Ls);
-        sL[d] = Ls;
+        for (int s2 = 0; s2 < S; ++s2) Ls = fmaf(sl[s2 * G + tid], sw[s2 * G + tid], Ls);
+        sL[tid] = Ls;
     }
-    named_barrier(1, kConsumerThreads);
-    const float *po = a.part_o + (int64_t)head * a.splits * G * kD + d;
+    // outputs: thread (q, d) sums the splits s = q, q + P, ... for channel d
+    const int d = tid & 127, q = tid >> 7;
+    const float *po = a.part_o + (int64_t)head * S * G * kD + d;
+    float acc[G];
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-        float O0 = 0.f, O1 = 0.f, O2 = 0.f, O3 = 0.f;
-        int s2 = 0;
-        for (; s2 + 4 <= a.splits; s2 += 4) {
-            O0 = fmaf(__ldcg(po + ((int64_t)(s2 + 0) * G + g) * kD), sw[(s2 + 0) * G + g], O0);
-            O1 = fmaf(__ldcg(po + ((int64_t)(s2 + 1) * G + g) * kD), sw[(s2 + 1) * G + g], O1);
-            O2 = fmaf(__ldcg(po + ((int64_t)(s2 + 2) * G + g) * kD), sw[(s2 + 2) * G + g], O2);
-            O3 = fmaf(__ldcg(po + ((int64_t)(s2 + 3) * G + g) * kD), sw[(s2 + 3) * G + g], O3);
+    for (int g = 0; g < G; ++g) acc[g] = 0.f;
+    constexpr int CH = 8;
+    for (int s0 = q; s0 < S; s0 += P * CH) {
+        float v[CH][G];
+#pragma unroll
+        for (int u = 0; u < CH; ++u) {
+            const int s2 = s0 + u * P;
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+                v[u][g] = (s2 < S) ? __ldcg(po + ((int64_t)s2 * G + g) * kD) : 0.f;
         }
-        for (; s2 < a.splits; ++s2)
-            O0 = fmaf(__ldcg(po + ((int64_t)s2 * G + g) * kD), sw[s2 * G + g], O0);
-        a.out[((int64_t)b * a.Hq + (int64_t)kv * G + g) * kD + d] = ((O0 + O1) + (O2 + O3)) / sL[g];
+#pragma unroll
+        for (int u = 0; u < CH; ++u) {
+            const int s2 = s0 + u * P;
+            if (s2 < S) {
+#pragma unroll
+                for (int g = 0; g < G; ++g) acc[g] = fmaf(v[u][g], sw[s2 * G + g], acc[g]);
+            }
+        }
     }
-    if (d == 0) a.tickets[head] = 0u;  // ready for the next call
+#pragma unroll
+    for (int g = 0; g < G; ++g) sp[(q * G + g) * kD + d] = acc[g];
+    named_barrier(bar, NT);
+    if (tid < 128) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            float o = sp[g * kD + d];
+#pragma unroll
+            for (int q2 = 1; q2 < P; ++q2) o += sp[(q2 * G + g) * kD + d];
+            a.out[((int64_t)b * a.Hq + (int64_t)kv * G + g) * kD + d] = o / sL[g];
+        }
+        if (tid == 0) a.tickets[head] = 0u;  // ready for the next call
+    }
 }
 
 template <typename TIn, int G>
@@ -245,36 +278,33 @@ __global__ void __launch_bounds__(kDecodeThreads)
         }
         fence_barrier_init();
     }
-    if (warp == kConsumerWarps && lane == 0) {
-        prefetch_tensormap(&tm_k);
-        prefetch_tensormap(&tm_v);
-    }
-    // q' = q[idx] for the G query heads of this KV head, pre-scaled to log2 units.
-    {
-        const TIn *q = reinterpret_cast<const TIn *>(a.q);
-        const int32_t *ih = a.idx + (int64_t)head * T;
-        for (int i = tid; i < T * G; i += kDecodeThreads) {
-            const int t = i / G, g = i % G;
-            const int c = ih[t];
-            float x = 0.f;
-            if ((unsigned)c < (unsigned)kD)
-                x = Elem<TIn>::to_float(q[((int64_t)b * a.Hq + (int64_t)kv * G + g) * kD + c]);
-            qs[i] = x * a.scale_log2;
-        }
-    }
-    __syncthreads();
+    __syncthreads();  // barriers initialised
 
     if (warp == kConsumerWarps) {
         // ------------------------------------------------------ producer
+        // starts at once; the consumers gather q' meanwhile
         if (lane == 0) {
+            prefetch_tensormap(&tm_k);
+            prefetch_tensormap(&tm_v);
             int issued = 0;
             bool ok = true;
+            const int pf = a.prefetch;
+            for (int it = 0; it < min(ntiles, pf); ++it) {
+                const int x = (int)((tile0 + it) * kBN);
+                tma_prefetch_l2_4d(&tm_k, x, 0, kv, b);
+                tma_prefetch_l2_4d(&tm_v, 0, x, kv, b);
+            }
             for (int it = 0; it < ntiles; ++it) {
                 const int s = it % stages, f = it / stages;
                 if (f > 0 && !mbar_wait_bounded(empty0 + 8 * s, (f - 1) & 1, a.status,
                                                 THINK_DEVICE_TIMEOUT_EMPTY)) {
                     ok = false;
                     break;
+                }
+                if (pf > 0 && it + pf < ntiles) {
+                    const int xp = (int)((tile0 + it + pf) * kBN);
+                    tma_prefetch_l2_4d(&tm_k, xp, 0, kv, b);
+                    tma_prefetch_l2_4d(&tm_v, 0, xp, kv, b);
                 }
                 const uint32_t full = full0 + 8 * s;
                 mbar_arrive_expect_tx(full, a.tx_bytes);
@@ -295,6 +325,20 @@ __global__ void __launch_bounds__(kDecodeThreads)
     }
 
     // ---------------------------------------------------------- consumers
+    // q' = q[idx] for the G query heads of this KV head, pre-scaled to log2 units.
+    {
+        const TIn *q = reinterpret_cast<const TIn *>(a.q);
+        const int32_t *ih = a.idx + (int64_t)head * T;
+        for (int i = tid; i < T * G; i += kConsumerThreads) {
+            const int t = i / G, g = i % G;
+            const int c = ih[t];
+            float x = 0.f;
+            if ((unsigned)c < (unsigned)kD)
+                x = Elem<TIn>::to_float(q[((int64_t)b * a.Hq + (int64_t)kv * G + g) * kD + c]);
+            qs[i] = x * a.scale_log2;
+        }
+    }
+    named_barrier(1, kConsumerThreads);
     float m[G], l[G];
     float2 acc[G][4];  // channels 8*(lane&15) .. +7 of the tokens of half-warp lane>>4
 #pragma unroll
@@ -402,7 +446,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
         }
     }
     named_barrier(1, kConsumerThreads);  // merge scratch below overwrites mo/mml
-    finish_split<G>(a, head, split, b, kv, d, O, M, L, reinterpret_cast<float *>(smem), flag);
+    finish_split<G, kConsumerThreads>(a, head, split, b, kv, d, O, M, L, reinterpret_cast<float *>(smem),
+                                      flag, 1);
 }
 
 }  // namespace think

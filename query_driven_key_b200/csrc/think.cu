@@ -23,22 +23,32 @@ namespace {
 constexpr int kTargetSMs = 148;             // B200
 constexpr int kScoreBlocksPerSM = 4;        // 256-thread score blocks resident per SM
 constexpr int kDecodeBlocksPerSM = 2;       // decode blocks the plan aims to keep per SM
+constexpr int kDecodePrefetchTiles = 0;     // tiles a decode block prefetches into L2 ahead of TMA
+constexpr int kTcBlocksPerSM = 1;           // tcgen05 decode: blocks per SM the plan aims for
 constexpr size_t kDecodeHeader = 256;       // status word + reserved, start of the workspace
 constexpr size_t kSmemPerSM = 233472;       // 228 KB
 constexpr size_t kSmemPerBlockMax = 232448; // 227 KB opt-in
 constexpr size_t kSmemReservedPerBlock = 1024;
-
-inline size_t esize(think_dtype_t t) { return t == THINK_BF16 ? 2 : 4; }
-inline bool dtype_ok(int t) { return t == THINK_F32 || t == THINK_BF16; }
-inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
-inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 inline bool env_flag(const char *name)
 {
     const char *v = std::getenv(name);
     return v && v[0] == '1';
 }
+
+inline int env_int(const char *name, int dflt, int lo, int hi)
+{
+    const char *v = std::getenv(name);
+    if (!v || !*v) return dflt;
+    const int x = std::atoi(v);
+    return x < lo ? lo : (x > hi ? hi : x);
+}
+
+inline size_t esize(think_dtype_t t) { return t == THINK_BF16 ? 2 : 4; }
+inline bool dtype_ok(int t) { return t == THINK_F32 || t == THINK_BF16; }
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 inline think_status_t launch_status()
 {
@@ -309,35 +319,30 @@ think_status_t launch_compact(const void *k, const int64_t k_strides[3], int B, 
 // --------------------------------------------------------- tcgen05 decode --
 
 struct TcPlan {
-    int stages, blocks_per_sm;
+    int stages_k, stages_v;
     size_t bytes;
 };
 
-// Two blocks per SM with as many stages (2..4) as fit; otherwise one block
-// per SM with up to 4 stages.
+// One block per SM: 4 V slots if possible, then as many K' slots (2..6) as
+// fit.  THINK_DECODE_STAGES_V / THINK_DECODE_STAGES_K cap the choice (tuning).
 TcPlan plan_decode_tc(int T)
 {
     TcPlan p;
-    const size_t per_block_2 = kSmemPerSM / 2 - kSmemReservedPerBlock;
-    for (int st = 4; st >= 2; --st) {
-        const size_t bytes = tc_layout(T, st).total + 1024;
-        if (bytes <= per_block_2) {
-            p.stages = st;
-            p.blocks_per_sm = 2;
-            p.bytes = bytes;
-            return p;
+    const int max_v = env_int("THINK_DECODE_STAGES_V", 4, 2, 6);
+    const int max_k = env_int("THINK_DECODE_STAGES_K", 6, 2, 8);
+    for (int v = max_v; v >= 2; --v)
+        for (int k = max_k; k >= 2; --k) {
+            const size_t bytes = tc_layout(T, k, v).total + 1024;
+            if (bytes <= kSmemPerBlockMax) {
+                p.stages_k = k;
+                p.stages_v = v;
+                p.bytes = bytes;
+                return p;
+            }
         }
-    }
-    for (int st = 4; st >= 2; --st) {
-        const size_t bytes = tc_layout(T, st).total + 1024;
-        if (bytes <= kSmemPerBlockMax) {
-            p.stages = st;
-            p.blocks_per_sm = 1;
-            p.bytes = bytes;
-            return p;
-        }
-    }
-    p.stages = 0;
+    p.stages_k = 0;
+    p.stages_v = 0;
+    p.bytes = 0;
     return p;
 }
 
@@ -512,8 +517,8 @@ think_status_t think_pruned_decode_attn(const void *q, const void *k_pruned, int
     const bool use_tc = dtype == THINK_BF16 && !env_flag("THINK_DECODE_CUDA_CORES");
     const TcPlan tp = plan_decode_tc(T);
     const DecodeSmem sm = plan_decode_smem(T, G, es);
-    if (use_tc ? tp.stages == 0 : sm.bytes > kSmemPerBlockMax) return THINK_ERR_UNSUPPORTED;
-    const DecodeSplit sp = plan_decode_split(heads, N, use_tc ? tp.blocks_per_sm : kDecodeBlocksPerSM);
+    if (use_tc ? tp.stages_k == 0 : sm.bytes > kSmemPerBlockMax) return THINK_ERR_UNSUPPORTED;
+    const DecodeSplit sp = plan_decode_split(heads, N, use_tc ? kTcBlocksPerSM : kDecodeBlocksPerSM);
     CUtensorMap mk, mv;
     if (use_tc) {
         // K'^T in 64-token halves, V in 64-channel halves, 128-byte swizzle (the
@@ -552,7 +557,9 @@ think_status_t think_pruned_decode_attn(const void *q, const void *k_pruned, int
     a.N = N;
     a.tiles_per_split = sp.tiles_per_split;
     a.splits = sp.splits;
-    a.stages = use_tc ? tp.stages : sm.stages;
+    a.stages = use_tc ? tp.stages_k : sm.stages;
+    a.stages_v = use_tc ? tp.stages_v : 0;
+    a.prefetch = env_int("THINK_DECODE_PREFETCH", kDecodePrefetchTiles, 0, 64);
     a.scale_log2 = scale * 1.4426950408889634f;
     a.stage_bytes = sm.stage_bytes;
     a.v_off = sm.v_off;
