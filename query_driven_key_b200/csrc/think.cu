@@ -511,10 +511,10 @@ think_status_t think_pruned_decode_attn(const void *q, const void *k_pruned, int
     const size_t need = think_decode_workspace_size(B, Hq, Hkv, N, d, dtype);
     if (workspace_bytes < need) return THINK_ERR_WORKSPACE;
 
-    // bf16: tcgen05 kernel; fp32 (kept exact in fp32): CUDA-core kernel.  The
-    // environment variable THINK_DECODE_CUDA_CORES=1 selects the CUDA-core
-    // kernel for bf16 too (for comparisons; same results within tolerance).
-    const bool use_tc = dtype == THINK_BF16 && !env_flag("THINK_DECODE_CUDA_CORES");
+    // CUDA-core kernel by default (the faster one on B200 for this HBM-bound
+    // scan); THINK_DECODE_TENSOR_CORES=1 selects the tcgen05 kernel for bf16
+    // (same results within tolerance).  fp32 inputs always use CUDA cores.
+    const bool use_tc = dtype == THINK_BF16 && env_flag("THINK_DECODE_TENSOR_CORES");
     const TcPlan tp = plan_decode_tc(T);
     const DecodeSmem sm = plan_decode_smem(T, G, es);
     if (use_tc ? tp.stages_k == 0 : sm.bytes > kSmemPerBlockMax) return THINK_ERR_UNSUPPORTED;

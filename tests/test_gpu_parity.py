@@ -202,6 +202,22 @@ def test_fused_prune_equals_stepwise_calls():
     assert torch.equal(a.idx, b.idx)
 
 
+@pytest.mark.parametrize("kernel", ["cuda_cores", "tensor_cores"])
+def test_both_bf16_decode_kernels(kernel, monkeypatch):
+    # the CUDA-core kernel (default) and the tcgen05 kernel on the same inputs
+    if kernel == "tensor_cores":
+        monkeypatch.setenv("THINK_DECODE_TENSOR_CORES", "1")
+    else:
+        monkeypatch.delenv("THINK_DECODE_TENSOR_CORES", raising=False)
+    w = W.WORKLOADS["mistral_7b_long"].with_(N=20000)
+    q_win, k, v = W.gen_layer(w)
+    _full_path_check(w, q_win, k, v, steps=[0, 1])
+    for G, Hq in [(1, 8), (2, 16), (8, 64)]:
+        wg = w.with_(Hq=Hq, N=3000)
+        q_win, k, v = W.gen_layer(wg)
+        _full_path_check(wg, q_win, k, v, steps=[0])
+
+
 def test_scores_are_deterministic():
     w = W.WORKLOADS["llama2_7b_mha"]
     q_win, k, _ = W.gen_slice(w, 0, 0)
