@@ -169,6 +169,32 @@ think_status_t think_pruned_decode_attn(const void *q, const void *k_pruned, int
                                         float *out, void *workspace, size_t workspace_bytes,
                                         void *stream);
 
+/* ---------------------------------------------- decode without allocation --
+ * No counterpart in the paper: an implementation convenience.  Some callers
+ * may not allocate device memory at all, e.g. a library running inside a
+ * host framework that owns the whole device-memory budget, or a
+ * latency-critical path where an allocation (which can synchronise the
+ * device) is not allowed.  This entry point is think_pruned_decode_attn with
+ * its workspace replaced by a scratch array that the library holds in device
+ * memory (think_noalloc_scratch_bytes() bytes, 4 MiB, on every GPU that loads
+ * the library, until the process exits).  Arguments and results are those of
+ * think_pruned_decode_attn.
+ *   - It calls no cudaMalloc or cudaFree.  The first call on a device looks
+ *     up the array's device address (cudaGetSymbolAddress) with that device
+ *     current; make that first call before any stream capture.
+ *   - Every call clears the array's counters (a stream-ordered memset) and
+ *     then uses the array; all calls share it, so calls that overlap on the
+ *     GPU (different streams, or different host threads without ordering)
+ *     race and give wrong results.  Order them on one stream.
+ *   - A problem whose workspace (think_decode_workspace_size) exceeds the
+ *     array returns THINK_ERR_WORKSPACE and launches nothing. */
+size_t think_noalloc_scratch_bytes(void);
+think_status_t think_pruned_decode_attn_noalloc(const void *q, const void *k_pruned, int64_t ldk,
+                                                const void *v, const int64_t v_strides[3],
+                                                const int32_t *idx, int B, int Hq, int Hkv,
+                                                int64_t N, int d, int T, think_dtype_t dtype,
+                                                float scale, float *out, void *stream);
+
 /* Zero a score or decode workspace (stream-ordered memset). */
 think_status_t think_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
 

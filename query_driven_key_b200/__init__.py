@@ -34,7 +34,8 @@ EXPORTED = (
     "think_status_string", "think_t_from_lambda", "think_pruned_ld",
     "think_score_workspace_size", "think_score_channels", "think_select_channels",
     "think_compact_keys", "think_prune", "think_decode_workspace_size", "think_pruned_decode_attn",
-    "think_workspace_init", "think_read_device_status",
+    "think_workspace_init", "think_read_device_status", "think_noalloc_scratch_bytes",
+    "think_pruned_decode_attn_noalloc",
 )
 
 
@@ -68,6 +69,11 @@ def _load() -> ctypes.CDLL:
     lib.think_pruned_decode_attn.argtypes = [P, P, I64, P, I64P, P, I, I, I, I64, I, I, I, F, P,
                                              P, SZ, P]
     lib.think_pruned_decode_attn.restype = I
+    lib.think_noalloc_scratch_bytes.argtypes = []
+    lib.think_noalloc_scratch_bytes.restype = SZ
+    lib.think_pruned_decode_attn_noalloc.argtypes = [P, P, I64, P, I64P, P, I, I, I, I64, I, I, I, F,
+                                                     P, P]
+    lib.think_pruned_decode_attn_noalloc.restype = I
     lib.think_workspace_init.argtypes = [P, SZ, P]
     lib.think_workspace_init.restype = I
     lib.think_read_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint32), P]
@@ -199,6 +205,26 @@ def think_pruned_decode_attn(q: torch.Tensor, k_pruned: torch.Tensor, ldk: int, 
                                         _ptr(out), _ptr(workspace),
                                         workspace.numel() * workspace.element_size(),
                                         _stream(stream)), "think_pruned_decode_attn")
+
+
+def think_pruned_decode_attn_noalloc(q: torch.Tensor, k_pruned: torch.Tensor, ldk: int,
+                                     v: torch.Tensor, idx: torch.Tensor, out: torch.Tensor,
+                                     scale: float | None = None, N: int | None = None,
+                                     stream=None) -> None:
+    """think_pruned_decode_attn with the library's built-in scratch instead of a
+    caller workspace (for callers that may not allocate device memory)."""
+    B, Hq, d = q.shape
+    _, Hkv, Nv, _ = v.shape
+    N = Nv if N is None else N
+    T = idx.shape[-1]
+    if scale is None:
+        scale = 1.0 / float(d) ** 0.5
+    if not q.is_contiguous() or out.dtype != torch.float32 or idx.dtype != torch.int32:
+        raise ThinkError(THINK_ERR_INVALID_ARG, "think_pruned_decode_attn_noalloc")
+    _check(lib.think_pruned_decode_attn_noalloc(_ptr(q), _ptr(k_pruned), int(ldk), _ptr(v),
+                                                _strides3(v), _ptr(idx), B, Hq, Hkv, N, d, T,
+                                                _dtype(q), float(scale), _ptr(out), _stream(stream)),
+           "think_pruned_decode_attn_noalloc")
 
 
 def think_workspace_init(workspace: torch.Tensor, stream=None) -> None:

@@ -374,6 +374,48 @@ think_status_t launch_decode_tc(int G, const CUtensorMap &mk, const CUtensorMap 
 }  // namespace
 }  // namespace think
 
+// ------------------------------------------------------ decode without allocation --
+// Callers that may not allocate device memory (a host framework that owns the
+// whole device-memory budget, or a latency-critical path where an allocation,
+// which can synchronise the device, is not allowed) use
+// think_pruned_decode_attn_noalloc, whose scratch lives in this file-scope
+// array.  Every GPU that loads the library holds it until the process exits.
+namespace think {
+namespace {
+constexpr size_t kNoAllocScratchBytes = (size_t)4 << 20;  // 4 MiB
+constexpr int kNoAllocMaxDevices = 64;
+}  // namespace
+}  // namespace think
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[think::kNoAllocScratchBytes];
+
+namespace think {
+namespace {
+std::mutex g_noalloc_mutex;
+void *g_noalloc_ptr[kNoAllocMaxDevices];  // device address of g_noalloc_scratch, per device
+
+// Device address of the scratch array on the current device, looked up once
+// per device (with that device current).  In host code the array's name only
+// stands for it; the kernel must be given this address.
+cudaError_t noalloc_scratch(void **out)
+{
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return cudaSuccess;
+}
+}  // namespace
+}  // namespace think
+
 using namespace think;
 
 extern "C" {
@@ -589,6 +631,32 @@ think_status_t think_read_device_status(const void *workspace, uint32_t *status,
         cudaSuccess)
         return THINK_ERR_CUDA;
     return cudaStreamSynchronize(st) == cudaSuccess ? THINK_OK : THINK_ERR_CUDA;
+}
+
+size_t think_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
+
+think_status_t think_pruned_decode_attn_noalloc(const void *q, const void *k_pruned, int64_t ldk,
+                                                const void *v, const int64_t v_strides[3],
+                                                const int32_t *idx, int B, int Hq, int Hkv,
+                                                int64_t N, int d, int T, think_dtype_t dtype,
+                                                float scale, float *out, void *stream)
+{
+    // Same validation as the workspace form; the problem must fit the array.
+    if (B < 0 || Hq < 0 || Hkv < 0 || N < 0) return THINK_ERR_INVALID_ARG;
+    if (B == 0 || Hkv == 0) return THINK_OK;
+    const size_t need = think_decode_workspace_size(B, Hq, Hkv, N, d, dtype);
+    if (need > kNoAllocScratchBytes) return THINK_ERR_WORKSPACE;
+    if (need == 0)  // shape rejected by the sizing rules: let the full check name the reason
+        return think_pruned_decode_attn(q, k_pruned, ldk, v, v_strides, idx, B, Hq, Hkv, N, d, T,
+                                        dtype, scale, out, nullptr, 0, stream);
+    void *ws = nullptr;
+    if (noalloc_scratch(&ws) != cudaSuccess) return THINK_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // the status word and the per-head arrival counters must start at zero
+    const size_t zero = kDecodeHeader + align_up((size_t)B * Hkv * sizeof(unsigned), 256);
+    if (cudaMemsetAsync(ws, 0, zero, st) != cudaSuccess) return THINK_ERR_CUDA;
+    return think_pruned_decode_attn(q, k_pruned, ldk, v, v_strides, idx, B, Hq, Hkv, N, d, T, dtype,
+                                    scale, out, ws, kNoAllocScratchBytes, stream);
 }
 
 }  // extern "C"
