@@ -56,23 +56,50 @@ struct ScoreArgs {
 // 16-byte loads (bf16: 16 threads x 8 channels per row, 16 rows per pass, 8
 // passes in flight); blocks split < G also sum the window-query energies of
 // query head kv*G + split.  The last block of the head to finish (ticket
-// counter) adds the partials in split order and forms
+// counter) adds the partials in a fixed order (even and odd splits in two
+// halves of the block, then the halves) and forms
 //     s[c] = sum_g sqrt(qn2[g][c]) * sqrt(kn2[c])
 // with each operation rounded as written, then optionally selects the top T.
 // The square of a bf16 or fp32 value is exact in fp64; only the order of the
 // additions differs from a sequential sum.
 // ---------------------------------------------------------------------------
+// fp64 value of a bf16 with a nonzero exponent field, built from its bits:
+// the fp64 exponent is the bf16 exponent + (1023 - 127) and the 7 mantissa
+// bits go to the top of the fp64 mantissa; the low word is zero.  The sign is
+// dropped (only squares are used).  Exact for every normal bf16 value.
+__device__ __forceinline__ double bf16_abs_to_f64_normal(uint32_t bits15)
+{
+    return __hiloint2double((int)(bits15 * 8192u + 0x38000000u), 0);
+}
+
 template <typename TIn>
 __device__ __forceinline__ void add_squares(const uint4 &w, double *acc)
 {
     const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
     if constexpr (sizeof(TIn) == 2) {
+        // Fast path (integer ops + fp64 FMA, no conversion unit) when no element
+        // of the 16 bytes has a zero exponent field (zero or subnormal); the
+        // exact conversion otherwise.  Both give the same fp64 squares.
+        const bool zero_exp = ((ww[0] & 0x7f80u) == 0u) | ((ww[0] & 0x7f800000u) == 0u) |
+                              ((ww[1] & 0x7f80u) == 0u) | ((ww[1] & 0x7f800000u) == 0u) |
+                              ((ww[2] & 0x7f80u) == 0u) | ((ww[2] & 0x7f800000u) == 0u) |
+                              ((ww[3] & 0x7f80u) == 0u) | ((ww[3] & 0x7f800000u) == 0u);
+        if (!zero_exp) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const double lo = (double)bf16lo(ww[e]);
-            const double hi = (double)bf16hi(ww[e]);
-            acc[2 * e] = fma(lo, lo, acc[2 * e]);
-            acc[2 * e + 1] = fma(hi, hi, acc[2 * e + 1]);
+            for (int e = 0; e < 4; ++e) {
+                const double lo = bf16_abs_to_f64_normal(ww[e] & 0x7fffu);
+                const double hi = bf16_abs_to_f64_normal((ww[e] >> 16) & 0x7fffu);
+                acc[2 * e] = fma(lo, lo, acc[2 * e]);
+                acc[2 * e + 1] = fma(hi, hi, acc[2 * e + 1]);
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const double lo = (double)bf16lo(ww[e]);
+                const double hi = (double)bf16hi(ww[e]);
+                acc[2 * e] = fma(lo, lo, acc[2 * e]);
+                acc[2 * e + 1] = fma(hi, hi, acc[2 * e + 1]);
+            }
         }
     } else {
 #pragma unroll
@@ -89,7 +116,7 @@ __global__ void __launch_bounds__(256, sizeof(TIn) == 2 ? 4 : 2) score_kernel(co
     constexpr int VEC = 16 / sizeof(TIn);  // channels per 16-byte load
     constexpr int TPR = kD / VEC;          // threads per row
     constexpr int RPP = 256 / TPR;         // rows per pass
-    constexpr int UNROLL = sizeof(TIn) == 2 ? 8 : 4;  // 16-byte loads in flight per thread
+    constexpr int UNROLL = 4;              // 16-byte loads per batch (two batches in flight)
     __shared__ double red[RPP][kD];
     __shared__ unsigned last;
 
@@ -129,14 +156,33 @@ __global__ void __launch_bounds__(256, sizeof(TIn) == 2 ? 4 : 2) score_kernel(co
     double acc[VEC];
 #pragma unroll
     for (int e = 0; e < VEC; ++e) acc[e] = 0.0;
+    // Software pipeline: the loads of the next batch of UNROLL rows are issued
+    // before the squares of the current batch are added, so about 2 * UNROLL
+    // 16-byte loads per thread stay in flight.
     int64_t n = n0 + r;
-    for (; n + (int64_t)(UNROLL - 1) * RPP < n1; n += (int64_t)RPP * UNROLL) {
-        uint4 w[UNROLL];
+    const int64_t step = (int64_t)RPP * UNROLL;
+    uint4 cur[UNROLL];
+    bool have = n + (int64_t)(UNROLL - 1) * RPP < n1;
+    if (have) {
 #pragma unroll
         for (int u = 0; u < UNROLL; ++u)
-            w[u] = __ldg(reinterpret_cast<const uint4 *>(base + (n + (int64_t)u * RPP) * a.sn));
+            cur[u] = __ldg(reinterpret_cast<const uint4 *>(base + (n + (int64_t)u * RPP) * a.sn));
+    }
+    while (have) {
+        const int64_t nn = n + step;
+        const bool have_next = nn + (int64_t)(UNROLL - 1) * RPP < n1;
+        uint4 nxt[UNROLL];
+        if (have_next) {
 #pragma unroll
-        for (int u = 0; u < UNROLL; ++u) add_squares<TIn>(w[u], acc);
+            for (int u = 0; u < UNROLL; ++u)
+                nxt[u] = __ldg(reinterpret_cast<const uint4 *>(base + (nn + (int64_t)u * RPP) * a.sn));
+        }
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u) add_squares<TIn>(cur[u], acc);
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u) cur[u] = nxt[u];
+        n = nn;
+        have = have_next;
     }
     for (; n < n1; n += RPP) add_squares<TIn>(__ldg(reinterpret_cast<const uint4 *>(base + n * a.sn)), acc);
 #pragma unroll
@@ -157,18 +203,28 @@ __global__ void __launch_bounds__(256, sizeof(TIn) == 2 ? 4 : 2) score_kernel(co
     if (!last) return;
     __threadfence();
     __shared__ unsigned long long sv[kD];
-    if (tid < kD) {
-        const double *p = a.part + (int64_t)head * a.splits * kD + tid;
-        double k0 = 0.0;
-        int s = 0;
-        for (; s + 8 <= a.splits; s += 8) {  // loads issued together, added in split order
-            double v[8];
+    __shared__ double khalf[kD];
+    // channel energy: the two halves of the block add the even and the odd
+    // splits (each in split order, 16 loads in flight), then half 0 adds half 1
+    const int c = tid & (kD - 1), hp = tid >> 7;
+    double k0 = 0.0;
+    {
+        const double *p = a.part + (int64_t)head * a.splits * kD + c;
+        for (int s = hp; s < a.splits; s += 32) {
+            double v[16];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) v[u] = __ldcg(p + (int64_t)(s + u) * kD);
+            for (int u = 0; u < 16; ++u) {
+                const int s2 = s + 2 * u;
+                v[u] = (s2 < a.splits) ? __ldcg(p + (int64_t)s2 * kD) : 0.0;
+            }
 #pragma unroll
-            for (int u = 0; u < 8; ++u) k0 = __dadd_rn(k0, v[u]);
+            for (int u = 0; u < 16; ++u) k0 = __dadd_rn(k0, v[u]);
         }
-        for (; s < a.splits; ++s) k0 = __dadd_rn(k0, __ldcg(p + (int64_t)s * kD));
+    }
+    if (hp == 1) khalf[c] = k0;
+    __syncthreads();
+    if (tid < kD) {
+        k0 = __dadd_rn(k0, khalf[tid]);
         const double knorm = sqrt(k0);
         double sc = 0.0;
         for (int g = 0; g < G; ++g)
@@ -200,7 +256,8 @@ __global__ void __launch_bounds__(128)
 }
 
 // ---------------------------------------------------------------------------
-// Compact: K'^T[t][n] = K[n][idx[t]] for a tile of 64 tokens of one head.
+// Compact: K'^T[t][n] = K[n][idx[t]] for a tile of 64
+// tokens of one head.
 // Each thread loads a 4-token x 8-channel block (four 16-byte loads, one per
 // token row), regroups it in registers into 8 channel runs of 4 tokens, and
 // stores those transposed into shared memory (channel-major, padded pitch).
@@ -234,12 +291,14 @@ template <> struct Transpose4<float> {
     }
 };
 
+template <typename TIn> struct CompactTokens { static constexpr int value = 64; };
+
 template <typename TIn>
 __global__ void __launch_bounds__(256)
     compact_kernel(const TIn *__restrict__ k, int64_t sb, int64_t sh, int64_t sn, int Hkv, int64_t N,
                    const int32_t *__restrict__ idx, int T, TIn *__restrict__ kp, int64_t ldk)
 {
-    constexpr int BNC = 64;                       // tokens per block
+    constexpr int BNC = CompactTokens<TIn>::value;  // tokens per block
     constexpr int VEC = 16 / sizeof(TIn);         // elements per 16 bytes (channels per load)
     constexpr int PITCH = BNC + VEC;              // padded smem row, elements (16-byte multiple)
     constexpr int CGROUPS = kD / VEC;             // channel groups of one row: 16 (bf16), 32 (fp32)
@@ -261,17 +320,21 @@ __global__ void __launch_bounds__(256)
     const int cgi = (CGROUPS == 16) ? (warp * 2 + (lane >> 4)) : (warp * 4 + (lane >> 3));
     const TIn *kh = k + (int64_t)b * sb + (int64_t)h * sh + cgi * VEC;
 
+    uint4 w[PASSES][4];  // every load of the block is issued before the first is used
 #pragma unroll
     for (int pass = 0; pass < PASSES; ++pass) {
         const int row0 = (pass * TGROUPS + tg) * 4;
-        uint4 w[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int64_t n = n0 + row0 + i;
-            w[i] = (n < N) ? __ldg(reinterpret_cast<const uint4 *>(kh + n * sn)) : make_uint4(0, 0, 0, 0);
+            w[pass][i] = (n < N) ? __ldg(reinterpret_cast<const uint4 *>(kh + n * sn)) : make_uint4(0, 0, 0, 0);
         }
+    }
+#pragma unroll
+    for (int pass = 0; pass < PASSES; ++pass) {
+        const int row0 = (pass * TGROUPS + tg) * 4;
         Run runs[Transpose4<TIn>::CH];
-        Transpose4<TIn>::run(w, runs);
+        Transpose4<TIn>::run(w[pass], runs);
 #pragma unroll
         for (int c = 0; c < Transpose4<TIn>::CH; ++c)
             *reinterpret_cast<Run *>(&sT[cgi * VEC + c][row0]) = runs[c];

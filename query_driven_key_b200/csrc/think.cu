@@ -303,7 +303,8 @@ think_status_t launch_compact(const void *k, const int64_t k_strides[3], int B, 
                               int64_t ldk, cudaStream_t st)
 {
     const int64_t heads = (int64_t)B * Hkv;
-    dim3 grid((unsigned)ceil_div(N, 64), (unsigned)heads);
+    const int bnc = dtype == THINK_BF16 ? CompactTokens<__nv_bfloat16>::value : CompactTokens<float>::value;
+    dim3 grid((unsigned)ceil_div(N, bnc), (unsigned)heads);
     if (dtype == THINK_BF16)
         compact_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
             static_cast<const __nv_bfloat16 *>(k), k_strides[0], k_strides[1], k_strides[2], Hkv, N,
