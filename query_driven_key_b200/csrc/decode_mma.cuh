@@ -1,0 +1,366 @@
+// decode_mma.cuh -- decode attention with the thinner key cache, tensor-core
+// contractions issued per warp (mma.sync m16n8k16, bf16 in, fp32 accumulate).
+//
+// "ThinK: Thinner Key Cache by Query-Driven Pruning", method section
+// (technical framework, last step): run inference with the pruned cache.
+//
+// Same split-N structure as the CUDA-core kernel (producer warp + four
+// consumer warps, TMA stage ring, each warp owns 32 tokens of every 128-token
+// tile and keeps its own online-softmax state), but each warp runs its two
+// small contractions on the tensor cores:
+//   logits  S[tok][g]  = K'[tok][t] q'[g][t]^T   m16n8k16: M = 16 tokens, N = 8
+//                                                 query heads (G <= 8), K = 16 channels
+//   values  O^T[c][g] += V[tok][c]^T P[g][tok]^T  M = 16 channels, N = 8, K = 16 tokens
+// K' and V tiles arrive by TMA with the 128-byte swizzle and are read with
+// ldmatrix.trans (conflict-free); the softmax weights are transposed from the
+// logits' accumulator layout to the values' operand layout in registers with
+// movmatrix, split into a bf16 high and low part (two MMAs; p = hi + lo keeps
+// the weights to about 2^-17 relative).  No block-wide barrier in the loop;
+// every mbarrier wait is bounded.
+#pragma once
+
+#include "decode_kernels.cuh"
+
+namespace think {
+
+namespace wmma16 {
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
+                                              uint32_t &r3)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+// D = A * B + D, A 16x16 bf16 (row), B 16x8 bf16 (col), D 16x8 fp32.
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// 8x8 16-bit matrix held one row per group of 4 lanes -> its transpose.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x)
+{
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
+// (lo, hi) floats -> bf16x2 with `lo` in the low half (round to nearest even).
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+}  // namespace wmma16
+
+struct MmaLayout {
+    uint32_t t_pad;   // T rounded up to 16
+    uint32_t k_half;  // one 64-token half of a K' tile: t_pad rows x 128 B
+    uint32_t v_off;   // V tile (two 64-channel halves of 128 tokens x 128 B) inside a stage
+    uint32_t stage;   // bytes per stage
+};
+
+__host__ __device__ inline MmaLayout mma_layout(int T)
+{
+    MmaLayout L;
+    L.t_pad = (uint32_t)((T + 15) & ~15);
+    L.k_half = L.t_pad * 128u;
+    L.v_off = 2u * L.k_half;
+    L.stage = L.v_off + 32768u;
+    return L;
+}
+
+// shared memory after the stages: q' [16 rows][t_pad] bf16, per-warp merge
+// area [4 warps][G][128] + [4 warps][G][2] floats, barriers, a flag
+__host__ __device__ inline size_t mma_smem_bytes(int T, int G, int stages)
+{
+    const MmaLayout L = mma_layout(T);
+    return (size_t)stages * L.stage + 32u * L.t_pad + (size_t)kConsumerWarps * G * 130 * 4 +
+           (size_t)2 * stages * 8 + 16 + 1024;
+}
+
+template <int G>
+__global__ void __launch_bounds__(kDecodeThreads)
+    pruned_decode_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
+                             const __grid_constant__ CUtensorMap tm_v, const DecodeArgs a)
+{
+    static_assert(G >= 1 && G <= 8, "the group's query heads fill at most the 8 MMA columns");
+    extern __shared__ unsigned char smem_dyn[];
+    unsigned char *smem = smem_dyn + ((1024u - (smem_addr(smem_dyn) & 1023u)) & 1023u);
+
+    const int split = blockIdx.x;
+    const int head = blockIdx.y;
+    const int b = head / a.Hkv, kv = head % a.Hkv;
+    const int T = a.T;
+    const int stages = a.stages;
+    const MmaLayout L = mma_layout(T);
+    const int64_t tile0 = (int64_t)split * a.tiles_per_split;
+    const int64_t tiles_all = (a.N + kBN - 1) / kBN;
+    const int ntiles = (int)min((int64_t)a.tiles_per_split, tiles_all - tile0);
+
+    unsigned char *qsm = smem + (size_t)stages * L.stage;                       // [16][t_pad] bf16
+    float *mo = reinterpret_cast<float *>(qsm + 32u * L.t_pad);                 // [warps][G][128]
+    float *mml = mo + kConsumerWarps * G * kD;                                  // [warps][G][2]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(mml + kConsumerWarps * G * 2);
+    unsigned *flag = reinterpret_cast<unsigned *>(bars + 2 * stages);
+    const uint32_t full0 = smem_addr(bars);
+    const uint32_t empty0 = smem_addr(bars + stages);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        for (int s = 0; s < stages; ++s) {
+            mbar_init(full0 + 8 * s, 1);
+            mbar_init(empty0 + 8 * s, kConsumerWarps);
+        }
+        fence_barrier_init();
+    }
+    __syncthreads();  // barriers initialised
+
+    if (warp == kConsumerWarps) {
+        // ------------------------------------------------------ producer
+        if (lane == 0) {
+            prefetch_tensormap(&tm_k);
+            prefetch_tensormap(&tm_v);
+            const uint32_t tx = 2u * 64u * (uint32_t)T * 2u + 32768u;
+            int issued = 0;
+            bool ok = true;
+            for (int it = 0; it < ntiles; ++it) {
+                const int s = it % stages, f = it / stages;
+                if (f > 0 && !mbar_wait_bounded(empty0 + 8 * s, (f - 1) & 1, a.status,
+                                                THINK_DEVICE_TIMEOUT_EMPTY)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t full = full0 + 8 * s;
+                mbar_arrive_expect_tx(full, tx);
+                const int x = (int)((tile0 + it) * kBN);
+                const uint32_t st = smem_addr(smem + (size_t)s * L.stage);
+                tma_load_4d(st, &tm_k, x, 0, kv, b, full);
+                tma_load_4d(st + L.k_half, &tm_k, x + 64, 0, kv, b, full);
+                tma_load_4d(st + L.v_off, &tm_v, 0, x, kv, b, full);
+                tma_load_4d(st + L.v_off + 16384u, &tm_v, 64, x, kv, b, full);
+                ++issued;
+            }
+            if (!ok) {
+                for (int it = max(0, issued - stages); it < issued; ++it)
+                    mbar_wait_bounded(full0 + 8 * (it % stages), (it / stages) & 1, a.status,
+                                      THINK_DEVICE_TIMEOUT_FULL);
+            }
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------- consumers
+    // Operand set-up (while the first tiles load): zero the K' rows T..t_pad-1
+    // of every stage (TMA writes rows 0..T-1 only; the matching q' columns are
+    // zero, but stale bits could be NaN), and stage q' = q[idx] as [g][t] bf16.
+    {
+        const uint32_t pad16 = (L.t_pad - (uint32_t)T) * 8u;  // 16-byte words per half
+        for (uint32_t i = tid; i < (uint32_t)stages * 2u * pad16; i += kConsumerThreads) {
+            const uint32_t hs = i / pad16, o = i % pad16;  // hs = stage * 2 + half
+            *reinterpret_cast<uint4 *>(smem + (hs >> 1) * L.stage + (hs & 1u) * L.k_half +
+                                       (uint32_t)T * 128u + o * 16u) = make_uint4(0, 0, 0, 0);
+        }
+        const __nv_bfloat16 *q = reinterpret_cast<const __nv_bfloat16 *>(a.q);
+        const int32_t *ih = a.idx + (int64_t)head * T;
+        __nv_bfloat16 *qs = reinterpret_cast<__nv_bfloat16 *>(qsm);
+        for (int i = tid; i < 16 * (int)L.t_pad; i += kConsumerThreads) {
+            const int g = i / (int)L.t_pad, t = i % (int)L.t_pad;
+            __nv_bfloat16 x = __float2bfloat16(0.f);
+            if (g < G && t < T) {
+                const int c = ih[t];
+                if ((unsigned)c < (unsigned)kD) x = q[((int64_t)b * a.Hq + (int64_t)kv * G + g) * kD + c];
+            }
+            qs[g * L.t_pad + t] = x;
+        }
+    }
+    named_barrier(1, kConsumerThreads);  // zeroed rows and q' visible to all consumers
+
+    const int q4 = lane & 3;   // accumulator column pair: query heads 2*q4, 2*q4+1
+    const int r8 = lane >> 2;  // accumulator row within an 8-row half
+    // q' as the B operand (k = channel, n = query head): per 16-channel step two
+    // registers: channels 2*q4, 2*q4+1 and +8 of query head r8.
+    constexpr int KS_MAX = kD / 16;
+    uint32_t qb[KS_MAX][2];
+    const int ksteps = (int)(L.t_pad / 16u);
+    {
+        const uint32_t *qs32 = reinterpret_cast<const uint32_t *>(qsm);
+#pragma unroll
+        for (int ks = 0; ks < KS_MAX; ++ks) {
+            if (ks < ksteps) {
+                qb[ks][0] = qs32[(r8 * L.t_pad + 16 * ks + 2 * q4) >> 1];
+                qb[ks][1] = qs32[(r8 * L.t_pad + 16 * ks + 8 + 2 * q4) >> 1];
+            } else {
+                qb[ks][0] = qb[ks][1] = 0u;
+            }
+        }
+    }
+
+    float m[2], l[2];          // running max (log2 units) and sum for heads 2*q4, 2*q4+1
+    float acc[8][4];           // O^T: channel rows 16*md + r8 (+8), head columns 2*q4 (+1)
+    m[0] = m[1] = -INFINITY;
+    l[0] = l[1] = 0.f;
+#pragma unroll
+    for (int md = 0; md < 8; ++md)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[md][e] = 0.f;
+
+    const int jm = lane >> 3, jr = lane & 7;  // ldmatrix: matrix index, row within it
+    const uint32_t sbase = smem_addr(smem);
+
+    for (int it = 0; it < ntiles; ++it) {
+        const int s = it % stages;
+        if (!mbar_wait_bounded(full0 + 8 * s, (it / stages) & 1, a.status, THINK_DEVICE_TIMEOUT_FULL))
+            break;
+        const uint32_t st = sbase + (uint32_t)s * L.stage;
+        const int64_t tok_base = (tile0 + it) * kBN + warp * 32;
+
+        // ---- logits for this warp's 32 tokens: two 16-token m-tiles
+        float sc[2][4];
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sc[mt][e] = 0.f;
+            const int tok = warp * 32 + mt * 16 + (jm & 1) * 8;   // first token of this lane's 8x8 block
+            const uint32_t kh = st + (uint32_t)(tok >> 6) * L.k_half;
+            const uint32_t chunk = (uint32_t)((tok & 63) >> 3);
+#pragma unroll
+            for (int ks = 0; ks < KS_MAX; ++ks) {
+                if (ks < ksteps) {
+                    const uint32_t t = (uint32_t)(16 * ks + (jm >> 1) * 8 + jr);
+                    uint32_t a0, a1, a2, a3;
+                    wmma16::ldsm_x4_trans(kh + t * 128u + ((chunk ^ (t & 7u)) << 4), a0, a1, a2, a3);
+                    wmma16::mma_bf16(sc[mt], a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+                }
+            }
+        }
+        // ---- online softmax per query head over the warp's 32 tokens
+        // sc[mt][0..1]: token 16*mt + r8, heads 2*q4, 2*q4+1; sc[mt][2..3]: token +8
+        float alpha[2];
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+            float xm = -INFINITY;
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int hr = 0; hr < 2; ++hr) {
+                    const int64_t n = tok_base + mt * 16 + hr * 8 + r8;
+                    const float x = (n < a.N) ? sc[mt][hr * 2 + h2] * a.scale_log2 : -INFINITY;
+                    sc[mt][hr * 2 + h2] = x;
+                    xm = fmaxf(xm, x);
+                }
+            xm = fmaxf(xm, __shfl_xor_sync(0xffffffffu, xm, 4));
+            xm = fmaxf(xm, __shfl_xor_sync(0xffffffffu, xm, 8));
+            xm = fmaxf(xm, __shfl_xor_sync(0xffffffffu, xm, 16));
+            const float mnew = fmaxf(m[h2], xm);
+            alpha[h2] = (m[h2] == mnew) ? 1.f : exp2_approx(m[h2] - mnew);
+            float ps = 0.f;
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int hr = 0; hr < 2; ++hr) {
+                    const float x = sc[mt][hr * 2 + h2];
+                    const float p = (x == -INFINITY) ? 0.f : exp2_approx(x - mnew);
+                    sc[mt][hr * 2 + h2] = p;
+                    ps += p;
+                }
+            l[h2] = fmaf(l[h2], alpha[h2], ps);
+            m[h2] = mnew;
+        }
+#pragma unroll
+        for (int md = 0; md < 8; ++md) {
+            acc[md][0] *= alpha[0];
+            acc[md][1] *= alpha[1];
+            acc[md][2] *= alpha[0];
+            acc[md][3] *= alpha[1];
+        }
+        // ---- weights as the B operand of the values MMA (k = token, n = head),
+        // high and low bf16 parts; one 16-token k-step per logits m-tile
+        uint32_t pbh[2][2], pbl[2][2];
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                const float p0 = sc[mt][hr * 2], p1 = sc[mt][hr * 2 + 1];
+                const uint32_t hi = wmma16::pack_bf16x2(p0, p1);
+                const float h0 = __uint_as_float(hi << 16), h1 = __uint_as_float(hi & 0xffff0000u);
+                const uint32_t lo = wmma16::pack_bf16x2(p0 - h0, p1 - h1);
+                pbh[mt][hr] = wmma16::movmatrix_trans(hi);
+                pbl[mt][hr] = wmma16::movmatrix_trans(lo);
+            }
+        // ---- values: O^T[c][g] += V^T[c][tok] P^T[tok][g] over the 32 tokens
+        const uint32_t vb = st + L.v_off;
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+            const uint32_t tok = (uint32_t)(warp * 32 + ks * 16 + (jm >> 1) * 8 + jr);
+#pragma unroll
+            for (int md = 0; md < 8; ++md) {
+                const uint32_t c0 = (uint32_t)(md * 16 + (jm & 1) * 8);   // first channel of the block
+                const uint32_t addr = vb + (c0 >> 6) * 16384u + tok * 128u +
+                                      ((((c0 & 63u) >> 3) ^ (tok & 7u)) << 4);
+                uint32_t a0, a1, a2, a3;
+                wmma16::ldsm_x4_trans(addr, a0, a1, a2, a3);
+                wmma16::mma_bf16(acc[md], a0, a1, a2, a3, pbh[ks][0], pbh[ks][1]);
+                wmma16::mma_bf16(acc[md], a0, a1, a2, a3, pbl[ks][0], pbl[ks][1]);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty0 + 8 * s);
+    }
+
+    // ------------------------------------------- merge the four warps
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+        l[h2] += __shfl_xor_sync(0xffffffffu, l[h2], 4);
+        l[h2] += __shfl_xor_sync(0xffffffffu, l[h2], 8);
+        l[h2] += __shfl_xor_sync(0xffffffffu, l[h2], 16);
+    }
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+        const int g = 2 * q4 + h2;
+        if (g < G) {
+#pragma unroll
+            for (int md = 0; md < 8; ++md) {
+                mo[(warp * G + g) * kD + md * 16 + r8] = acc[md][h2];
+                mo[(warp * G + g) * kD + md * 16 + 8 + r8] = acc[md][2 + h2];
+            }
+            if (r8 == 0) {
+                mml[(warp * G + g) * 2] = m[h2];
+                mml[(warp * G + g) * 2 + 1] = l[h2];
+            }
+        }
+    }
+    named_barrier(1, kConsumerThreads);
+    const int d = tid;  // 0..127: one output channel per consumer thread
+    float O[G], M[G], Lsum[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        M[g] = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) M[g] = fmaxf(M[g], mml[(w * G + g) * 2]);
+        O[g] = 0.f;
+        Lsum[g] = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) {
+            const float mw = mml[(w * G + g) * 2];
+            if (mw == -INFINITY) continue;
+            const float sw = exp2_approx(mw - M[g]);
+            O[g] = fmaf(mo[(w * G + g) * kD + d], sw, O[g]);
+            Lsum[g] = fmaf(mml[(w * G + g) * 2 + 1], sw, Lsum[g]);
+        }
+    }
+    named_barrier(1, kConsumerThreads);  // the split merge below reuses stage memory
+    finish_split<G, kConsumerThreads>(a, head, split, b, kv, d, O, M, Lsum, reinterpret_cast<float *>(smem),
+                                      flag, 1);
+}
+
+}  // namespace think

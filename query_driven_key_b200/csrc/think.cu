@@ -13,6 +13,7 @@
 #include <mutex>
 
 #include "decode_kernels.cuh"
+#include "decode_mma.cuh"
 #include "decode_tc.cuh"
 #include "prune_kernels.cuh"
 #include "think.h"
@@ -317,6 +318,59 @@ think_status_t launch_compact(const void *k, const int64_t k_strides[3], int B, 
 }
 
 
+// ---------------------------------------------------- warp-MMA decode --
+
+struct MmaPlan {
+    int stages, blocks_per_sm;
+    size_t bytes;
+};
+
+// Two blocks per SM with 2..4 stages if they fit, else one block per SM.
+MmaPlan plan_decode_mma(int T, int G)
+{
+    MmaPlan p;
+    const size_t per_block_2 = kSmemPerSM / 2 - kSmemReservedPerBlock;
+    for (int bps = 2; bps >= 1; --bps)
+        for (int st = 4; st >= 2; --st) {
+            const size_t bytes = mma_smem_bytes(T, G, st);
+            if (bytes <= (bps == 2 ? per_block_2 : kSmemPerBlockMax)) {
+                p.stages = st;
+                p.blocks_per_sm = bps;
+                p.bytes = bytes;
+                return p;
+            }
+        }
+    p.stages = 0;
+    p.blocks_per_sm = 1;
+    p.bytes = 0;
+    return p;
+}
+
+template <int G>
+think_status_t launch_decode_mma_g(const CUtensorMap &mk, const CUtensorMap &mv, const DecodeArgs &a,
+                                   size_t bytes, int heads, cudaStream_t st)
+{
+    auto kern = pruned_decode_mma_kernel<G>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+        cudaSuccess)
+        return THINK_ERR_CUDA;
+    dim3 grid(a.splits, heads);
+    kern<<<grid, kDecodeThreads, bytes, st>>>(mk, mv, a);
+    return launch_status();
+}
+
+think_status_t launch_decode_mma(int G, const CUtensorMap &mk, const CUtensorMap &mv,
+                                 const DecodeArgs &a, size_t bytes, int heads, cudaStream_t st)
+{
+    switch (G) {
+    case 1: return launch_decode_mma_g<1>(mk, mv, a, bytes, heads, st);
+    case 2: return launch_decode_mma_g<2>(mk, mv, a, bytes, heads, st);
+    case 4: return launch_decode_mma_g<4>(mk, mv, a, bytes, heads, st);
+    case 8: return launch_decode_mma_g<8>(mk, mv, a, bytes, heads, st);
+    default: return THINK_ERR_UNSUPPORTED;
+    }
+}
+
 // --------------------------------------------------------- tcgen05 decode --
 
 struct TcPlan {
@@ -554,16 +608,26 @@ think_status_t think_pruned_decode_attn(const void *q, const void *k_pruned, int
     const size_t need = think_decode_workspace_size(B, Hq, Hkv, N, d, dtype);
     if (workspace_bytes < need) return THINK_ERR_WORKSPACE;
 
-    // CUDA-core kernel by default (the faster one on B200 for this HBM-bound
-    // scan); THINK_DECODE_TENSOR_CORES=1 selects the tcgen05 kernel for bf16
-    // (same results within tolerance).  fp32 inputs always use CUDA cores.
-    const bool use_tc = dtype == THINK_BF16 && env_flag("THINK_DECODE_TENSOR_CORES");
+    // bf16: warp-level tensor-core kernel (mma.sync) by default;
+    // THINK_DECODE_TENSOR_CORES=1 selects the tcgen05 kernel and
+    // THINK_DECODE_CUDA_CORES=1 the CUDA-core kernel (same results within
+    // tolerance; for comparisons).  fp32 inputs always use the CUDA-core kernel.
+    enum { kSimt, kMma, kTc } kind = kSimt;
+    if (dtype == THINK_BF16) {
+        kind = kMma;
+        if (env_flag("THINK_DECODE_TENSOR_CORES")) kind = kTc;
+        else if (env_flag("THINK_DECODE_CUDA_CORES")) kind = kSimt;
+    }
+    const bool use_tc = kind == kTc;
     const TcPlan tp = plan_decode_tc(T);
+    const MmaPlan mp = plan_decode_mma(T, G);
     const DecodeSmem sm = plan_decode_smem(T, G, es);
-    if (use_tc ? tp.stages_k == 0 : sm.bytes > kSmemPerBlockMax) return THINK_ERR_UNSUPPORTED;
-    const DecodeSplit sp = plan_decode_split(heads, N, use_tc ? kTcBlocksPerSM : kDecodeBlocksPerSM);
+    if (kind == kTc ? tp.stages_k == 0 : kind == kMma ? mp.stages == 0 : sm.bytes > kSmemPerBlockMax)
+        return THINK_ERR_UNSUPPORTED;
+    const int bps = kind == kTc ? kTcBlocksPerSM : kind == kMma ? mp.blocks_per_sm : kDecodeBlocksPerSM;
+    const DecodeSplit sp = plan_decode_split(heads, N, bps);
     CUtensorMap mk, mv;
-    if (use_tc) {
+    if (kind != kSimt) {
         // K'^T in 64-token halves, V in 64-channel halves, 128-byte swizzle (the
         // tensor core's MN-major canonical layout)
         if (!make_map_4d(&mk, dtype, k_pruned, (uint64_t)N, (uint64_t)T, (uint64_t)Hkv, (uint64_t)B,
@@ -600,7 +664,7 @@ think_status_t think_pruned_decode_attn(const void *q, const void *k_pruned, int
     a.N = N;
     a.tiles_per_split = sp.tiles_per_split;
     a.splits = sp.splits;
-    a.stages = use_tc ? tp.stages_k : sm.stages;
+    a.stages = use_tc ? tp.stages_k : kind == kMma ? mp.stages : sm.stages;
     a.stages_v = use_tc ? tp.stages_v : 0;
     a.prefetch = env_int("THINK_DECODE_PREFETCH", kDecodePrefetchTiles, 0, 64);
     a.scale_log2 = scale * 1.4426950408889634f;
@@ -610,6 +674,7 @@ think_status_t think_pruned_decode_attn(const void *q, const void *k_pruned, int
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (use_tc) return launch_decode_tc(G, mk, mv, a, tp.bytes, (int)heads, st);
+    if (kind == kMma) return launch_decode_mma(G, mk, mv, a, mp.bytes, (int)heads, st);
     if (dtype == THINK_BF16) return launch_decode<__nv_bfloat16>(G, mk, mv, a, sm, (int)heads, st);
     return launch_decode<float>(G, mk, mv, a, sm, (int)heads, st);
 }

@@ -202,13 +202,16 @@ def test_fused_prune_equals_stepwise_calls():
     assert torch.equal(a.idx, b.idx)
 
 
-@pytest.mark.parametrize("kernel", ["cuda_cores", "tensor_cores"])
-def test_both_bf16_decode_kernels(kernel, monkeypatch):
-    # the CUDA-core kernel (default) and the tcgen05 kernel on the same inputs
+@pytest.mark.parametrize("kernel", ["warp_mma", "cuda_cores", "tensor_cores"])
+def test_every_bf16_decode_kernel(kernel, monkeypatch):
+    # the three bf16 decode kernels on the same inputs: warp-level mma (default),
+    # CUDA cores, tcgen05
+    monkeypatch.delenv("THINK_DECODE_TENSOR_CORES", raising=False)
+    monkeypatch.delenv("THINK_DECODE_CUDA_CORES", raising=False)
     if kernel == "tensor_cores":
         monkeypatch.setenv("THINK_DECODE_TENSOR_CORES", "1")
-    else:
-        monkeypatch.delenv("THINK_DECODE_TENSOR_CORES", raising=False)
+    elif kernel == "cuda_cores":
+        monkeypatch.setenv("THINK_DECODE_CUDA_CORES", "1")
     w = W.WORKLOADS["mistral_7b_long"].with_(N=20000)
     q_win, k, v = W.gen_layer(w)
     _full_path_check(w, q_win, k, v, steps=[0, 1])
