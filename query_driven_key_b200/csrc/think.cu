@@ -94,6 +94,15 @@ DecodeSplit plan_decode_split(int64_t heads, int64_t N, int blocks_per_sm = kDec
     return d;
 }
 
+double decode_fill(int64_t heads, int64_t N, int blocks_per_sm)
+{
+    const DecodeSplit d = plan_decode_split(heads, N, blocks_per_sm);
+    const int64_t blocks = heads * d.splits;
+    const int64_t slots = (int64_t)kTargetSMs * blocks_per_sm;
+    const int64_t waves = ceil_div(blocks, slots);
+    return (double)blocks / (double)(waves * slots);
+}
+
 struct DecodeSmem {
     uint32_t stage_bytes, v_off, tx_bytes;
     int stages;
@@ -325,13 +334,19 @@ struct MmaPlan {
     size_t bytes;
 };
 
-// Two blocks per SM with 2..4 stages if they fit, else one block per SM.
-MmaPlan plan_decode_mma(int T, int G)
+// One block per SM with up to 4 stages (the deeper ring streams faster) when
+// that keeps at least 95% of the SMs busy, else two blocks per SM.
+// THINK_DECODE_BLOCKS_PER_SM (1, 2) and THINK_DECODE_STAGES (2..4) cap the
+// choice (tuning only).
+MmaPlan plan_decode_mma(int T, int G, int64_t heads, int64_t N)
 {
     MmaPlan p;
     const size_t per_block_2 = kSmemPerSM / 2 - kSmemReservedPerBlock;
-    for (int bps = 2; bps >= 1; --bps)
-        for (int st = 4; st >= 2; --st) {
+    const int pref_bps = decode_fill(heads, N, 1) >= 0.95 ? 1 : 2;
+    const int max_bps = env_int("THINK_DECODE_BLOCKS_PER_SM", pref_bps, 1, 2);
+    const int max_st = env_int("THINK_DECODE_STAGES", 4, 2, 4);
+    for (int bps = max_bps; bps >= 1; --bps)
+        for (int st = max_st; st >= 2; --st) {
             const size_t bytes = mma_smem_bytes(T, G, st);
             if (bytes <= (bps == 2 ? per_block_2 : kSmemPerBlockMax)) {
                 p.stages = st;
@@ -620,7 +635,7 @@ think_status_t think_pruned_decode_attn(const void *q, const void *k_pruned, int
     }
     const bool use_tc = kind == kTc;
     const TcPlan tp = plan_decode_tc(T);
-    const MmaPlan mp = plan_decode_mma(T, G);
+    const MmaPlan mp = plan_decode_mma(T, G, heads, N);
     const DecodeSmem sm = plan_decode_smem(T, G, es);
     if (kind == kTc ? tp.stages_k == 0 : kind == kMma ? mp.stages == 0 : sm.bytes > kSmemPerBlockMax)
         return THINK_ERR_UNSUPPORTED;
