@@ -35,6 +35,12 @@ METRIC = "pruned-K decode attention HBM GB/s (% of 8 TB/s); prune pass µs/layer
 WORKLOAD = "mistral_7b_long"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the
+# default bf16 decode kernel, pruned_decode_mma_kernel<4>, on the long-context
+# workload, from one ncu capture of that kernel; reported only for that
+# workload and to be reset to None whenever the kernel changes.
+DECODE_TRAFFIC_BYTES = 375_440_128 + 3_847_168
+DECODE_TRAFFIC_WORKLOAD = WORKLOAD
 
 
 def parse():
@@ -351,11 +357,12 @@ def run_native(args):
         "decode_us_per_step": dec_us,
         "prune_us_per_layer": prune_us,
         "prune_gbs_1read": W.prune_bytes(w, T) / (prune_us * 1e-6) / 1e9,
-        "roofline": {"kernel": "pruned_decode_kernel (think_pruned_decode_attn, one launch), "
+        "roofline": {"kernel": "pruned_decode_mma_kernel<4> (think_pruned_decode_attn, one launch), "
                                "CUDA events around each step's 256 decode calls",
                      "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": f"{peak_kind} hbm_gbs",
-                     "algorithmic_bytes_per_launch": dec_bytes, "traffic": None},
+                     "algorithmic_bytes_per_launch": dec_bytes,
+                     "traffic": DECODE_TRAFFIC_BYTES if w.name == DECODE_TRAFFIC_WORKLOAD else None},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
         "e2e": e2e,
