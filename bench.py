@@ -40,7 +40,6 @@ FALLBACK_HBM_GBS = 6650.0
 # workload, from one ncu capture of that kernel; reported only for that
 # workload and to be reset to None whenever the kernel changes.
 DECODE_TRAFFIC_BYTES = 375_440_128 + 3_847_168
-DECODE_TRAFFIC_WORKLOAD = WORKLOAD
 
 
 def parse():
@@ -51,6 +50,13 @@ def parse():
     p.add_argument("--impl", default="native", choices=["native", "reference"])
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--workload", default=WORKLOAD,
+                   help="workload name from query_driven_key_b200.workloads (default: the "
+                        "long-context layer the metric is quoted on)")
+    p.add_argument("--batch", type=int, default=None, help="override the workload's B")
+    p.add_argument("--lam", type=float, default=None, help="override the workload's lambda")
+    p.add_argument("--decode-steps", type=int, default=None,
+                   help="override the workload's decode steps per bench step")
     return p.parse_args()
 
 
@@ -150,14 +156,72 @@ def aggregate_gbs(world: int, bytes_per_rank_step: int, ms_per_step: float) -> f
 
 # ----------------------------------------------------------- workload ---
 
-def workload():
+def workload(args):
     from query_driven_key_b200 import workloads as W
-    return W.WORKLOADS[WORKLOAD]
+    w = W.WORKLOADS[args.workload]
+    kw = {}
+    if args.batch is not None:
+        kw["B"] = args.batch
+    if args.lam is not None:
+        kw["lam"] = args.lam
+    if args.decode_steps is not None:
+        kw["decode_steps"] = args.decode_steps
+    return w.with_(**kw) if kw else w
+
+
+def default_workload(args):
+    return (args.workload == WORKLOAD and args.batch is None and args.lam is None
+            and args.decode_steps is None)
+
+
+L2_BYTES = 126 * 1000 * 1000
+
+
+def resident_layers(w, T):
+    """How many layers' buffers a step cycles through: all layers of a
+    multi-layer workload, else enough copies of the one layer that a pass over
+    them reads at least twice the L2 capacity (so no step finds its K, K' or V
+    in L2 from the previous one)."""
+    if w.layers > 1:
+        return w.layers
+    e = torch_elem_size(w.dtype)
+    heads = w.B * w.Hkv
+    footprint = heads * w.N * (2 * w.d + T) * e        # K + V + K'
+    return max(1, -(-2 * L2_BYTES // footprint))
+
+
+def torch_elem_size(dtype):
+    import torch
+    return torch.empty((), dtype=dtype).element_size()
 
 
 def step_bytes(w, T):
     from query_driven_key_b200 import workloads as W
     return W.prune_bytes(w, T) + w.decode_steps * W.decode_bytes(w, T)
+
+
+def data_recipe(w):
+    if w.k_kind == "lowrank":
+        keys = f"rank-{w.k_rank} N(0,1) factors + {w.k_noise} N(0,1) noise, LogNormal(0,{w.k_sigma}) channel scales"
+    else:
+        keys = f"LogNormal(0,{w.k_sigma}) channel-scaled N(0,1) keys"
+    return f"synthetic (seeded {keys}, N(0,1) values/queries)"
+
+
+def l2_note(w, T, R):
+    e = torch_elem_size(w.dtype)
+    heads = w.B * w.Hkv
+    kvp = heads * w.N * (w.d + T) * e
+    k = heads * w.N * w.d * e
+    return (f"inputs larger than L2: {R} resident layer(s); a pass over them reads "
+            f"K {R * k / 1e6:.0f} MB (prune) and K'+V {R * kvp / 1e6:.0f} MB (decode), no flush")
+
+
+def decode_kernel_name(w):
+    import torch
+    if w.dtype == torch.bfloat16:
+        return f"pruned_decode_mma_kernel<{w.G}>"
+    return f"pruned_decode_kernel<float, {w.G}>"
 
 
 def cpu_baseline(w, T, seed_layer=0, budget_s=12.0):
@@ -195,7 +259,7 @@ def run_reference(args):
     import oracle
     from query_driven_key_b200 import workloads as W
 
-    w = workload()
+    w = workload(args)
     T = oracle.t_from_lambda(w.d, w.lam)
     q_win, k, v = W.gen_layer(w)
     f64 = lambda t: t.to(torch.float64).numpy()
@@ -249,35 +313,48 @@ def run_native(args):
     import query_driven_key_b200 as qdk
     from query_driven_key_b200 import workloads as W
 
-    w = workload()
+    w = workload(args)
     T = qdk.think_t_from_lambda(w.d, w.lam)
-    # each rank: an independent replica on its own data
+    R = resident_layers(w, T)
+    # each rank: an independent replica on its own data; one generated layer
+    # is copied into R device buffers (distinct addresses, so L2 cannot serve
+    # one layer's reads from another's)
     q_win, k, v = W.gen_layer(w, layer=rank)
     qs = torch.stack([W.gen_decode_q(w, s, layer=rank) for s in range(w.decode_steps)])
     stream = torch.cuda.Stream(device=dev)
     with torch.cuda.stream(stream):
-        qw_d, k_d, v_d, qs_d = (t.to(dev) for t in (q_win, k, v, qs))
-        cache = qdk.PrunedCache(w.B, w.Hq, w.Hkv, w.N, T, w.d, dtype=w.dtype, device=dev)
-        outs = torch.empty((w.decode_steps, w.B, w.Hq, w.d), dtype=torch.float32, device=dev)
+        qw_d = [q_win.to(dev) for _ in range(R)]
+        k_d = [k.to(dev) for _ in range(R)]
+        v_d = [v.to(dev) for _ in range(R)]
+        qs_d = qs.to(dev)
+        caches = [qdk.PrunedCache(w.B, w.Hq, w.Hkv, w.N, T, w.d, dtype=w.dtype, device=dev)
+                  for _ in range(R)]
+        outs = torch.empty((w.decode_steps, R, w.B, w.Hq, w.d), dtype=torch.float32, device=dev)
     stream.synchronize()
 
-    launches_per_step = 2 + w.decode_steps  # prune: score+select, compact; one kernel per decode
+    # prune: score+select, compact; one kernel per decode
+    launches_per_step = R * (2 + w.decode_steps)
 
     def one_step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        cache.prune(qw_d, k_d, stream=stream)
+        for r in range(R):
+            caches[r].prune(qw_d[r], k_d[r], stream=stream)
         if ev is not None:
             ev[1].record(stream)
         for s in range(w.decode_steps):
-            cache.decode(qs_d[s], v_d, outs[s], stream=stream)
+            for r in range(R):
+                caches[r].decode(qs_d[s], v_d[r], outs[s, r], stream=stream)
         if ev is not None:
             ev[2].record(stream)
+
+    def device_status():
+        return max(qdk.think_read_device_status(c.decode_ws, stream) for c in caches)
 
     for _ in range(args.warmup):
         one_step()
     stream.synchronize()
-    assert qdk.think_read_device_status(cache.decode_ws, stream) == 0
+    assert device_status() == 0
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -296,14 +373,14 @@ def run_native(args):
     prune_ms = [e[0].elapsed_time(e[1]) for e in evs]
     decode_ms = [e[1].elapsed_time(e[2]) for e in evs]
     total_ms, prune_sum, decode_sum = max_over_ranks([total_ms, sum(prune_ms), sum(decode_ms)], dev)
-    assert qdk.think_read_device_status(cache.decode_ws, stream) == 0
+    assert device_status() == 0
 
     ms_per_step = total_ms / args.steps
-    nbytes = step_bytes(w, T)
+    nbytes = R * step_bytes(w, T)
     value = aggregate_gbs(world, nbytes, ms_per_step)
     dec_bytes = W.decode_bytes(w, T)
-    dec_us = decode_sum / args.steps / w.decode_steps * 1e3
-    prune_us = prune_sum / args.steps * 1e3
+    dec_us = decode_sum / args.steps / (w.decode_steps * R) * 1e3
+    prune_us = prune_sum / args.steps / R * 1e3
     achieved = dec_bytes / (dec_us * 1e-6) / 1e9
     peak, peak_kind = measured_peaks()
 
@@ -313,18 +390,21 @@ def run_native(args):
         pin = lambda t: t.pin_memory()
         h_qw, h_k, h_v, h_qs = pin(q_win), pin(k), pin(v), pin(qs)
         h_out = torch.empty(outs.shape, dtype=torch.float32).pin_memory()
-        h_idx = torch.empty(cache.idx.shape, dtype=torch.int32).pin_memory()
-        h2d = sum(t.numel() * t.element_size() for t in (h_qw, h_k, h_v, h_qs))
+        h_idx = torch.empty((R,) + tuple(caches[0].idx.shape), dtype=torch.int32).pin_memory()
+        h2d = R * sum(t.numel() * t.element_size() for t in (h_qw, h_k, h_v)) \
+            + h_qs.numel() * h_qs.element_size()
         d2h = h_out.numel() * 4 + h_idx.numel() * 4
 
         def e2e_step():
-            qw_d.copy_(h_qw, non_blocking=True)
-            k_d.copy_(h_k, non_blocking=True)
-            v_d.copy_(h_v, non_blocking=True)
+            for r in range(R):
+                qw_d[r].copy_(h_qw, non_blocking=True)
+                k_d[r].copy_(h_k, non_blocking=True)
+                v_d[r].copy_(h_v, non_blocking=True)
             qs_d.copy_(h_qs, non_blocking=True)
             one_step()
             h_out.copy_(outs, non_blocking=True)
-            h_idx.copy_(cache.idx, non_blocking=True)
+            for r in range(R):
+                h_idx[r].copy_(caches[r].idx, non_blocking=True)
 
         with torch.cuda.stream(stream):
             e2e_step()
@@ -345,24 +425,26 @@ def run_native(args):
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded LogNormal(0,1.5) channel-scaled N(0,1) keys, N(0,1) values/queries)",
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32",
+        "data": data_recipe(w),
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
                    "S_obs": w.S_obs, "lambda": w.lam, "T": T, "decode_steps_per_step": w.decode_steps,
+                   "layers_per_step": R,
                    "parallelism": f"{world} independent replica(s), no collective",
-                   "l2": "inputs larger than L2 (K 268 MB, K'+V 375 MB per decode step), no flush"},
+                   "l2": l2_note(w, T, R)},
         "pct_of_8tbs": value / world / NOMINAL_HBM_GBS * 100.0,
         "decode_gbs": achieved,
         "decode_pct_of_8tbs": achieved / NOMINAL_HBM_GBS * 100.0,
         "decode_us_per_step": dec_us,
         "prune_us_per_layer": prune_us,
         "prune_gbs_1read": W.prune_bytes(w, T) / (prune_us * 1e-6) / 1e9,
-        "roofline": {"kernel": "pruned_decode_mma_kernel<4> (think_pruned_decode_attn, one launch), "
-                               "CUDA events around each step's 256 decode calls",
+        "roofline": {"kernel": f"{decode_kernel_name(w)} (think_pruned_decode_attn, one launch), "
+                               f"CUDA events around each step's {w.decode_steps * R} decode calls",
                      "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": f"{peak_kind} hbm_gbs",
                      "algorithmic_bytes_per_launch": dec_bytes,
-                     "traffic": DECODE_TRAFFIC_BYTES if w.name == DECODE_TRAFFIC_WORKLOAD else None},
+                     "traffic": DECODE_TRAFFIC_BYTES if default_workload(args) else None},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
         "e2e": e2e,
