@@ -349,7 +349,8 @@ def run_native(args):
             ev[2].record(stream)
 
     def device_status():
-        return max(qdk.think_read_device_status(c.decode_ws, stream) for c in caches)
+        return max(max(qdk.think_read_device_status(c.decode_ws, stream),
+                       qdk.think_read_device_status(c.score_ws, stream)) for c in caches)
 
     for _ in range(args.warmup):
         one_step()

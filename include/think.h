@@ -59,12 +59,14 @@ typedef enum {
 
 typedef enum { THINK_F32 = 0, THINK_BF16 = 1 } think_dtype_t;
 
-/* Device-side status bits written into the first 4 bytes of a decode
- * workspace when a bounded wait inside the decode kernel gives up (the kernel
- * then returns early and its output is invalid).  Read them with
+/* Device-side status bits written into the first 4 bytes of a decode or
+ * score workspace when a bounded wait (2 s) inside a kernel gives up (the
+ * kernel then returns early and its outputs are invalid).  Read them with
  * think_read_device_status; clear them with think_workspace_init. */
-#define THINK_DEVICE_TIMEOUT_FULL  0x1u   /* a tile load never arrived */
-#define THINK_DEVICE_TIMEOUT_EMPTY 0x2u   /* a stage was never released */
+#define THINK_DEVICE_TIMEOUT_FULL    0x1u   /* a tile load never arrived */
+#define THINK_DEVICE_TIMEOUT_EMPTY   0x2u   /* a stage was never released */
+#define THINK_DEVICE_TIMEOUT_READY   0x4u   /* a head's channel selection never became ready */
+#define THINK_DEVICE_TIMEOUT_BARRIER 0x8u   /* a block-internal barrier was not reached */
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char *think_status_string(think_status_t status);
@@ -83,10 +85,14 @@ int64_t think_pruned_ld(int64_t N, think_dtype_t dtype);
  * method section: "compute each channel's relevance to the query"; abstract:
  * keep the attention weights Qwin K^T).  For each batch item b and KV head
  * h_kv, with the group's query heads g = h_kv*G .. h_kv*G+G-1:
- *     kn2[c]  = sum_n K[b,h_kv,n,c]^2                 (fp64)
+ *     kn2[c]  = sum_n K[b,h_kv,n,c]^2
  *     s[c]    = sum_g sqrt(sum_s Qwin[b,g,s,c]^2) * sqrt(kn2[c])
  * which is the Frobenius norm of channel c's rank-one share Qwin_g[:,c]K[:,c]^T
- * of the window's attention logits, summed over the group.
+ * of the window's attention logits, summed over the group.  Arithmetic:
+ * fp32 keys are squared and summed in fp64; bf16 keys are squared exactly,
+ * summed four tokens at a time in fp32, then in fp64 (kn2 within 1.8e-7
+ * relative for keys of magnitude in [2^-63, 2^64)); window energies and the
+ * score in fp64.
  *
  *   q_win     [B][Hq][S_obs][d] contiguous, dtype.  May be NULL if S_obs == 0.
  *   k         key cache; element (b,h,n,c) at k[b*k_strides[0] + h*k_strides[1]
@@ -131,8 +137,11 @@ think_status_t think_compact_keys(const void *k, const int64_t k_strides[3], int
 /* ---------------------------------------------------------------- prune --
  * The whole prune step of one layer in two launches: scores and the top-T
  * selection in one kernel (the last block of each head selects), then the
- * compaction.  Same results as think_score_channels, think_select_channels
- * and think_compact_keys called in a row; arguments as documented there.
+ * compaction.  Same results, bit for bit, as think_score_channels,
+ * think_select_channels and think_compact_keys called in a row; arguments as
+ * documented there.  With THINK_PRUNE_FUSED=1 in the environment a bf16 prune
+ * runs as one persistent kernel instead (same results; its bounded waits
+ * report through the workspace's status word, see think_read_device_status).
  * workspace: think_score_workspace_size() bytes, zeroed once before first use. */
 think_status_t think_prune(const void *q_win, const void *k, const int64_t k_strides[3], int B,
                            int Hq, int Hkv, int64_t N, int S_obs, int d, think_dtype_t dtype,
@@ -198,8 +207,9 @@ think_status_t think_pruned_decode_attn_noalloc(const void *q, const void *k_pru
 /* Zero a score or decode workspace (stream-ordered memset). */
 think_status_t think_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
 
-/* Copy the device status bits of a decode workspace to *status after the
- * stream's queued work has finished (synchronises `stream`). */
+/* Copy the device status bits of a decode or score workspace (its first 4
+ * bytes) to *status after the stream's queued work has finished
+ * (synchronises `stream`). */
 think_status_t think_read_device_status(const void *workspace, uint32_t *status, void *stream);
 
 #ifdef __cplusplus

@@ -29,6 +29,8 @@ THINK_F32 = 0
 THINK_BF16 = 1
 THINK_DEVICE_TIMEOUT_FULL = 0x1
 THINK_DEVICE_TIMEOUT_EMPTY = 0x2
+THINK_DEVICE_TIMEOUT_READY = 0x4
+THINK_DEVICE_TIMEOUT_BARRIER = 0x8
 
 EXPORTED = (
     "think_status_string", "think_t_from_lambda", "think_pruned_ld",

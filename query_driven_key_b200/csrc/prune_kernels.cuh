@@ -52,7 +52,7 @@ struct ScoreArgs {
 };
 
 // ---------------------------------------------------------------------------
-// Score.  Block (split, head) sums K[n,c]^2 (fp64) over its run of tokens with
+// Score.  Block (split, head) sums K[n,c]^2 over its run of tokens with
 // 16-byte loads (bf16: 16 threads x 8 channels per row, 16 rows per pass, 8
 // passes in flight); blocks split < G also sum the window-query energies of
 // query head kv*G + split.  The last block of the head to finish (ticket
@@ -60,58 +60,53 @@ struct ScoreArgs {
 // halves of the block, then the halves) and forms
 //     s[c] = sum_g sqrt(qn2[g][c]) * sqrt(kn2[c])
 // with each operation rounded as written, then optionally selects the top T.
-// The square of a bf16 or fp32 value is exact in fp64; only the order of the
-// additions differs from a sequential sum.
+// fp32 keys: every square is exact in fp64 and only the order of the fp64
+// additions differs from a sequential sum.  bf16 keys: four-row fp32 partials
+// (add_squares4_bf16), then fp64.  The order of all additions is fixed by the
+// split plan, so the result is deterministic.
 // ---------------------------------------------------------------------------
-// fp64 value of a bf16 with a nonzero exponent field, built from its bits:
-// the fp64 exponent is the bf16 exponent + (1023 - 127) and the 7 mantissa
-// bits go to the top of the fp64 mantissa; the low word is zero.  The sign is
-// dropped (only squares are used).  Exact for every normal bf16 value.
-__device__ __forceinline__ double bf16_abs_to_f64_normal(uint32_t bits15)
-{
-    return __hiloint2double((int)(bits15 * 8192u + 0x38000000u), 0);
-}
-
-template <typename TIn>
-__device__ __forceinline__ void add_squares(const uint4 &w, double *acc)
+// fp32 keys: the square of an fp32 value is exact in fp64; one FMA per element.
+__device__ __forceinline__ void add_squares_f32(const uint4 &w, double *acc)
 {
     const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-    if constexpr (sizeof(TIn) == 2) {
-        // Fast path (integer ops + fp64 FMA, no conversion unit) when no element
-        // of the 16 bytes has a zero exponent field (zero or subnormal); the
-        // exact conversion otherwise.  Both give the same fp64 squares.
-        const bool zero_exp = ((ww[0] & 0x7f80u) == 0u) | ((ww[0] & 0x7f800000u) == 0u) |
-                              ((ww[1] & 0x7f80u) == 0u) | ((ww[1] & 0x7f800000u) == 0u) |
-                              ((ww[2] & 0x7f80u) == 0u) | ((ww[2] & 0x7f800000u) == 0u) |
-                              ((ww[3] & 0x7f80u) == 0u) | ((ww[3] & 0x7f800000u) == 0u);
-        if (!zero_exp) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const double lo = bf16_abs_to_f64_normal(ww[e] & 0x7fffu);
-                const double hi = bf16_abs_to_f64_normal((ww[e] >> 16) & 0x7fffu);
-                acc[2 * e] = fma(lo, lo, acc[2 * e]);
-                acc[2 * e + 1] = fma(hi, hi, acc[2 * e + 1]);
-            }
-        } else {
+    for (int e = 0; e < 4; ++e) {
+        const double x = (double)__uint_as_float(ww[e]);
+        acc[e] = fma(x, x, acc[e]);
+    }
+}
+
+// bf16: the squares of one thread's four rows of a 64-token tile (rows r,
+// r+16, r+32, r+48; 8 channels each) are added in fp32 (FFMA2 on channel
+// pairs; each product is exact, three roundings of at most 2^-24 relative),
+// then the four-term partial of each channel is added to its fp64 running sum.
+// So every channel energy carries a relative error below 3 * 2^-24 = 1.8e-7,
+// for keys of magnitude in [2^-63, 2^64) (outside it the fp32 square
+// underflows or overflows).  Rows past the end of the keys are passed as zero
+// words, which add nothing.
+__device__ __forceinline__ void add_squares4_bf16(const uint4 (&w)[4], double *acc)
+{
+    float2 p[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const double lo = (double)bf16lo(ww[e]);
-                const double hi = (double)bf16hi(ww[e]);
-                acc[2 * e] = fma(lo, lo, acc[2 * e]);
-                acc[2 * e + 1] = fma(hi, hi, acc[2 * e + 1]);
-            }
-        }
-    } else {
+    for (int e = 0; e < 4; ++e) p[e] = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const uint32_t ww[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const double x = (double)__uint_as_float(ww[e]);
-            acc[e] = fma(x, x, acc[e]);
+            const float2 x = make_float2(__uint_as_float(ww[e] << 16), __uint_as_float(ww[e] & 0xffff0000u));
+            p[e] = __ffma2_rn(x, x, p[e]);
         }
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        acc[2 * e] += (double)p[e].x;
+        acc[2 * e + 1] += (double)p[e].y;
     }
 }
 
 template <typename TIn>
-__global__ void __launch_bounds__(256, sizeof(TIn) == 2 ? 4 : 2) score_kernel(const ScoreArgs a)
+__global__ void __launch_bounds__(256, 3) score_kernel(const ScoreArgs a)
 {
     constexpr int VEC = 16 / sizeof(TIn);  // channels per 16-byte load
     constexpr int TPR = kD / VEC;          // threads per row
@@ -177,14 +172,29 @@ __global__ void __launch_bounds__(256, sizeof(TIn) == 2 ? 4 : 2) score_kernel(co
             for (int u = 0; u < UNROLL; ++u)
                 nxt[u] = __ldg(reinterpret_cast<const uint4 *>(base + (nn + (int64_t)u * RPP) * a.sn));
         }
+        if constexpr (sizeof(TIn) == 2) {
+            add_squares4_bf16(cur, acc);
+        } else {
 #pragma unroll
-        for (int u = 0; u < UNROLL; ++u) add_squares<TIn>(cur[u], acc);
+            for (int u = 0; u < UNROLL; ++u) add_squares_f32(cur[u], acc);
+        }
 #pragma unroll
         for (int u = 0; u < UNROLL; ++u) cur[u] = nxt[u];
         n = nn;
         have = have_next;
     }
-    for (; n < n1; n += RPP) add_squares<TIn>(__ldg(reinterpret_cast<const uint4 *>(base + n * a.sn)), acc);
+    if constexpr (sizeof(TIn) == 2) {
+        if (n < n1) {  // the rows of the last, partial tile
+#pragma unroll
+            for (int u = 0; u < UNROLL; ++u)
+                cur[u] = (n + (int64_t)u * RPP < n1)
+                             ? __ldg(reinterpret_cast<const uint4 *>(base + (n + (int64_t)u * RPP) * a.sn))
+                             : make_uint4(0u, 0u, 0u, 0u);
+            add_squares4_bf16(cur, acc);
+        }
+    } else {
+        for (; n < n1; n += RPP) add_squares_f32(__ldg(reinterpret_cast<const uint4 *>(base + n * a.sn)), acc);
+    }
 #pragma unroll
     for (int e = 0; e < VEC; ++e) red[r][cg * VEC + e] = acc[e];
     __syncthreads();

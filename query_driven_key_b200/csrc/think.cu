@@ -15,6 +15,7 @@
 #include "decode_kernels.cuh"
 #include "decode_mma.cuh"
 #include "decode_tc.cuh"
+#include "prune_fused.cuh"
 #include "prune_kernels.cuh"
 #include "think.h"
 
@@ -58,19 +59,28 @@ inline think_status_t launch_status()
 
 // ---------------------------------------------------------------- plans --
 
+// Split of each head's tokens for scoring, shared by score_kernel and the
+// fused prune kernel (so that both add the squares in the same order): runs of
+// s_tiles 64-token tiles, about kScoreBlocksPerSM runs per SM over all heads,
+// 4 to 32 tiles per run.
 struct ScorePlan {
-    int splits;
-    int64_t rows_per_split;
+    int splits;              // runs per head
+    int s_tiles;             // 64-token tiles per run
+    int64_t rows_per_split;  // = 64 * s_tiles
+    int64_t tiles_per_head;
 };
 
 ScorePlan plan_score(int64_t heads, int64_t N)
 {
     ScorePlan p;
-    const int64_t target = (int64_t)kTargetSMs * kScoreBlocksPerSM;
-    int64_t s = heads >= target ? 1 : target / heads;
-    s = std::max<int64_t>(1, std::min<int64_t>(s, ceil_div(std::max<int64_t>(N, 1), 256)));
-    p.rows_per_split = ceil_div(std::max<int64_t>(N, 1), s);
-    p.splits = (int)ceil_div(std::max<int64_t>(N, 1), p.rows_per_split);
+    p.tiles_per_head = std::max<int64_t>(1, ceil_div(N, kPfTile));
+    const int64_t total = heads * p.tiles_per_head;
+    int64_t st = total / ((int64_t)kTargetSMs * kScoreBlocksPerSM);
+    st = std::min<int64_t>(std::max<int64_t>(st, 4), 32);
+    st = std::min(st, p.tiles_per_head);
+    p.s_tiles = (int)st;
+    p.rows_per_split = st * kPfTile;
+    p.splits = (int)ceil_div(p.tiles_per_head, st);
     return p;
 }
 
@@ -217,15 +227,25 @@ think_status_t launch_decode(int G, const CUtensorMap &mk, const CUtensorMap &mv
 
 // ---------------------------------------------------------------- score --
 
+// Score workspace: a 256-byte header (status word at 0; the fused kernel's
+// score-queue counter at 8, front compact head at 16, block-exit counter at
+// 24), per-head arrival counters, per-head ready flags, per-head compact
+// counters, window-query energies, per-run channel energies.
 struct ScoreWs {
-    size_t tickets, qn2, part, total;  // byte offsets and total size
+    size_t status, s_next, c_front, exits, tickets, ready, c_cnt, qn2, part, total;  // byte offsets, size
 };
 
 ScoreWs score_ws_layout(int64_t heads, int G, const ScorePlan &p)
 {
     ScoreWs w;
-    w.tickets = 0;
-    w.qn2 = align_up((size_t)heads * sizeof(unsigned), 256);
+    w.status = 0;
+    w.s_next = 8;
+    w.c_front = 16;
+    w.exits = 24;
+    w.tickets = 256;
+    w.ready = w.tickets + align_up((size_t)heads * sizeof(unsigned), 256);
+    w.c_cnt = w.ready + align_up((size_t)heads * sizeof(unsigned), 256);
+    w.qn2 = w.c_cnt + align_up((size_t)heads * sizeof(unsigned), 256);
     w.part = w.qn2 + align_up((size_t)heads * G * kD * sizeof(double), 256);
     w.total = w.part + (size_t)heads * p.splits * kD * sizeof(double);
     return w;
@@ -323,6 +343,76 @@ think_status_t launch_compact(const void *k, const int64_t k_strides[3], int B, 
         compact_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float *>(k), k_strides[0],
                                                     k_strides[1], k_strides[2], Hkv, N, idx, T,
                                                     static_cast<float *>(k_pruned), ldk);
+    return launch_status();
+}
+
+
+// ---------------------------------------------------------- fused prune --
+
+struct PrunePlan {
+    ScorePlan sp;
+    int c_tiles, c_items, grid;
+};
+
+// Compact items have the score items' size; one block per SM.
+PrunePlan plan_prune(int64_t heads, int64_t N)
+{
+    PrunePlan p;
+    p.sp = plan_score(heads, N);
+    p.c_tiles = p.sp.s_tiles;
+    p.c_items = p.sp.splits;
+    p.grid = (int)std::min<int64_t>(kTargetSMs, heads * (p.sp.splits + p.c_items));
+    return p;
+}
+
+// The fused prune (bf16, N > 0).  Returns THINK_ERR_UNSUPPORTED, having
+// launched nothing, when a tensor map cannot be built for these strides.
+think_status_t launch_prune_fused(const void *q_win, const void *k, const int64_t k_strides[3], int B,
+                                  int Hq, int Hkv, int64_t N, int S_obs, int T, double *scores,
+                                  int32_t *idx, void *k_pruned, int64_t ldk, void *workspace,
+                                  cudaStream_t st)
+{
+    const int64_t heads = (int64_t)B * Hkv;
+    const PrunePlan p = plan_prune(heads, N);
+    const ScoreWs w = score_ws_layout(heads, Hq / Hkv, p.sp);
+    CUtensorMap mk;
+    if (!make_map_4d(&mk, THINK_BF16, k, kD, (uint64_t)N, (uint64_t)Hkv, (uint64_t)B, k_strides[2],
+                     k_strides[1], k_strides[0], 64, kPfTile, true))
+        return THINK_ERR_UNSUPPORTED;
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    PruneFusedArgs a;
+    a.qwin = static_cast<const __nv_bfloat16 *>(q_win);
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.S = S_obs;
+    a.G = Hq / Hkv;
+    a.T = T;
+    a.heads = (int)heads;
+    a.tiles_per_head = (int)p.sp.tiles_per_head;
+    a.s_tiles = p.sp.s_tiles;
+    a.s_items = p.sp.splits;
+    a.c_tiles = p.c_tiles;
+    a.c_items = p.c_items;
+    a.l2_hints = env_int("THINK_PRUNE_L2_HINTS", 1, 0, 1);
+    a.s_total = (long long)heads * p.sp.splits;
+    a.part = reinterpret_cast<double *>(ws + w.part);
+    a.qn2 = reinterpret_cast<double *>(ws + w.qn2);
+    a.tickets = reinterpret_cast<unsigned *>(ws + w.tickets);
+    a.ready = reinterpret_cast<unsigned *>(ws + w.ready);
+    a.status = reinterpret_cast<unsigned *>(ws + w.status);
+    a.s_next = reinterpret_cast<unsigned long long *>(ws + w.s_next);
+    a.c_front = reinterpret_cast<unsigned *>(ws + w.c_front);
+    a.c_cnt = reinterpret_cast<unsigned *>(ws + w.c_cnt);
+    a.exits = reinterpret_cast<unsigned *>(ws + w.exits);
+    a.scores = scores;
+    a.idx = idx;
+    a.kp = static_cast<__nv_bfloat16 *>(k_pruned);
+    a.ldk = ldk;
+    a.N = N;
+    if (cudaFuncSetAttribute(prune_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kPfSmemBytes) != cudaSuccess)
+        return THINK_ERR_CUDA;
+    prune_fused_kernel<<<p.grid, kPfThreads, kPfSmemBytes, st>>>(mk, a);
     return launch_status();
 }
 
@@ -579,6 +669,13 @@ think_status_t think_prune(const void *q_win, const void *k, const int64_t k_str
     v = validate_compact(k, k_strides, B, Hkv, N, d, dtype, idx, T, k_pruned, ldk);
     if (v != THINK_OK || B == 0 || Hkv == 0) return v;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // Two launches (score + select, then compact).  THINK_PRUNE_FUSED=1 selects
+    // the one-kernel prune for bf16 (same results; not faster on B200 yet).
+    if (dtype == THINK_BF16 && N > 0 && env_flag("THINK_PRUNE_FUSED")) {
+        v = launch_prune_fused(q_win, k, k_strides, B, Hq, Hkv, N, S_obs, T, scores, idx, k_pruned,
+                               ldk, workspace, st);
+        if (v != THINK_ERR_UNSUPPORTED) return v;
+    }
     v = launch_score(q_win, k, k_strides, B, Hq, Hkv, N, S_obs, dtype, T, scores, idx, workspace, st);
     if (v != THINK_OK || N == 0) return v;
     return launch_compact(k, k_strides, B, Hkv, N, dtype, idx, T, k_pruned, ldk, st);

@@ -27,6 +27,7 @@ def _prune_gpu(q_win, k, T):
     _, Hkv, N, _ = k.shape
     cache = qdk.PrunedCache(B, Hq, Hkv, N, T, d, dtype=k.dtype)
     cache.prune(q_win, k)
+    assert qdk.think_read_device_status(cache.score_ws) == 0
     return cache
 
 
@@ -37,7 +38,7 @@ def _full_path_check(w, q_win, k, v, steps, T=None):
     cache = _prune_gpu(qd, kd, T)
     torch.cuda.synchronize()
     ora_scores, ora_idx, ora_kp = oracle.oracle_prune(f64(q_win), f64(k), T)
-    check_scores(cache.scores, ora_scores)
+    check_scores(cache.scores, ora_scores, dtype=w.dtype)
     gpu_idx = cache.idx.cpu().numpy()
     ties = idx_mismatch_heads(gpu_idx, ora_idx, ora_scores, T)
     if ties:
@@ -154,7 +155,7 @@ def test_edge_shapes(case, dtype):
     cache.decode(q.to(DEV), vd, out)
     torch.cuda.synchronize()
     ora_scores, ora_idx, ora_kp = oracle.oracle_prune(f64(q_win), f64(k), T)
-    check_scores(cache.scores, ora_scores)
+    check_scores(cache.scores, ora_scores, dtype=dtype)
     assert not idx_mismatch_heads(cache.idx.cpu().numpy(), ora_idx, ora_scores, T)
     assert np.array_equal(kp_logical(cache.k_pruned, N), ora_kp)
     check_out(out, oracle.oracle_decode(f64(q), ora_kp, f64(v), ora_idx), dtype, where=str(case))
@@ -200,6 +201,36 @@ def test_fused_prune_equals_stepwise_calls():
     a.prune(qd, kd)
     torch.cuda.synchronize()
     assert torch.equal(a.idx, b.idx)
+
+
+@pytest.mark.parametrize("env", [{"THINK_PRUNE_FUSED": "1"},
+                                 {"THINK_PRUNE_FUSED": "1", "THINK_PRUNE_L2_HINTS": "0"}])
+def test_prune_schedules_give_identical_results(env, monkeypatch):
+    # the two-launch prune (default) and the one-kernel prune (with and without
+    # its L2 hints) must agree bit for bit: same split plan, same order of
+    # additions, pure copies
+    shapes = [(2, 32, 8, 5000, 64), (1, 8, 1, 70, 51), (4, 4, 4, 3000, 128), (3, 16, 8, 1, 1),
+              (1, 32, 8, 40000, 51)]
+    for i, (B, Hq, Hkv, N, T) in enumerate(shapes):
+        q_win, k, _, _ = _random_case(100 + i, B, Hq, Hkv, N, 32, torch.bfloat16, k_pad=8)
+        kd = torch.empty((B, Hkv, N + 8, 128), dtype=torch.bfloat16, device=DEV)[:, :, :N].copy_(k)
+        qd = q_win.to(DEV)
+        for key in ("THINK_PRUNE_FUSED", "THINK_PRUNE_L2_HINTS"):
+            monkeypatch.delenv(key, raising=False)
+        a = _prune_gpu(qd, kd, T)
+        for key, val in env.items():
+            monkeypatch.setenv(key, val)
+        b = _prune_gpu(qd, kd, T)
+        b.prune(qd, kd)  # a second call on the same workspace: counters and flags were reset
+        torch.cuda.synchronize()
+        assert qdk.think_read_device_status(b.score_ws) == 0
+        assert torch.equal(a.scores, b.scores), (env, B, Hq, Hkv, N, T)
+        assert torch.equal(a.idx, b.idx)
+        assert torch.equal(a.k_pruned[..., :N], b.k_pruned[..., :N])
+        ora_scores, ora_idx, ora_kp = oracle.oracle_prune(f64(q_win), f64(k), T)
+        check_scores(a.scores, ora_scores)
+        assert not idx_mismatch_heads(a.idx.cpu().numpy(), ora_idx, ora_scores, T)
+        assert np.array_equal(kp_logical(a.k_pruned, N), ora_kp)
 
 
 @pytest.mark.parametrize("kernel", ["warp_mma", "cuda_cores", "tensor_cores"])
