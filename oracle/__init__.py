@@ -16,7 +16,9 @@ Python because they are definitions, not kernels:
 * ``attention_loss`` -- the attention-weight loss ||Q K^T - Q_S K_S^T||_F that
   the abstract says the pruning keeps small;
 * ``bruteforce_best_subset`` -- the exhaustive minimiser of that loss over all
-  channel subsets of a given size (tiny d only).
+  channel subsets of a given size (tiny d only);
+* ``oracle_append`` -- the growing cache: new tokens' keys compacted with the
+  fixed kept channels and appended (a composition of ``oracle_compact``).
 
 Parity pins: every function here is pinned by ``tests/test_oracle_pins.py``
 (closed forms, brute force, library routines, a hand-worked example).
@@ -215,6 +217,15 @@ def oracle_dense_decode(q, k, v, scale=None):
 
 def oracle_prune(q_win, k, T):
     return default_oracle().prune(q_win, k, T)
+
+
+def oracle_append(kp, k_new, idx):
+    """Growing cache: after the prune, the keys of new tokens are compacted with
+    each head's kept channels (fixed at prune time) and appended along N:
+    [K' | compact(k_new, idx)].  The ThinK pages only say that inference runs
+    with the pruned cache; the new tokens' keys are read here the same way as
+    the cached ones.  kp [B,Hkv,N,T], k_new [B,Hkv,n,d] -> [B,Hkv,N+n,T]."""
+    return np.concatenate([_f64(kp), oracle_compact(k_new, idx)], axis=2)
 
 
 def attention_loss(q_win_head, k_head, keep) -> float:

@@ -13,7 +13,11 @@ worked example and no formula, so the oracle is pinned by:
 * library routines: Python's sort for the selection order, numpy's gather for
   the compaction, torch's fp64 scaled_dot_product_attention for decode;
 * invariants: lambda = 0 reproduces dense attention bit for bit, softmax
-  weights sum to one, all-zero channels make pruning lossless.
+  weights sum to one, all-zero channels make pruning lossless;
+* growing cache: appending keys chunk by chunk equals compacting the whole
+  cache at once, lambda = 0 over a grown cache equals dense attention over all
+  keys, and an appended token that dominates the logits takes the whole
+  softmax weight (closed form).
 """
 import itertools
 import json
@@ -314,3 +318,50 @@ def test_decode_rejects_empty_cache():
 def test_t_from_lambda_rule():
     for d, lam, T in GOLDEN["t_from_lambda"]["cases"]:
         assert oracle.t_from_lambda(d, lam) == T, (d, lam)
+
+
+# -------------------------------------------------------- growing cache ---
+
+def test_append_in_chunks_equals_compacting_everything():
+    r = rng(70)
+    B, Hkv, N, d, T = 2, 3, 41, 16, 6
+    k = r.standard_normal((B, Hkv, N, d))
+    idx = np.sort(np.stack([np.stack([r.choice(d, T, replace=False) for _ in range(Hkv)])
+                            for _ in range(B)]), axis=-1).astype(np.int32)
+    kp = oracle.oracle_compact(k[:, :, :10], idx)
+    for a, b in [(10, 11), (11, 18), (18, 18), (18, 40), (40, 41)]:
+        kp = oracle.oracle_append(kp, k[:, :, a:b], idx)
+    assert kp.shape == (B, Hkv, N, T)
+    assert np.array_equal(kp, oracle.oracle_compact(k, idx))
+    assert np.array_equal(kp, np.take_along_axis(k, idx[:, :, None, :].repeat(N, 2), axis=3))
+
+
+def test_grown_cache_at_lambda_zero_is_dense_attention():
+    r = rng(71)
+    B, Hq, Hkv, N0, n, d = 1, 4, 2, 20, 13, 8
+    q = r.standard_normal((B, Hq, d))
+    k = r.standard_normal((B, Hkv, N0 + n, d))
+    v = r.standard_normal((B, Hkv, N0 + n, d))
+    idx = np.broadcast_to(np.arange(d, dtype=np.int32), (B, Hkv, d)).copy()
+    kp = oracle.oracle_append(oracle.oracle_compact(k[:, :, :N0], idx), k[:, :, N0:], idx)
+    np.testing.assert_array_equal(oracle.oracle_decode(q, kp, v, idx), oracle.oracle_dense_decode(q, k, v))
+    np.testing.assert_allclose(oracle.oracle_decode(q, kp, v, idx), _sdpa(q, k, v, Hq // Hkv),
+                               rtol=1e-12, atol=1e-13)
+
+
+def test_dominant_appended_token_takes_all_weight():
+    # the appended token's key on the kept channels is 800 q' / |q'|^2, so its
+    # logit is 800 / sqrt(16) = 200; the cached keys are tiny (logits ~ 0.01),
+    # so every other softmax weight is below e^-190
+    r = rng(72)
+    B, Hq, Hkv, N0, d, T = 1, 1, 1, 30, 16, 4
+    idx = np.array([[[2, 5, 11, 13]]], dtype=np.int32)
+    q = r.standard_normal((B, Hq, d))
+    k_old = 0.01 * r.standard_normal((B, Hkv, N0, d))
+    k_new = np.zeros((B, Hkv, 1, d))
+    qk = q[0, 0, idx[0, 0]]
+    k_new[0, 0, 0, idx[0, 0]] = 800.0 * qk / np.dot(qk, qk)
+    v = r.standard_normal((B, Hkv, N0 + 1, d))
+    kp = oracle.oracle_append(oracle.oracle_compact(k_old, idx), k_new, idx)
+    out = oracle.oracle_decode(q, kp, v, idx)
+    np.testing.assert_allclose(out[0, 0], v[0, 0, N0], rtol=0, atol=1e-12)
