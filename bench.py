@@ -200,6 +200,37 @@ def step_bytes(w, T):
     return W.prune_bytes(w, T) + w.decode_steps * W.decode_bytes(w, T)
 
 
+def measure_append(w, T, dev, stream, qw_d, k_d, chunk=4096, reps=50):
+    """Growing cache, outside the timed step: device time of appending one new
+    token's keys (all heads) and a chunk of new tokens' keys to a pruned cache
+    with room for them (the new keys are views of cached ones)."""
+    import torch
+    import query_driven_key_b200 as qdk
+    chunk = min(chunk, w.N)
+    cache = qdk.PrunedCache(w.B, w.Hq, w.Hkv, w.N, T, w.d, dtype=w.dtype, device=dev,
+                            capacity=w.N + chunk)
+    cache.prune(qw_d, k_d, stream=stream)
+
+    def timed(n_new):
+        knew = k_d[:, :, :n_new]
+        for _ in range(3):
+            qdk.think_append_keys(knew, cache.idx, cache.k_pruned, cache.ldk, w.N, stream)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            qdk.think_append_keys(knew, cache.idx, cache.k_pruned, cache.ldk, w.N, stream)
+        e1.record(stream)
+        stream.synchronize()
+        return e0.elapsed_time(e1) * 1e3 / reps
+
+    e = torch_elem_size(w.dtype)
+    one_us, chunk_us = timed(1), timed(chunk)
+    chunk_bytes = w.B * w.Hkv * chunk * (w.d + T) * e + w.B * w.Hkv * T * 4
+    return {"one_token_us": one_us, "chunk_tokens": chunk, "chunk_us": chunk_us,
+            "chunk_gbs": chunk_bytes / (chunk_us * 1e-6) / 1e9,
+            "note": "think_append_keys, device time per call (CUDA events), not part of the step"}
+
+
 def data_recipe(w):
     if w.k_kind == "lowrank":
         keys = f"rank-{w.k_rank} N(0,1) factors + {w.k_noise} N(0,1) noise, LogNormal(0,{w.k_sigma}) channel scales"
@@ -423,6 +454,8 @@ def run_native(args):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                "steps": args.e2e_steps}
 
+    append = measure_append(w, T, dev, stream, qw_d[0], k_d[0]) if rank == 0 else None
+
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -446,6 +479,7 @@ def run_native(args):
                      "frac": achieved / peak, "peak_source": f"{peak_kind} hbm_gbs",
                      "algorithmic_bytes_per_launch": dec_bytes,
                      "traffic": DECODE_TRAFFIC_BYTES if default_workload(args) else None},
+        "append": append,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
         "e2e": e2e,

@@ -14,7 +14,8 @@
  *   think_compact_keys        K'[n,t] = K[n, idx[t]]   (V is not touched)
  *   think_pruned_decode_attn  out = softmax((q[idx] . K'^T) / sqrt(d)) V
  *
- * plus think_prune, the first three in two launches.
+ * plus think_prune, the first three in two launches, and think_append_keys,
+ * which appends new tokens' keys to the thinner cache.
  *
  * Conventions shared by every call
  *   - Shapes: B batch, Hq query heads, Hkv KV heads (G = Hq/Hkv query heads
@@ -133,6 +134,27 @@ think_status_t think_select_channels(const double *scores, int B, int Hkv, int d
 think_status_t think_compact_keys(const void *k, const int64_t k_strides[3], int B, int Hkv,
                                   int64_t N, int d, think_dtype_t dtype, const int32_t *idx,
                                   int T, void *k_pruned, int64_t ldk, void *stream);
+
+/* --------------------------------------------------------------- append --
+ * Growing cache (after the prune; the ThinK pages only say that inference
+ * runs with the pruned cache, and this library reads new tokens' keys the
+ * same way as the cached ones): the keys of n_new new tokens are compacted
+ * with each head's kept channels, fixed at prune time, and written to token
+ * columns [n_at, n_at + n_new) of K':
+ *     K'[b,h,t, n_at + n] = k_new[b,h,n, idx[b,h,t]]      (a pure copy)
+ *   k_new, k_strides  [B][Hkv][n_new][d] keys of the new tokens (layout as K
+ *                     in think_score_channels).
+ *   idx, T, k_pruned, ldk  as for think_compact_keys.
+ *   n_at              first column to write, usually the current cache
+ *                     length; n_at + n_new <= ldk (the capacity of a K' row),
+ *                     else THINK_ERR_INVALID_ARG.  Other columns are not
+ *                     touched; V is the caller's (append its rows as usual).
+ * Decode the grown cache with think_pruned_decode_attn and N = n_at + n_new
+ * (its workspace must be sized for that N).  n_new == 0 launches nothing.
+ * One launch (the compaction kernel with a column offset). */
+think_status_t think_append_keys(const void *k_new, const int64_t k_strides[3], int B, int Hkv,
+                                 int64_t n_new, int d, think_dtype_t dtype, const int32_t *idx,
+                                 int T, void *k_pruned, int64_t ldk, int64_t n_at, void *stream);
 
 /* ---------------------------------------------------------------- prune --
  * The whole prune step of one layer in two launches: scores and the top-T

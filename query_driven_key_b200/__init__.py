@@ -35,7 +35,8 @@ THINK_DEVICE_TIMEOUT_BARRIER = 0x8
 EXPORTED = (
     "think_status_string", "think_t_from_lambda", "think_pruned_ld",
     "think_score_workspace_size", "think_score_channels", "think_select_channels",
-    "think_compact_keys", "think_prune", "think_decode_workspace_size", "think_pruned_decode_attn",
+    "think_compact_keys", "think_append_keys", "think_prune", "think_decode_workspace_size",
+    "think_pruned_decode_attn",
     "think_workspace_init", "think_read_device_status", "think_noalloc_scratch_bytes",
     "think_pruned_decode_attn_noalloc",
 )
@@ -66,6 +67,8 @@ def _load() -> ctypes.CDLL:
     lib.think_compact_keys.restype = I
     lib.think_prune.argtypes = [P, P, I64P, I, I, I, I64, I, I, I, I, P, P, P, I64, P, SZ, P]
     lib.think_prune.restype = I
+    lib.think_append_keys.argtypes = [P, I64P, I, I, I64, I, I, P, I, P, I64, I64, P]
+    lib.think_append_keys.restype = I
     lib.think_decode_workspace_size.argtypes = [I, I, I, I64, I, I]
     lib.think_decode_workspace_size.restype = SZ
     lib.think_pruned_decode_attn.argtypes = [P, P, I64, P, I64P, P, I, I, I, I64, I, I, I, F, P,
@@ -174,6 +177,18 @@ def think_compact_keys(k: torch.Tensor, idx: torch.Tensor, k_pruned: torch.Tenso
                                   _ptr(k_pruned), int(ldk), _stream(stream)), "think_compact_keys")
 
 
+def think_append_keys(k_new: torch.Tensor, idx: torch.Tensor, k_pruned: torch.Tensor, ldk: int,
+                      n_at: int, stream=None) -> None:
+    """k_new [B,Hkv,n,d] -> K' columns [n_at, n_at + n) of every kept channel."""
+    B, Hkv, n, d = k_new.shape
+    T = idx.shape[-1]
+    if idx.dtype != torch.int32 or k_pruned.dtype != k_new.dtype:
+        raise ThinkError(THINK_ERR_INVALID_ARG, "think_append_keys")
+    _check(lib.think_append_keys(_ptr(k_new), _strides3(k_new), B, Hkv, n, d, _dtype(k_new),
+                                 _ptr(idx), T, _ptr(k_pruned), int(ldk), int(n_at), _stream(stream)),
+           "think_append_keys")
+
+
 def think_prune(q_win: torch.Tensor, k: torch.Tensor, T: int, scores: torch.Tensor,
                 idx: torch.Tensor, k_pruned: torch.Tensor, ldk: int, workspace: torch.Tensor,
                 stream=None) -> None:
@@ -242,33 +257,46 @@ def think_read_device_status(workspace: torch.Tensor, stream=None) -> int:
 
 
 class PrunedCache:
-    """Device buffers of one pruned layer: kept channels, thinner K, V, workspaces.
+    """Device buffers of one pruned layer: kept channels, thinner K, workspaces.
 
     A convenience holder for callers of the functions above; it allocates with
-    torch on construction and then only calls the C entry points."""
+    torch on construction and then only calls the C entry points.  ``N`` is
+    the cache length at prune time, ``capacity`` (>= N) the longest the cache
+    may grow to by ``append``; ``n`` is the current length."""
 
     def __init__(self, B: int, Hq: int, Hkv: int, N: int, T: int, d: int = 128,
-                 dtype: torch.dtype = torch.bfloat16, device="cuda"):
+                 dtype: torch.dtype = torch.bfloat16, device="cuda", capacity: int | None = None):
         self.B, self.Hq, self.Hkv, self.N, self.T, self.d, self.dtype = B, Hq, Hkv, N, T, d, dtype
-        self.ldk = think_pruned_ld(N, dtype)
+        self.capacity = N if capacity is None else max(N, capacity)
+        self.n = N
+        self.ldk = think_pruned_ld(self.capacity, dtype)
         self.scores = torch.empty((B, Hkv, d), dtype=torch.float64, device=device)
         self.idx = torch.empty((B, Hkv, T), dtype=torch.int32, device=device)
         self.k_pruned = torch.empty((B, Hkv, T, self.ldk), dtype=dtype, device=device)
         self.score_ws = torch.zeros(max(256, think_score_workspace_size(B, Hq, Hkv, N, d)),
                                     dtype=torch.uint8, device=device)
-        self.decode_ws = torch.zeros(max(256, think_decode_workspace_size(B, Hq, Hkv, N, d, dtype)),
-                                     dtype=torch.uint8, device=device)
+        self.decode_ws = torch.zeros(
+            max(256, think_decode_workspace_size(B, Hq, Hkv, self.capacity, d, dtype)),
+            dtype=torch.uint8, device=device)
 
     def prune(self, q_win, k, stream=None):
         think_prune(q_win, k, self.T, self.scores, self.idx, self.k_pruned, self.ldk,
                     self.score_ws, stream)
+        self.n = self.N
+
+    def append(self, k_new, stream=None):
+        """Append the keys of k_new.shape[2] new tokens (compacted with the kept channels)."""
+        think_append_keys(k_new, self.idx, self.k_pruned, self.ldk, self.n, stream)
+        self.n += k_new.shape[2]
 
     def prune_stepwise(self, q_win, k, stream=None):
         """The same prune through the three separate entry points."""
         think_score_channels(q_win, k, self.scores, self.score_ws, stream)
         think_select_channels(self.scores, self.T, self.idx, stream)
         think_compact_keys(k, self.idx, self.k_pruned, self.ldk, stream)
+        self.n = self.N
 
     def decode(self, q, v, out, scale=None, stream=None):
+        """Attend over the current n tokens (v holds at least n token rows)."""
         think_pruned_decode_attn(q, self.k_pruned, self.ldk, v, self.idx, out, self.decode_ws,
-                                 scale=scale, N=self.N, stream=stream)
+                                 scale=scale, N=self.n, stream=stream)

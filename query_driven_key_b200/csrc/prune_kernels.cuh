@@ -266,8 +266,9 @@ __global__ void __launch_bounds__(128)
 }
 
 // ---------------------------------------------------------------------------
-// Compact: K'^T[t][n] = K[n][idx[t]] for a tile of 64
-// tokens of one head.
+// Compact: K'^T[t][col0 + n] = K[n][idx[t]] for a tile of 64 tokens of one
+// head (col0 = 0 for a whole cache, the current length when new tokens'
+// keys are appended).
 // Each thread loads a 4-token x 8-channel block (four 16-byte loads, one per
 // token row), regroups it in registers into 8 channel runs of 4 tokens, and
 // stores those transposed into shared memory (channel-major, padded pitch).
@@ -306,7 +307,7 @@ template <typename TIn> struct CompactTokens { static constexpr int value = 64; 
 template <typename TIn>
 __global__ void __launch_bounds__(256)
     compact_kernel(const TIn *__restrict__ k, int64_t sb, int64_t sh, int64_t sn, int Hkv, int64_t N,
-                   const int32_t *__restrict__ idx, int T, TIn *__restrict__ kp, int64_t ldk)
+                   const int32_t *__restrict__ idx, int T, TIn *__restrict__ kp, int64_t ldk, int64_t col0)
 {
     constexpr int BNC = CompactTokens<TIn>::value;  // tokens per block
     constexpr int VEC = 16 / sizeof(TIn);         // elements per 16 bytes (channels per load)
@@ -353,12 +354,13 @@ __global__ void __launch_bounds__(256)
 
     const int seg = lane % LPR;
     const int tok = seg * VEC;
+    const bool vec_ok = (col0 % VEC) == 0;  // 16-byte aligned output runs
     for (int t = warp * RPI + lane / LPR; t < T; t += 8 * RPI) {
         const int c = idx[(int64_t)head * T + t];
         uint4 val = make_uint4(0, 0, 0, 0);
         if ((unsigned)c < (unsigned)kD) val = *reinterpret_cast<const uint4 *>(&sT[c][tok]);
-        TIn *out = kp + ((int64_t)head * T + t) * ldk + n0 + tok;
-        if (n0 + tok + VEC <= N) {
+        TIn *out = kp + ((int64_t)head * T + t) * ldk + col0 + n0 + tok;
+        if (vec_ok && n0 + tok + VEC <= N) {
             *reinterpret_cast<uint4 *>(out) = val;
         } else {
             const TIn *e = reinterpret_cast<const TIn *>(&val);

@@ -330,7 +330,7 @@ think_status_t validate_compact(const void *k, const int64_t k_strides[3], int B
 
 think_status_t launch_compact(const void *k, const int64_t k_strides[3], int B, int Hkv, int64_t N,
                               think_dtype_t dtype, const int32_t *idx, int T, void *k_pruned,
-                              int64_t ldk, cudaStream_t st)
+                              int64_t ldk, cudaStream_t st, int64_t col0 = 0)
 {
     const int64_t heads = (int64_t)B * Hkv;
     const int bnc = dtype == THINK_BF16 ? CompactTokens<__nv_bfloat16>::value : CompactTokens<float>::value;
@@ -338,11 +338,11 @@ think_status_t launch_compact(const void *k, const int64_t k_strides[3], int B, 
     if (dtype == THINK_BF16)
         compact_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
             static_cast<const __nv_bfloat16 *>(k), k_strides[0], k_strides[1], k_strides[2], Hkv, N,
-            idx, T, static_cast<__nv_bfloat16 *>(k_pruned), ldk);
+            idx, T, static_cast<__nv_bfloat16 *>(k_pruned), ldk, col0);
     else
         compact_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float *>(k), k_strides[0],
                                                     k_strides[1], k_strides[2], Hkv, N, idx, T,
-                                                    static_cast<float *>(k_pruned), ldk);
+                                                    static_cast<float *>(k_pruned), ldk, col0);
     return launch_status();
 }
 
@@ -653,6 +653,19 @@ think_status_t think_compact_keys(const void *k, const int64_t k_strides[3], int
     if (v != THINK_OK || B == 0 || Hkv == 0 || N == 0) return v;
     return launch_compact(k, k_strides, B, Hkv, N, dtype, idx, T, k_pruned, ldk,
                           static_cast<cudaStream_t>(stream));
+}
+
+think_status_t think_append_keys(const void *k_new, const int64_t k_strides[3], int B, int Hkv,
+                                 int64_t n_new, int d, think_dtype_t dtype, const int32_t *idx, int T,
+                                 void *k_pruned, int64_t ldk, int64_t n_at, void *stream)
+{
+    if (n_new < 0 || n_at < 0) return THINK_ERR_INVALID_ARG;
+    if (n_new > 0 && n_at > ldk - n_new) return THINK_ERR_INVALID_ARG;  // past the row capacity
+    const think_status_t v = validate_compact(k_new, k_strides, B, Hkv, n_new, d, dtype, idx, T,
+                                              k_pruned, ldk);
+    if (v != THINK_OK || B == 0 || Hkv == 0 || n_new == 0) return v;
+    return launch_compact(k_new, k_strides, B, Hkv, n_new, dtype, idx, T, k_pruned, ldk,
+                          static_cast<cudaStream_t>(stream), n_at);
 }
 
 think_status_t think_prune(const void *q_win, const void *k, const int64_t k_strides[3], int B,

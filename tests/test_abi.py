@@ -119,6 +119,20 @@ def test_compact_validation():
     assert f(FAKE, s, 1, 2, 0, 128, 1, FAKE, 10, FAKE, 0, None) == qdk.THINK_OK                  # N == 0
 
 
+def test_append_validation():
+    s = I64x3(128 * 64, 128 * 64, 128)
+    f = lib.think_append_keys
+    # (k_new, strides, B, Hkv, n_new, d, dtype, idx, T, k_pruned, ldk, n_at, stream)
+    assert f(FAKE, s, 1, 2, 8, 128, 1, FAKE, 10, FAKE, 64, 57, None) == qdk.THINK_ERR_INVALID_ARG  # past capacity
+    assert f(FAKE, s, 1, 2, -1, 128, 1, FAKE, 10, FAKE, 64, 0, None) == qdk.THINK_ERR_INVALID_ARG
+    assert f(FAKE, s, 1, 2, 8, 128, 1, FAKE, 10, FAKE, 64, -1, None) == qdk.THINK_ERR_INVALID_ARG
+    assert f(FAKE, s, 1, 2, 8, 96, 1, FAKE, 10, FAKE, 64, 56, None) == qdk.THINK_ERR_UNSUPPORTED
+    assert f(FAKE, s, 1, 2, 8, 128, 1, FAKE, 0, FAKE, 64, 56, None) == qdk.THINK_ERR_INVALID_ARG    # T = 0
+    assert f(FAKE, s, 1, 2, 8, 128, 1, FAKE, 10, FAKE, 68, 60, None) == qdk.THINK_ERR_ALIGNMENT     # 136 B pitch
+    assert f(FAKE, s, 1, 2, 8, 128, 1, None, 10, FAKE, 64, 56, None) == qdk.THINK_ERR_INVALID_ARG
+    assert f(FAKE, s, 1, 2, 0, 128, 1, FAKE, 10, FAKE, 64, 64, None) == qdk.THINK_OK              # nothing to append
+
+
 def test_decode_validation():
     s = I64x3(128 * 64 * 2, 128 * 64, 128)
     f = lib.think_pruned_decode_attn

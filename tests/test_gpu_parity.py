@@ -163,6 +163,41 @@ def test_edge_shapes(case, dtype):
         assert np.array_equal(cache.idx.cpu().numpy()[0, 0], np.arange(T))
 
 
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_growing_cache(dtype):
+    # prune on the first N0 tokens, then append new tokens' keys in chunks of
+    # odd sizes (unaligned columns included) and decode after every append
+    B, Hq, Hkv, N0, S, T = 2, 8, 2, 300, 16, 51
+    chunks = [1, 7, 64, 100, 1, 500, 3]
+    n_tot = N0 + sum(chunks)
+    q_win, k, v, q = _random_case(77, B, Hq, Hkv, n_tot, S, dtype)
+    kd, vd, qd = k.to(DEV), v.to(DEV), q.to(DEV)
+    cache = qdk.PrunedCache(B, Hq, Hkv, N0, T, dtype=dtype, capacity=n_tot + 5)
+    cache.k_pruned.fill_(7.0)
+    cache.prune(q_win.to(DEV), kd[:, :, :N0])
+    torch.cuda.synchronize()
+    ora_scores, ora_idx, ora_kp = oracle.oracle_prune(f64(q_win), f64(k[:, :, :N0]), T)
+    if idx_mismatch_heads(cache.idx.cpu().numpy(), ora_idx, ora_scores, T):
+        cache.idx.copy_(torch.from_numpy(ora_idx))
+        qdk.think_compact_keys(kd[:, :, :N0], cache.idx, cache.k_pruned, cache.ldk)
+    out = torch.empty((B, Hq, 128), dtype=torch.float32, device=DEV)
+    n = N0
+    for c in chunks:
+        cache.append(kd[:, :, n:n + c])
+        ora_kp = oracle.oracle_append(ora_kp, f64(k[:, :, n:n + c]), ora_idx)
+        n += c
+        assert cache.n == n
+        cache.decode(qd, vd, out)
+        torch.cuda.synchronize()
+        assert np.array_equal(kp_logical(cache.k_pruned, n), ora_kp), f"K' after growing to {n}"
+        assert torch.all(cache.k_pruned[..., n:] == 7.0), "columns past the cache length are not written"
+        check_out(out, oracle.oracle_decode(f64(q), ora_kp, f64(v[:, :, :n]), ora_idx), dtype,
+                  where=f"grown to {n}")
+    with pytest.raises(qdk.ThinkError):  # past the capacity of a K' row
+        qdk.think_append_keys(kd[:, :, :cache.ldk - n + 1], cache.idx, cache.k_pruned, cache.ldk, n)
+    assert qdk.think_read_device_status(cache.decode_ws) == 0
+
+
 def test_ldk_larger_than_needed_and_exact_ties():
     # duplicate channels give exact score ties: lower index must win on both sides
     B, Hq, Hkv, N, S, T = 1, 4, 2, 300, 6, 40
