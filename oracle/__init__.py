@@ -20,6 +20,9 @@ Python because they are definitions, not kernels:
 * ``oracle_append`` -- the growing cache: new tokens' keys compacted with the
   fixed kept channels and appended (a composition of ``oracle_compact``).
 
+The 4-bit thinner cache (``oracle_quantize_q4`` / ``oracle_dequantize_q4``)
+is plain C in ``think_oracle.c`` (fp32 steps as defined there).
+
 Parity pins: every function here is pinned by ``tests/test_oracle_pins.py``
 (closed forms, brute force, library routines, a hand-worked example).
 """
@@ -77,10 +80,12 @@ class Oracle:
         lib.oracle_compact.argtypes = [P, P, I, I, I, I, I, P]
         lib.oracle_decode.argtypes = [P, P, P, P, I, I, I, I, I, I, D, P]
         lib.oracle_dense_decode.argtypes = [P, P, P, I, I, I, I, I, D, P]
+        lib.oracle_quantize_q4.argtypes = [P, I, I, I, I, I, P, P]
+        lib.oracle_dequantize_q4.argtypes = [P, P, I, I, I, I, I, P]
         lib.oracle_num_threads.restype = I
         lib.oracle_set_num_threads.argtypes = [I]
         for f in ("oracle_score", "oracle_score_explicit", "oracle_select", "oracle_compact",
-                  "oracle_decode", "oracle_dense_decode"):
+                  "oracle_decode", "oracle_dense_decode", "oracle_quantize_q4", "oracle_dequantize_q4"):
             getattr(lib, f).restype = I
         self.lib = lib
 
@@ -156,6 +161,28 @@ class Oracle:
                                             float(scale), _ptr(out)), "oracle_dense_decode")
         return out
 
+    def quantize_q4(self, kp, group: int = 128):
+        """K' [B,Hkv,N,T] (bf16 values) -> codes uint8 [B,Hkv,N,T] (0..15) and group
+        parameters fp32 [B,Hkv,ceil(N/group),T,2] = (scale, min)."""
+        kp = _f64(kp)
+        B, Hkv, N, T = kp.shape
+        ng = -(-N // group)
+        codes = np.zeros((B, Hkv, N, T), dtype=np.uint8)
+        gs = np.zeros((B, Hkv, ng, T, 2), dtype=np.float32)
+        _check(self.lib.oracle_quantize_q4(_ptr(kp), B, Hkv, N, T, group, _ptr(codes), _ptr(gs)),
+               "oracle_quantize_q4")
+        return codes, gs
+
+    def dequantize_q4(self, codes, gs, group: int = 128) -> np.ndarray:
+        """codes [B,Hkv,N,T], group parameters -> dequantised K' (bf16 values, fp64)."""
+        codes = np.ascontiguousarray(codes, dtype=np.uint8)
+        gs = np.ascontiguousarray(gs, dtype=np.float32)
+        B, Hkv, N, T = codes.shape
+        out = np.zeros((B, Hkv, N, T), dtype=np.float64)
+        _check(self.lib.oracle_dequantize_q4(_ptr(codes), _ptr(gs), B, Hkv, N, T, group, _ptr(out)),
+               "oracle_dequantize_q4")
+        return out
+
     def prune(self, q_win, k, T: int):
         """The whole prune step: scores, kept channels, thinner key cache."""
         scores = self.score(q_win, k)
@@ -226,6 +253,14 @@ def oracle_append(kp, k_new, idx):
     with the pruned cache; the new tokens' keys are read here the same way as
     the cached ones.  kp [B,Hkv,N,T], k_new [B,Hkv,n,d] -> [B,Hkv,N+n,T]."""
     return np.concatenate([_f64(kp), oracle_compact(k_new, idx)], axis=2)
+
+
+def oracle_quantize_q4(kp, group: int = 128):
+    return default_oracle().quantize_q4(kp, group)
+
+
+def oracle_dequantize_q4(codes, gs, group: int = 128):
+    return default_oracle().dequantize_q4(codes, gs, group)
 
 
 def attention_loss(q_win_head, k_head, keep) -> float:

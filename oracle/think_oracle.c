@@ -264,3 +264,82 @@ int oracle_dense_decode(const double *q, const double *k, const double *v, int B
     }
     return 0;
 }
+
+/*
+ * 4-bit thinner key cache (ThinK composed with per-channel key quantisation,
+ * as in the ThinK + KIVI combination of the experiments section; KIVI
+ * quantises keys per channel over groups of tokens).  Reading used here, for
+ * each (b, h_kv), kept channel t and group of `group` consecutive tokens:
+ *
+ *   mn    = min of the group's K'[n,t]      mx = max            (fp32, exact)
+ *   scale = (mx - mn) / 15                                      (fp32 division)
+ *   code  = 0 if scale == 0, else clamp(rint((K'[n,t] - mn) / scale), 0, 15)
+ *           (fp32 subtraction and division, rint = round half to even)
+ *   K^[n,t] = bf16(fma(code, scale, mn))    (fp32 fused multiply-add, then
+ *                                            round to nearest-even bf16)
+ *
+ * The inputs are bf16 values (carried as doubles); every step is the fp32
+ * operation written, so the codes, the group parameters and the dequantised
+ * keys are defined exactly.
+ *
+ *   kp    [B][Hkv][N][T]     values of the thinner key cache (bf16-exact)
+ *   codes [B][Hkv][N][T]     uint8, 0..15
+ *   gs    [B][Hkv][ng][T][2] fp32 (scale, mn), ng = ceil(N / group)
+ */
+static float bf16_round(float x)
+{
+    uint32_t u;
+    memcpy(&u, &x, 4);
+    u = (u + 0x7fffu + ((u >> 16) & 1u)) & 0xffff0000u;   /* finite inputs only */
+    float y;
+    memcpy(&y, &u, 4);
+    return y;
+}
+
+int oracle_quantize_q4(const double *kp, int B, int Hkv, int N, int T, int group, uint8_t *codes,
+                       float *gs)
+{
+    if (B < 0 || Hkv < 0 || N < 0 || T < 1 || group < 1) return -1;
+    const int ng = (N + group - 1) / group;
+    for (int bh = 0; bh < B * Hkv; ++bh)
+        for (int g = 0; g < ng; ++g) {
+            const int n0 = g * group, n1 = (n0 + group < N) ? n0 + group : N;
+            for (int t = 0; t < T; ++t) {
+                float mn = (float)kp[((size_t)bh * N + n0) * T + t], mx = mn;
+                for (int n = n0 + 1; n < n1; ++n) {
+                    const float x = (float)kp[((size_t)bh * N + n) * T + t];
+                    if (x < mn) mn = x;
+                    if (x > mx) mx = x;
+                }
+                const float scale = (mx - mn) / 15.0f;
+                gs[(((size_t)bh * ng + g) * T + t) * 2 + 0] = scale;
+                gs[(((size_t)bh * ng + g) * T + t) * 2 + 1] = mn;
+                for (int n = n0; n < n1; ++n) {
+                    const float x = (float)kp[((size_t)bh * N + n) * T + t];
+                    float c = 0.0f;
+                    if (scale != 0.0f) {
+                        c = rintf((x - mn) / scale);
+                        if (c < 0.0f) c = 0.0f;
+                        if (c > 15.0f) c = 15.0f;
+                    }
+                    codes[((size_t)bh * N + n) * T + t] = (uint8_t)c;
+                }
+            }
+        }
+    return 0;
+}
+
+int oracle_dequantize_q4(const uint8_t *codes, const float *gs, int B, int Hkv, int N, int T,
+                         int group, double *khat)
+{
+    if (B < 0 || Hkv < 0 || N < 0 || T < 1 || group < 1) return -1;
+    const int ng = (N + group - 1) / group;
+    for (int bh = 0; bh < B * Hkv; ++bh)
+        for (int n = 0; n < N; ++n)
+            for (int t = 0; t < T; ++t) {
+                const size_t gi = (((size_t)bh * ng + n / group) * T + t) * 2;
+                const float c = (float)codes[((size_t)bh * N + n) * T + t];
+                khat[((size_t)bh * N + n) * T + t] = (double)bf16_round(fmaf(c, gs[gi], gs[gi + 1]));
+            }
+    return 0;
+}

@@ -37,6 +37,11 @@ MUTATIONS = {
                                 "kv = h % Hkv;\n        const size_t kvh = (size_t)b * Hkv + (size_t)kv;\n"
                                 "        const int32_t *ih"),
     "query_not_gathered": ("qp[t] = q[(size_t)bhq * d + ih[t]];", "qp[t] = q[(size_t)bhq * d + t];"),
+    "q4_step_of_16_levels": ("const float scale = (mx - mn) / 15.0f;", "const float scale = (mx - mn) / 16.0f;"),
+    "q4_truncated_codes": ("c = rintf((x - mn) / scale);", "c = floorf((x - mn) / scale);"),
+    "q4_min_not_added": ("bf16_round(fmaf(c, gs[gi], gs[gi + 1]))", "bf16_round(c * gs[gi])"),
+    "q4_group_index_of_next_group": ("(((size_t)bh * ng + n / group) * T + t) * 2;",
+                                     "(((size_t)bh * ng + (n + 1) / group) * T + t) * 2;"),
 }
 
 
@@ -90,6 +95,19 @@ def _pins(o: oracle.Oracle):
     vt = torch.from_numpy(v).repeat_interleave(G, 1)
     ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt)[:, :, 0].numpy()
     yield "sdpa_masked", np.allclose(out, ref, rtol=1e-12, atol=1e-13)
+    # 4-bit thinner K: grid values are exact; min -> 0 and max -> 15; error bound
+    kgrid = np.zeros((1, 1, 130, 2))
+    kq = r.integers(0, 16, size=(130, 2))
+    kq[0], kq[1], kq[128], kq[129] = 0, 15, 0, 15
+    kgrid[0, 0] = -1.0 + kq / 8.0
+    codes, gs = o.quantize_q4(kgrid)
+    ok = np.array_equal(codes[0, 0], kq) and np.array_equal(o.dequantize_q4(codes, gs), kgrid)
+    yield "q4_grid", ok
+    kr = torch.from_numpy(r.standard_normal((1, 1, 200, 3)) * 2).to(torch.bfloat16).double().numpy()
+    codes, gs = o.quantize_q4(kr)
+    khat = o.dequantize_q4(codes, gs)
+    step = np.repeat(gs[..., 0], 128, axis=2)[:, :, :200].astype(np.float64)
+    yield "q4_bound", bool(np.all(np.abs(khat - kr) <= 0.5 * step * (1 + 1e-5) + np.abs(khat) * 2.0 ** -8))
 
 
 def _all_pass(o):

@@ -365,3 +365,75 @@ def test_dominant_appended_token_takes_all_weight():
     kp = oracle.oracle_append(oracle.oracle_compact(k_old, idx), k_new, idx)
     out = oracle.oracle_decode(q, kp, v, idx)
     np.testing.assert_allclose(out[0, 0], v[0, 0, N0], rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------- 4-bit thinner K ---
+
+def _bf16_values(a):
+    return torch.from_numpy(np.asarray(a, dtype=np.float64)).to(torch.bfloat16).to(torch.float64).numpy()
+
+
+def test_q4_codes_span_each_group():
+    r = rng(80)
+    B, Hkv, N, T, group = 2, 2, 300, 5, 128
+    kp = _bf16_values(r.standard_normal((B, Hkv, N, T)) * r.lognormal(0, 1, (1, 1, 1, T)))
+    codes, gs = oracle.oracle_quantize_q4(kp, group)
+    assert codes.max() <= 15
+    for g0 in range(0, N, group):
+        blk = kp[:, :, g0:g0 + group]
+        cb = codes[:, :, g0:g0 + group]
+        gi = g0 // group
+        # the group's parameters are its own min and (max - min) / 15
+        np.testing.assert_array_equal(gs[:, :, gi, :, 1], blk.min(axis=2).astype(np.float32))
+        np.testing.assert_array_equal(gs[:, :, gi, :, 0],
+                                      ((blk.max(axis=2) - blk.min(axis=2)).astype(np.float32) / np.float32(15)))
+        # the minimum maps to code 0 and the maximum to code 15
+        amin, amax = blk.argmin(axis=2), blk.argmax(axis=2)
+        assert np.all(np.take_along_axis(cb, amin[:, :, None, :], 2) == 0)
+        assert np.all(np.take_along_axis(cb, amax[:, :, None, :], 2) == 15)
+
+
+def test_q4_error_is_within_half_a_step_plus_bf16_rounding():
+    r = rng(81)
+    B, Hkv, N, T = 1, 3, 257, 7
+    kp = _bf16_values(r.standard_normal((B, Hkv, N, T)) * 3)
+    codes, gs = oracle.oracle_quantize_q4(kp)
+    khat = oracle.oracle_dequantize_q4(codes, gs)
+    scale = np.repeat(gs[..., 0], 128, axis=2)[:, :, :N].astype(np.float64)
+    bound = 0.5 * scale * (1 + 1e-5) + np.abs(khat) * 2.0 ** -8
+    assert np.all(np.abs(khat - kp) <= bound)
+    # a dequantised key is a bf16 value
+    np.testing.assert_array_equal(_bf16_values(khat), khat)
+
+
+def test_q4_constant_group_is_exact():
+    kp = np.full((1, 1, 100, 3), 0.3125)
+    kp[0, 0, :, 1] = -2.5
+    codes, gs = oracle.oracle_quantize_q4(kp)
+    assert np.all(codes == 0) and np.all(gs[..., 0] == 0)
+    np.testing.assert_array_equal(oracle.oracle_dequantize_q4(codes, gs), kp)
+
+
+def test_q4_values_on_the_grid_are_exact():
+    # values mn + k * s with s = 1/8 and k covering 0..15: the step is s exactly,
+    # every value is a grid point, so codes are k and dequantisation is exact
+    r = rng(82)
+    k = r.integers(0, 16, size=(1, 2, 128, 4))
+    k[0, :, 0, :], k[0, :, 1, :] = 0, 15
+    kp = -1.0 + k / 8.0
+    codes, gs = oracle.oracle_quantize_q4(kp)
+    np.testing.assert_array_equal(gs[..., 0], 0.125)
+    np.testing.assert_array_equal(codes, k)
+    np.testing.assert_array_equal(oracle.oracle_dequantize_q4(codes, gs), kp)
+
+
+def test_q4_last_group_uses_only_its_tokens():
+    # N = 130: the second group holds two tokens, its range is theirs alone
+    kp = np.zeros((1, 1, 130, 1))
+    kp[0, 0, :128, 0] = np.linspace(-4, 4, 128)
+    kp[0, 0, 128:, 0] = [1.0, 2.5]
+    kp = _bf16_values(kp)
+    codes, gs = oracle.oracle_quantize_q4(kp)
+    assert gs.shape == (1, 1, 2, 1, 2)
+    assert gs[0, 0, 1, 0, 1] == 1.0 and gs[0, 0, 1, 0, 0] == np.float32(1.5) / np.float32(15)
+    assert list(codes[0, 0, 128:, 0]) == [0, 15]
