@@ -231,6 +231,35 @@ def measure_append(w, T, dev, stream, qw_d, k_d, chunk=4096, reps=50):
             "note": "think_append_keys, device time per call (CUDA events), not part of the step"}
 
 
+def measure_q4(w, T, stream, cache, qs_d, v_d, outs, bf16_us, peak):
+    """The 4-bit thinner cache on the same layer, outside the timed step:
+    device time of quantising K' and of the step's decode calls over the codes."""
+    import torch
+    from query_driven_key_b200 import workloads as W
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    for _ in range(3):
+        cache.quantize_q4(stream)
+    e0, e1 = ev(), ev()
+    e0.record(stream)
+    cache.quantize_q4(stream)
+    e1.record(stream)
+    for s in range(3):
+        cache.decode_q4(qs_d[s], v_d, outs[s], stream=stream)
+    e2, e3 = ev(), ev()
+    e2.record(stream)
+    for s in range(w.decode_steps):
+        cache.decode_q4(qs_d[s], v_d, outs[s], stream=stream)
+    e3.record(stream)
+    stream.synchronize()
+    us = e2.elapsed_time(e3) * 1e3 / w.decode_steps
+    nbytes = W.decode_bytes_q4(w, T)
+    gbs = nbytes / (us * 1e-6) / 1e9
+    return {"decode_us_per_step": us, "decode_gbs": gbs, "frac_of_measured_peak": gbs / peak,
+            "algorithmic_bytes_per_launch": nbytes, "speedup_vs_bf16_decode": bf16_us / us,
+            "quantize_us": e0.elapsed_time(e1) * 1e3,
+            "kernel": "pruned_decode_q4_kernel (think_pruned_decode_attn_q4), not part of the step"}
+
+
 def data_recipe(w):
     if w.k_kind == "lowrank":
         keys = f"rank-{w.k_rank} N(0,1) factors + {w.k_noise} N(0,1) noise, LogNormal(0,{w.k_sigma}) channel scales"
@@ -455,6 +484,8 @@ def run_native(args):
                "steps": args.e2e_steps}
 
     append = measure_append(w, T, dev, stream, qw_d[0], k_d[0]) if rank == 0 else None
+    q4 = (measure_q4(w, T, stream, caches[0], qs_d, v_d[0], outs[:, 0], dec_us, peak)
+          if rank == 0 and w.dtype == torch.bfloat16 else None)
 
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -480,6 +511,7 @@ def run_native(args):
                      "algorithmic_bytes_per_launch": dec_bytes,
                      "traffic": DECODE_TRAFFIC_BYTES if default_workload(args) else None},
         "append": append,
+        "q4": q4,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
         "e2e": e2e,

@@ -14,8 +14,9 @@
  *   think_compact_keys        K'[n,t] = K[n, idx[t]]   (V is not touched)
  *   think_pruned_decode_attn  out = softmax((q[idx] . K'^T) / sqrt(d)) V
  *
- * plus think_prune, the first three in two launches, and think_append_keys,
- * which appends new tokens' keys to the thinner cache.
+ * plus think_prune, the first three in two launches; think_append_keys,
+ * which appends new tokens' keys to the thinner cache; and a 4-bit thinner
+ * cache (think_quantize_keys_q4, think_pruned_decode_attn_q4).
  *
  * Conventions shared by every call
  *   - Shapes: B batch, Hq query heads, Hkv KV heads (G = Hq/Hkv query heads
@@ -225,6 +226,38 @@ think_status_t think_pruned_decode_attn_noalloc(const void *q, const void *k_pru
                                                 const int32_t *idx, int B, int Hq, int Hkv,
                                                 int64_t N, int d, int T, think_dtype_t dtype,
                                                 float scale, float *out, void *stream);
+
+/* ---------------------------------------------------------- 4-bit K' --
+ * The thinner key cache at 4 bits per element (ThinK abstract and method
+ * section, technical framework: the pruned cache combines with KV-cache
+ * quantisation such as KIVI; MiniKV page, quantisation: keys quantised per
+ * (sub-)channel).  Reading used here: for each (b, h_kv), kept channel t and
+ * group of 128 consecutive tokens,
+ *     mn = min, scale = (max - mn) / 15                          (fp32)
+ *     code = 0 if scale == 0, else clamp(rint((K'[n,t] - mn) / scale), 0, 15)
+ *     dequantised key = bf16(fma(code, scale, mn))               (fp32, RNE)
+ * each step the IEEE fp32 operation written (rint rounds half to even).
+ *   codes   [B][Hkv][T][ldq] bytes: token n of row t in byte n/2, the even
+ *           token in the low nibble; ldq >= think_q4_ld(N), a multiple of 64.
+ *   groups  [B][Hkv][ldq/64][T2][2] fp32 (scale, mn) per 128-token group,
+ *           T2 = T rounded up to even (the pad row is zero);
+ *           think_q4_groups_bytes(B, Hkv, ldq*2, T) bytes.
+ * bf16 only.  Token columns past N in the last group get code 0. */
+int64_t think_q4_ld(int64_t N);   /* bytes per codes row: 64 per 128 tokens; -1 if N < 0 */
+size_t think_q4_groups_bytes(int B, int Hkv, int64_t N, int T);
+/* Quantise the bf16 thinner cache k_pruned (layout of think_compact_keys,
+ * pitch ldk) into codes and group parameters.  One launch. */
+think_status_t think_quantize_keys_q4(const void *k_pruned, int64_t ldk, int B, int Hkv, int64_t N, int T,
+                                      uint8_t *codes, int64_t ldq, float *groups, void *stream);
+/* think_pruned_decode_attn over the 4-bit thinner cache: the keys are the
+ * dequantised values above; q, v bf16; everything else (layouts, scale,
+ * workspace of think_decode_workspace_size(..., THINK_BF16), status bits) as
+ * there.  One launch. */
+think_status_t think_pruned_decode_attn_q4(const void *q, const uint8_t *codes, int64_t ldq,
+                                           const float *groups, const void *v, const int64_t v_strides[3],
+                                           const int32_t *idx, int B, int Hq, int Hkv, int64_t N, int d, int T,
+                                           float scale, float *out, void *workspace, size_t workspace_bytes,
+                                           void *stream);
 
 /* Zero a score or decode workspace (stream-ordered memset). */
 think_status_t think_workspace_init(void *workspace, size_t workspace_bytes, void *stream);

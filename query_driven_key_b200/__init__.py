@@ -38,7 +38,8 @@ EXPORTED = (
     "think_compact_keys", "think_append_keys", "think_prune", "think_decode_workspace_size",
     "think_pruned_decode_attn",
     "think_workspace_init", "think_read_device_status", "think_noalloc_scratch_bytes",
-    "think_pruned_decode_attn_noalloc",
+    "think_pruned_decode_attn_noalloc", "think_q4_ld", "think_q4_groups_bytes",
+    "think_quantize_keys_q4", "think_pruned_decode_attn_q4",
 )
 
 
@@ -69,6 +70,14 @@ def _load() -> ctypes.CDLL:
     lib.think_prune.restype = I
     lib.think_append_keys.argtypes = [P, I64P, I, I, I64, I, I, P, I, P, I64, I64, P]
     lib.think_append_keys.restype = I
+    lib.think_q4_ld.argtypes = [I64]
+    lib.think_q4_ld.restype = I64
+    lib.think_q4_groups_bytes.argtypes = [I, I, I64, I]
+    lib.think_q4_groups_bytes.restype = SZ
+    lib.think_quantize_keys_q4.argtypes = [P, I64, I, I, I64, I, P, I64, P, P]
+    lib.think_quantize_keys_q4.restype = I
+    lib.think_pruned_decode_attn_q4.argtypes = [P, P, I64, P, P, I64P, P, I, I, I, I64, I, I, F, P, P, SZ, P]
+    lib.think_pruned_decode_attn_q4.restype = I
     lib.think_decode_workspace_size.argtypes = [I, I, I, I64, I, I]
     lib.think_decode_workspace_size.restype = SZ
     lib.think_pruned_decode_attn.argtypes = [P, P, I64, P, I64P, P, I, I, I, I64, I, I, I, F, P,
@@ -244,6 +253,42 @@ def think_pruned_decode_attn_noalloc(q: torch.Tensor, k_pruned: torch.Tensor, ld
            "think_pruned_decode_attn_noalloc")
 
 
+def think_q4_ld(N: int) -> int:
+    return lib.think_q4_ld(int(N))
+
+
+def think_q4_groups_bytes(B: int, Hkv: int, N: int, T: int) -> int:
+    return lib.think_q4_groups_bytes(B, Hkv, int(N), T)
+
+
+def think_quantize_keys_q4(k_pruned: torch.Tensor, ldk: int, N: int, codes: torch.Tensor, ldq: int,
+                           groups: torch.Tensor, stream=None) -> None:
+    """bf16 K' [B,Hkv,T,ldk] -> codes [B,Hkv,T,ldq] uint8 and groups (scale, mn) fp32."""
+    B, Hkv, T, _ = k_pruned.shape
+    if k_pruned.dtype != torch.bfloat16 or codes.dtype != torch.uint8 or groups.dtype != torch.float32:
+        raise ThinkError(THINK_ERR_INVALID_ARG, "think_quantize_keys_q4")
+    _check(lib.think_quantize_keys_q4(_ptr(k_pruned), int(ldk), B, Hkv, int(N), T, _ptr(codes), int(ldq),
+                                      _ptr(groups), _stream(stream)), "think_quantize_keys_q4")
+
+
+def think_pruned_decode_attn_q4(q: torch.Tensor, codes: torch.Tensor, ldq: int, groups: torch.Tensor,
+                                v: torch.Tensor, idx: torch.Tensor, out: torch.Tensor, workspace: torch.Tensor,
+                                N: int, scale: float | None = None, stream=None) -> None:
+    """Decode attention over the 4-bit thinner cache (keys = dequantised codes)."""
+    B, Hq, d = q.shape
+    _, Hkv, _, _ = v.shape
+    T = idx.shape[-1]
+    if scale is None:
+        scale = 1.0 / float(d) ** 0.5
+    if (not q.is_contiguous() or q.dtype != torch.bfloat16 or v.dtype != torch.bfloat16
+            or out.dtype != torch.float32 or idx.dtype != torch.int32):
+        raise ThinkError(THINK_ERR_INVALID_ARG, "think_pruned_decode_attn_q4")
+    _check(lib.think_pruned_decode_attn_q4(_ptr(q), _ptr(codes), int(ldq), _ptr(groups), _ptr(v), _strides3(v),
+                                           _ptr(idx), B, Hq, Hkv, int(N), d, T, float(scale), _ptr(out),
+                                           _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                           _stream(stream)), "think_pruned_decode_attn_q4")
+
+
 def think_workspace_init(workspace: torch.Tensor, stream=None) -> None:
     _check(lib.think_workspace_init(_ptr(workspace), workspace.numel() * workspace.element_size(),
                                     _stream(stream)), "think_workspace_init")
@@ -295,6 +340,22 @@ class PrunedCache:
         think_select_channels(self.scores, self.T, self.idx, stream)
         think_compact_keys(k, self.idx, self.k_pruned, self.ldk, stream)
         self.n = self.N
+
+    def quantize_q4(self, stream=None):
+        """Build the 4-bit thinner cache (codes, groups) from the current K' (bf16)."""
+        if not hasattr(self, "codes"):
+            self.ldq = think_q4_ld(self.capacity)
+            self.codes = torch.zeros((self.B, self.Hkv, self.T, self.ldq), dtype=torch.uint8,
+                                     device=self.k_pruned.device)
+            T2 = (self.T + 1) // 2 * 2
+            self.groups = torch.zeros((self.B, self.Hkv, self.ldq // 64, T2, 2), dtype=torch.float32,
+                                      device=self.k_pruned.device)
+        think_quantize_keys_q4(self.k_pruned, self.ldk, self.n, self.codes, self.ldq, self.groups, stream)
+
+    def decode_q4(self, q, v, out, scale=None, stream=None):
+        """Attend over the current n tokens with the 4-bit thinner cache."""
+        think_pruned_decode_attn_q4(q, self.codes, self.ldq, self.groups, v, self.idx, out, self.decode_ws,
+                                    N=self.n, scale=scale, stream=stream)
 
     def decode(self, q, v, out, scale=None, stream=None):
         """Attend over the current n tokens (v holds at least n token rows)."""

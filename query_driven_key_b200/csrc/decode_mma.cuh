@@ -82,6 +82,219 @@ __host__ __device__ inline size_t mma_smem_bytes(int T, int G, int stages)
            (size_t)2 * stages * 8 + 16 + 1024;
 }
 
+// q' = q[idx] of the group's query heads as [16 rows (g)][t_pad] bf16 (rows
+// g >= G and columns t >= T zero), by the consumer threads.
+template <int G>
+__device__ __forceinline__ void mma_stage_q(const DecodeArgs &a, unsigned char *qsm, uint32_t t_pad, int T,
+                                            int head, int b, int kv, int tid)
+{
+    const __nv_bfloat16 *q = reinterpret_cast<const __nv_bfloat16 *>(a.q);
+    const int32_t *ih = a.idx + (int64_t)head * T;
+    __nv_bfloat16 *qs = reinterpret_cast<__nv_bfloat16 *>(qsm);
+    for (int i = tid; i < 16 * (int)t_pad; i += kConsumerThreads) {
+        const int g = i / (int)t_pad, t = i % (int)t_pad;
+        __nv_bfloat16 x = __float2bfloat16(0.f);
+        if (g < G && t < T) {
+            const int c = ih[t];
+            if ((unsigned)c < (unsigned)kD) x = q[((int64_t)b * a.Hq + (int64_t)kv * G + g) * kD + c];
+        }
+        qs[g * t_pad + t] = x;
+    }
+}
+
+// q' as the B operand of the logits MMA (k = channel, n = query head): per
+// 16-channel step two registers, channels 2*q4, 2*q4+1 and +8 of head r8.
+__device__ __forceinline__ void mma_load_qb(const unsigned char *qsm, uint32_t t_pad, int lane,
+                                            uint32_t (&qb)[kD / 16][2])
+{
+    const int q4 = lane & 3, r8 = lane >> 2;
+    const int ksteps = (int)(t_pad / 16u);
+    const uint32_t *qs32 = reinterpret_cast<const uint32_t *>(qsm);
+#pragma unroll
+    for (int ks = 0; ks < kD / 16; ++ks) {
+        if (ks < ksteps) {
+            qb[ks][0] = qs32[(r8 * t_pad + 16 * ks + 2 * q4) >> 1];
+            qb[ks][1] = qs32[(r8 * t_pad + 16 * ks + 8 + 2 * q4) >> 1];
+        } else {
+            qb[ks][0] = qb[ks][1] = 0u;
+        }
+    }
+}
+
+// Online-softmax state of one consumer warp: running max (log2 units) and sum
+// for query heads 2*q4, 2*q4+1, and O^T (channel rows 16*md + r8 (+8), head
+// columns 2*q4 (+1)).
+struct MmaState {
+    float m[2], l[2];
+    float acc[8][4];
+};
+
+// One 128-token tile for one consumer warp (its 32 tokens): logits from the
+// K' tile (two 64-token halves of t_pad channel rows x 128 B, 128-byte
+// swizzle, starting at kbase), online softmax, values from the V tile (two
+// 64-channel halves of 128 tokens x 128 B, swizzled, at vbase).
+__device__ __forceinline__ void mma_tile(uint32_t kbase, uint32_t k_half, uint32_t vbase,
+                                         const uint32_t (&qb)[kD / 16][2], int ksteps, int warp, int lane,
+                                         int64_t tok_base, int64_t N, float scale_log2, MmaState &S)
+{
+    constexpr int KS_MAX = kD / 16;
+    const int q4 = lane & 3, r8 = lane >> 2;
+    const int jm = lane >> 3, jr = lane & 7;  // ldmatrix: matrix index, row within it
+
+    // ---- logits for this warp's 32 tokens: two 16-token m-tiles
+    float sc[2][4];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sc[mt][e] = 0.f;
+        const int tok = warp * 32 + mt * 16 + (jm & 1) * 8;   // first token of this lane's 8x8 block
+        const uint32_t kh = kbase + (uint32_t)(tok >> 6) * k_half;
+        const uint32_t chunk = (uint32_t)((tok & 63) >> 3);
+#pragma unroll
+        for (int ks = 0; ks < KS_MAX; ++ks) {
+            if (ks < ksteps) {
+                const uint32_t t = (uint32_t)(16 * ks + (jm >> 1) * 8 + jr);
+                uint32_t a0, a1, a2, a3;
+                wmma16::ldsm_x4_trans(kh + t * 128u + ((chunk ^ (t & 7u)) << 4), a0, a1, a2, a3);
+                wmma16::mma_bf16(sc[mt], a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+            }
+        }
+    }
+    // ---- online softmax per query head over the warp's 32 tokens
+    // sc[mt][0..1]: token 16*mt + r8, heads 2*q4, 2*q4+1; sc[mt][2..3]: token +8
+    float alpha[2];
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+        float xm = -INFINITY;
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                const int64_t n = tok_base + mt * 16 + hr * 8 + r8;
+                const float x = (n < N) ? sc[mt][hr * 2 + h2] * scale_log2 : -INFINITY;
+                sc[mt][hr * 2 + h2] = x;
+                xm = fmaxf(xm, x);
+            }
+        xm = fmaxf(xm, __shfl_xor_sync(0xffffffffu, xm, 4));
+        xm = fmaxf(xm, __shfl_xor_sync(0xffffffffu, xm, 8));
+        xm = fmaxf(xm, __shfl_xor_sync(0xffffffffu, xm, 16));
+        const float mnew = fmaxf(S.m[h2], xm);
+        alpha[h2] = (S.m[h2] == mnew) ? 1.f : exp2_approx(S.m[h2] - mnew);
+        float ps = 0.f;
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                const float x = sc[mt][hr * 2 + h2];
+                const float p = (x == -INFINITY) ? 0.f : exp2_approx(x - mnew);
+                sc[mt][hr * 2 + h2] = p;
+                ps += p;
+            }
+        S.l[h2] = fmaf(S.l[h2], alpha[h2], ps);
+        S.m[h2] = mnew;
+    }
+#pragma unroll
+    for (int md = 0; md < 8; ++md) {
+        S.acc[md][0] *= alpha[0];
+        S.acc[md][1] *= alpha[1];
+        S.acc[md][2] *= alpha[0];
+        S.acc[md][3] *= alpha[1];
+    }
+    // ---- weights as the B operand of the values MMA (k = token, n = head),
+    // high and low bf16 parts; one 16-token k-step per logits m-tile
+    uint32_t pbh[2][2], pbl[2][2];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+            const float p0 = sc[mt][hr * 2], p1 = sc[mt][hr * 2 + 1];
+            const uint32_t hi = wmma16::pack_bf16x2(p0, p1);
+            const float h0 = __uint_as_float(hi << 16), h1 = __uint_as_float(hi & 0xffff0000u);
+            const uint32_t lo = wmma16::pack_bf16x2(p0 - h0, p1 - h1);
+            pbh[mt][hr] = wmma16::movmatrix_trans(hi);
+            pbl[mt][hr] = wmma16::movmatrix_trans(lo);
+        }
+    // ---- values: O^T[c][g] += V^T[c][tok] P^T[tok][g] over the 32 tokens
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+        const uint32_t tok = (uint32_t)(warp * 32 + ks * 16 + (jm >> 1) * 8 + jr);
+#pragma unroll
+        for (int md = 0; md < 8; ++md) {
+            const uint32_t c0 = (uint32_t)(md * 16 + (jm & 1) * 8);   // first channel of the block
+            const uint32_t addr = vbase + (c0 >> 6) * 16384u + tok * 128u +
+                                  ((((c0 & 63u) >> 3) ^ (tok & 7u)) << 4);
+            uint32_t a0, a1, a2, a3;
+            wmma16::ldsm_x4_trans(addr, a0, a1, a2, a3);
+            wmma16::mma_bf16(S.acc[md], a0, a1, a2, a3, pbh[ks][0], pbh[ks][1]);
+            wmma16::mma_bf16(S.acc[md], a0, a1, a2, a3, pbl[ks][0], pbl[ks][1]);
+        }
+    }
+    (void)q4;
+}
+
+// Merge the four consumer warps of the block (through mo/mml in shared
+// memory), then the split merge (finish_split, which reuses `scratch`).
+template <int G>
+__device__ __forceinline__ void mma_merge_and_finish(const DecodeArgs &a, MmaState &S, float *mo, float *mml,
+                                                     float *scratch, unsigned *flag, int head, int split,
+                                                     int b, int kv, int tid)
+{
+    const int warp = tid >> 5, lane = tid & 31;
+    const int q4 = lane & 3, r8 = lane >> 2;
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+        S.l[h2] += __shfl_xor_sync(0xffffffffu, S.l[h2], 4);
+        S.l[h2] += __shfl_xor_sync(0xffffffffu, S.l[h2], 8);
+        S.l[h2] += __shfl_xor_sync(0xffffffffu, S.l[h2], 16);
+    }
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+        const int g = 2 * q4 + h2;
+        if (g < G) {
+#pragma unroll
+            for (int md = 0; md < 8; ++md) {
+                mo[(warp * G + g) * kD + md * 16 + r8] = S.acc[md][h2];
+                mo[(warp * G + g) * kD + md * 16 + 8 + r8] = S.acc[md][2 + h2];
+            }
+            if (r8 == 0) {
+                mml[(warp * G + g) * 2] = S.m[h2];
+                mml[(warp * G + g) * 2 + 1] = S.l[h2];
+            }
+        }
+    }
+    named_barrier(1, kConsumerThreads);
+    const int d = tid;  // 0..127: one output channel per consumer thread
+    float O[G], M[G], Lsum[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        M[g] = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) M[g] = fmaxf(M[g], mml[(w * G + g) * 2]);
+        O[g] = 0.f;
+        Lsum[g] = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) {
+            const float mw = mml[(w * G + g) * 2];
+            if (mw == -INFINITY) continue;
+            const float sw = exp2_approx(mw - M[g]);
+            O[g] = fmaf(mo[(w * G + g) * kD + d], sw, O[g]);
+            Lsum[g] = fmaf(mml[(w * G + g) * 2 + 1], sw, Lsum[g]);
+        }
+    }
+    named_barrier(1, kConsumerThreads);  // the split merge below reuses stage memory
+    finish_split<G, kConsumerThreads>(a, head, split, b, kv, d, O, M, Lsum, scratch, flag, 1);
+}
+
+__device__ __forceinline__ void mma_state_init(MmaState &S)
+{
+    S.m[0] = S.m[1] = -INFINITY;
+    S.l[0] = S.l[1] = 0.f;
+#pragma unroll
+    for (int md = 0; md < 8; ++md)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) S.acc[md][e] = 0.f;
+}
+
 template <int G>
 __global__ void __launch_bounds__(kDecodeThreads)
     pruned_decode_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
@@ -164,51 +377,15 @@ __global__ void __launch_bounds__(kDecodeThreads)
             *reinterpret_cast<uint4 *>(smem + (hs >> 1) * L.stage + (hs & 1u) * L.k_half +
                                        (uint32_t)T * 128u + o * 16u) = make_uint4(0, 0, 0, 0);
         }
-        const __nv_bfloat16 *q = reinterpret_cast<const __nv_bfloat16 *>(a.q);
-        const int32_t *ih = a.idx + (int64_t)head * T;
-        __nv_bfloat16 *qs = reinterpret_cast<__nv_bfloat16 *>(qsm);
-        for (int i = tid; i < 16 * (int)L.t_pad; i += kConsumerThreads) {
-            const int g = i / (int)L.t_pad, t = i % (int)L.t_pad;
-            __nv_bfloat16 x = __float2bfloat16(0.f);
-            if (g < G && t < T) {
-                const int c = ih[t];
-                if ((unsigned)c < (unsigned)kD) x = q[((int64_t)b * a.Hq + (int64_t)kv * G + g) * kD + c];
-            }
-            qs[g * L.t_pad + t] = x;
-        }
+        mma_stage_q<G>(a, qsm, L.t_pad, T, head, b, kv, tid);
     }
     named_barrier(1, kConsumerThreads);  // zeroed rows and q' visible to all consumers
 
-    const int q4 = lane & 3;   // accumulator column pair: query heads 2*q4, 2*q4+1
-    const int r8 = lane >> 2;  // accumulator row within an 8-row half
-    // q' as the B operand (k = channel, n = query head): per 16-channel step two
-    // registers: channels 2*q4, 2*q4+1 and +8 of query head r8.
-    constexpr int KS_MAX = kD / 16;
-    uint32_t qb[KS_MAX][2];
+    uint32_t qb[kD / 16][2];
+    mma_load_qb(qsm, L.t_pad, lane, qb);
     const int ksteps = (int)(L.t_pad / 16u);
-    {
-        const uint32_t *qs32 = reinterpret_cast<const uint32_t *>(qsm);
-#pragma unroll
-        for (int ks = 0; ks < KS_MAX; ++ks) {
-            if (ks < ksteps) {
-                qb[ks][0] = qs32[(r8 * L.t_pad + 16 * ks + 2 * q4) >> 1];
-                qb[ks][1] = qs32[(r8 * L.t_pad + 16 * ks + 8 + 2 * q4) >> 1];
-            } else {
-                qb[ks][0] = qb[ks][1] = 0u;
-            }
-        }
-    }
-
-    float m[2], l[2];          // running max (log2 units) and sum for heads 2*q4, 2*q4+1
-    float acc[8][4];           // O^T: channel rows 16*md + r8 (+8), head columns 2*q4 (+1)
-    m[0] = m[1] = -INFINITY;
-    l[0] = l[1] = 0.f;
-#pragma unroll
-    for (int md = 0; md < 8; ++md)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[md][e] = 0.f;
-
-    const int jm = lane >> 3, jr = lane & 7;  // ldmatrix: matrix index, row within it
+    MmaState S;
+    mma_state_init(S);
     const uint32_t sbase = smem_addr(smem);
 
     for (int it = 0; it < ntiles; ++it) {
@@ -217,144 +394,11 @@ __global__ void __launch_bounds__(kDecodeThreads)
             break;
         const uint32_t st = sbase + (uint32_t)s * L.stage;
         const int64_t tok_base = (tile0 + it) * kBN + warp * 32;
-
-        // ---- logits for this warp's 32 tokens: two 16-token m-tiles
-        float sc[2][4];
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) sc[mt][e] = 0.f;
-            const int tok = warp * 32 + mt * 16 + (jm & 1) * 8;   // first token of this lane's 8x8 block
-            const uint32_t kh = st + (uint32_t)(tok >> 6) * L.k_half;
-            const uint32_t chunk = (uint32_t)((tok & 63) >> 3);
-#pragma unroll
-            for (int ks = 0; ks < KS_MAX; ++ks) {
-                if (ks < ksteps) {
-                    const uint32_t t = (uint32_t)(16 * ks + (jm >> 1) * 8 + jr);
-                    uint32_t a0, a1, a2, a3;
-                    wmma16::ldsm_x4_trans(kh + t * 128u + ((chunk ^ (t & 7u)) << 4), a0, a1, a2, a3);
-                    wmma16::mma_bf16(sc[mt], a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
-                }
-            }
-        }
-        // ---- online softmax per query head over the warp's 32 tokens
-        // sc[mt][0..1]: token 16*mt + r8, heads 2*q4, 2*q4+1; sc[mt][2..3]: token +8
-        float alpha[2];
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-            float xm = -INFINITY;
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-                for (int hr = 0; hr < 2; ++hr) {
-                    const int64_t n = tok_base + mt * 16 + hr * 8 + r8;
-                    const float x = (n < a.N) ? sc[mt][hr * 2 + h2] * a.scale_log2 : -INFINITY;
-                    sc[mt][hr * 2 + h2] = x;
-                    xm = fmaxf(xm, x);
-                }
-            xm = fmaxf(xm, __shfl_xor_sync(0xffffffffu, xm, 4));
-            xm = fmaxf(xm, __shfl_xor_sync(0xffffffffu, xm, 8));
-            xm = fmaxf(xm, __shfl_xor_sync(0xffffffffu, xm, 16));
-            const float mnew = fmaxf(m[h2], xm);
-            alpha[h2] = (m[h2] == mnew) ? 1.f : exp2_approx(m[h2] - mnew);
-            float ps = 0.f;
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-                for (int hr = 0; hr < 2; ++hr) {
-                    const float x = sc[mt][hr * 2 + h2];
-                    const float p = (x == -INFINITY) ? 0.f : exp2_approx(x - mnew);
-                    sc[mt][hr * 2 + h2] = p;
-                    ps += p;
-                }
-            l[h2] = fmaf(l[h2], alpha[h2], ps);
-            m[h2] = mnew;
-        }
-#pragma unroll
-        for (int md = 0; md < 8; ++md) {
-            acc[md][0] *= alpha[0];
-            acc[md][1] *= alpha[1];
-            acc[md][2] *= alpha[0];
-            acc[md][3] *= alpha[1];
-        }
-        // ---- weights as the B operand of the values MMA (k = token, n = head),
-        // high and low bf16 parts; one 16-token k-step per logits m-tile
-        uint32_t pbh[2][2], pbl[2][2];
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-            for (int hr = 0; hr < 2; ++hr) {
-                const float p0 = sc[mt][hr * 2], p1 = sc[mt][hr * 2 + 1];
-                const uint32_t hi = wmma16::pack_bf16x2(p0, p1);
-                const float h0 = __uint_as_float(hi << 16), h1 = __uint_as_float(hi & 0xffff0000u);
-                const uint32_t lo = wmma16::pack_bf16x2(p0 - h0, p1 - h1);
-                pbh[mt][hr] = wmma16::movmatrix_trans(hi);
-                pbl[mt][hr] = wmma16::movmatrix_trans(lo);
-            }
-        // ---- values: O^T[c][g] += V^T[c][tok] P^T[tok][g] over the 32 tokens
-        const uint32_t vb = st + L.v_off;
-#pragma unroll
-        for (int ks = 0; ks < 2; ++ks) {
-            const uint32_t tok = (uint32_t)(warp * 32 + ks * 16 + (jm >> 1) * 8 + jr);
-#pragma unroll
-            for (int md = 0; md < 8; ++md) {
-                const uint32_t c0 = (uint32_t)(md * 16 + (jm & 1) * 8);   // first channel of the block
-                const uint32_t addr = vb + (c0 >> 6) * 16384u + tok * 128u +
-                                      ((((c0 & 63u) >> 3) ^ (tok & 7u)) << 4);
-                uint32_t a0, a1, a2, a3;
-                wmma16::ldsm_x4_trans(addr, a0, a1, a2, a3);
-                wmma16::mma_bf16(acc[md], a0, a1, a2, a3, pbh[ks][0], pbh[ks][1]);
-                wmma16::mma_bf16(acc[md], a0, a1, a2, a3, pbl[ks][0], pbl[ks][1]);
-            }
-        }
+        mma_tile(st, L.k_half, st + L.v_off, qb, ksteps, warp, lane, tok_base, a.N, a.scale_log2, S);
         __syncwarp();
         if (lane == 0) mbar_arrive(empty0 + 8 * s);
     }
-
-    // ------------------------------------------- merge the four warps
-#pragma unroll
-    for (int h2 = 0; h2 < 2; ++h2) {
-        l[h2] += __shfl_xor_sync(0xffffffffu, l[h2], 4);
-        l[h2] += __shfl_xor_sync(0xffffffffu, l[h2], 8);
-        l[h2] += __shfl_xor_sync(0xffffffffu, l[h2], 16);
-    }
-#pragma unroll
-    for (int h2 = 0; h2 < 2; ++h2) {
-        const int g = 2 * q4 + h2;
-        if (g < G) {
-#pragma unroll
-            for (int md = 0; md < 8; ++md) {
-                mo[(warp * G + g) * kD + md * 16 + r8] = acc[md][h2];
-                mo[(warp * G + g) * kD + md * 16 + 8 + r8] = acc[md][2 + h2];
-            }
-            if (r8 == 0) {
-                mml[(warp * G + g) * 2] = m[h2];
-                mml[(warp * G + g) * 2 + 1] = l[h2];
-            }
-        }
-    }
-    named_barrier(1, kConsumerThreads);
-    const int d = tid;  // 0..127: one output channel per consumer thread
-    float O[G], M[G], Lsum[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-        M[g] = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) M[g] = fmaxf(M[g], mml[(w * G + g) * 2]);
-        O[g] = 0.f;
-        Lsum[g] = 0.f;
-#pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) {
-            const float mw = mml[(w * G + g) * 2];
-            if (mw == -INFINITY) continue;
-            const float sw = exp2_approx(mw - M[g]);
-            O[g] = fmaf(mo[(w * G + g) * kD + d], sw, O[g]);
-            Lsum[g] = fmaf(mml[(w * G + g) * 2 + 1], sw, Lsum[g]);
-        }
-    }
-    named_barrier(1, kConsumerThreads);  // the split merge below reuses stage memory
-    finish_split<G, kConsumerThreads>(a, head, split, b, kv, d, O, M, Lsum, reinterpret_cast<float *>(smem),
-                                      flag, 1);
+    mma_merge_and_finish<G>(a, S, mo, mml, reinterpret_cast<float *>(smem), flag, head, split, b, kv, tid);
 }
 
 }  // namespace think

@@ -14,6 +14,7 @@
 
 #include "decode_kernels.cuh"
 #include "decode_mma.cuh"
+#include "decode_q4.cuh"
 #include "decode_tc.cuh"
 #include "prune_fused.cuh"
 #include "prune_kernels.cuh"
@@ -186,6 +187,22 @@ bool make_map_4d(CUtensorMap *m, think_dtype_t dt, const void *base, uint64_t dx
                           swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+// 4-D map of any element type with byte strides; box (bx, by, 1, 1), no swizzle.
+bool make_map_raw_4d(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t dx, uint64_t dy,
+                     uint64_t dz, uint64_t dw, uint64_t sy_bytes, uint64_t sz_bytes, uint64_t sw_bytes,
+                     uint32_t bx, uint32_t by)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {dx, dy, dz, dw};
+    cuuint64_t strides[3] = {sy_bytes, sz_bytes, sw_bytes};
+    cuuint32_t box[4] = {bx, by, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(m, dt, 4, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // ---------------------------------------------------------- validation --
@@ -472,6 +489,56 @@ think_status_t launch_decode_mma(int G, const CUtensorMap &mk, const CUtensorMap
     case 2: return launch_decode_mma_g<2>(mk, mv, a, bytes, heads, st);
     case 4: return launch_decode_mma_g<4>(mk, mv, a, bytes, heads, st);
     case 8: return launch_decode_mma_g<8>(mk, mv, a, bytes, heads, st);
+    default: return THINK_ERR_UNSUPPORTED;
+    }
+}
+
+// ------------------------------------------------------------ 4-bit K' --
+
+MmaPlan plan_decode_q4(int T, int G, int64_t heads, int64_t N)
+{
+    MmaPlan p;
+    const size_t per_block_2 = kSmemPerSM / 2 - kSmemReservedPerBlock;
+    const int pref_bps = decode_fill(heads, N, 1) >= 0.95 ? 1 : 2;
+    const int max_bps = env_int("THINK_DECODE_BLOCKS_PER_SM", pref_bps, 1, 2);
+    const int max_st = env_int("THINK_DECODE_STAGES", 6, 2, 6);
+    for (int bps = max_bps; bps >= 1; --bps)
+        for (int st = max_st; st >= 2; --st) {
+            const size_t bytes = q4_smem_bytes(T, G, st);
+            if (bytes <= (bps == 2 ? per_block_2 : kSmemPerBlockMax)) {
+                p.stages = st;
+                p.blocks_per_sm = bps;
+                p.bytes = bytes;
+                return p;
+            }
+        }
+    p.stages = 0;
+    p.blocks_per_sm = 1;
+    p.bytes = 0;
+    return p;
+}
+
+template <int G>
+think_status_t launch_decode_q4_g(const CUtensorMap &mc, const CUtensorMap &mg, const CUtensorMap &mv,
+                                  const DecodeArgs &a, size_t bytes, int heads, cudaStream_t st)
+{
+    auto kern = pruned_decode_q4_kernel<G>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+        cudaSuccess)
+        return THINK_ERR_CUDA;
+    dim3 grid(a.splits, heads);
+    kern<<<grid, kDecodeThreads, bytes, st>>>(mc, mg, mv, a);
+    return launch_status();
+}
+
+think_status_t launch_decode_q4(int G, const CUtensorMap &mc, const CUtensorMap &mg, const CUtensorMap &mv,
+                                const DecodeArgs &a, size_t bytes, int heads, cudaStream_t st)
+{
+    switch (G) {
+    case 1: return launch_decode_q4_g<1>(mc, mg, mv, a, bytes, heads, st);
+    case 2: return launch_decode_q4_g<2>(mc, mg, mv, a, bytes, heads, st);
+    case 4: return launch_decode_q4_g<4>(mc, mg, mv, a, bytes, heads, st);
+    case 8: return launch_decode_q4_g<8>(mc, mg, mv, a, bytes, heads, st);
     default: return THINK_ERR_UNSUPPORTED;
     }
 }
@@ -802,6 +869,100 @@ think_status_t think_pruned_decode_attn(const void *q, const void *k_pruned, int
     if (kind == kMma) return launch_decode_mma(G, mk, mv, a, mp.bytes, (int)heads, st);
     if (dtype == THINK_BF16) return launch_decode<__nv_bfloat16>(G, mk, mv, a, sm, (int)heads, st);
     return launch_decode<float>(G, mk, mv, a, sm, (int)heads, st);
+}
+
+int64_t think_q4_ld(int64_t N)
+{
+    if (N < 0) return -1;
+    return ceil_div(N, kQ4Group) * 64;
+}
+
+size_t think_q4_groups_bytes(int B, int Hkv, int64_t N, int T)
+{
+    if (B < 0 || Hkv < 0 || N < 0 || T < 1) return 0;
+    return (size_t)B * Hkv * (size_t)ceil_div(N, kQ4Group) * (size_t)((T + 1) & ~1) * 2 * sizeof(float);
+}
+
+think_status_t think_quantize_keys_q4(const void *k_pruned, int64_t ldk, int B, int Hkv, int64_t N, int T,
+                                      uint8_t *codes, int64_t ldq, float *groups, void *stream)
+{
+    if (B < 0 || Hkv < 0 || N < 0 || T < 1 || T > kD || ldk < N) return THINK_ERR_INVALID_ARG;
+    if (B == 0 || Hkv == 0 || N == 0) return THINK_OK;
+    if (!k_pruned || !codes || !groups) return THINK_ERR_INVALID_ARG;
+    if (ldq < think_q4_ld(N) || ldq % 64 != 0) return THINK_ERR_INVALID_ARG;
+    const int64_t heads = (int64_t)B * Hkv;
+    if (heads > 65535 || ceil_div(N, kQ4Group) > INT32_MAX) return THINK_ERR_UNSUPPORTED;
+    if (!aligned16(k_pruned) || !aligned16(codes) || !aligned16(groups) || (ldk * 2) % 16 != 0)
+        return THINK_ERR_ALIGNMENT;
+    dim3 grid((unsigned)ceil_div(N, kQ4Group), (unsigned)heads);
+    quantize_q4_kernel<<<grid, 128, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const __nv_bfloat16 *>(k_pruned), ldk, T, N, codes, ldq, reinterpret_cast<float2 *>(groups));
+    return launch_status();
+}
+
+think_status_t think_pruned_decode_attn_q4(const void *q, const uint8_t *codes, int64_t ldq,
+                                           const float *groups, const void *v, const int64_t v_strides[3],
+                                           const int32_t *idx, int B, int Hq, int Hkv, int64_t N, int d, int T,
+                                           float scale, float *out, void *workspace, size_t workspace_bytes,
+                                           void *stream)
+{
+    if (B < 0 || Hq < 0 || Hkv < 0 || N < 0 || !std::isfinite(scale)) return THINK_ERR_INVALID_ARG;
+    if (d != kD) return THINK_ERR_UNSUPPORTED;
+    if (T < 1 || T > d) return THINK_ERR_INVALID_ARG;
+    if (B == 0 || Hkv == 0) return THINK_OK;
+    if (Hq < Hkv || Hq % Hkv != 0) return THINK_ERR_INVALID_ARG;
+    const int G = Hq / Hkv;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return THINK_ERR_UNSUPPORTED;
+    if (N == 0 || ldq < think_q4_ld(N) || ldq % 64 != 0) return THINK_ERR_INVALID_ARG;
+    if (!q || !codes || !groups || !v || !v_strides || !idx || !out || !workspace)
+        return THINK_ERR_INVALID_ARG;
+    const int64_t heads = (int64_t)B * Hkv;
+    if (heads > 65535 || N > (int64_t)INT32_MAX - kBN) return THINK_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(codes) || !aligned16(groups) || !aligned16(v) || !aligned16(workspace) ||
+        !aligned16(out) || !strides_ok(v_strides, 2) || (reinterpret_cast<uintptr_t>(idx) & 3u))
+        return THINK_ERR_ALIGNMENT;
+    if (workspace_bytes < think_decode_workspace_size(B, Hq, Hkv, N, d, THINK_BF16)) return THINK_ERR_WORKSPACE;
+
+    const MmaPlan mp = plan_decode_q4(T, G, heads, N);
+    if (mp.stages == 0) return THINK_ERR_UNSUPPORTED;
+    const DecodeSplit sp = plan_decode_split(heads, N, mp.blocks_per_sm);
+    const int64_t ng = ldq / 64;
+    const uint64_t T2 = (uint64_t)((T + 1) & ~1);
+    CUtensorMap mc, mg, mv;
+    // codes: x = byte (two tokens), y = kept channel, z = KV head, w = batch; box 64 B x T
+    if (!make_map_raw_4d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, (uint64_t)ldq, (uint64_t)T, (uint64_t)Hkv,
+                         (uint64_t)B, (uint64_t)ldq, (uint64_t)T * ldq, (uint64_t)Hkv * T * ldq, 64,
+                         (uint32_t)T))
+        return THINK_ERR_CUDA;
+    // group parameters: x = (scale, mn) of the T2 rows, y = group, z = KV head, w = batch
+    if (!make_map_raw_4d(&mg, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, groups, 2 * T2, (uint64_t)ng, (uint64_t)Hkv,
+                         (uint64_t)B, 2 * T2 * 4, (uint64_t)ng * 2 * T2 * 4, (uint64_t)Hkv * ng * 2 * T2 * 4,
+                         (uint32_t)(2 * T2), 1))
+        return THINK_ERR_CUDA;
+    if (!make_map_4d(&mv, THINK_BF16, v, kD, (uint64_t)N, (uint64_t)Hkv, (uint64_t)B, v_strides[2],
+                     v_strides[1], v_strides[0], 64, kBN, true))
+        return THINK_ERR_CUDA;
+
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    const size_t slots = (size_t)heads * sp.splits * G;
+    DecodeArgs a;
+    memset(&a, 0, sizeof(a));
+    a.q = q;
+    a.idx = idx;
+    a.status = reinterpret_cast<unsigned *>(ws);
+    a.tickets = reinterpret_cast<unsigned *>(ws + kDecodeHeader);
+    a.part_o = reinterpret_cast<float *>(ws + kDecodeHeader + align_up((size_t)heads * sizeof(unsigned), 256));
+    a.out = out;
+    a.part_ml = a.part_o + slots * kD;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.T = T;
+    a.N = N;
+    a.tiles_per_split = sp.tiles_per_split;
+    a.splits = sp.splits;
+    a.stages = mp.stages;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    return launch_decode_q4(G, mc, mg, mv, a, mp.bytes, (int)heads, static_cast<cudaStream_t>(stream));
 }
 
 think_status_t think_workspace_init(void *workspace, size_t workspace_bytes, void *stream)

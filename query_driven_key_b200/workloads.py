@@ -128,6 +128,15 @@ def decode_bytes(w: Workload, T: int) -> int:
             + w.B * w.Hq * w.d * 4 + heads * T * 4)
 
 
+def decode_bytes_q4(w: Workload, T: int) -> int:
+    """Algorithmic HBM bytes of one decode step over the 4-bit thinner cache:
+    codes (half a byte per kept element) + group parameters (8 bytes per kept
+    channel and 128 tokens) + V + q + out(fp32) + idx."""
+    heads = w.B * w.Hkv
+    return (heads * w.N * T // 2 + heads * (-(-w.N // 128)) * T * 8 + heads * w.N * w.d * 2
+            + w.B * w.Hq * w.d * 2 + w.B * w.Hq * w.d * 4 + heads * T * 4)
+
+
 def prune_bytes(w: Workload, T: int, k_reads: int = 1) -> int:
     """Algorithmic HBM bytes of one prune pass: K read k_reads times + K' written +
     Q_win read + idx written."""

@@ -133,6 +133,37 @@ def test_append_validation():
     assert f(FAKE, s, 1, 2, 0, 128, 1, FAKE, 10, FAKE, 64, 64, None) == qdk.THINK_OK              # nothing to append
 
 
+def test_q4_sizes_and_validation():
+    assert qdk.think_q4_ld(0) == 0 and qdk.think_q4_ld(1) == 64 and qdk.think_q4_ld(128) == 64
+    assert qdk.think_q4_ld(129) == 128 and qdk.think_q4_ld(-1) == -1
+    assert qdk.think_q4_groups_bytes(2, 8, 131072, 51) == 2 * 8 * 1024 * 52 * 8
+    f = lib.think_quantize_keys_q4
+    # (k_pruned, ldk, B, Hkv, N, T, codes, ldq, groups, stream)
+    assert f(FAKE, 256, 1, 2, 200, 10, FAKE, 64, FAKE, None) == qdk.THINK_ERR_INVALID_ARG     # ldq < q4_ld(200)
+    assert f(FAKE, 256, 1, 2, 200, 10, FAKE, 160, FAKE, None) == qdk.THINK_ERR_INVALID_ARG    # not a multiple of 64
+    assert f(FAKE, 100, 1, 2, 200, 10, FAKE, 128, FAKE, None) == qdk.THINK_ERR_INVALID_ARG    # ldk < N
+    assert f(FAKE, 260, 1, 2, 200, 10, FAKE, 128, FAKE, None) == qdk.THINK_ERR_ALIGNMENT      # 520 B pitch
+    assert f(FAKE, 256, 1, 2, 200, 129, FAKE, 128, FAKE, None) == qdk.THINK_ERR_INVALID_ARG   # T > 128
+    assert f(None, 256, 1, 2, 200, 10, FAKE, 128, FAKE, None) == qdk.THINK_ERR_INVALID_ARG
+    assert f(FAKE, 256, 1, 2, 0, 10, FAKE, 0, FAKE, None) == qdk.THINK_OK                     # N == 0
+    s = I64x3(128 * 64 * 2, 128 * 64, 128)
+    g = lib.think_pruned_decode_attn_q4
+    ws = qdk.think_decode_workspace_size(1, 4, 2, 200)
+    def call(**kw):
+        a = dict(q=FAKE, codes=FAKE, ldq=128, groups=FAKE, v=FAKE, vs=s, idx=FAKE, B=1, Hq=4, Hkv=2,
+                 N=200, d=128, T=10, scale=0.088, out=FAKE, ws=FAKE, wsb=ws)
+        a.update(kw)
+        return g(*a.values(), None)
+    assert call(ldq=64) == qdk.THINK_ERR_INVALID_ARG
+    assert call(d=64) == qdk.THINK_ERR_UNSUPPORTED
+    assert call(Hq=12) == qdk.THINK_ERR_UNSUPPORTED          # G = 6
+    assert call(N=0) == qdk.THINK_ERR_INVALID_ARG
+    assert call(wsb=ws - 16) == qdk.THINK_ERR_WORKSPACE
+    assert call(codes=MISALIGNED) == qdk.THINK_ERR_ALIGNMENT
+    assert call(scale=float("nan")) == qdk.THINK_ERR_INVALID_ARG
+    assert call(B=0) == qdk.THINK_OK
+
+
 def test_decode_validation():
     s = I64x3(128 * 64 * 2, 128 * 64, 128)
     f = lib.think_pruned_decode_attn

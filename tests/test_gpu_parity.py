@@ -198,6 +198,52 @@ def test_growing_cache(dtype):
     assert qdk.think_read_device_status(cache.decode_ws) == 0
 
 
+def _q4_codes_logical(cache, N):
+    """GPU codes [B,Hkv,T,ldq] (two tokens per byte) -> [B,Hkv,N,T] uint8."""
+    c = cache.codes.cpu().numpy()
+    both = np.stack([c & 15, c >> 4], axis=-1).reshape(c.shape[:3] + (-1,))[..., :N]
+    return np.ascontiguousarray(both.transpose(0, 1, 3, 2))
+
+
+def _q4_check(cache, q_win, k, v, q, T, where):
+    B, Hkv, N, _ = k.shape
+    ora_scores, ora_idx, ora_kp = oracle.oracle_prune(f64(q_win), f64(k), T)
+    if idx_mismatch_heads(cache.idx.cpu().numpy(), ora_idx, ora_scores, T):
+        cache.idx.copy_(torch.from_numpy(ora_idx))
+        qdk.think_compact_keys(k.to(DEV), cache.idx, cache.k_pruned, cache.ldk)
+    cache.quantize_q4()
+    torch.cuda.synchronize()
+    codes, gs = oracle.oracle_quantize_q4(ora_kp)
+    assert np.array_equal(_q4_codes_logical(cache, N), codes), f"{where}: 4-bit codes differ"
+    ng = -(-N // 128)
+    gpu_gs = cache.groups[:, :, :ng, :T].cpu().numpy()
+    assert np.array_equal(gpu_gs, gs), f"{where}: group parameters differ"
+    out = torch.empty((B, q.shape[1], 128), dtype=torch.float32, device=DEV)
+    cache.decode_q4(q.to(DEV), v.to(DEV), out)
+    torch.cuda.synchronize()
+    khat = oracle.oracle_dequantize_q4(codes, gs)
+    check_out(out, oracle.oracle_decode(f64(q), khat, f64(v), ora_idx), torch.bfloat16, where=where)
+    assert qdk.think_read_device_status(cache.decode_ws) == 0
+
+
+@pytest.mark.parametrize("case", [(1, 32, 8, 20000, 51), (2, 8, 2, 1000, 64), (1, 4, 4, 130, 13),
+                                  (1, 8, 1, 5000, 128), (2, 16, 8, 257, 1), (3, 16, 8, 128, 77)])
+def test_q4_thinner_cache(case):
+    B, Hq, Hkv, N, T = case
+    q_win, k, v, q = _random_case(hash(case) & 0xFFFF, B, Hq, Hkv, N, 16, torch.bfloat16)
+    cache = _prune_gpu(q_win.to(DEV), k.to(DEV), T)
+    _q4_check(cache, q_win, k, v, q, T, str(case))
+
+
+def test_q4_long_context_full_size():
+    # the bench workload at full size: codes, parameters and one decode step
+    w = W.WORKLOADS["mistral_7b_long"]
+    T = qdk.think_t_from_lambda(w.d, w.lam)
+    q_win, k, v = W.gen_layer(w)
+    cache = _prune_gpu(q_win.to(DEV), k.to(DEV), T)
+    _q4_check(cache, q_win, k, v, W.gen_decode_q(w, 0), T, "mistral_7b_long q4")
+
+
 def test_ldk_larger_than_needed_and_exact_ties():
     # duplicate channels give exact score ties: lower index must win on both sides
     B, Hq, Hkv, N, S, T = 1, 4, 2, 300, 6, 40
