@@ -280,7 +280,7 @@ def l2_note(w, T, R):
 def decode_kernel_name(w):
     import torch
     if w.dtype == torch.bfloat16:
-        return f"pruned_decode_mma_kernel<{w.G}>"
+        return f"pruned_decode_mma_kernel<{w.G}, 4>"
     return f"pruned_decode_kernel<float, {w.G}>"
 
 

@@ -74,24 +74,24 @@ __host__ __device__ inline MmaLayout mma_layout(int T)
 }
 
 // shared memory after the stages: q' [16 rows][t_pad] bf16, per-warp merge
-// area [4 warps][G][128] + [4 warps][G][2] floats, barriers, a flag
-__host__ __device__ inline size_t mma_smem_bytes(int T, int G, int stages)
+// area [CW warps][G][128] + [CW warps][G][2] floats, barriers, a flag
+__host__ __device__ inline size_t mma_smem_bytes(int T, int G, int stages, int CW = kConsumerWarps)
 {
     const MmaLayout L = mma_layout(T);
-    return (size_t)stages * L.stage + 32u * L.t_pad + (size_t)kConsumerWarps * G * 130 * 4 +
+    return (size_t)stages * L.stage + 32u * L.t_pad + (size_t)CW * G * 130 * 4 +
            (size_t)2 * stages * 8 + 16 + 1024;
 }
 
 // q' = q[idx] of the group's query heads as [16 rows (g)][t_pad] bf16 (rows
 // g >= G and columns t >= T zero), by the consumer threads.
-template <int G>
+template <int G, int NT>
 __device__ __forceinline__ void mma_stage_q(const DecodeArgs &a, unsigned char *qsm, uint32_t t_pad, int T,
                                             int head, int b, int kv, int tid)
 {
     const __nv_bfloat16 *q = reinterpret_cast<const __nv_bfloat16 *>(a.q);
     const int32_t *ih = a.idx + (int64_t)head * T;
     __nv_bfloat16 *qs = reinterpret_cast<__nv_bfloat16 *>(qsm);
-    for (int i = tid; i < 16 * (int)t_pad; i += kConsumerThreads) {
+    for (int i = tid; i < 16 * (int)t_pad; i += NT) {
         const int g = i / (int)t_pad, t = i % (int)t_pad;
         __nv_bfloat16 x = __float2bfloat16(0.f);
         if (g < G && t < T) {
@@ -129,25 +129,28 @@ struct MmaState {
     float acc[8][4];
 };
 
-// One 128-token tile for one consumer warp (its 32 tokens): logits from the
-// K' tile (two 64-token halves of t_pad channel rows x 128 B, 128-byte
-// swizzle, starting at kbase), online softmax, values from the V tile (two
-// 64-channel halves of 128 tokens x 128 B, swizzled, at vbase).
+// One 128-token tile for one consumer warp (its TPW = 32 or 16 tokens):
+// logits from the K' tile (two 64-token halves of t_pad channel rows x 128 B,
+// 128-byte swizzle, starting at kbase), online softmax, values from the V
+// tile (two 64-channel halves of 128 tokens x 128 B, swizzled, at vbase).
+template <int TPW>
 __device__ __forceinline__ void mma_tile(uint32_t kbase, uint32_t k_half, uint32_t vbase,
                                          const uint32_t (&qb)[kD / 16][2], int ksteps, int warp, int lane,
                                          int64_t tok_base, int64_t N, float scale_log2, MmaState &S)
 {
+    static_assert(TPW == 32 || TPW == 16, "one or two 16-token m-tiles per warp");
     constexpr int KS_MAX = kD / 16;
+    constexpr int MT = TPW / 16;
     const int q4 = lane & 3, r8 = lane >> 2;
     const int jm = lane >> 3, jr = lane & 7;  // ldmatrix: matrix index, row within it
 
-    // ---- logits for this warp's 32 tokens: two 16-token m-tiles
-    float sc[2][4];
+    // ---- logits for this warp's tokens: MT 16-token m-tiles
+    float sc[MT][4];
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt) {
+    for (int mt = 0; mt < MT; ++mt) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) sc[mt][e] = 0.f;
-        const int tok = warp * 32 + mt * 16 + (jm & 1) * 8;   // first token of this lane's 8x8 block
+        const int tok = warp * TPW + mt * 16 + (jm & 1) * 8;   // first token of this lane's 8x8 block
         const uint32_t kh = kbase + (uint32_t)(tok >> 6) * k_half;
         const uint32_t chunk = (uint32_t)((tok & 63) >> 3);
 #pragma unroll
@@ -160,14 +163,14 @@ __device__ __forceinline__ void mma_tile(uint32_t kbase, uint32_t k_half, uint32
             }
         }
     }
-    // ---- online softmax per query head over the warp's 32 tokens
+    // ---- online softmax per query head over the warp's tokens
     // sc[mt][0..1]: token 16*mt + r8, heads 2*q4, 2*q4+1; sc[mt][2..3]: token +8
     float alpha[2];
 #pragma unroll
     for (int h2 = 0; h2 < 2; ++h2) {
         float xm = -INFINITY;
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
+        for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
             for (int hr = 0; hr < 2; ++hr) {
                 const int64_t n = tok_base + mt * 16 + hr * 8 + r8;
@@ -182,7 +185,7 @@ __device__ __forceinline__ void mma_tile(uint32_t kbase, uint32_t k_half, uint32
         alpha[h2] = (S.m[h2] == mnew) ? 1.f : exp2_approx(S.m[h2] - mnew);
         float ps = 0.f;
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
+        for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
             for (int hr = 0; hr < 2; ++hr) {
                 const float x = sc[mt][hr * 2 + h2];
@@ -202,9 +205,9 @@ __device__ __forceinline__ void mma_tile(uint32_t kbase, uint32_t k_half, uint32
     }
     // ---- weights as the B operand of the values MMA (k = token, n = head),
     // high and low bf16 parts; one 16-token k-step per logits m-tile
-    uint32_t pbh[2][2], pbl[2][2];
+    uint32_t pbh[MT][2], pbl[MT][2];
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
+    for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
         for (int hr = 0; hr < 2; ++hr) {
             const float p0 = sc[mt][hr * 2], p1 = sc[mt][hr * 2 + 1];
@@ -214,10 +217,10 @@ __device__ __forceinline__ void mma_tile(uint32_t kbase, uint32_t k_half, uint32
             pbh[mt][hr] = wmma16::movmatrix_trans(hi);
             pbl[mt][hr] = wmma16::movmatrix_trans(lo);
         }
-    // ---- values: O^T[c][g] += V^T[c][tok] P^T[tok][g] over the 32 tokens
+    // ---- values: O^T[c][g] += V^T[c][tok] P^T[tok][g] over the warp's tokens
 #pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
-        const uint32_t tok = (uint32_t)(warp * 32 + ks * 16 + (jm >> 1) * 8 + jr);
+    for (int ks = 0; ks < MT; ++ks) {
+        const uint32_t tok = (uint32_t)(warp * TPW + ks * 16 + (jm >> 1) * 8 + jr);
 #pragma unroll
         for (int md = 0; md < 8; ++md) {
             const uint32_t c0 = (uint32_t)(md * 16 + (jm & 1) * 8);   // first channel of the block
@@ -232,9 +235,9 @@ __device__ __forceinline__ void mma_tile(uint32_t kbase, uint32_t k_half, uint32
     (void)q4;
 }
 
-// Merge the four consumer warps of the block (through mo/mml in shared
+// Merge the CW consumer warps of the block (through mo/mml in shared
 // memory), then the split merge (finish_split, which reuses `scratch`).
-template <int G>
+template <int G, int CW>
 __device__ __forceinline__ void mma_merge_and_finish(const DecodeArgs &a, MmaState &S, float *mo, float *mml,
                                                      float *scratch, unsigned *flag, int head, int split,
                                                      int b, int kv, int tid)
@@ -262,18 +265,18 @@ __device__ __forceinline__ void mma_merge_and_finish(const DecodeArgs &a, MmaSta
             }
         }
     }
-    named_barrier(1, kConsumerThreads);
-    const int d = tid;  // 0..127: one output channel per consumer thread
+    named_barrier(1, CW * 32);
+    const int d = tid & (kD - 1);  // one output channel per thread (threads >= 128 repeat it)
     float O[G], M[G], Lsum[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
         M[g] = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) M[g] = fmaxf(M[g], mml[(w * G + g) * 2]);
+        for (int w = 0; w < CW; ++w) M[g] = fmaxf(M[g], mml[(w * G + g) * 2]);
         O[g] = 0.f;
         Lsum[g] = 0.f;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) {
+        for (int w = 0; w < CW; ++w) {
             const float mw = mml[(w * G + g) * 2];
             if (mw == -INFINITY) continue;
             const float sw = exp2_approx(mw - M[g]);
@@ -281,8 +284,8 @@ __device__ __forceinline__ void mma_merge_and_finish(const DecodeArgs &a, MmaSta
             Lsum[g] = fmaf(mml[(w * G + g) * 2 + 1], sw, Lsum[g]);
         }
     }
-    named_barrier(1, kConsumerThreads);  // the split merge below reuses stage memory
-    finish_split<G, kConsumerThreads>(a, head, split, b, kv, d, O, M, Lsum, scratch, flag, 1);
+    named_barrier(1, CW * 32);  // the split merge below reuses stage memory
+    finish_split<G, CW * 32>(a, head, split, b, kv, tid, O, M, Lsum, scratch, flag, 1);
 }
 
 __device__ __forceinline__ void mma_state_init(MmaState &S)
@@ -295,12 +298,15 @@ __device__ __forceinline__ void mma_state_init(MmaState &S)
         for (int e = 0; e < 4; ++e) S.acc[md][e] = 0.f;
 }
 
-template <int G>
-__global__ void __launch_bounds__(kDecodeThreads)
+template <int G, int CW>
+__global__ void __launch_bounds__(CW * 32 + 32)
     pruned_decode_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_v, const DecodeArgs a)
 {
     static_assert(G >= 1 && G <= 8, "the group's query heads fill at most the 8 MMA columns");
+    static_assert(CW == 4 || CW == 8, "32 or 16 tokens of a tile per consumer warp");
+    constexpr int TPW = kBN / CW;
+    constexpr int NT = CW * 32;
     extern __shared__ unsigned char smem_dyn[];
     unsigned char *smem = smem_dyn + ((1024u - (smem_addr(smem_dyn) & 1023u)) & 1023u);
 
@@ -315,9 +321,9 @@ __global__ void __launch_bounds__(kDecodeThreads)
     const int ntiles = (int)min((int64_t)a.tiles_per_split, tiles_all - tile0);
 
     unsigned char *qsm = smem + (size_t)stages * L.stage;                       // [16][t_pad] bf16
-    float *mo = reinterpret_cast<float *>(qsm + 32u * L.t_pad);                 // [warps][G][128]
-    float *mml = mo + kConsumerWarps * G * kD;                                  // [warps][G][2]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(mml + kConsumerWarps * G * 2);
+    float *mo = reinterpret_cast<float *>(qsm + 32u * L.t_pad);                 // [CW][G][128]
+    float *mml = mo + CW * G * kD;                                              // [CW][G][2]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(mml + CW * G * 2);
     unsigned *flag = reinterpret_cast<unsigned *>(bars + 2 * stages);
     const uint32_t full0 = smem_addr(bars);
     const uint32_t empty0 = smem_addr(bars + stages);
@@ -326,13 +332,13 @@ __global__ void __launch_bounds__(kDecodeThreads)
     if (tid == 0) {
         for (int s = 0; s < stages; ++s) {
             mbar_init(full0 + 8 * s, 1);
-            mbar_init(empty0 + 8 * s, kConsumerWarps);
+            mbar_init(empty0 + 8 * s, CW);
         }
         fence_barrier_init();
     }
     __syncthreads();  // barriers initialised
 
-    if (warp == kConsumerWarps) {
+    if (warp == CW) {
         // ------------------------------------------------------ producer
         if (lane == 0) {
             prefetch_tensormap(&tm_k);
@@ -372,14 +378,14 @@ __global__ void __launch_bounds__(kDecodeThreads)
     // zero, but stale bits could be NaN), and stage q' = q[idx] as [g][t] bf16.
     {
         const uint32_t pad16 = (L.t_pad - (uint32_t)T) * 8u;  // 16-byte words per half
-        for (uint32_t i = tid; i < (uint32_t)stages * 2u * pad16; i += kConsumerThreads) {
+        for (uint32_t i = tid; i < (uint32_t)stages * 2u * pad16; i += NT) {
             const uint32_t hs = i / pad16, o = i % pad16;  // hs = stage * 2 + half
             *reinterpret_cast<uint4 *>(smem + (hs >> 1) * L.stage + (hs & 1u) * L.k_half +
                                        (uint32_t)T * 128u + o * 16u) = make_uint4(0, 0, 0, 0);
         }
-        mma_stage_q<G>(a, qsm, L.t_pad, T, head, b, kv, tid);
+        mma_stage_q<G, NT>(a, qsm, L.t_pad, T, head, b, kv, tid);
     }
-    named_barrier(1, kConsumerThreads);  // zeroed rows and q' visible to all consumers
+    named_barrier(1, NT);  // zeroed rows and q' visible to all consumers
 
     uint32_t qb[kD / 16][2];
     mma_load_qb(qsm, L.t_pad, lane, qb);
@@ -393,12 +399,12 @@ __global__ void __launch_bounds__(kDecodeThreads)
         if (!mbar_wait_bounded(full0 + 8 * s, (it / stages) & 1, a.status, THINK_DEVICE_TIMEOUT_FULL))
             break;
         const uint32_t st = sbase + (uint32_t)s * L.stage;
-        const int64_t tok_base = (tile0 + it) * kBN + warp * 32;
-        mma_tile(st, L.k_half, st + L.v_off, qb, ksteps, warp, lane, tok_base, a.N, a.scale_log2, S);
+        const int64_t tok_base = (tile0 + it) * kBN + warp * TPW;
+        mma_tile<TPW>(st, L.k_half, st + L.v_off, qb, ksteps, warp, lane, tok_base, a.N, a.scale_log2, S);
         __syncwarp();
         if (lane == 0) mbar_arrive(empty0 + 8 * s);
     }
-    mma_merge_and_finish<G>(a, S, mo, mml, reinterpret_cast<float *>(smem), flag, head, split, b, kv, tid);
+    mma_merge_and_finish<G, CW>(a, S, mo, mml, reinterpret_cast<float *>(smem), flag, head, split, b, kv, tid);
 }
 
 }  // namespace think

@@ -121,21 +121,26 @@ __host__ __device__ inline Q4Layout q4_layout(int T)
 }
 
 // stages, then the bf16 tile (two halves), q' [16][t_pad] bf16, the warp merge
-// area [4][G][128] + [4][G][2] floats, barriers, a flag
-__host__ __device__ inline size_t q4_smem_bytes(int T, int G, int stages)
+// area [CW][G][128] + [CW][G][2] floats, barriers, a flag
+__host__ __device__ inline size_t q4_smem_bytes(int T, int G, int stages, int CW)
 {
     const Q4Layout L = q4_layout(T);
-    return (size_t)stages * L.stage + 2u * L.k_half + 32u * L.t_pad + (size_t)kConsumerWarps * G * 130 * 4 +
+    return (size_t)stages * L.stage + 2u * L.k_half + 32u * L.t_pad + (size_t)CW * G * 130 * 4 +
            (size_t)2 * stages * 8 + 16 + 1024;
 }
 
-template <int G>
-__global__ void __launch_bounds__(kDecodeThreads)
+template <int G, int CW>
+__global__ void __launch_bounds__(CW * 32 + 32)
     pruned_decode_q4_kernel(const __grid_constant__ CUtensorMap tm_codes,
                             const __grid_constant__ CUtensorMap tm_groups,
                             const __grid_constant__ CUtensorMap tm_v, const DecodeArgs a)
 {
     static_assert(G >= 1 && G <= 8, "the group's query heads fill at most the 8 MMA columns");
+    static_assert(CW == 4 || CW == 8, "32 or 16 tokens of a tile per consumer warp");
+    constexpr int TPW = kBN / CW;        // tokens per consumer warp
+    constexpr int NT = CW * 32;
+    constexpr int PARTS = TPW / 8;       // 8-token chunks per warp and channel row
+    constexpr int RPP = 32 / PARTS;      // channel rows per pass of a warp
     extern __shared__ unsigned char smem_dyn[];
     unsigned char *smem = smem_dyn + ((1024u - (smem_addr(smem_dyn) & 1023u)) & 1023u);
 
@@ -151,9 +156,9 @@ __global__ void __launch_bounds__(kDecodeThreads)
 
     unsigned char *kbf = smem + (size_t)stages * L.stage;                        // bf16 K' tile
     unsigned char *qsm = kbf + 2u * L.k_half;                                    // [16][t_pad] bf16
-    float *mo = reinterpret_cast<float *>(qsm + 32u * L.t_pad);                  // [warps][G][128]
-    float *mml = mo + kConsumerWarps * G * kD;                                   // [warps][G][2]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(mml + kConsumerWarps * G * 2);
+    float *mo = reinterpret_cast<float *>(qsm + 32u * L.t_pad);                  // [CW][G][128]
+    float *mml = mo + CW * G * kD;                                               // [CW][G][2]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(mml + CW * G * 2);
     unsigned *flag = reinterpret_cast<unsigned *>(bars + 2 * stages);
     const uint32_t full0 = smem_addr(bars);
     const uint32_t empty0 = smem_addr(bars + stages);
@@ -162,13 +167,13 @@ __global__ void __launch_bounds__(kDecodeThreads)
     if (tid == 0) {
         for (int s = 0; s < stages; ++s) {
             mbar_init(full0 + 8 * s, 1);
-            mbar_init(empty0 + 8 * s, kConsumerWarps);
+            mbar_init(empty0 + 8 * s, CW);
         }
         fence_barrier_init();
     }
     __syncthreads();  // barriers initialised
 
-    if (warp == kConsumerWarps) {
+    if (warp == CW) {
         // ------------------------------------------------------ producer
         if (lane == 0) {
             prefetch_tensormap(&tm_codes);
@@ -208,12 +213,12 @@ __global__ void __launch_bounds__(kDecodeThreads)
     // 0..T-1 only), stage q'
     {
         const uint32_t pad16 = (L.t_pad - (uint32_t)T) * 8u;  // 16-byte words per half
-        for (uint32_t i = tid; i < 2u * pad16; i += kConsumerThreads)
+        for (uint32_t i = tid; i < 2u * pad16; i += NT)
             *reinterpret_cast<uint4 *>(kbf + (i / pad16) * L.k_half + (uint32_t)T * 128u + (i % pad16) * 16u) =
                 make_uint4(0, 0, 0, 0);
-        mma_stage_q<G>(a, qsm, L.t_pad, T, head, b, kv, tid);
+        mma_stage_q<G, NT>(a, qsm, L.t_pad, T, head, b, kv, tid);
     }
-    named_barrier(1, kConsumerThreads);
+    named_barrier(1, NT);
 
     uint32_t qb[kD / 16][2];
     mma_load_qb(qsm, L.t_pad, lane, qb);
@@ -222,31 +227,40 @@ __global__ void __launch_bounds__(kDecodeThreads)
     mma_state_init(S);
     const uint32_t sbase = smem_addr(smem);
     const uint32_t kbase = smem_addr(kbf);
-    // dequantisation: lane = 4 * rr + p handles rows t = 8 i + rr, tokens
-    // 32 * warp + 8 p .. +7 (one 16-byte chunk of the bf16 tile)
-    const int rr = lane >> 2, p = lane & 3;
-    const uint32_t dq_dst = kbase + (uint32_t)(warp >> 1) * L.k_half;
-    const uint32_t dq_chunk = (uint32_t)(4 * (warp & 1) + p);
+    // dequantisation: lane = PARTS * rr + p handles rows t = RPP i + rr, tokens
+    // TPW * warp + 8 p .. +7 (one 16-byte chunk of the bf16 tile)
+    const int rr = lane / PARTS, p = lane % PARTS;
+    const uint32_t dq_dst = kbase + (uint32_t)((TPW * warp) >> 6) * L.k_half;
+    const uint32_t dq_chunk = (uint32_t)(((TPW * warp) & 63) / 8 + p);
+    const uint32_t dq_src = (uint32_t)(TPW / 2 * warp + 4 * p);   // byte of the codes row
 
     for (int it = 0; it < ntiles; ++it) {
         const int s = it % stages;
         if (!mbar_wait_bounded(full0 + 8 * s, (it / stages) & 1, a.status, THINK_DEVICE_TIMEOUT_FULL))
             break;
         const uint32_t st = sbase + (uint32_t)s * L.stage;
-        for (int t = rr; t < T; t += 8) {
+        for (int t = rr; t < T; t += RPP) {
             uint32_t w;
             float2 sm;
-            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w) : "r"(st + (uint32_t)t * 64u + 16u * warp + 4u * p));
+            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w) : "r"(st + (uint32_t)t * 64u + dq_src));
             asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];"
                          : "=f"(sm.x), "=f"(sm.y)
                          : "r"(st + L.meta_off + (uint32_t)t * 8u));
+            // even and odd tokens' codes, one per byte; a byte permute builds the
+            // float 2^23 + code, from which an exact subtraction gives the code;
+            // then fma(code, scale, mn) per element (packed pairs) and bf16 RNE
+            const uint32_t ev = w & 0x0F0F0F0Fu, od = (w >> 4) & 0x0F0F0F0Fu;
+            const float2 sc2 = make_float2(sm.x, sm.x), mn2 = make_float2(sm.y, sm.y);
+            const float2 bias = make_float2(-8388608.f, -8388608.f);
             uint32_t o[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                // codes 2j, 2j+1 as exact floats (2^23 + c - 2^23), then fma, then bf16
-                const float c0 = __uint_as_float(0x4B000000u | ((w >> (8 * j)) & 15u)) - 8388608.f;
-                const float c1 = __uint_as_float(0x4B000000u | ((w >> (8 * j + 4)) & 15u)) - 8388608.f;
-                o[j] = wmma16::pack_bf16x2(__fmaf_rn(c0, sm.x, sm.y), __fmaf_rn(c1, sm.x, sm.y));
+                const uint32_t sel = 0x7440u | (uint32_t)j;
+                const float2 c = __fadd2_rn(make_float2(__uint_as_float(__byte_perm(ev, 0x4B000000u, sel)),
+                                                        __uint_as_float(__byte_perm(od, 0x4B000000u, sel))),
+                                            bias);
+                const float2 y = __ffma2_rn(c, sc2, mn2);
+                o[j] = wmma16::pack_bf16x2(y.x, y.y);
             }
             const uint32_t dst = dq_dst + (uint32_t)t * 128u + ((dq_chunk ^ ((uint32_t)t & 7u)) << 4);
             asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(o[0]), "r"(o[1]), "r"(o[2]),
@@ -254,12 +268,12 @@ __global__ void __launch_bounds__(kDecodeThreads)
                          : "memory");
         }
         __syncwarp();
-        const int64_t tok_base = (tile0 + it) * kBN + warp * 32;
-        mma_tile(kbase, L.k_half, st + L.v_off, qb, ksteps, warp, lane, tok_base, a.N, a.scale_log2, S);
+        const int64_t tok_base = (tile0 + it) * kBN + warp * TPW;
+        mma_tile<TPW>(kbase, L.k_half, st + L.v_off, qb, ksteps, warp, lane, tok_base, a.N, a.scale_log2, S);
         __syncwarp();
         if (lane == 0) mbar_arrive(empty0 + 8 * s);
     }
-    mma_merge_and_finish<G>(a, S, mo, mml, reinterpret_cast<float *>(smem), flag, head, split, b, kv, tid);
+    mma_merge_and_finish<G, CW>(a, S, mo, mml, reinterpret_cast<float *>(smem), flag, head, split, b, kv, tid);
 }
 
 }  // namespace think

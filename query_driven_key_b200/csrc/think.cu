@@ -437,9 +437,11 @@ think_status_t launch_prune_fused(const void *q_win, const void *k, const int64_
 // ---------------------------------------------------- warp-MMA decode --
 
 struct MmaPlan {
-    int stages, blocks_per_sm;
+    int stages, blocks_per_sm, warps;  // warps: consumer warps per block (4 or 8)
     size_t bytes;
 };
+
+inline int consumer_warps(int dflt) { return env_int("THINK_DECODE_WARPS", dflt, 4, 8) >= 6 ? 8 : 4; }
 
 // One block per SM with up to 4 stages (the deeper ring streams faster) when
 // that keeps at least 95% of the SMs busy, else two blocks per SM.
@@ -452,9 +454,10 @@ MmaPlan plan_decode_mma(int T, int G, int64_t heads, int64_t N)
     const int pref_bps = decode_fill(heads, N, 1) >= 0.95 ? 1 : 2;
     const int max_bps = env_int("THINK_DECODE_BLOCKS_PER_SM", pref_bps, 1, 2);
     const int max_st = env_int("THINK_DECODE_STAGES", 4, 2, 4);
+    p.warps = consumer_warps(4);
     for (int bps = max_bps; bps >= 1; --bps)
         for (int st = max_st; st >= 2; --st) {
-            const size_t bytes = mma_smem_bytes(T, G, st);
+            const size_t bytes = mma_smem_bytes(T, G, st, p.warps);
             if (bytes <= (bps == 2 ? per_block_2 : kSmemPerBlockMax)) {
                 p.stages = st;
                 p.blocks_per_sm = bps;
@@ -468,43 +471,56 @@ MmaPlan plan_decode_mma(int T, int G, int64_t heads, int64_t N)
     return p;
 }
 
-template <int G>
-think_status_t launch_decode_mma_g(const CUtensorMap &mk, const CUtensorMap &mv, const DecodeArgs &a,
-                                   size_t bytes, int heads, cudaStream_t st)
+template <int G, int CW>
+think_status_t launch_decode_mma_gw(const CUtensorMap &mk, const CUtensorMap &mv, const DecodeArgs &a,
+                                    size_t bytes, int heads, cudaStream_t st)
 {
-    auto kern = pruned_decode_mma_kernel<G>;
+    auto kern = pruned_decode_mma_kernel<G, CW>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
         cudaSuccess)
         return THINK_ERR_CUDA;
     dim3 grid(a.splits, heads);
-    kern<<<grid, kDecodeThreads, bytes, st>>>(mk, mv, a);
+    kern<<<grid, CW * 32 + 32, bytes, st>>>(mk, mv, a);
     return launch_status();
 }
 
-think_status_t launch_decode_mma(int G, const CUtensorMap &mk, const CUtensorMap &mv,
+template <int G>
+think_status_t launch_decode_mma_g(int cw, const CUtensorMap &mk, const CUtensorMap &mv, const DecodeArgs &a,
+                                   size_t bytes, int heads, cudaStream_t st)
+{
+    return cw == 8 ? launch_decode_mma_gw<G, 8>(mk, mv, a, bytes, heads, st)
+                   : launch_decode_mma_gw<G, 4>(mk, mv, a, bytes, heads, st);
+}
+
+think_status_t launch_decode_mma(int G, int cw, const CUtensorMap &mk, const CUtensorMap &mv,
                                  const DecodeArgs &a, size_t bytes, int heads, cudaStream_t st)
 {
     switch (G) {
-    case 1: return launch_decode_mma_g<1>(mk, mv, a, bytes, heads, st);
-    case 2: return launch_decode_mma_g<2>(mk, mv, a, bytes, heads, st);
-    case 4: return launch_decode_mma_g<4>(mk, mv, a, bytes, heads, st);
-    case 8: return launch_decode_mma_g<8>(mk, mv, a, bytes, heads, st);
+    case 1: return launch_decode_mma_g<1>(cw, mk, mv, a, bytes, heads, st);
+    case 2: return launch_decode_mma_g<2>(cw, mk, mv, a, bytes, heads, st);
+    case 4: return launch_decode_mma_g<4>(cw, mk, mv, a, bytes, heads, st);
+    case 8: return launch_decode_mma_g<8>(cw, mk, mv, a, bytes, heads, st);
     default: return THINK_ERR_UNSUPPORTED;
     }
 }
 
 // ------------------------------------------------------------ 4-bit K' --
 
+// Two blocks per SM (eight consumer warps) first: the dequantisation makes
+// the consumers' latency, not the stream, the limit with four warps per SM
+// (long-context workload: 64 us at two blocks per SM, 94 us at one).
 MmaPlan plan_decode_q4(int T, int G, int64_t heads, int64_t N)
 {
     MmaPlan p;
+    (void)heads;
+    (void)N;
     const size_t per_block_2 = kSmemPerSM / 2 - kSmemReservedPerBlock;
-    const int pref_bps = decode_fill(heads, N, 1) >= 0.95 ? 1 : 2;
-    const int max_bps = env_int("THINK_DECODE_BLOCKS_PER_SM", pref_bps, 1, 2);
+    const int max_bps = env_int("THINK_DECODE_BLOCKS_PER_SM", 2, 1, 2);
     const int max_st = env_int("THINK_DECODE_STAGES", 6, 2, 6);
+    p.warps = consumer_warps(8);
     for (int bps = max_bps; bps >= 1; --bps)
         for (int st = max_st; st >= 2; --st) {
-            const size_t bytes = q4_smem_bytes(T, G, st);
+            const size_t bytes = q4_smem_bytes(T, G, st, p.warps);
             if (bytes <= (bps == 2 ? per_block_2 : kSmemPerBlockMax)) {
                 p.stages = st;
                 p.blocks_per_sm = bps;
@@ -518,27 +534,36 @@ MmaPlan plan_decode_q4(int T, int G, int64_t heads, int64_t N)
     return p;
 }
 
-template <int G>
-think_status_t launch_decode_q4_g(const CUtensorMap &mc, const CUtensorMap &mg, const CUtensorMap &mv,
-                                  const DecodeArgs &a, size_t bytes, int heads, cudaStream_t st)
+template <int G, int CW>
+think_status_t launch_decode_q4_gw(const CUtensorMap &mc, const CUtensorMap &mg, const CUtensorMap &mv,
+                                   const DecodeArgs &a, size_t bytes, int heads, cudaStream_t st)
 {
-    auto kern = pruned_decode_q4_kernel<G>;
+    auto kern = pruned_decode_q4_kernel<G, CW>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
         cudaSuccess)
         return THINK_ERR_CUDA;
     dim3 grid(a.splits, heads);
-    kern<<<grid, kDecodeThreads, bytes, st>>>(mc, mg, mv, a);
+    kern<<<grid, CW * 32 + 32, bytes, st>>>(mc, mg, mv, a);
     return launch_status();
 }
 
-think_status_t launch_decode_q4(int G, const CUtensorMap &mc, const CUtensorMap &mg, const CUtensorMap &mv,
-                                const DecodeArgs &a, size_t bytes, int heads, cudaStream_t st)
+template <int G>
+think_status_t launch_decode_q4_g(int cw, const CUtensorMap &mc, const CUtensorMap &mg, const CUtensorMap &mv,
+                                  const DecodeArgs &a, size_t bytes, int heads, cudaStream_t st)
+{
+    return cw == 8 ? launch_decode_q4_gw<G, 8>(mc, mg, mv, a, bytes, heads, st)
+                   : launch_decode_q4_gw<G, 4>(mc, mg, mv, a, bytes, heads, st);
+}
+
+think_status_t launch_decode_q4(int G, int cw, const CUtensorMap &mc, const CUtensorMap &mg,
+                                const CUtensorMap &mv, const DecodeArgs &a, size_t bytes, int heads,
+                                cudaStream_t st)
 {
     switch (G) {
-    case 1: return launch_decode_q4_g<1>(mc, mg, mv, a, bytes, heads, st);
-    case 2: return launch_decode_q4_g<2>(mc, mg, mv, a, bytes, heads, st);
-    case 4: return launch_decode_q4_g<4>(mc, mg, mv, a, bytes, heads, st);
-    case 8: return launch_decode_q4_g<8>(mc, mg, mv, a, bytes, heads, st);
+    case 1: return launch_decode_q4_g<1>(cw, mc, mg, mv, a, bytes, heads, st);
+    case 2: return launch_decode_q4_g<2>(cw, mc, mg, mv, a, bytes, heads, st);
+    case 4: return launch_decode_q4_g<4>(cw, mc, mg, mv, a, bytes, heads, st);
+    case 8: return launch_decode_q4_g<8>(cw, mc, mg, mv, a, bytes, heads, st);
     default: return THINK_ERR_UNSUPPORTED;
     }
 }
@@ -866,7 +891,7 @@ think_status_t think_pruned_decode_attn(const void *q, const void *k_pruned, int
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (use_tc) return launch_decode_tc(G, mk, mv, a, tp.bytes, (int)heads, st);
-    if (kind == kMma) return launch_decode_mma(G, mk, mv, a, mp.bytes, (int)heads, st);
+    if (kind == kMma) return launch_decode_mma(G, mp.warps, mk, mv, a, mp.bytes, (int)heads, st);
     if (dtype == THINK_BF16) return launch_decode<__nv_bfloat16>(G, mk, mv, a, sm, (int)heads, st);
     return launch_decode<float>(G, mk, mv, a, sm, (int)heads, st);
 }
@@ -962,7 +987,7 @@ think_status_t think_pruned_decode_attn_q4(const void *q, const uint8_t *codes, 
     a.splits = sp.splits;
     a.stages = mp.stages;
     a.scale_log2 = scale * 1.4426950408889634f;
-    return launch_decode_q4(G, mc, mg, mv, a, mp.bytes, (int)heads, static_cast<cudaStream_t>(stream));
+    return launch_decode_q4(G, mp.warps, mc, mg, mv, a, mp.bytes, (int)heads, static_cast<cudaStream_t>(stream));
 }
 
 think_status_t think_workspace_init(void *workspace, size_t workspace_bytes, void *stream)

@@ -48,5 +48,5 @@ def test_l2_note_and_kernel_name():
     w = W.WORKLOADS["mistral_7b_long"]
     note = bench.l2_note(w, _T(w), 1)
     assert "K 268 MB" in note and "K'+V 375 MB" in note
-    assert bench.decode_kernel_name(w) == "pruned_decode_mma_kernel<4>"
+    assert bench.decode_kernel_name(w) == "pruned_decode_mma_kernel<4, 4>"
     assert bench.decode_kernel_name(W.WORKLOADS["tiny_fp32"]).startswith("pruned_decode_kernel<float")

@@ -235,6 +235,16 @@ def test_q4_thinner_cache(case):
     _q4_check(cache, q_win, k, v, q, T, str(case))
 
 
+@pytest.mark.parametrize("warps", ["4", "8"])
+def test_q4_consumer_warp_variants(warps, monkeypatch):
+    monkeypatch.setenv("THINK_DECODE_WARPS", warps)
+    for case in [(1, 32, 8, 3000, 51), (2, 8, 1, 1000, 128), (1, 16, 8, 300, 1)]:
+        B, Hq, Hkv, N, T = case
+        q_win, k, v, q = _random_case(hash(case) & 0xFFFF, B, Hq, Hkv, N, 16, torch.bfloat16)
+        cache = _prune_gpu(q_win.to(DEV), k.to(DEV), T)
+        _q4_check(cache, q_win, k, v, q, T, f"{case} warps={warps}")
+
+
 def test_q4_long_context_full_size():
     # the bench workload at full size: codes, parameters and one decode step
     w = W.WORKLOADS["mistral_7b_long"]
@@ -314,16 +324,18 @@ def test_prune_schedules_give_identical_results(env, monkeypatch):
         assert np.array_equal(kp_logical(a.k_pruned, N), ora_kp)
 
 
-@pytest.mark.parametrize("kernel", ["warp_mma", "cuda_cores", "tensor_cores"])
+@pytest.mark.parametrize("kernel", ["warp_mma", "warp_mma_8_warps", "cuda_cores", "tensor_cores"])
 def test_every_bf16_decode_kernel(kernel, monkeypatch):
-    # the three bf16 decode kernels on the same inputs: warp-level mma (default),
-    # CUDA cores, tcgen05
-    monkeypatch.delenv("THINK_DECODE_TENSOR_CORES", raising=False)
-    monkeypatch.delenv("THINK_DECODE_CUDA_CORES", raising=False)
+    # the bf16 decode kernels on the same inputs: warp-level mma (default; four
+    # and eight consumer warps), CUDA cores, tcgen05
+    for key in ("THINK_DECODE_TENSOR_CORES", "THINK_DECODE_CUDA_CORES", "THINK_DECODE_WARPS"):
+        monkeypatch.delenv(key, raising=False)
     if kernel == "tensor_cores":
         monkeypatch.setenv("THINK_DECODE_TENSOR_CORES", "1")
     elif kernel == "cuda_cores":
         monkeypatch.setenv("THINK_DECODE_CUDA_CORES", "1")
+    elif kernel == "warp_mma_8_warps":
+        monkeypatch.setenv("THINK_DECODE_WARPS", "8")
     w = W.WORKLOADS["mistral_7b_long"].with_(N=20000)
     q_win, k, v = W.gen_layer(w)
     _full_path_check(w, q_win, k, v, steps=[0, 1])
