@@ -21,7 +21,9 @@ Python because they are definitions, not kernels:
   fixed kept channels and appended (a composition of ``oracle_compact``).
 
 The 4-bit thinner cache (``oracle_quantize_q4`` / ``oracle_dequantize_q4``)
-is plain C in ``think_oracle.c`` (fp32 steps as defined there).
+and the adaptive kept width (``oracle_select_adaptive``) are plain C in
+``think_oracle.c``; ``oracle_decode_ragged`` composes the per-head oracle
+calls for a kept width that differs between heads.
 
 Parity pins: every function here is pinned by ``tests/test_oracle_pins.py``
 (closed forms, brute force, library routines, a hand-worked example).
@@ -82,10 +84,12 @@ class Oracle:
         lib.oracle_dense_decode.argtypes = [P, P, P, I, I, I, I, I, D, P]
         lib.oracle_quantize_q4.argtypes = [P, I, I, I, I, I, P, P]
         lib.oracle_dequantize_q4.argtypes = [P, P, I, I, I, I, I, P]
+        lib.oracle_select_adaptive.argtypes = [P, I, I, I, D, I, I, P, P, P, I]
         lib.oracle_num_threads.restype = I
         lib.oracle_set_num_threads.argtypes = [I]
         for f in ("oracle_score", "oracle_score_explicit", "oracle_select", "oracle_compact",
-                  "oracle_decode", "oracle_dense_decode", "oracle_quantize_q4", "oracle_dequantize_q4"):
+                  "oracle_decode", "oracle_dense_decode", "oracle_quantize_q4", "oracle_dequantize_q4",
+                  "oracle_select_adaptive"):
             getattr(lib, f).restype = I
         self.lib = lib
 
@@ -183,6 +187,18 @@ class Oracle:
                "oracle_dequantize_q4")
         return out
 
+    def select_adaptive(self, scores, tau: float, T_min: int, T_max: int):
+        """scores [B,Hkv,d] -> (T_h [B,Hkv], off [B*Hkv+1], idx [total]) of the adaptive rule."""
+        scores = _f64(scores)
+        B, Hkv, d = scores.shape
+        Th = np.zeros(B * Hkv, dtype=np.int32)
+        off = np.zeros(B * Hkv + 1, dtype=np.int32)
+        idx = np.zeros(max(1, B * Hkv * T_max), dtype=np.int32)
+        rows = self.lib.oracle_select_adaptive(_ptr(scores), B, Hkv, d, float(tau), int(T_min), int(T_max),
+                                               _ptr(Th), _ptr(off), _ptr(idx), idx.size)
+        _check(min(rows, 0), "oracle_select_adaptive")
+        return Th.reshape(B, Hkv), off, idx[:rows].copy()
+
     def prune(self, q_win, k, T: int):
         """The whole prune step: scores, kept channels, thinner key cache."""
         scores = self.score(q_win, k)
@@ -261,6 +277,29 @@ def oracle_quantize_q4(kp, group: int = 128):
 
 def oracle_dequantize_q4(codes, gs, group: int = 128):
     return default_oracle().dequantize_q4(codes, gs, group)
+
+
+def oracle_select_adaptive(scores, tau, T_min, T_max):
+    return default_oracle().select_adaptive(scores, tau, T_min, T_max)
+
+
+def oracle_decode_ragged(q, k, v, Th, off, idx, scale=None):
+    """Decode with a kept width per head: each (b, h_kv) attends with its own
+    kept channels idx[off_h : off_h + T_h] (oracle_compact and oracle_decode
+    per head).  q [B,Hq,d], k, v [B,Hkv,N,d] -> out [B,Hq,d]."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, d = q.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
+    out = np.zeros((B, Hq, d))
+    for b in range(B):
+        for h in range(Hkv):
+            bh = b * Hkv + h
+            ih = np.asarray(idx[off[bh]:off[bh] + Th[b, h]], dtype=np.int32)[None, None, :]
+            kp = oracle_compact(k[b:b + 1, h:h + 1], ih)
+            out[b:b + 1, h * G:(h + 1) * G] = oracle_decode(q[b:b + 1, h * G:(h + 1) * G], kp,
+                                                             v[b:b + 1, h:h + 1], ih, scale)
+    return out
 
 
 def attention_loss(q_win_head, k_head, keep) -> float:

@@ -343,3 +343,64 @@ int oracle_dequantize_q4(const uint8_t *codes, const float *gs, int B, int Hkv, 
             }
     return 0;
 }
+
+/*
+ * Adaptive kept width per head (ThinK method section, key design 3: the
+ * pruning ratio adapts to the query and the cache; key design 2: the pruning
+ * keeps the attention-weight loss small).  Reading used here: rank the
+ * channels as oracle_select does (score descending, index ascending); with
+ * E = the sum of the squared scores taken in rank order and cum_k the sum of
+ * the first k squared scores in rank order (fp64, sequential),
+ *     T_h = the smallest k in [T_min, T_max] with cum_k >= tau * E,
+ *           T_max if there is none, T_min if E == 0;
+ * the kept channels are the first T_h in rank order, written ascending at
+ * idx[off_h .. off_h + T_h), off_h = T_0 + ... + T_{h-1} over the heads in
+ * (b, h_kv) order.  For one query head and orthogonal window queries the
+ * squared score of a channel is exactly its share of the squared attention
+ * loss, so T_h is then the fewest channels whose dropped loss^2 stays within
+ * (1 - tau) E.
+ *   scores [B][Hkv][d]; Th [B*Hkv] int32; off [B*Hkv + 1] int32 (off[B*Hkv] =
+ *   total rows); idx [total rows] int32.  Returns the total number of rows.
+ */
+int oracle_select_adaptive(const double *scores, int B, int Hkv, int d, double tau, int T_min, int T_max,
+                           int32_t *Th, int32_t *off, int32_t *idx, int idx_cap)
+{
+    if (B < 0 || Hkv < 0 || d < 1 || T_min < 1 || T_max < T_min || T_max > d) return -1;
+    if (!(tau >= 0.0 && tau <= 1.0)) return -1;
+    int *order = (int *)malloc(sizeof(int) * (size_t)d);
+    if (!order) return -2;
+    int32_t rows = 0;
+    for (int bh = 0; bh < B * Hkv; ++bh) {
+        const double *s = scores + (size_t)bh * d;
+        g_sort_scores = s;
+        for (int c = 0; c < d; ++c) order[c] = c;
+        qsort(order, (size_t)d, sizeof(int), by_score_desc);
+        double E = 0.0;
+        for (int i = 0; i < d; ++i) E += s[order[i]] * s[order[i]];
+        int T = T_max;
+        if (E == 0.0) {
+            T = T_min;
+        } else {
+            double cum = 0.0;
+            for (int k = 1; k <= T_max; ++k) {
+                cum += s[order[k - 1]] * s[order[k - 1]];
+                if (k >= T_min && cum >= tau * E) {
+                    T = k;
+                    break;
+                }
+            }
+        }
+        Th[bh] = T;
+        off[bh] = rows;
+        if (rows + T > idx_cap) {
+            free(order);
+            return -3;
+        }
+        qsort(order, (size_t)T, sizeof(int), ascending_int);
+        for (int t = 0; t < T; ++t) idx[rows + t] = order[t];
+        rows += T;
+    }
+    off[B * Hkv] = rows;
+    free(order);
+    return rows;
+}

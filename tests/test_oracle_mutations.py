@@ -24,7 +24,8 @@ MUTATIONS = {
     "group_rows_concatenated": ("s += sqrt(qn2) * sqrt(kn2[c]);", "s += qn2 * kn2[c];"),
     "tie_to_higher_index": ("    return (a > b) - (a < b);\n}\n\nstatic int ascending",
                             "    return (b > a) - (b < a);\n}\n\nstatic int ascending"),
-    "kept_list_not_reordered": ("qsort(order, (size_t)T, sizeof(int), ascending_int);", ""),
+    "kept_list_not_reordered": ("qsort(order, (size_t)T, sizeof(int), ascending_int);\n        for (int t = 0; t < T; ++t) idx[(size_t)bh * T + t]",
+                                "for (int t = 0; t < T; ++t) idx[(size_t)bh * T + t]"),
     "gather_uses_position": ("k[((size_t)bh * N + (size_t)n) * d + ih[t]];",
                              "k[((size_t)bh * N + (size_t)n) * d + t];"),
     "gather_transposed": ("k[((size_t)bh * N + (size_t)n) * d + ih[t]];",
@@ -42,6 +43,10 @@ MUTATIONS = {
     "q4_min_not_added": ("bf16_round(fmaf(c, gs[gi], gs[gi + 1]))", "bf16_round(c * gs[gi])"),
     "q4_group_index_of_next_group": ("(((size_t)bh * ng + n / group) * T + t) * 2;",
                                      "(((size_t)bh * ng + (n + 1) / group) * T + t) * 2;"),
+    "adaptive_strict_threshold": ("if (k >= T_min && cum >= tau * E) {", "if (k >= T_min && cum > tau * E) {"),
+    "adaptive_energy_unsquared": ("cum += s[order[k - 1]] * s[order[k - 1]];", "cum += s[order[k - 1]];"),
+    "adaptive_offsets_not_advanced": ("        rows += T;\n    }\n    off[B * Hkv] = rows;",
+                                      "    }\n    off[B * Hkv] = rows;"),
 }
 
 
@@ -108,6 +113,14 @@ def _pins(o: oracle.Oracle):
     khat = o.dequantize_q4(codes, gs)
     step = np.repeat(gs[..., 0], 128, axis=2)[:, :, :200].astype(np.float64)
     yield "q4_bound", bool(np.all(np.abs(khat - kr) <= 0.5 * step * (1 + 1e-5) + np.abs(khat) * 2.0 ** -8))
+    # adaptive kept width: hand-worked thresholds and ragged offsets
+    sc2 = np.array([[[3.0, 4.0, 0.0, 0.0], [1.0, 1.0, 1.0, 1.0]]])
+    ok = True
+    for tau, T0, T1 in [(0.64, 1, 3), (0.65, 2, 3), (0.26, 1, 2)]:
+        Th, off, ix = o.select_adaptive(sc2, tau, 1, 4)
+        ok &= Th.tolist() == [[T0, T1]] and list(off) == [0, T0, T0 + T1]
+        ok &= list(ix[:T0]) == ([1] if T0 == 1 else [0, 1])
+    yield "adaptive_hand", bool(ok)
 
 
 def _all_pass(o):

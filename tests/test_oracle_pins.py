@@ -437,3 +437,82 @@ def test_q4_last_group_uses_only_its_tokens():
     assert gs.shape == (1, 1, 2, 1, 2)
     assert gs[0, 0, 1, 0, 1] == 1.0 and gs[0, 0, 1, 0, 0] == np.float32(1.5) / np.float32(15)
     assert list(codes[0, 0, 128:, 0]) == [0, 15]
+
+
+# ----------------------------------------------------- adaptive kept width ---
+
+def test_adaptive_width_hand_worked():
+    # scores (3, 4, 0, 0): squared 16 and 9 of E = 25, rank order channel 1, 0
+    s = np.array([[[3.0, 4.0, 0.0, 0.0]]])
+    for tau, T, idx in [(0.5, 1, [1]), (0.64, 1, [1]), (0.65, 2, [0, 1]), (1.0, 2, [0, 1]), (0.0, 1, [1])]:
+        Th, off, ix = oracle.oracle_select_adaptive(s, tau, 1, 4)
+        assert Th[0, 0] == T and list(ix) == idx and list(off) == [0, T], (tau, Th, ix)
+    # clamps: T_min = 3 keeps the two zero channels by index; T_max = 1 caps
+    Th, _, ix = oracle.oracle_select_adaptive(s, 0.5, 3, 4)
+    assert Th[0, 0] == 3 and list(ix) == [0, 1, 2]
+    Th, _, ix = oracle.oracle_select_adaptive(s, 1.0, 1, 1)
+    assert Th[0, 0] == 1 and list(ix) == [1]
+    # all-zero scores keep T_min channels, lowest indices first
+    Th, _, ix = oracle.oracle_select_adaptive(np.zeros((1, 1, 4)), 0.9, 2, 4)
+    assert Th[0, 0] == 2 and list(ix) == [0, 1]
+
+
+def test_adaptive_width_ragged_offsets_and_monotone_in_tau():
+    r = rng(90)
+    s = np.abs(r.standard_normal((2, 3, 16))) * r.lognormal(0, 1, (2, 3, 16))
+    prev = None
+    for tau in (0.0, 0.3, 0.6, 0.9, 0.99, 1.0):
+        Th, off, ix = oracle.oracle_select_adaptive(s, tau, 2, 12)
+        assert np.all((Th >= 2) & (Th <= 12))
+        assert list(off) == [0] + list(np.cumsum(Th.ravel()))
+        for bh in range(6):
+            seg = ix[off[bh]:off[bh + 1]]
+            assert np.all(np.diff(seg) > 0)
+            # the kept channels are the top T_h of the ranking
+            order = sorted(range(16), key=lambda c: (-s.reshape(6, 16)[bh, c], c))
+            assert sorted(order[:Th.ravel()[bh]]) == list(seg)
+        if prev is not None:
+            assert np.all(Th >= prev)
+        prev = Th
+
+
+def test_adaptive_width_is_the_fewest_channels_within_the_loss_budget():
+    # one query head with orthogonal window queries: the squared attention loss
+    # of dropping a set of channels is the sum of their squared scores, so the
+    # chosen width must be the smallest subset size (over every subset, brute
+    # force) whose loss^2 is within (1 - tau) of the total
+    r = rng(91)
+    d, S, N = 8, 8, 12
+    q, _ = np.linalg.qr(r.standard_normal((S, S)))
+    q_win = (q[:, :d] * r.lognormal(0, 1, d))[None, None]
+    k = r.standard_normal((1, 1, N, d)) * r.lognormal(0, 1, (1, 1, 1, d))
+    s = oracle.oracle_score(q_win, k)
+    total = oracle.attention_loss(q_win[0, 0], k[0, 0], [])
+    for tau in (0.5, 0.8, 0.95):
+        Th, _, ix = oracle.oracle_select_adaptive(s, tau, 1, d)
+        kept_loss = oracle.attention_loss(q_win[0, 0], k[0, 0], list(ix))
+        assert kept_loss ** 2 <= (1 - tau) * total ** 2 * (1 + 1e-9)
+        best = min(T for T in range(1, d + 1)
+                   if any(oracle.attention_loss(q_win[0, 0], k[0, 0], list(c)) ** 2 <= (1 - tau) * total ** 2 * (1 + 1e-9)
+                          for c in itertools.combinations(range(d), T)))
+        assert Th[0, 0] == best, (tau, Th, best)
+
+
+def test_ragged_decode_equals_per_head_pruned_decode():
+    r = rng(92)
+    B, Hq, Hkv, N, d = 2, 4, 2, 20, 8
+    q = r.standard_normal((B, Hq, d))
+    k = r.standard_normal((B, Hkv, N, d))
+    v = r.standard_normal((B, Hkv, N, d))
+    Th = np.array([[3, 5], [8, 1]], dtype=np.int32)
+    off = np.array([0, 3, 8, 16, 17], dtype=np.int32)
+    idx = np.array([0, 4, 7, 1, 2, 3, 5, 6, 0, 1, 2, 3, 4, 5, 6, 7, 2], dtype=np.int32)
+    out = oracle.oracle_decode_ragged(q, k, v, Th, off, idx)
+    # head (1, 0) keeps every channel: dense attention for its two query heads
+    np.testing.assert_allclose(out[1, 0:2], oracle.oracle_dense_decode(q[1:2, 0:2], k[1:2, 0:1], v[1:2, 0:1])[0],
+                               rtol=1e-12, atol=1e-13)
+    # head (0, 0): masked-key SDPA with channels {0, 4, 7}
+    mask = np.zeros(d)
+    mask[[0, 4, 7]] = 1
+    np.testing.assert_allclose(out[0, 0:2], _sdpa(q[0:1, 0:2], k[0:1, 0:1] * mask, v[0:1, 0:1], 2)[0],
+                               rtol=1e-12, atol=1e-13)
