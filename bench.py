@@ -260,6 +260,39 @@ def measure_q4(w, T, stream, cache, qs_d, v_d, outs, bf16_us, peak):
             "kernel": "pruned_decode_q4_kernel (think_pruned_decode_attn_q4), not part of the step"}
 
 
+def measure_adaptive(w, dev, stream, qw_d, k_d, qs_d, v_d, outs, peak, tau=0.9, T_min=8, T_max=128):
+    """A kept width per head on the same layer, outside the timed step: prune
+    with the adaptive rule, then the step's decode calls over the ragged cache."""
+    import torch
+    import query_driven_key_b200 as qdk
+    cache = qdk.AdaptiveCache(w.B, w.Hq, w.Hkv, w.N, tau, T_min, T_max, w.d, dtype=w.dtype, device=dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    for _ in range(3):
+        cache.prune(qw_d, k_d, stream=stream)
+    e0, e1 = ev(), ev()
+    e0.record(stream)
+    cache.prune(qw_d, k_d, stream=stream)
+    e1.record(stream)
+    for s in range(3):
+        cache.decode(qs_d[s], v_d, outs[s], stream=stream)
+    e2, e3 = ev(), ev()
+    e2.record(stream)
+    for s in range(w.decode_steps):
+        cache.decode(qs_d[s], v_d, outs[s], stream=stream)
+    e3.record(stream)
+    stream.synchronize()
+    Th = cache.Th.cpu()
+    kept = int(Th.sum())
+    heads = w.B * w.Hkv
+    nbytes = (kept * w.N * 2 + heads * w.N * w.d * 2 + w.B * w.Hq * w.d * 2 + w.B * w.Hq * w.d * 4 + kept * 4)
+    us = e2.elapsed_time(e3) * 1e3 / w.decode_steps
+    return {"tau": tau, "T_min": T_min, "T_max": T_max, "T_per_head": Th.tolist(),
+            "mean_T": kept / heads, "prune_us": e0.elapsed_time(e1) * 1e3, "decode_us_per_step": us,
+            "decode_gbs": nbytes / (us * 1e-6) / 1e9, "frac_of_measured_peak": nbytes / (us * 1e-6) / 1e9 / peak,
+            "algorithmic_bytes_per_launch": nbytes,
+            "kernel": "pruned_decode_mma_kernel, ragged mode (think_pruned_decode_attn_ragged), not part of the step"}
+
+
 def data_recipe(w):
     if w.k_kind == "lowrank":
         keys = f"rank-{w.k_rank} N(0,1) factors + {w.k_noise} N(0,1) noise, LogNormal(0,{w.k_sigma}) channel scales"
@@ -486,6 +519,8 @@ def run_native(args):
     append = measure_append(w, T, dev, stream, qw_d[0], k_d[0]) if rank == 0 else None
     q4 = (measure_q4(w, T, stream, caches[0], qs_d, v_d[0], outs[:, 0], dec_us, peak)
           if rank == 0 and w.dtype == torch.bfloat16 else None)
+    adaptive = (measure_adaptive(w, dev, stream, qw_d[0], k_d[0], qs_d, v_d[0], outs[:, 0], peak)
+                if rank == 0 and w.dtype == torch.bfloat16 else None)
 
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -512,6 +547,7 @@ def run_native(args):
                      "traffic": DECODE_TRAFFIC_BYTES if default_workload(args) else None},
         "append": append,
         "q4": q4,
+        "adaptive": adaptive,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
         "e2e": e2e,

@@ -15,8 +15,9 @@
  *   think_pruned_decode_attn  out = softmax((q[idx] . K'^T) / sqrt(d)) V
  *
  * plus think_prune, the first three in two launches; think_append_keys,
- * which appends new tokens' keys to the thinner cache; and a 4-bit thinner
- * cache (think_quantize_keys_q4, think_pruned_decode_attn_q4).
+ * which appends new tokens' keys to the thinner cache; a 4-bit thinner
+ * cache (think_quantize_keys_q4, think_pruned_decode_attn_q4); and a kept
+ * width per head (think_select_adaptive and the _ragged calls).
  *
  * Conventions shared by every call
  *   - Shapes: B batch, Hq query heads, Hkv KV heads (G = Hq/Hkv query heads
@@ -258,6 +259,42 @@ think_status_t think_pruned_decode_attn_q4(const void *q, const uint8_t *codes, 
                                            const int32_t *idx, int B, int Hq, int Hkv, int64_t N, int d, int T,
                                            float scale, float *out, void *workspace, size_t workspace_bytes,
                                            void *stream);
+
+/* ------------------------------------------------- adaptive kept width --
+ * A kept width per head (ThinK method section, key design 3: the pruning
+ * ratio adapts to the query and the cache; key design 2: keep the
+ * attention-weight loss small).  Reading used here: rank a head's channels as
+ * think_select_channels does; with E the sum of the squared scores in rank
+ * order and cum_k the sum of the first k of them (fp64, sequential),
+ *     T_h = the smallest k in [T_min, T_max] with cum_k >= tau * E
+ *           (T_max if none, T_min if E == 0).
+ * Ragged layout: head h = b*Hkv + h_kv owns rows rowoff[h] .. rowoff[h] +
+ * P_h - 1 of K' and of idx, P_h = T_h rounded up to a multiple of 16;
+ * rowoff[h] = P_0 + ... + P_{h-1}, rowoff[B*Hkv] = the rows in use.  Rows
+ * T_h .. P_h - 1 of K' are zero (their idx entries are unspecified).  K' rows
+ * have pitch ldk as in think_compact_keys; allocate think_ragged_rows() rows
+ * for K' and idx.
+ *   Th      [B*Hkv] int32 output;  rowoff [B*Hkv + 1] int32 output;
+ *   idx     [rows] int32 output, each head's kept channels ascending. */
+int64_t think_ragged_rows(int B, int Hkv, int T_max);   /* B*Hkv*roundup16(T_max); -1 on bad input */
+/* One launch (one block for every head).  scores as written by
+ * think_score_channels; 0 <= tau <= 1, 1 <= T_min <= T_max <= d. */
+think_status_t think_select_adaptive(const double *scores, int B, int Hkv, int d, double tau, int T_min,
+                                     int T_max, int32_t *Th, int32_t *rowoff, int32_t *idx, void *stream);
+/* think_compact_keys for the ragged layout (writes the zero pad rows too).
+ * One launch. */
+think_status_t think_compact_keys_ragged(const void *k, const int64_t k_strides[3], int B, int Hkv, int64_t N,
+                                         int d, think_dtype_t dtype, const int32_t *idx, const int32_t *Th,
+                                         const int32_t *rowoff, int T_max, void *k_pruned, int64_t ldk,
+                                         void *stream);
+/* think_pruned_decode_attn for the ragged layout: query heads of KV head h
+ * use its T_h kept channels; bf16 only; workspace as for
+ * think_pruned_decode_attn.  One launch. */
+think_status_t think_pruned_decode_attn_ragged(const void *q, const void *k_pruned, int64_t ldk, const void *v,
+                                               const int64_t v_strides[3], const int32_t *idx,
+                                               const int32_t *Th, const int32_t *rowoff, int T_max, int B, int Hq,
+                                               int Hkv, int64_t N, int d, float scale, float *out,
+                                               void *workspace, size_t workspace_bytes, void *stream);
 
 /* Zero a score or decode workspace (stream-ordered memset). */
 think_status_t think_workspace_init(void *workspace, size_t workspace_bytes, void *stream);

@@ -39,7 +39,8 @@ EXPORTED = (
     "think_pruned_decode_attn",
     "think_workspace_init", "think_read_device_status", "think_noalloc_scratch_bytes",
     "think_pruned_decode_attn_noalloc", "think_q4_ld", "think_q4_groups_bytes",
-    "think_quantize_keys_q4", "think_pruned_decode_attn_q4",
+    "think_quantize_keys_q4", "think_pruned_decode_attn_q4", "think_ragged_rows", "think_select_adaptive",
+    "think_compact_keys_ragged", "think_pruned_decode_attn_ragged",
 )
 
 
@@ -78,6 +79,14 @@ def _load() -> ctypes.CDLL:
     lib.think_quantize_keys_q4.restype = I
     lib.think_pruned_decode_attn_q4.argtypes = [P, P, I64, P, P, I64P, P, I, I, I, I64, I, I, F, P, P, SZ, P]
     lib.think_pruned_decode_attn_q4.restype = I
+    lib.think_ragged_rows.argtypes = [I, I, I]
+    lib.think_ragged_rows.restype = I64
+    lib.think_select_adaptive.argtypes = [P, I, I, I, D, I, I, P, P, P, P]
+    lib.think_select_adaptive.restype = I
+    lib.think_compact_keys_ragged.argtypes = [P, I64P, I, I, I64, I, I, P, P, P, I, P, I64, P]
+    lib.think_compact_keys_ragged.restype = I
+    lib.think_pruned_decode_attn_ragged.argtypes = [P, P, I64, P, I64P, P, P, P, I, I, I, I, I64, I, F, P, P, SZ, P]
+    lib.think_pruned_decode_attn_ragged.restype = I
     lib.think_decode_workspace_size.argtypes = [I, I, I, I64, I, I]
     lib.think_decode_workspace_size.restype = SZ
     lib.think_pruned_decode_attn.argtypes = [P, P, I64, P, I64P, P, I, I, I, I64, I, I, I, F, P,
@@ -287,6 +296,76 @@ def think_pruned_decode_attn_q4(q: torch.Tensor, codes: torch.Tensor, ldq: int, 
                                            _ptr(idx), B, Hq, Hkv, int(N), d, T, float(scale), _ptr(out),
                                            _ptr(workspace), workspace.numel() * workspace.element_size(),
                                            _stream(stream)), "think_pruned_decode_attn_q4")
+
+
+def think_ragged_rows(B: int, Hkv: int, T_max: int) -> int:
+    return lib.think_ragged_rows(B, Hkv, T_max)
+
+
+def think_select_adaptive(scores: torch.Tensor, tau: float, T_min: int, T_max: int, Th: torch.Tensor,
+                          rowoff: torch.Tensor, idx: torch.Tensor, stream=None) -> None:
+    """scores [B,Hkv,d] fp64 -> Th [B*Hkv], rowoff [B*Hkv+1], idx [rows] (int32, ragged layout)."""
+    B, Hkv, d = scores.shape
+    _check(lib.think_select_adaptive(_ptr(scores), B, Hkv, d, float(tau), int(T_min), int(T_max), _ptr(Th),
+                                     _ptr(rowoff), _ptr(idx), _stream(stream)), "think_select_adaptive")
+
+
+def think_compact_keys_ragged(k: torch.Tensor, idx: torch.Tensor, Th: torch.Tensor, rowoff: torch.Tensor,
+                              T_max: int, k_pruned: torch.Tensor, ldk: int, stream=None) -> None:
+    B, Hkv, N, d = k.shape
+    _check(lib.think_compact_keys_ragged(_ptr(k), _strides3(k), B, Hkv, N, d, _dtype(k), _ptr(idx), _ptr(Th),
+                                         _ptr(rowoff), int(T_max), _ptr(k_pruned), int(ldk), _stream(stream)),
+           "think_compact_keys_ragged")
+
+
+def think_pruned_decode_attn_ragged(q: torch.Tensor, k_pruned: torch.Tensor, ldk: int, v: torch.Tensor,
+                                    idx: torch.Tensor, Th: torch.Tensor, rowoff: torch.Tensor, T_max: int,
+                                    out: torch.Tensor, workspace: torch.Tensor, N: int | None = None,
+                                    scale: float | None = None, stream=None) -> None:
+    B, Hq, d = q.shape
+    _, Hkv, Nv, _ = v.shape
+    N = Nv if N is None else N
+    if scale is None:
+        scale = 1.0 / float(d) ** 0.5
+    if not q.is_contiguous() or out.dtype != torch.float32:
+        raise ThinkError(THINK_ERR_INVALID_ARG, "think_pruned_decode_attn_ragged")
+    _check(lib.think_pruned_decode_attn_ragged(_ptr(q), _ptr(k_pruned), int(ldk), _ptr(v), _strides3(v), _ptr(idx),
+                                               _ptr(Th), _ptr(rowoff), int(T_max), B, Hq, Hkv, int(N), d,
+                                               float(scale), _ptr(out), _ptr(workspace),
+                                               workspace.numel() * workspace.element_size(), _stream(stream)),
+           "think_pruned_decode_attn_ragged")
+
+
+class AdaptiveCache:
+    """Device buffers of one layer pruned with a kept width per head (ragged
+    thinner K).  Allocates with torch on construction, then only calls the C
+    entry points: prune = scores, adaptive selection, ragged compaction."""
+
+    def __init__(self, B: int, Hq: int, Hkv: int, N: int, tau: float, T_min: int, T_max: int, d: int = 128,
+                 dtype: torch.dtype = torch.bfloat16, device="cuda"):
+        self.B, self.Hq, self.Hkv, self.N, self.d, self.dtype = B, Hq, Hkv, N, d, dtype
+        self.tau, self.T_min, self.T_max = tau, T_min, T_max
+        self.ldk = think_pruned_ld(N, dtype)
+        rows = think_ragged_rows(B, Hkv, T_max)
+        self.scores = torch.empty((B, Hkv, d), dtype=torch.float64, device=device)
+        self.Th = torch.empty(B * Hkv, dtype=torch.int32, device=device)
+        self.rowoff = torch.empty(B * Hkv + 1, dtype=torch.int32, device=device)
+        self.idx = torch.empty(rows, dtype=torch.int32, device=device)
+        self.k_pruned = torch.empty((rows, self.ldk), dtype=dtype, device=device)
+        self.score_ws = torch.zeros(max(256, think_score_workspace_size(B, Hq, Hkv, N, d)),
+                                    dtype=torch.uint8, device=device)
+        self.decode_ws = torch.zeros(max(256, think_decode_workspace_size(B, Hq, Hkv, N, d, dtype)),
+                                     dtype=torch.uint8, device=device)
+
+    def prune(self, q_win, k, stream=None):
+        think_score_channels(q_win, k, self.scores, self.score_ws, stream)
+        think_select_adaptive(self.scores, self.tau, self.T_min, self.T_max, self.Th, self.rowoff, self.idx,
+                              stream)
+        think_compact_keys_ragged(k, self.idx, self.Th, self.rowoff, self.T_max, self.k_pruned, self.ldk, stream)
+
+    def decode(self, q, v, out, scale=None, stream=None):
+        think_pruned_decode_attn_ragged(q, self.k_pruned, self.ldk, v, self.idx, self.Th, self.rowoff, self.T_max,
+                                        out, self.decode_ws, N=self.N, scale=scale, stream=stream)
 
 
 def think_workspace_init(workspace: torch.Tensor, stream=None) -> None:

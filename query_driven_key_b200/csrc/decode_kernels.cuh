@@ -46,6 +46,8 @@ struct DecodeArgs {
     uint32_t stage_bytes;   // bytes per ring stage (multiple of 1024)
     uint32_t v_off;         // offset of the V tile inside a stage
     uint32_t tx_bytes;      // bytes one stage's two TMA loads deliver
+    const int32_t *Th;      // kept width per head (ragged thinner cache), or null: T for all
+    const int32_t *rowoff;  // first K' row (and idx entry) of each head when Th is set
 };
 
 __device__ __forceinline__ float warp_max(float x)

@@ -86,10 +86,9 @@ __host__ __device__ inline size_t mma_smem_bytes(int T, int G, int stages, int C
 // g >= G and columns t >= T zero), by the consumer threads.
 template <int G, int NT>
 __device__ __forceinline__ void mma_stage_q(const DecodeArgs &a, unsigned char *qsm, uint32_t t_pad, int T,
-                                            int head, int b, int kv, int tid)
+                                            const int32_t *ih, int b, int kv, int tid)
 {
     const __nv_bfloat16 *q = reinterpret_cast<const __nv_bfloat16 *>(a.q);
-    const int32_t *ih = a.idx + (int64_t)head * T;
     __nv_bfloat16 *qs = reinterpret_cast<__nv_bfloat16 *>(qsm);
     for (int i = tid; i < 16 * (int)t_pad; i += NT) {
         const int g = i / (int)t_pad, t = i % (int)t_pad;
@@ -103,12 +102,12 @@ __device__ __forceinline__ void mma_stage_q(const DecodeArgs &a, unsigned char *
 }
 
 // q' as the B operand of the logits MMA (k = channel, n = query head): per
-// 16-channel step two registers, channels 2*q4, 2*q4+1 and +8 of head r8.
-__device__ __forceinline__ void mma_load_qb(const unsigned char *qsm, uint32_t t_pad, int lane,
+// 16-channel step two registers, channels 2*q4, 2*q4+1 and +8 of head r8
+// (q' rows t_pad apart; ksteps 16-channel steps used).
+__device__ __forceinline__ void mma_load_qb(const unsigned char *qsm, uint32_t t_pad, int ksteps, int lane,
                                             uint32_t (&qb)[kD / 16][2])
 {
     const int q4 = lane & 3, r8 = lane >> 2;
-    const int ksteps = (int)(t_pad / 16u);
     const uint32_t *qs32 = reinterpret_cast<const uint32_t *>(qsm);
 #pragma unroll
     for (int ks = 0; ks < kD / 16; ++ks) {
@@ -313,9 +312,18 @@ __global__ void __launch_bounds__(CW * 32 + 32)
     const int split = blockIdx.x;
     const int head = blockIdx.y;
     const int b = head / a.Hkv, kv = head % a.Hkv;
-    const int T = a.T;
+    // Ragged thinner cache (a.Th set): this head keeps Th[head] channels, its
+    // K' rows start at rowoff[head] and are padded with zero rows to a
+    // multiple of 16; the stage layout is that of the widest head (a.T).
+    const bool ragged = a.Th != nullptr;
+    const int T = ragged ? min(max(a.Th[head], 1), a.T) : a.T;
+    // rows of all heads: gridDim.y * roundup16(a.T); an offset outside it is
+    // clamped (garbage in, no access outside K' or idx)
+    const int64_t row_cap = (int64_t)gridDim.y * ((a.T + 15) & ~15);
+    const int64_t row0 = ragged ? min(max((int64_t)a.rowoff[head], (int64_t)0), row_cap - ((T + 15) & ~15)) : 0;
     const int stages = a.stages;
-    const MmaLayout L = mma_layout(T);
+    const MmaLayout L = mma_layout(a.T);
+    const uint32_t t_rows = ragged ? (uint32_t)((T + 15) & ~15) : L.t_pad;  // K' rows used
     const int64_t tile0 = (int64_t)split * a.tiles_per_split;
     const int64_t tiles_all = (a.N + kBN - 1) / kBN;
     const int ntiles = (int)min((int64_t)a.tiles_per_split, tiles_all - tile0);
@@ -343,7 +351,7 @@ __global__ void __launch_bounds__(CW * 32 + 32)
         if (lane == 0) {
             prefetch_tensormap(&tm_k);
             prefetch_tensormap(&tm_v);
-            const uint32_t tx = 2u * 64u * (uint32_t)T * 2u + 32768u;
+            const uint32_t tx = ragged ? 2u * t_rows * 128u + 32768u : 2u * 64u * (uint32_t)T * 2u + 32768u;
             int issued = 0;
             bool ok = true;
             for (int it = 0; it < ntiles; ++it) {
@@ -357,8 +365,16 @@ __global__ void __launch_bounds__(CW * 32 + 32)
                 mbar_arrive_expect_tx(full, tx);
                 const int x = (int)((tile0 + it) * kBN);
                 const uint32_t st = smem_addr(smem + (size_t)s * L.stage);
-                tma_load_4d(st, &tm_k, x, 0, kv, b, full);
-                tma_load_4d(st + L.k_half, &tm_k, x + 64, 0, kv, b, full);
+                if (ragged) {
+                    // 16-row boxes of this head's rows (its zero pad rows included)
+                    for (uint32_t j = 0; j < t_rows / 16u; ++j) {
+                        tma_load_4d(st + 2048u * j, &tm_k, x, (int)(row0 + 16 * j), 0, 0, full);
+                        tma_load_4d(st + L.k_half + 2048u * j, &tm_k, x + 64, (int)(row0 + 16 * j), 0, 0, full);
+                    }
+                } else {
+                    tma_load_4d(st, &tm_k, x, 0, kv, b, full);
+                    tma_load_4d(st + L.k_half, &tm_k, x + 64, 0, kv, b, full);
+                }
                 tma_load_4d(st + L.v_off, &tm_v, 0, x, kv, b, full);
                 tma_load_4d(st + L.v_off + 16384u, &tm_v, 64, x, kv, b, full);
                 ++issued;
@@ -377,19 +393,19 @@ __global__ void __launch_bounds__(CW * 32 + 32)
     // of every stage (TMA writes rows 0..T-1 only; the matching q' columns are
     // zero, but stale bits could be NaN), and stage q' = q[idx] as [g][t] bf16.
     {
-        const uint32_t pad16 = (L.t_pad - (uint32_t)T) * 8u;  // 16-byte words per half
+        const uint32_t pad16 = ragged ? 0u : (L.t_pad - (uint32_t)T) * 8u;  // 16-byte words per half
         for (uint32_t i = tid; i < (uint32_t)stages * 2u * pad16; i += NT) {
             const uint32_t hs = i / pad16, o = i % pad16;  // hs = stage * 2 + half
             *reinterpret_cast<uint4 *>(smem + (hs >> 1) * L.stage + (hs & 1u) * L.k_half +
                                        (uint32_t)T * 128u + o * 16u) = make_uint4(0, 0, 0, 0);
         }
-        mma_stage_q<G, NT>(a, qsm, L.t_pad, T, head, b, kv, tid);
+        mma_stage_q<G, NT>(a, qsm, L.t_pad, T, a.idx + (ragged ? row0 : (int64_t)head * T), b, kv, tid);
     }
     named_barrier(1, NT);  // zeroed rows and q' visible to all consumers
 
     uint32_t qb[kD / 16][2];
-    mma_load_qb(qsm, L.t_pad, lane, qb);
-    const int ksteps = (int)(L.t_pad / 16u);
+    const int ksteps = (int)(t_rows / 16u);
+    mma_load_qb(qsm, L.t_pad, ksteps, lane, qb);
     MmaState S;
     mma_state_init(S);
     const uint32_t sbase = smem_addr(smem);

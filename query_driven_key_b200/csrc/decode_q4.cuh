@@ -216,13 +216,13 @@ __global__ void __launch_bounds__(CW * 32 + 32)
         for (uint32_t i = tid; i < 2u * pad16; i += NT)
             *reinterpret_cast<uint4 *>(kbf + (i / pad16) * L.k_half + (uint32_t)T * 128u + (i % pad16) * 16u) =
                 make_uint4(0, 0, 0, 0);
-        mma_stage_q<G, NT>(a, qsm, L.t_pad, T, head, b, kv, tid);
+        mma_stage_q<G, NT>(a, qsm, L.t_pad, T, a.idx + (int64_t)head * T, b, kv, tid);
     }
     named_barrier(1, NT);
 
     uint32_t qb[kD / 16][2];
-    mma_load_qb(qsm, L.t_pad, lane, qb);
     const int ksteps = (int)(L.t_pad / 16u);
+    mma_load_qb(qsm, L.t_pad, ksteps, lane, qb);
     MmaState S;
     mma_state_init(S);
     const uint32_t sbase = smem_addr(smem);

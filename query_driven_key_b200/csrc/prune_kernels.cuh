@@ -266,6 +266,128 @@ __global__ void __launch_bounds__(128)
 }
 
 // ---------------------------------------------------------------------------
+// Adaptive kept width (ThinK method section, key design 3: the pruning ratio
+// adapts to the query and the cache).  One block does every head: a warp per
+// head ranks the channels (score descending, index ascending; scores are
+// non-negative doubles, ordered by their bits), and lane 0 adds the squared
+// scores in rank order (fp64, each product and sum rounded as written) to
+// find the shortest prefix holding tau of the total:
+//     T_h = min { k in [T_min, T_max] : cum_k >= tau * E }, else T_max;
+//     T_h = T_min when E == 0.
+// The padded widths (multiples of 16) are then scanned into the heads' first
+// rows, and the kept channels are written ascending at idx[rowoff[h] ..].
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int rank_of(const unsigned long long *sv, unsigned long long mine, int c)
+{
+    int rank = 0;
+#pragma unroll 8
+    for (int c2 = 0; c2 < kD; ++c2) {
+        const unsigned long long u = sv[c2];
+        rank += (u > mine) | ((u == mine) & (c2 < c));
+    }
+    return rank;
+}
+
+__global__ void __launch_bounds__(1024)
+    select_adaptive_kernel(const double *__restrict__ scores, int heads, double tau, int T_min, int T_max,
+                           int32_t *__restrict__ Th, int32_t *__restrict__ rowoff, int32_t *__restrict__ idx)
+{
+    __shared__ unsigned long long sv[32][kD];
+    __shared__ unsigned char order[32][kD];   // channel at each rank
+    __shared__ int32_t wsum[32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // ---- widths
+    for (int h = warp; h < heads; h += 32) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            sv[warp][lane + 32 * j] = __double_as_longlong(scores[(int64_t)h * kD + lane + 32 * j]);
+        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int c = lane + 32 * j;
+            order[warp][rank_of(sv[warp], sv[warp][c], c)] = (unsigned char)c;
+        }
+        __syncwarp();
+        if (lane == 0) {
+            double E = 0.0;
+            for (int i = 0; i < kD; ++i) {
+                const double x = __longlong_as_double(sv[warp][order[warp][i]]);
+                E = __dadd_rn(E, __dmul_rn(x, x));
+            }
+            int T = T_max;
+            if (E == 0.0) {
+                T = T_min;
+            } else {
+                const double target = __dmul_rn(tau, E);
+                double cum = 0.0;
+                for (int k = 1; k <= T_max; ++k) {
+                    const double x = __longlong_as_double(sv[warp][order[warp][k - 1]]);
+                    cum = __dadd_rn(cum, __dmul_rn(x, x));
+                    if (k >= T_min && cum >= target) {
+                        T = k;
+                        break;
+                    }
+                }
+            }
+            Th[h] = T;
+        }
+        __syncwarp();
+    }
+    __syncthreads();
+
+    // ---- first rows: exclusive scan of the padded widths over the heads
+    const int per = (heads + 1023) / 1024;
+    const int h0 = min(heads, (int)threadIdx.x * per), h1 = min(heads, h0 + per);
+    int32_t local = 0;
+    for (int h = h0; h < h1; ++h) local += (Th[h] + 15) & ~15;
+    int32_t incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int32_t w = wsum[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t y = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += y;
+        }
+        wsum[lane] = w;  // inclusive sums over warps
+    }
+    __syncthreads();
+    int32_t run = incl - local + (warp > 0 ? wsum[warp - 1] : 0);
+    for (int h = h0; h < h1; ++h) {
+        rowoff[h] = run;
+        run += (Th[h] + 15) & ~15;
+    }
+    if (threadIdx.x == 1023) rowoff[heads] = run;
+    __syncthreads();
+
+    // ---- kept channels, ascending
+    for (int h = warp; h < heads; h += 32) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            sv[warp][lane + 32 * j] = __double_as_longlong(scores[(int64_t)h * kD + lane + 32 * j]);
+        __syncwarp();
+        const int T = Th[h];
+        int base = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int c = lane + 32 * j;
+            const bool keep = rank_of(sv[warp], sv[warp][c], c) < T;
+            const unsigned ball = __ballot_sync(0xffffffffu, keep);
+            if (keep) idx[rowoff[h] + base + __popc(ball & ((1u << lane) - 1u))] = c;
+            base += __popc(ball);
+        }
+        __syncwarp();
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Compact: K'^T[t][col0 + n] = K[n][idx[t]] for a tile of 64 tokens of one
 // head (col0 = 0 for a whole cache, the current length when new tokens'
 // keys are appended).
@@ -307,7 +429,8 @@ template <typename TIn> struct CompactTokens { static constexpr int value = 64; 
 template <typename TIn>
 __global__ void __launch_bounds__(256)
     compact_kernel(const TIn *__restrict__ k, int64_t sb, int64_t sh, int64_t sn, int Hkv, int64_t N,
-                   const int32_t *__restrict__ idx, int T, TIn *__restrict__ kp, int64_t ldk, int64_t col0)
+                   const int32_t *__restrict__ idx, int T, TIn *__restrict__ kp, int64_t ldk, int64_t col0,
+                   const int32_t *__restrict__ Th, const int32_t *__restrict__ rowoff)
 {
     constexpr int BNC = CompactTokens<TIn>::value;  // tokens per block
     constexpr int VEC = 16 / sizeof(TIn);         // elements per 16 bytes (channels per load)
@@ -355,11 +478,17 @@ __global__ void __launch_bounds__(256)
     const int seg = lane % LPR;
     const int tok = seg * VEC;
     const bool vec_ok = (col0 % VEC) == 0;  // 16-byte aligned output runs
-    for (int t = warp * RPI + lane / LPR; t < T; t += 8 * RPI) {
-        const int c = idx[(int64_t)head * T + t];
+    // ragged (Th set): this head keeps Th[head] rows from rowoff[head], then
+    // zero rows up to a multiple of 16
+    const int Tk = Th ? min(max(Th[head], 0), T) : T;
+    const int Tw = Th ? ((Tk + 15) & ~15) : T;
+    const int64_t r0 = Th ? (int64_t)rowoff[head] : (int64_t)head * T;
+    if (Th && (r0 < 0 || r0 + Tw > (int64_t)gridDim.y * ((T + 15) & ~15))) return;  // not from the selection
+    for (int t = warp * RPI + lane / LPR; t < Tw; t += 8 * RPI) {
+        const int c = t < Tk ? idx[r0 + t] : -1;
         uint4 val = make_uint4(0, 0, 0, 0);
         if ((unsigned)c < (unsigned)kD) val = *reinterpret_cast<const uint4 *>(&sT[c][tok]);
-        TIn *out = kp + ((int64_t)head * T + t) * ldk + col0 + n0 + tok;
+        TIn *out = kp + (r0 + t) * ldk + col0 + n0 + tok;
         if (vec_ok && n0 + tok + VEC <= N) {
             *reinterpret_cast<uint4 *>(out) = val;
         } else {

@@ -347,7 +347,8 @@ think_status_t validate_compact(const void *k, const int64_t k_strides[3], int B
 
 think_status_t launch_compact(const void *k, const int64_t k_strides[3], int B, int Hkv, int64_t N,
                               think_dtype_t dtype, const int32_t *idx, int T, void *k_pruned,
-                              int64_t ldk, cudaStream_t st, int64_t col0 = 0)
+                              int64_t ldk, cudaStream_t st, int64_t col0 = 0, const int32_t *Th = nullptr,
+                              const int32_t *rowoff = nullptr)
 {
     const int64_t heads = (int64_t)B * Hkv;
     const int bnc = dtype == THINK_BF16 ? CompactTokens<__nv_bfloat16>::value : CompactTokens<float>::value;
@@ -355,11 +356,11 @@ think_status_t launch_compact(const void *k, const int64_t k_strides[3], int B, 
     if (dtype == THINK_BF16)
         compact_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
             static_cast<const __nv_bfloat16 *>(k), k_strides[0], k_strides[1], k_strides[2], Hkv, N,
-            idx, T, static_cast<__nv_bfloat16 *>(k_pruned), ldk, col0);
+            idx, T, static_cast<__nv_bfloat16 *>(k_pruned), ldk, col0, Th, rowoff);
     else
         compact_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float *>(k), k_strides[0],
                                                     k_strides[1], k_strides[2], Hkv, N, idx, T,
-                                                    static_cast<float *>(k_pruned), ldk, col0);
+                                                    static_cast<float *>(k_pruned), ldk, col0, Th, rowoff);
     return launch_status();
 }
 
@@ -867,6 +868,7 @@ think_status_t think_pruned_decode_attn(const void *q, const void *k_pruned, int
     unsigned char *ws = static_cast<unsigned char *>(workspace);
     const size_t slots = (size_t)heads * sp.splits * G;
     DecodeArgs a;
+    memset(&a, 0, sizeof(a));  // Th = rowoff = null: one kept width for every head
     a.q = q;
     a.idx = idx;
     a.status = reinterpret_cast<unsigned *>(ws);
@@ -988,6 +990,103 @@ think_status_t think_pruned_decode_attn_q4(const void *q, const uint8_t *codes, 
     a.stages = mp.stages;
     a.scale_log2 = scale * 1.4426950408889634f;
     return launch_decode_q4(G, mp.warps, mc, mg, mv, a, mp.bytes, (int)heads, static_cast<cudaStream_t>(stream));
+}
+
+int64_t think_ragged_rows(int B, int Hkv, int T_max)
+{
+    if (B < 0 || Hkv < 0 || T_max < 1 || T_max > kD) return -1;
+    return (int64_t)B * Hkv * ((T_max + 15) & ~15);
+}
+
+think_status_t think_select_adaptive(const double *scores, int B, int Hkv, int d, double tau, int T_min,
+                                     int T_max, int32_t *Th, int32_t *rowoff, int32_t *idx, void *stream)
+{
+    if (B < 0 || Hkv < 0) return THINK_ERR_INVALID_ARG;
+    if (d != kD) return THINK_ERR_UNSUPPORTED;
+    if (!(tau >= 0.0 && tau <= 1.0) || T_min < 1 || T_max < T_min || T_max > d) return THINK_ERR_INVALID_ARG;
+    if (B == 0 || Hkv == 0) return THINK_OK;
+    if (!scores || !Th || !rowoff || !idx) return THINK_ERR_INVALID_ARG;
+    const int64_t heads = (int64_t)B * Hkv;
+    if (heads > 65535) return THINK_ERR_UNSUPPORTED;
+    if ((reinterpret_cast<uintptr_t>(scores) & 7u) || (reinterpret_cast<uintptr_t>(Th) & 3u) ||
+        (reinterpret_cast<uintptr_t>(rowoff) & 3u) || (reinterpret_cast<uintptr_t>(idx) & 3u))
+        return THINK_ERR_ALIGNMENT;
+    select_adaptive_kernel<<<1, 1024, 0, static_cast<cudaStream_t>(stream)>>>(scores, (int)heads, tau, T_min,
+                                                                             T_max, Th, rowoff, idx);
+    return launch_status();
+}
+
+think_status_t think_compact_keys_ragged(const void *k, const int64_t k_strides[3], int B, int Hkv, int64_t N,
+                                         int d, think_dtype_t dtype, const int32_t *idx, const int32_t *Th,
+                                         const int32_t *rowoff, int T_max, void *k_pruned, int64_t ldk,
+                                         void *stream)
+{
+    think_status_t v = validate_compact(k, k_strides, B, Hkv, N, d, dtype, idx, T_max, k_pruned, ldk);
+    if (v != THINK_OK || B == 0 || Hkv == 0 || N == 0) return v;
+    if (!Th || !rowoff) return THINK_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(Th) & 3u) || (reinterpret_cast<uintptr_t>(rowoff) & 3u))
+        return THINK_ERR_ALIGNMENT;
+    return launch_compact(k, k_strides, B, Hkv, N, dtype, idx, T_max, k_pruned, ldk,
+                          static_cast<cudaStream_t>(stream), 0, Th, rowoff);
+}
+
+think_status_t think_pruned_decode_attn_ragged(const void *q, const void *k_pruned, int64_t ldk, const void *v,
+                                               const int64_t v_strides[3], const int32_t *idx,
+                                               const int32_t *Th, const int32_t *rowoff, int T_max, int B, int Hq,
+                                               int Hkv, int64_t N, int d, float scale, float *out,
+                                               void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (B < 0 || Hq < 0 || Hkv < 0 || N < 0 || !std::isfinite(scale)) return THINK_ERR_INVALID_ARG;
+    if (d != kD) return THINK_ERR_UNSUPPORTED;
+    if (T_max < 1 || T_max > d) return THINK_ERR_INVALID_ARG;
+    if (B == 0 || Hkv == 0) return THINK_OK;
+    if (Hq < Hkv || Hq % Hkv != 0) return THINK_ERR_INVALID_ARG;
+    const int G = Hq / Hkv;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return THINK_ERR_UNSUPPORTED;
+    if (N == 0 || ldk < N) return THINK_ERR_INVALID_ARG;
+    if (!q || !k_pruned || !v || !v_strides || !idx || !Th || !rowoff || !out || !workspace)
+        return THINK_ERR_INVALID_ARG;
+    const int64_t heads = (int64_t)B * Hkv;
+    if (heads > 65535 || N > (int64_t)INT32_MAX - kBN) return THINK_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k_pruned) || !aligned16(v) || !aligned16(workspace) || !aligned16(out) ||
+        !strides_ok(v_strides, 2) || (ldk * 2) % 16 != 0 || (reinterpret_cast<uintptr_t>(idx) & 3u) ||
+        (reinterpret_cast<uintptr_t>(Th) & 3u) || (reinterpret_cast<uintptr_t>(rowoff) & 3u))
+        return THINK_ERR_ALIGNMENT;
+    if (workspace_bytes < think_decode_workspace_size(B, Hq, Hkv, N, d, THINK_BF16)) return THINK_ERR_WORKSPACE;
+    const MmaPlan mp = plan_decode_mma(T_max, G, heads, N);
+    if (mp.stages == 0) return THINK_ERR_UNSUPPORTED;
+    const DecodeSplit sp = plan_decode_split(heads, N, mp.blocks_per_sm);
+    const int64_t rows = think_ragged_rows(B, Hkv, T_max);
+    CUtensorMap mk, mv;
+    // K' rows of every head in one 2-D range (x = token, y = row), 16-row boxes
+    if (!make_map_4d(&mk, THINK_BF16, k_pruned, (uint64_t)N, (uint64_t)rows, 1, 1, ldk, rows * ldk, rows * ldk, 64,
+                     16, true))
+        return THINK_ERR_CUDA;
+    if (!make_map_4d(&mv, THINK_BF16, v, kD, (uint64_t)N, (uint64_t)Hkv, (uint64_t)B, v_strides[2], v_strides[1],
+                     v_strides[0], 64, kBN, true))
+        return THINK_ERR_CUDA;
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    const size_t slots = (size_t)heads * sp.splits * G;
+    DecodeArgs a;
+    memset(&a, 0, sizeof(a));
+    a.q = q;
+    a.idx = idx;
+    a.status = reinterpret_cast<unsigned *>(ws);
+    a.tickets = reinterpret_cast<unsigned *>(ws + kDecodeHeader);
+    a.part_o = reinterpret_cast<float *>(ws + kDecodeHeader + align_up((size_t)heads * sizeof(unsigned), 256));
+    a.out = out;
+    a.part_ml = a.part_o + slots * kD;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.T = T_max;
+    a.N = N;
+    a.tiles_per_split = sp.tiles_per_split;
+    a.splits = sp.splits;
+    a.stages = mp.stages;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.Th = Th;
+    a.rowoff = rowoff;
+    return launch_decode_mma(G, mp.warps, mk, mv, a, mp.bytes, (int)heads, static_cast<cudaStream_t>(stream));
 }
 
 think_status_t think_workspace_init(void *workspace, size_t workspace_bytes, void *stream)

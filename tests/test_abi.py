@@ -164,6 +164,30 @@ def test_q4_sizes_and_validation():
     assert call(B=0) == qdk.THINK_OK
 
 
+def test_adaptive_validation():
+    assert qdk.think_ragged_rows(2, 8, 51) == 2 * 8 * 64 and qdk.think_ragged_rows(1, 1, 129) == -1
+    f = lib.think_select_adaptive
+    # (scores, B, Hkv, d, tau, T_min, T_max, Th, rowoff, idx, stream)
+    assert f(FAKE, 1, 2, 128, 1.5, 1, 64, FAKE, FAKE, FAKE, None) == qdk.THINK_ERR_INVALID_ARG
+    assert f(FAKE, 1, 2, 128, float("nan"), 1, 64, FAKE, FAKE, FAKE, None) == qdk.THINK_ERR_INVALID_ARG
+    assert f(FAKE, 1, 2, 128, 0.5, 8, 4, FAKE, FAKE, FAKE, None) == qdk.THINK_ERR_INVALID_ARG
+    assert f(FAKE, 1, 2, 128, 0.5, 0, 4, FAKE, FAKE, FAKE, None) == qdk.THINK_ERR_INVALID_ARG
+    assert f(FAKE, 1, 2, 96, 0.5, 1, 4, FAKE, FAKE, FAKE, None) == qdk.THINK_ERR_UNSUPPORTED
+    assert f(FAKE, 1, 2, 128, 0.5, 1, 4, None, FAKE, FAKE, None) == qdk.THINK_ERR_INVALID_ARG
+    assert f(FAKE, 0, 2, 128, 0.5, 1, 4, FAKE, FAKE, FAKE, None) == qdk.THINK_OK
+    s = I64x3(128 * 64, 128 * 64, 128)
+    g = lib.think_compact_keys_ragged
+    assert g(FAKE, s, 1, 2, 64, 128, 1, FAKE, None, FAKE, 10, FAKE, 64, None) == qdk.THINK_ERR_INVALID_ARG
+    assert g(FAKE, s, 1, 2, 64, 128, 1, FAKE, FAKE, FAKE, 129, FAKE, 64, None) == qdk.THINK_ERR_INVALID_ARG
+    h = lib.think_pruned_decode_attn_ragged
+    vs = I64x3(128 * 64 * 2, 128 * 64, 128)
+    ws = qdk.think_decode_workspace_size(1, 4, 2, 64)
+    assert h(FAKE, FAKE, 64, FAKE, vs, FAKE, FAKE, FAKE, 0, 1, 4, 2, 64, 128, 0.1, FAKE, FAKE, ws, None) == qdk.THINK_ERR_INVALID_ARG
+    assert h(FAKE, FAKE, 64, FAKE, vs, FAKE, None, FAKE, 32, 1, 4, 2, 64, 128, 0.1, FAKE, FAKE, ws, None) == qdk.THINK_ERR_INVALID_ARG
+    assert h(FAKE, FAKE, 64, FAKE, vs, FAKE, FAKE, FAKE, 32, 1, 4, 2, 64, 128, 0.1, FAKE, FAKE, ws - 8, None) == qdk.THINK_ERR_WORKSPACE
+    assert h(FAKE, FAKE, 64, FAKE, vs, FAKE, FAKE, FAKE, 32, 0, 4, 2, 64, 128, 0.1, FAKE, FAKE, 0, None) == qdk.THINK_OK
+
+
 def test_decode_validation():
     s = I64x3(128 * 64 * 2, 128 * 64, 128)
     f = lib.think_pruned_decode_attn

@@ -254,6 +254,45 @@ def test_q4_long_context_full_size():
     _q4_check(cache, q_win, k, v, W.gen_decode_q(w, 0), T, "mistral_7b_long q4")
 
 
+@pytest.mark.parametrize("case", [(1, 32, 8, 20000, 0.9, 16, 96), (2, 8, 2, 1000, 0.5, 1, 128),
+                                  (1, 16, 8, 300, 1.0, 8, 64), (2, 32, 32, 257, 0.0, 4, 40),
+                                  (1, 8, 8, 2000, 0.8, 33, 33), (3, 8, 1, 129, 0.95, 1, 17)])
+def test_adaptive_width(case):
+    B, Hq, Hkv, N, tau, T_min, T_max = case
+    q_win, k, v, q = _random_case(hash(case) & 0xFFFF, B, Hq, Hkv, N, 16, torch.bfloat16, k_pad=8)
+    kd = torch.empty((B, Hkv, N + 8, 128), dtype=torch.bfloat16, device=DEV)[:, :, :N].copy_(k)
+    cache = qdk.AdaptiveCache(B, Hq, Hkv, N, tau, T_min, T_max)
+    cache.k_pruned.fill_(7.0)
+    cache.prune(q_win.to(DEV), kd)
+    out = torch.empty((B, Hq, 128), dtype=torch.float32, device=DEV)
+    cache.decode(q.to(DEV), v.to(DEV), out)
+    torch.cuda.synchronize()
+    ora_scores = oracle.oracle_score(f64(q_win), f64(k))
+    check_scores(cache.scores, ora_scores)
+    # the width rule decides on the GPU's scores: the oracle's rule on the same
+    # scores must give the same widths and kept channels
+    oTh, ooff, oidx = oracle.oracle_select_adaptive(f64(cache.scores), tau, T_min, T_max)
+    Th = cache.Th.cpu().numpy().reshape(B, Hkv)
+    assert np.array_equal(Th, oTh), (Th, oTh)
+    rowoff = cache.rowoff.cpu().numpy()
+    assert np.array_equal(rowoff, np.concatenate([[0], np.cumsum((oTh.ravel() + 15) // 16 * 16)]))
+    gidx = cache.idx.cpu().numpy()
+    kp = cache.k_pruned.cpu()
+    kf = f64(k)
+    for bh in range(B * Hkv):
+        b, h = divmod(bh, Hkv)
+        T = int(Th[b, h])
+        ih = oidx[ooff[bh]:ooff[bh] + T]
+        assert np.array_equal(gidx[rowoff[bh]:rowoff[bh] + T], ih)
+        rows = f64(kp[rowoff[bh]:rowoff[bh + 1], :N])
+        assert np.array_equal(rows[:T], kf[b, h][:, ih].T), f"K' rows of head {bh}"
+        assert np.all(rows[T:] == 0), "pad rows are zero"
+    assert torch.all(kp[rowoff[-1]:, :N] == 7.0) if rowoff[-1] < kp.shape[0] else True
+    check_out(out, oracle.oracle_decode_ragged(f64(q), kf, f64(v), oTh, ooff, oidx), torch.bfloat16,
+              where=str(case))
+    assert qdk.think_read_device_status(cache.decode_ws) == 0
+
+
 def test_ldk_larger_than_needed_and_exact_ties():
     # duplicate channels give exact score ties: lower index must win on both sides
     B, Hq, Hkv, N, S, T = 1, 4, 2, 300, 6, 40
