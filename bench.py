@@ -50,6 +50,8 @@ def parse():
     p.add_argument("--impl", default="native", choices=["native", "reference"])
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-extras", action="store_true",
+                   help="skip the measurements outside the step (append, 4-bit and adaptive-width decode)")
     p.add_argument("--workload", default=WORKLOAD,
                    help="workload name from query_driven_key_b200.workloads (default: the "
                         "long-context layer the metric is quoted on)")
@@ -516,11 +518,12 @@ def run_native(args):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                "steps": args.e2e_steps}
 
-    append = measure_append(w, T, dev, stream, qw_d[0], k_d[0]) if rank == 0 else None
+    extras = rank == 0 and not args.no_extras
+    append = measure_append(w, T, dev, stream, qw_d[0], k_d[0]) if extras else None
     q4 = (measure_q4(w, T, stream, caches[0], qs_d, v_d[0], outs[:, 0], dec_us, peak)
-          if rank == 0 and w.dtype == torch.bfloat16 else None)
+          if extras and w.dtype == torch.bfloat16 else None)
     adaptive = (measure_adaptive(w, dev, stream, qw_d[0], k_d[0], qs_d, v_d[0], outs[:, 0], peak)
-                if rank == 0 and w.dtype == torch.bfloat16 else None)
+                if extras and w.dtype == torch.bfloat16 else None)
 
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
