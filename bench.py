@@ -36,10 +36,10 @@ WORKLOAD = "mistral_7b_long"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the
-# default bf16 decode kernel, pruned_decode_mma_kernel<4>, on the long-context
+# default bf16 decode kernel, pruned_decode_mma_kernel<4, 4>, on the long-context
 # workload, from one ncu capture of that kernel; reported only for that
 # workload and to be reset to None whenever the kernel changes.
-DECODE_TRAFFIC_BYTES = 375_440_128 + 3_847_168
+DECODE_TRAFFIC_BYTES = 375_456_512 + 4_305_408
 
 
 def parse():
