@@ -23,7 +23,9 @@ Python because they are definitions, not kernels:
 The 4-bit thinner cache (``oracle_quantize_q4`` / ``oracle_dequantize_q4``)
 and the adaptive kept width (``oracle_select_adaptive``) are plain C in
 ``think_oracle.c``; ``oracle_decode_ragged`` composes the per-head oracle
-calls for a kept width that differs between heads.
+calls for a kept width that differs between heads.  Token eviction
+(``oracle_token_mass``, ``oracle_select_tokens``) is plain C too;
+``oracle_evict_and_prune`` composes it with the prune.
 
 Parity pins: every function here is pinned by ``tests/test_oracle_pins.py``
 (closed forms, brute force, library routines, a hand-worked example).
@@ -85,11 +87,13 @@ class Oracle:
         lib.oracle_quantize_q4.argtypes = [P, I, I, I, I, I, P, P]
         lib.oracle_dequantize_q4.argtypes = [P, P, I, I, I, I, I, P]
         lib.oracle_select_adaptive.argtypes = [P, I, I, I, D, I, I, P, P, P, I]
+        lib.oracle_token_mass.argtypes = [P, P, I, I, I, I, I, I, D, P]
+        lib.oracle_select_tokens.argtypes = [P, I, I, I, I, P]
         lib.oracle_num_threads.restype = I
         lib.oracle_set_num_threads.argtypes = [I]
         for f in ("oracle_score", "oracle_score_explicit", "oracle_select", "oracle_compact",
                   "oracle_decode", "oracle_dense_decode", "oracle_quantize_q4", "oracle_dequantize_q4",
-                  "oracle_select_adaptive"):
+                  "oracle_select_adaptive", "oracle_token_mass", "oracle_select_tokens"):
             getattr(lib, f).restype = I
         self.lib = lib
 
@@ -199,6 +203,25 @@ class Oracle:
         _check(min(rows, 0), "oracle_select_adaptive")
         return Th.reshape(B, Hkv), off, idx[:rows].copy()
 
+    def token_mass(self, q_win, k, scale: float | None = None) -> np.ndarray:
+        """q_win [B,Hq,S,d], k [B,Hkv,N,d] -> observation-window attention mass [B,Hkv,N]."""
+        q_win, k = _f64(q_win), _f64(k)
+        B, Hq, S, d = q_win.shape
+        _, Hkv, N, _ = k.shape
+        scale = default_scale(d) if scale is None else scale
+        mass = np.zeros((B, Hkv, N), dtype=np.float64)
+        _check(self.lib.oracle_token_mass(_ptr(q_win), _ptr(k), B, Hq, Hkv, S, N, d, float(scale), _ptr(mass)),
+               "oracle_token_mass")
+        return mass
+
+    def select_tokens(self, mass, M: int) -> np.ndarray:
+        """mass [B,Hkv,N] -> the M kept tokens per head [B,Hkv,M] (ascending)."""
+        mass = _f64(mass)
+        B, Hkv, N = mass.shape
+        kept = np.zeros((B, Hkv, M), dtype=np.int32)
+        _check(self.lib.oracle_select_tokens(_ptr(mass), B, Hkv, N, M, _ptr(kept)), "oracle_select_tokens")
+        return kept
+
     def prune(self, q_win, k, T: int):
         """The whole prune step: scores, kept channels, thinner key cache."""
         scores = self.score(q_win, k)
@@ -300,6 +323,29 @@ def oracle_decode_ragged(q, k, v, Th, off, idx, scale=None):
             out[b:b + 1, h * G:(h + 1) * G] = oracle_decode(q[b:b + 1, h * G:(h + 1) * G], kp,
                                                              v[b:b + 1, h:h + 1], ih, scale)
     return out
+
+
+def oracle_token_mass(q_win, k, scale=None):
+    return default_oracle().token_mass(q_win, k, scale)
+
+
+def oracle_select_tokens(mass, M):
+    return default_oracle().select_tokens(mass, M)
+
+
+def oracle_gather_tokens(x, kept):
+    """x [B,Hkv,N,d], kept [B,Hkv,M] -> x[b,h,kept[b,h],:] [B,Hkv,M,d] (numpy gather)."""
+    x = _f64(x)
+    return np.take_along_axis(x, np.asarray(kept)[..., None].astype(np.int64), axis=2)
+
+
+def oracle_evict_and_prune(q_win, k, M, T):
+    """Token eviction then channel pruning: kept tokens by window attention
+    mass, then oracle_prune on the kept tokens' keys.  Returns (kept, scores,
+    idx, K' over the kept tokens)."""
+    kept = oracle_select_tokens(oracle_token_mass(q_win, k), M)
+    scores, idx, kp = oracle_prune(q_win, oracle_gather_tokens(k, kept), T)
+    return kept, scores, idx, kp
 
 
 def attention_loss(q_win_head, k_head, keep) -> float:

@@ -404,3 +404,69 @@ int oracle_select_adaptive(const double *scores, int B, int Hkv, int d, double t
     free(order);
     return rows;
 }
+
+/*
+ * Token eviction composed with channel pruning (ThinK abstract and
+ * experiments: compared with and combined with KV-cache eviction; Keyformer
+ * page: keep the "key tokens" that receive the most attention).  Reading used
+ * here (the observation-window attention mass): for each (b, h_kv) and cached
+ * token n,
+ *     mass[n] = sum over the group's query heads g and window rows s of
+ *               softmax_n( scale * Qwin[b,g,s,:] . K[b,h_kv,n,:] )
+ * (fp64; for each row the max, then the sum of exp(z - max) over n ascending,
+ * then the rows added in (g, s) order); keep the M tokens with the largest
+ * mass (ties to the lower index), in ascending order; the channel pruning then
+ * runs on the kept tokens' keys.
+ *   qwin [B][Hq][S][d], k [B][Hkv][N][d] -> mass [B][Hkv][N];
+ *   kept [B][Hkv][M] int32.
+ */
+int oracle_token_mass(const double *qwin, const double *k, int B, int Hq, int Hkv, int S, int N, int d,
+                      double scale, double *mass)
+{
+    if (B < 0 || Hq < 0 || Hkv < 1 || S < 0 || N < 1 || d < 1 || Hq % Hkv) return -1;
+    const int G = Hq / Hkv;
+    double *z = (double *)malloc(sizeof(double) * (size_t)N);
+    if (!z) return -2;
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < Hkv; ++h) {
+            const double *kh = k + ((size_t)b * Hkv + h) * (size_t)N * d;
+            double *mh = mass + ((size_t)b * Hkv + h) * (size_t)N;
+            for (int n = 0; n < N; ++n) mh[n] = 0.0;
+            for (int g = 0; g < G; ++g)
+                for (int s = 0; s < S; ++s) {
+                    const double *qv = qwin + (((size_t)b * Hq + (size_t)h * G + g) * S + s) * d;
+                    double m = -INFINITY;
+                    for (int n = 0; n < N; ++n) {
+                        double dot = 0.0;
+                        for (int c = 0; c < d; ++c) dot += qv[c] * kh[(size_t)n * d + c];
+                        z[n] = dot * scale;
+                        if (z[n] > m) m = z[n];
+                    }
+                    double l = 0.0;
+                    for (int n = 0; n < N; ++n) {
+                        z[n] = exp(z[n] - m);
+                        l += z[n];
+                    }
+                    for (int n = 0; n < N; ++n) mh[n] += z[n] / l;
+                }
+        }
+    free(z);
+    return 0;
+}
+
+int oracle_select_tokens(const double *mass, int B, int Hkv, int N, int M, int32_t *kept)
+{
+    if (B < 0 || Hkv < 0 || N < 1 || M < 1 || M > N) return -1;
+    int *order = (int *)malloc((size_t)N * sizeof(int));
+    if (!order) return -2;
+    for (long long bh = 0; bh < (long long)B * Hkv; ++bh) {
+        for (int n = 0; n < N; ++n) order[n] = n;
+        g_sort_scores = mass + (size_t)bh * N;
+        qsort(order, (size_t)N, sizeof(int), by_score_desc);
+        qsort(order, (size_t)M, sizeof(int), ascending_int);
+        for (int t = 0; t < M; ++t) kept[(size_t)bh * M + t] = order[t];
+    }
+    free(order);
+    g_sort_scores = NULL;
+    return 0;
+}

@@ -30,8 +30,8 @@ MUTATIONS = {
                              "k[((size_t)bh * N + (size_t)n) * d + t];"),
     "gather_transposed": ("k[((size_t)bh * N + (size_t)n) * d + ih[t]];",
                           "k[((size_t)bh * N + (size_t)(ih[t] % N)) * d + (n % d)];"),
-    "scale_of_kept_width": ("z[n] = dot * scale;", "z[n] = dot * scale * sqrt((double)d / W);"),
-    "softmax_sign": ("z[n] = exp(z[n] - m);", "z[n] = exp(m - z[n]);"),
+    "scale_of_kept_width": ("\n        z[n] = dot * scale;", "\n        z[n] = dot * scale * sqrt((double)d / W);"),
+    "softmax_sign": ("\n        z[n] = exp(z[n] - m);", "\n        z[n] = exp(m - z[n]);"),
     "softmax_not_normalised": ("const double p = z[n] / l;", "const double p = z[n];"),
     "gqa_head_mapping_modulo": ("kv = h / G;\n        const size_t kvh = (size_t)b * Hkv + (size_t)kv;\n"
                                 "        const int32_t *ih",
@@ -45,6 +45,10 @@ MUTATIONS = {
                                      "(((size_t)bh * ng + (n + 1) / group) * T + t) * 2;"),
     "adaptive_strict_threshold": ("if (k >= T_min && cum >= tau * E) {", "if (k >= T_min && cum > tau * E) {"),
     "adaptive_energy_unsquared": ("cum += s[order[k - 1]] * s[order[k - 1]];", "cum += s[order[k - 1]];"),
+    "mass_without_scale": ("z[n] = dot * scale;\n                        if (z[n] > m) m = z[n];",
+                           "z[n] = dot;\n                        if (z[n] > m) m = z[n];"),
+    "mass_not_normalised": ("for (int n = 0; n < N; ++n) mh[n] += z[n] / l;",
+                            "for (int n = 0; n < N; ++n) mh[n] += z[n];"),
     "adaptive_offsets_not_advanced": ("        rows += T;\n    }\n    off[B * Hkv] = rows;",
                                       "    }\n    off[B * Hkv] = rows;"),
 }
@@ -121,6 +125,12 @@ def _pins(o: oracle.Oracle):
         ok &= Th.tolist() == [[T0, T1]] and list(off) == [0, T0, T0 + T1]
         ok &= list(ix[:T0]) == ([1] if T0 == 1 else [0, 1])
     yield "adaptive_hand", bool(ok)
+    # token mass against torch's softmax, and its row-sum closed form
+    qw = r.standard_normal((1, 2, 3, 8))
+    kk = r.standard_normal((1, 1, 11, 8))
+    mass = o.token_mass(qw, kk)
+    p = torch.softmax(torch.from_numpy(qw[0].reshape(6, 8)) @ torch.from_numpy(kk[0, 0]).T / math.sqrt(8), -1)
+    yield "mass_softmax", bool(np.allclose(mass[0, 0], p.sum(0).numpy(), rtol=1e-12, atol=1e-15))
 
 
 def _all_pass(o):

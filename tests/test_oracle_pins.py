@@ -516,3 +516,60 @@ def test_ragged_decode_equals_per_head_pruned_decode():
     mask[[0, 4, 7]] = 1
     np.testing.assert_allclose(out[0, 0:2], _sdpa(q[0:1, 0:2], k[0:1, 0:1] * mask, v[0:1, 0:1], 2)[0],
                                rtol=1e-12, atol=1e-13)
+
+
+# ------------------------------------------------------- token eviction ---
+
+def test_token_mass_equals_torch_softmax_and_sums_to_rows():
+    r = rng(100)
+    B, Hq, Hkv, S, N, d = 2, 4, 2, 5, 37, 16
+    q_win = r.standard_normal((B, Hq, S, d)) * 2
+    k = r.standard_normal((B, Hkv, N, d))
+    mass = oracle.oracle_token_mass(q_win, k)
+    G = Hq // Hkv
+    for b in range(B):
+        for h in range(Hkv):
+            qg = torch.from_numpy(q_win[b, h * G:(h + 1) * G].reshape(G * S, d))
+            p = torch.softmax(qg @ torch.from_numpy(k[b, h]).T / math.sqrt(d), dim=-1)
+            np.testing.assert_allclose(mass[b, h], p.sum(0).numpy(), rtol=1e-12, atol=1e-15)
+    # every softmax row sums to one: the mass of a head sums to G * S
+    np.testing.assert_allclose(mass.sum(-1), G * S, rtol=1e-12)
+
+
+def test_token_mass_of_equal_keys_is_uniform():
+    r = rng(101)
+    q_win = r.standard_normal((1, 2, 3, 8))
+    k = np.broadcast_to(r.standard_normal(8), (1, 1, 9, 8)).copy()
+    np.testing.assert_allclose(oracle.oracle_token_mass(q_win, k), 2 * 3 / 9, rtol=1e-13)
+
+
+def test_select_tokens_matches_python_sort():
+    r = rng(102)
+    mass = r.integers(0, 6, size=(2, 3, 40)).astype(np.float64)  # many exact ties
+    for M in (1, 7, 40):
+        kept = oracle.oracle_select_tokens(mass, M)
+        for b in range(2):
+            for h in range(3):
+                order = sorted(range(40), key=lambda n: (-mass[b, h, n], n))
+                assert kept[b, h].tolist() == sorted(order[:M])
+
+
+def test_keeping_every_token_is_the_plain_prune():
+    r = rng(103)
+    q_win = r.standard_normal((1, 4, 6, 16))
+    k = r.standard_normal((1, 2, 25, 16)) * r.lognormal(0, 1, (1, 1, 1, 16))
+    kept, scores, idx, kp = oracle.oracle_evict_and_prune(q_win, k, 25, 6)
+    assert np.array_equal(kept, np.broadcast_to(np.arange(25), (1, 2, 25)))
+    s2, i2, kp2 = oracle.oracle_prune(q_win, k, 6)
+    assert np.array_equal(scores, s2) and np.array_equal(idx, i2) and np.array_equal(kp, kp2)
+
+
+def test_eviction_keeps_the_attended_token():
+    # a key aligned with every window query gets almost all of the mass
+    r = rng(104)
+    d = 16
+    q_win = np.abs(r.standard_normal((1, 2, 4, d)))
+    k = 0.01 * r.standard_normal((1, 1, 30, d))
+    k[0, 0, 17] = 8.0
+    kept = oracle.oracle_select_tokens(oracle.oracle_token_mass(q_win, k), 1)
+    assert kept[0, 0, 0] == 17
