@@ -295,6 +295,41 @@ def measure_adaptive(w, dev, stream, qw_d, k_d, qs_d, v_d, outs, peak, tau=0.9, 
             "kernel": "pruned_decode_mma_kernel, ragged mode (think_pruned_decode_attn_ragged), not part of the step"}
 
 
+def measure_evict(w, T, dev, stream, qw_d, k_d, v_d, qs_d, outs, peak, keep=0.25):
+    """Token eviction then channel pruning on the same layer, outside the timed
+    step: the M = keep * N tokens of largest window attention mass are kept,
+    then pruned to T channels; device time of that whole prune and of the
+    step's decode calls over the M kept tokens."""
+    import torch
+    import query_driven_key_b200 as qdk
+    from query_driven_key_b200 import workloads as W
+    M = max(1, int(w.N * keep))
+    cache = qdk.EvictedCache(w.B, w.Hq, w.Hkv, w.N, w.S_obs, M, T, w.d, dtype=w.dtype, device=dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    for _ in range(3):
+        cache.prune(qw_d, k_d, v_d, stream=stream)
+    e0, e1 = ev(), ev()
+    e0.record(stream)
+    cache.prune(qw_d, k_d, v_d, stream=stream)
+    e1.record(stream)
+    for s in range(3):
+        cache.decode(qs_d[s], outs[s], stream=stream)
+    e2, e3 = ev(), ev()
+    e2.record(stream)
+    for s in range(w.decode_steps):
+        cache.decode(qs_d[s], outs[s], stream=stream)
+    e3.record(stream)
+    stream.synchronize()
+    wm = w.with_(N=M)
+    nbytes = W.decode_bytes(wm, T)
+    us = e2.elapsed_time(e3) * 1e3 / w.decode_steps
+    return {"kept_tokens": M, "T": T, "evict_and_prune_us": e0.elapsed_time(e1) * 1e3,
+            "decode_us_per_step": us, "decode_gbs": nbytes / (us * 1e-6) / 1e9,
+            "frac_of_measured_peak": nbytes / (us * 1e-6) / 1e9 / peak, "algorithmic_bytes_per_launch": nbytes,
+            "note": "token_mass (2 launches) + select_tokens + 2 gathers + prune; decode over the kept tokens; "
+                    "not part of the step"}
+
+
 def data_recipe(w):
     if w.k_kind == "lowrank":
         keys = f"rank-{w.k_rank} N(0,1) factors + {w.k_noise} N(0,1) noise, LogNormal(0,{w.k_sigma}) channel scales"
@@ -524,6 +559,8 @@ def run_native(args):
           if extras and w.dtype == torch.bfloat16 else None)
     adaptive = (measure_adaptive(w, dev, stream, qw_d[0], k_d[0], qs_d, v_d[0], outs[:, 0], peak)
                 if extras and w.dtype == torch.bfloat16 else None)
+    evict = (measure_evict(w, T, dev, stream, qw_d[0], k_d[0], v_d[0], qs_d, outs[:, 0], peak)
+             if extras and w.dtype == torch.bfloat16 else None)
 
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -551,6 +588,7 @@ def run_native(args):
         "append": append,
         "q4": q4,
         "adaptive": adaptive,
+        "evict": evict,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
         "e2e": e2e,

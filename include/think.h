@@ -16,8 +16,10 @@
  *
  * plus think_prune, the first three in two launches; think_append_keys,
  * which appends new tokens' keys to the thinner cache; a 4-bit thinner
- * cache (think_quantize_keys_q4, think_pruned_decode_attn_q4); and a kept
- * width per head (think_select_adaptive and the _ragged calls).
+ * cache (think_quantize_keys_q4, think_pruned_decode_attn_q4); a kept
+ * width per head (think_select_adaptive and the _ragged calls); and token
+ * eviction to compose with it (think_token_mass, think_select_tokens,
+ * think_gather_tokens).
  *
  * Conventions shared by every call
  *   - Shapes: B batch, Hq query heads, Hkv KV heads (G = Hq/Hkv query heads
@@ -295,6 +297,37 @@ think_status_t think_pruned_decode_attn_ragged(const void *q, const void *k_prun
                                                const int32_t *Th, const int32_t *rowoff, int T_max, int B, int Hq,
                                                int Hkv, int64_t N, int d, float scale, float *out,
                                                void *workspace, size_t workspace_bytes, void *stream);
+
+/* ----------------------------------------------------- token eviction --
+ * Token eviction composed with the channel pruning (ThinK abstract and
+ * experiments: compared with and combined with KV-cache eviction; Keyformer
+ * page: keep the tokens that receive the most attention).  Reading used here:
+ *     mass[n] = sum over the group's query heads g and window rows s of
+ *               softmax_n(scale * Qwin[b,g,s,:] . K[b,h_kv,n,:])
+ * (the observation-window attention mass); each head keeps the M tokens of
+ * largest mass, ties to the lower index, ascending.  The pipeline is
+ * think_token_mass -> think_select_tokens -> think_gather_tokens (K and V)
+ * -> think_prune on the gathered keys -> decode with N = M.
+ *
+ * think_token_mass: two launches (row statistics, then the masses) on the
+ *   tensor cores; bf16 only; G * S_obs <= 512.  q_win [B][Hq][S_obs][d]
+ *   contiguous; k, k_strides as for think_score_channels; mass [B][Hkv][N]
+ *   fp32 output; workspace of think_token_mass_workspace_size() bytes, zeroed
+ *   once before first use (per-head counters that every call leaves at zero;
+ *   its first 4 bytes are the device status word). */
+size_t think_token_mass_workspace_size(int B, int Hq, int Hkv, int64_t N, int S_obs);
+think_status_t think_token_mass(const void *q_win, const void *k, const int64_t k_strides[3], int B, int Hq,
+                                int Hkv, int64_t N, int S_obs, int d, think_dtype_t dtype, float scale, float *mass,
+                                void *workspace, size_t workspace_bytes, void *stream);
+/* kept [B][Hkv][M] int32 output: the M tokens of largest mass per head (ties
+ * to the lower index), ascending; 1 <= M <= N.  One launch (a block per
+ * head, radix select on the masses' bits). */
+think_status_t think_select_tokens(const float *mass, int B, int Hkv, int64_t N, int M, int32_t *kept,
+                                   void *stream);
+/* out[b,h,j,:] = x[b,h,kept[b,h,j],:], out contiguous [B][Hkv][M][d] (a copy;
+ * an out-of-range index gives a zero row).  One launch. */
+think_status_t think_gather_tokens(const void *x, const int64_t x_strides[3], int B, int Hkv, int64_t N, int d,
+                                   think_dtype_t dtype, const int32_t *kept, int M, void *out, void *stream);
 
 /* Zero a score or decode workspace (stream-ordered memset). */
 think_status_t think_workspace_init(void *workspace, size_t workspace_bytes, void *stream);

@@ -40,7 +40,8 @@ EXPORTED = (
     "think_workspace_init", "think_read_device_status", "think_noalloc_scratch_bytes",
     "think_pruned_decode_attn_noalloc", "think_q4_ld", "think_q4_groups_bytes",
     "think_quantize_keys_q4", "think_pruned_decode_attn_q4", "think_ragged_rows", "think_select_adaptive",
-    "think_compact_keys_ragged", "think_pruned_decode_attn_ragged",
+    "think_compact_keys_ragged", "think_pruned_decode_attn_ragged", "think_token_mass_workspace_size",
+    "think_token_mass", "think_select_tokens", "think_gather_tokens",
 )
 
 
@@ -87,6 +88,14 @@ def _load() -> ctypes.CDLL:
     lib.think_compact_keys_ragged.restype = I
     lib.think_pruned_decode_attn_ragged.argtypes = [P, P, I64, P, I64P, P, P, P, I, I, I, I, I64, I, F, P, P, SZ, P]
     lib.think_pruned_decode_attn_ragged.restype = I
+    lib.think_token_mass_workspace_size.argtypes = [I, I, I, I64, I]
+    lib.think_token_mass_workspace_size.restype = SZ
+    lib.think_token_mass.argtypes = [P, P, I64P, I, I, I, I64, I, I, I, F, P, P, SZ, P]
+    lib.think_token_mass.restype = I
+    lib.think_select_tokens.argtypes = [P, I, I, I64, I, P, P]
+    lib.think_select_tokens.restype = I
+    lib.think_gather_tokens.argtypes = [P, I64P, I, I, I64, I, I, P, I, P, P]
+    lib.think_gather_tokens.restype = I
     lib.think_decode_workspace_size.argtypes = [I, I, I, I64, I, I]
     lib.think_decode_workspace_size.restype = SZ
     lib.think_pruned_decode_attn.argtypes = [P, P, I64, P, I64P, P, I, I, I, I64, I, I, I, F, P,
@@ -366,6 +375,69 @@ class AdaptiveCache:
     def decode(self, q, v, out, scale=None, stream=None):
         think_pruned_decode_attn_ragged(q, self.k_pruned, self.ldk, v, self.idx, self.Th, self.rowoff, self.T_max,
                                         out, self.decode_ws, N=self.N, scale=scale, stream=stream)
+
+
+def think_token_mass_workspace_size(B: int, Hq: int, Hkv: int, N: int, S_obs: int) -> int:
+    return lib.think_token_mass_workspace_size(B, Hq, Hkv, int(N), S_obs)
+
+
+def think_token_mass(q_win: torch.Tensor, k: torch.Tensor, mass: torch.Tensor, workspace: torch.Tensor,
+                     scale: float | None = None, stream=None) -> None:
+    """q_win [B,Hq,S,d], k [B,Hkv,N,d] (bf16) -> mass [B,Hkv,N] fp32 (window attention mass)."""
+    B, Hq, S, d = q_win.shape
+    _, Hkv, N, _ = k.shape
+    if scale is None:
+        scale = 1.0 / float(d) ** 0.5
+    if not q_win.is_contiguous() or mass.dtype != torch.float32:
+        raise ThinkError(THINK_ERR_INVALID_ARG, "think_token_mass")
+    _check(lib.think_token_mass(_ptr(q_win), _ptr(k), _strides3(k), B, Hq, Hkv, N, S, d, _dtype(k), float(scale),
+                                _ptr(mass), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                _stream(stream)), "think_token_mass")
+
+
+def think_select_tokens(mass: torch.Tensor, M: int, kept: torch.Tensor, stream=None) -> None:
+    """mass [B,Hkv,N] fp32 -> kept [B,Hkv,M] int32 (largest mass, ties to the lower index, ascending)."""
+    B, Hkv, N = mass.shape
+    _check(lib.think_select_tokens(_ptr(mass), B, Hkv, N, int(M), _ptr(kept), _stream(stream)),
+           "think_select_tokens")
+
+
+def think_gather_tokens(x: torch.Tensor, kept: torch.Tensor, out: torch.Tensor, stream=None) -> None:
+    """x [B,Hkv,N,d], kept [B,Hkv,M] -> out [B,Hkv,M,d] (contiguous)."""
+    B, Hkv, N, d = x.shape
+    M = kept.shape[-1]
+    if not out.is_contiguous() or out.dtype != x.dtype or kept.dtype != torch.int32:
+        raise ThinkError(THINK_ERR_INVALID_ARG, "think_gather_tokens")
+    _check(lib.think_gather_tokens(_ptr(x), _strides3(x), B, Hkv, N, d, _dtype(x), _ptr(kept), int(M), _ptr(out),
+                                   _stream(stream)), "think_gather_tokens")
+
+
+class EvictedCache:
+    """Token eviction then channel pruning of one layer: keep the M tokens of
+    largest window attention mass per head, gather their K and V rows, prune
+    the channels of the kept keys (a PrunedCache over M tokens).  Allocates
+    with torch on construction, then only calls the C entry points."""
+
+    def __init__(self, B: int, Hq: int, Hkv: int, N: int, S_obs: int, M: int, T: int, d: int = 128,
+                 dtype: torch.dtype = torch.bfloat16, device="cuda"):
+        self.B, self.Hq, self.Hkv, self.N, self.M, self.T, self.d = B, Hq, Hkv, N, M, T, d
+        self.mass = torch.empty((B, Hkv, N), dtype=torch.float32, device=device)
+        self.kept = torch.empty((B, Hkv, M), dtype=torch.int32, device=device)
+        self.k_kept = torch.empty((B, Hkv, M, d), dtype=dtype, device=device)
+        self.v_kept = torch.empty((B, Hkv, M, d), dtype=dtype, device=device)
+        self.mass_ws = torch.zeros(max(256, think_token_mass_workspace_size(B, Hq, Hkv, N, S_obs)),
+                                   dtype=torch.uint8, device=device)
+        self.pruned = PrunedCache(B, Hq, Hkv, M, T, d, dtype=dtype, device=device)
+
+    def prune(self, q_win, k, v, stream=None):
+        think_token_mass(q_win, k, self.mass, self.mass_ws, stream=stream)
+        think_select_tokens(self.mass, self.M, self.kept, stream)
+        think_gather_tokens(k, self.kept, self.k_kept, stream)
+        think_gather_tokens(v, self.kept, self.v_kept, stream)
+        self.pruned.prune(q_win, self.k_kept, stream)
+
+    def decode(self, q, out, scale=None, stream=None):
+        self.pruned.decode(q, self.v_kept, out, scale=scale, stream=stream)
 
 
 def think_workspace_init(workspace: torch.Tensor, stream=None) -> None:

@@ -1,0 +1,384 @@
+// evict.cuh -- token eviction by observation-window attention mass, to be
+// composed with the channel pruning (the prune then runs on the kept tokens).
+//
+// "ThinK: Thinner Key Cache by Query-Driven Pruning", abstract and
+// experiments: ThinK is compared with and combined with KV-cache eviction;
+// the Keyformer page keeps the "key tokens" that receive the most attention.
+// Reading used here, for each (b, h_kv) and cached token n:
+//     mass[n] = sum over the group's query heads g and window rows s of
+//               softmax_n( scale * Qwin[b,g,s,:] . K[b,h_kv,n,:] )
+// and each head keeps the M tokens of largest mass (ties to the lower index),
+// in ascending order.
+//
+// The mass is an attention of R = G * S_obs query rows over the N keys,
+// computed in two passes on the tensor cores (mma.sync m16n8k16, bf16 in,
+// fp32 accumulate): pass 1 the row statistics (max and sum of exponentials,
+// per split, merged by the last block of the head), pass 2 the column sums of
+// the normalised weights.  K streams through a TMA ring as 128-token tiles
+// (two 64-channel halves, 128-byte swizzle); the window queries stay in
+// shared memory (same swizzle) for the whole block.
+#pragma once
+
+#include "decode_mma.cuh"
+
+namespace think {
+
+constexpr int kMassWarps = 4;
+constexpr int kMassThreads = kMassWarps * 32 + 32;  // + TMA producer warp
+constexpr int kMassRowsMax = 512;                   // G * S_obs
+
+struct MassArgs {
+    const __nv_bfloat16 *qwin;  // [B][Hq][S][128]
+    int Hq, Hkv, S, G, R, r_pad;  // R = G * S rows; r_pad = R rounded up to 8 * kMassWarps
+    int64_t N;
+    int tiles_per_split, splits, stages;
+    float scale_log2;           // scale * log2(e)
+    float2 *part;               // [heads][splits][R] (max, sum) of each split (pass 1)
+    float2 *stats;              // [heads][R] (max, 1 / sum) (written by pass 1, read by pass 2)
+    unsigned *tickets;          // [heads], zero between calls
+    unsigned *status;           // device status word
+    float *mass;                // [heads][N] (pass 2)
+};
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+// shared memory: stages x K tile (32 KB), the window queries (two 64-channel
+// halves of r_pad rows x 128 B), pass 2's row statistics and per-warp token
+// sums, barriers, a flag
+__host__ __device__ inline size_t mass_smem_bytes(int r_pad, int stages)
+{
+    return (size_t)stages * 32768u + (size_t)2 * r_pad * 128u + (size_t)r_pad * 8u +
+           (size_t)kMassWarps * kBN * 4u + (size_t)2 * stages * 8u + 16u + 1024u;
+}
+
+// NTW: 8-row query groups per warp (r_pad = 32 * NTW).
+template <int PASS, int NTW>
+__global__ void __launch_bounds__(kMassThreads)
+    token_mass_kernel(const __grid_constant__ CUtensorMap tm_k, const MassArgs a)
+{
+    extern __shared__ unsigned char smem_dyn[];
+    unsigned char *smem = smem_dyn + ((1024u - (smem_addr(smem_dyn) & 1023u)) & 1023u);
+    const int split = blockIdx.x;
+    const int head = blockIdx.y;
+    const int b = head / a.Hkv, kv = head % a.Hkv;
+    const int stages = a.stages;
+    const int64_t tile0 = (int64_t)split * a.tiles_per_split;
+    const int64_t tiles_all = (a.N + kBN - 1) / kBN;
+    const int ntiles = (int)min((int64_t)a.tiles_per_split, tiles_all - tile0);
+    const uint32_t q_half = (uint32_t)a.r_pad * 128u;
+
+    unsigned char *qs = smem + (size_t)stages * 32768u;                 // queries, swizzled
+    float2 *rstat = reinterpret_cast<float2 *>(qs + 2u * q_half);        // [r_pad] (max, 1/sum)
+    float *tsum = reinterpret_cast<float *>(rstat + a.r_pad);            // [warps][128]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(tsum + kMassWarps * kBN);
+    unsigned *flag = reinterpret_cast<unsigned *>(bars + 2 * stages);
+    const uint32_t full0 = smem_addr(bars), empty0 = smem_addr(bars + stages);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        for (int s = 0; s < stages; ++s) {
+            mbar_init(full0 + 8 * s, 1);
+            mbar_init(empty0 + 8 * s, kMassWarps);
+        }
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    if (warp == kMassWarps) {
+        // ------------------------------------------------------ producer
+        if (lane == 0) {
+            prefetch_tensormap(&tm_k);
+            int issued = 0;
+            bool ok = true;
+            for (int it = 0; it < ntiles; ++it) {
+                const int s = it % stages, f = it / stages;
+                if (f > 0 && !mbar_wait_bounded(empty0 + 8 * s, (f - 1) & 1, a.status,
+                                                THINK_DEVICE_TIMEOUT_EMPTY)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t full = full0 + 8 * s;
+                mbar_arrive_expect_tx(full, 32768u);
+                const int x = (int)((tile0 + it) * kBN);
+                const uint32_t st = smem_addr(smem + (size_t)s * 32768u);
+                tma_load_4d(st, &tm_k, 0, x, kv, b, full);
+                tma_load_4d(st + 16384u, &tm_k, 64, x, kv, b, full);
+                ++issued;
+            }
+            if (!ok) {
+                for (int it = max(0, issued - stages); it < issued; ++it)
+                    mbar_wait_bounded(full0 + 8 * (it % stages), (it / stages) & 1, a.status,
+                                      THINK_DEVICE_TIMEOUT_FULL);
+            }
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------- consumers
+    constexpr int NT = kMassWarps * 32;
+    // the window queries of the group, row r = g * S + s (rows >= R zero), in
+    // two 64-channel halves with the 128-byte swizzle
+    for (int i = tid; i < a.r_pad * 16; i += NT) {
+        const int r = i >> 4, c16 = i & 15;  // row, 16-byte chunk (8 channels)
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (r < a.R) {
+            const int g = r / a.S, s = r % a.S;
+            v = *reinterpret_cast<const uint4 *>(
+                a.qwin + (((int64_t)b * a.Hq + (int64_t)kv * a.G + g) * a.S + s) * kD + 8 * c16);
+        }
+        *reinterpret_cast<uint4 *>(qs + (c16 >> 3) * q_half + (uint32_t)r * 128u +
+                                   ((((uint32_t)c16 & 7u) ^ ((uint32_t)r & 7u)) << 4)) = v;
+    }
+    if (PASS == 2) {
+        for (int r = tid; r < a.r_pad; r += NT)
+            rstat[r] = r < a.R ? __ldcg(a.stats + (int64_t)head * a.R + r) : make_float2(0.f, 0.f);
+    }
+    named_barrier(1, NT);
+
+    const int q4 = lane & 3, r8 = lane >> 2;
+    const uint32_t qbase = smem_addr(qs);
+    // pass 1: running (max, lane-partial sum) for the warp's n-tiles (warp,
+    // warp + 4, ...), 2 columns each
+    float rm[NTW][2], rl[NTW][2];
+#pragma unroll
+    for (int j = 0; j < NTW; ++j)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            rm[j][h] = -INFINITY;
+            rl[j][h] = 0.f;
+        }
+
+    for (int it = 0; it < ntiles; ++it) {
+        const int s = it % stages;
+        if (!mbar_wait_bounded(full0 + 8 * s, (it / stages) & 1, a.status, THINK_DEVICE_TIMEOUT_FULL)) break;
+        const uint32_t kb = smem_addr(smem + (size_t)s * 32768u);
+        const int64_t tok0 = (tile0 + it) * kBN;
+#pragma unroll 1
+        for (int mt = 0; mt < 8; ++mt) {
+            float tacc[2] = {0.f, 0.f};  // pass 2: this lane's sums for tokens 16 mt + r8, + 8
+            // A fragments: tokens 16 mt .. +15, all 8 channel steps
+            uint32_t af[8][4];
+            const int mi = lane >> 3, rr = lane & 7;
+            const uint32_t tok = (uint32_t)(16 * mt + (mi & 1) * 8 + rr);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t chunk = (uint32_t)(2 * ks + (mi >> 1));
+                ldsm_x4(kb + (chunk >> 3) * 16384u + tok * 128u + (((chunk & 7u) ^ (tok & 7u)) << 4), af[ks][0],
+                        af[ks][1], af[ks][2], af[ks][3]);
+            }
+            const bool v0 = tok0 + 16 * mt + r8 < a.N, v1 = tok0 + 16 * mt + 8 + r8 < a.N;
+#pragma unroll
+            for (int j = 0; j < NTW; ++j) {
+                const int nt = warp + kMassWarps * j;
+                float c[4] = {0.f, 0.f, 0.f, 0.f};
+                const uint32_t n = (uint32_t)(8 * nt + rr);
+#pragma unroll
+                for (int kp = 0; kp < 4; ++kp) {
+                    uint32_t b0, b1, b2, b3;
+                    const uint32_t chunk = (uint32_t)(4 * kp + mi);
+                    ldsm_x4(qbase + (chunk >> 3) * q_half + n * 128u + (((chunk & 7u) ^ (n & 7u)) << 4), b0, b1,
+                            b2, b3);
+                    wmma16::mma_bf16(c, af[2 * kp][0], af[2 * kp][1], af[2 * kp][2], af[2 * kp][3], b0, b1);
+                    wmma16::mma_bf16(c, af[2 * kp + 1][0], af[2 * kp + 1][1], af[2 * kp + 1][2],
+                                     af[2 * kp + 1][3], b2, b3);
+                }
+                // c[0], c[1]: token 16 mt + r8, rows 8 nt + 2 q4 (+1); c[2], c[3]: token + 8
+                if (PASS == 1) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const float z0 = v0 ? c[h] * a.scale_log2 : -INFINITY;
+                        const float z1 = v1 ? c[2 + h] * a.scale_log2 : -INFINITY;
+                        float xm = fmaxf(z0, z1);
+                        xm = fmaxf(xm, __shfl_xor_sync(0xffffffffu, xm, 4));
+                        xm = fmaxf(xm, __shfl_xor_sync(0xffffffffu, xm, 8));
+                        xm = fmaxf(xm, __shfl_xor_sync(0xffffffffu, xm, 16));
+                        const float mnew = fmaxf(rm[j][h], xm);
+                        if (mnew != -INFINITY) {
+                            const float alpha = rm[j][h] == -INFINITY ? 0.f : exp2_approx(rm[j][h] - mnew);
+                            rl[j][h] = rl[j][h] * alpha + (v0 ? exp2_approx(z0 - mnew) : 0.f) +
+                                       (v1 ? exp2_approx(z1 - mnew) : 0.f);
+                            rm[j][h] = mnew;
+                        }
+                    }
+                } else {
+                    const float2 s0 = rstat[8 * nt + 2 * q4], s1 = rstat[8 * nt + 2 * q4 + 1];
+                    tacc[0] += exp2_approx(c[0] * a.scale_log2 - s0.x) * s0.y +
+                               exp2_approx(c[1] * a.scale_log2 - s1.x) * s1.y;
+                    tacc[1] += exp2_approx(c[2] * a.scale_log2 - s0.x) * s0.y +
+                               exp2_approx(c[3] * a.scale_log2 - s1.x) * s1.y;
+                }
+            }
+            if (PASS == 2) {
+                // the warp's rows for these 16 tokens (the 4 lanes of a token)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    float x = tacc[h];
+                    x += __shfl_xor_sync(0xffffffffu, x, 1);
+                    x += __shfl_xor_sync(0xffffffffu, x, 2);
+                    if (q4 == 0) tsum[warp * kBN + 16 * mt + 8 * h + r8] = x;
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty0 + 8 * s);
+        if (PASS == 2) {
+            // the four warps' row groups in order: the tile's masses
+            named_barrier(1, NT);
+            if (tid < kBN && tok0 + tid < a.N) {
+                float m = 0.f;
+#pragma unroll
+                for (int w = 0; w < kMassWarps; ++w) m += tsum[w * kBN + tid];
+                a.mass[(int64_t)head * a.N + tok0 + tid] = m;
+            }
+            named_barrier(1, NT);
+        }
+    }
+    if (PASS == 2) return;
+
+    // ---- pass 1: the block's row statistics, then the last block of the head merges
+#pragma unroll
+    for (int j = 0; j < NTW; ++j)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            float l = rl[j][h];
+            l += __shfl_xor_sync(0xffffffffu, l, 4);
+            l += __shfl_xor_sync(0xffffffffu, l, 8);
+            l += __shfl_xor_sync(0xffffffffu, l, 16);
+            const int r = 8 * (warp + kMassWarps * j) + 2 * q4 + h;
+            if (r8 == 0 && r < a.R)
+                a.part[((int64_t)head * a.splits + split) * a.R + r] = make_float2(rm[j][h], l);
+        }
+    __threadfence();
+    named_barrier(1, NT);
+    if (tid == 0) *flag = (atomicAdd(a.tickets + head, 1u) == (unsigned)(a.splits - 1)) ? 1u : 0u;
+    named_barrier(1, NT);
+    if (*flag == 0u) return;
+    __threadfence();
+    for (int r = tid; r < a.R; r += NT) {
+        float M = -INFINITY;
+        for (int s = 0; s < a.splits; ++s) M = fmaxf(M, __ldcg(a.part + ((int64_t)head * a.splits + s) * a.R + r).x);
+        float L = 0.f;
+        for (int s = 0; s < a.splits; ++s) {
+            const float2 p = __ldcg(a.part + ((int64_t)head * a.splits + s) * a.R + r);
+            if (p.x != -INFINITY) L = fmaf(p.y, exp2_approx(p.x - M), L);
+        }
+        a.stats[(int64_t)head * a.R + r] = make_float2(M, L > 0.f ? 1.f / L : 0.f);
+    }
+    if (tid == 0) a.tickets[head] = 0u;
+}
+
+// ---------------------------------------------------------------------------
+// Top-M tokens of each head by mass (one block of 1024 threads per head):
+// a radix select on the masses' bits (non-negative floats order like their
+// bits) finds the M-th largest value, then one ordered pass keeps every token
+// above it and the lowest-indexed ties, writing the kept indices ascending.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int block_exclusive_scan_1024(int x, int *wsum, int &total)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int w = wsum[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += y;
+        }
+        wsum[lane] = w;
+    }
+    __syncthreads();
+    total = wsum[31];
+    const int excl = incl - x + (warp > 0 ? wsum[warp - 1] : 0);
+    __syncthreads();
+    return excl;
+}
+
+__global__ void __launch_bounds__(1024)
+    select_tokens_kernel(const float *__restrict__ mass, int64_t N, int M, int32_t *__restrict__ kept)
+{
+    __shared__ int hist[256];
+    __shared__ int wsum[32];
+    __shared__ uint32_t s_prefix, s_mask;
+    __shared__ int s_need;
+    const int head = blockIdx.x;
+    const uint32_t *key = reinterpret_cast<const uint32_t *>(mass + (int64_t)head * N);
+    const int tid = threadIdx.x;
+    if (tid == 0) {
+        s_prefix = 0u;
+        s_mask = 0u;
+        s_need = M;
+    }
+    __syncthreads();
+    // four 8-bit digits from the top: the M-th largest key
+    for (int shift = 24; shift >= 0; shift -= 8) {
+        if (tid < 256) hist[tid] = 0;
+        __syncthreads();
+        const uint32_t prefix = s_prefix, mask = s_mask;
+        for (int64_t n = tid; n < N; n += 1024) {
+            const uint32_t k = key[n];
+            if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1);
+        }
+        __syncthreads();
+        if (tid == 0) {
+            int need = s_need, dg = 255;
+            for (; dg > 0 && hist[dg] < need; --dg) need -= hist[dg];
+            s_need = need;  // how many of the keys with this digit are still to take
+            s_prefix = prefix | ((uint32_t)dg << shift);
+            s_mask = mask | (255u << shift);
+        }
+        __syncthreads();
+    }
+    const uint32_t kth = s_prefix;
+    const int ties = s_need;  // keys equal to kth that are kept: the lowest-indexed ones
+    // ordered pass: keep key > kth, and the first `ties` keys == kth
+    int written = 0, ties_seen = 0;
+    for (int64_t base = 0; base < N; base += 1024) {
+        const int64_t n = base + tid;
+        const uint32_t k = n < N ? key[n] : 0u;
+        const int eq = (n < N && k == kth) ? 1 : 0;
+        int eq_total;
+        const int eq_before = block_exclusive_scan_1024(eq, wsum, eq_total);
+        const int keep = (n < N) && (k > kth || (eq && ties_seen + eq_before < ties)) ? 1 : 0;
+        int keep_total;
+        const int pos = block_exclusive_scan_1024(keep, wsum, keep_total);
+        if (keep && written + pos < M) kept[(int64_t)head * M + written + pos] = (int32_t)n;
+        written += keep_total;
+        ties_seen += eq_total;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Gather the kept tokens' rows: out[b,h,j,:] = x[b,h,kept[b,h,j],:] (a copy).
+// A warp per row (16-byte lanes).
+// ---------------------------------------------------------------------------
+template <typename TIn>
+__global__ void __launch_bounds__(256)
+    gather_tokens_kernel(const TIn *__restrict__ x, int64_t sb, int64_t sh, int64_t sn, int Hkv, int M,
+                         const int32_t *__restrict__ kept, int64_t N, TIn *__restrict__ out)
+{
+    constexpr int VEC = 16 / sizeof(TIn);
+    constexpr int LANES = kD / VEC;  // 16 (bf16) or 32 (fp32) lanes per row
+    const int64_t row = (int64_t)blockIdx.x * (256 / LANES) + threadIdx.x / LANES;
+    const int head = blockIdx.y;
+    if (row >= M) return;
+    const int b = head / Hkv, h = head % Hkv;
+    const int n = kept[(int64_t)head * M + row];
+    const int c = (threadIdx.x % LANES) * VEC;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if ((unsigned)n < (unsigned)N) v = *reinterpret_cast<const uint4 *>(x + (int64_t)b * sb + (int64_t)h * sh + (int64_t)n * sn + c);
+    *reinterpret_cast<uint4 *>(out + ((int64_t)head * M + row) * kD + c) = v;
+}
+
+}  // namespace think

@@ -15,6 +15,7 @@
 #include "decode_kernels.cuh"
 #include "decode_mma.cuh"
 #include "decode_q4.cuh"
+#include "evict.cuh"
 #include "decode_tc.cuh"
 #include "prune_fused.cuh"
 #include "prune_kernels.cuh"
@@ -503,6 +504,68 @@ think_status_t launch_decode_mma(int G, int cw, const CUtensorMap &mk, const CUt
     case 8: return launch_decode_mma_g<8>(cw, mk, mv, a, bytes, heads, st);
     default: return THINK_ERR_UNSUPPORTED;
     }
+}
+
+// ------------------------------------------------------- token eviction --
+
+struct MassPlan {
+    int ntw, r_pad, stages, blocks_per_sm;
+    size_t bytes;
+    DecodeSplit sp;
+};
+
+MassPlan plan_mass(int R, int64_t heads, int64_t N)
+{
+    MassPlan p;
+    p.ntw = R <= 64 ? 2 : R <= 128 ? 4 : R <= 256 ? 8 : 16;
+    p.r_pad = 32 * p.ntw;
+    const size_t per_block_2 = kSmemPerSM / 2 - kSmemReservedPerBlock;
+    p.blocks_per_sm = mass_smem_bytes(p.r_pad, 2) <= per_block_2 ? 2 : 1;
+    const size_t cap = p.blocks_per_sm == 2 ? per_block_2 : kSmemPerBlockMax;
+    p.stages = 0;
+    p.bytes = 0;
+    for (int st = 4; st >= 2; --st)
+        if (mass_smem_bytes(p.r_pad, st) <= cap) {
+            p.stages = st;
+            p.bytes = mass_smem_bytes(p.r_pad, st);
+            break;
+        }
+    p.sp = plan_decode_split(heads, N, p.blocks_per_sm);
+    return p;
+}
+
+struct MassWs {
+    size_t tickets, part, stats, total;
+};
+
+MassWs mass_ws_layout(int64_t heads, int R, int splits)
+{
+    MassWs w;
+    w.tickets = 256;
+    w.part = w.tickets + align_up((size_t)heads * sizeof(unsigned), 256);
+    w.stats = w.part + align_up((size_t)heads * splits * R * sizeof(float2), 256);
+    w.total = w.stats + (size_t)heads * R * sizeof(float2);
+    return w;
+}
+
+template <int PASS, int NTW>
+think_status_t launch_mass_kernel(const CUtensorMap &mk, const MassArgs &a, const MassPlan &p, int heads,
+                                  cudaStream_t st)
+{
+    auto kern = token_mass_kernel<PASS, NTW>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.bytes) != cudaSuccess)
+        return THINK_ERR_CUDA;
+    dim3 grid(a.splits, heads);
+    kern<<<grid, kMassThreads, p.bytes, st>>>(mk, a);
+    return launch_status();
+}
+
+template <int NTW>
+think_status_t launch_mass(const CUtensorMap &mk, const MassArgs &a, const MassPlan &p, int heads, cudaStream_t st)
+{
+    const think_status_t v = launch_mass_kernel<1, NTW>(mk, a, p, heads, st);
+    if (v != THINK_OK) return v;
+    return launch_mass_kernel<2, NTW>(mk, a, p, heads, st);
 }
 
 // ------------------------------------------------------------ 4-bit K' --
@@ -1087,6 +1150,109 @@ think_status_t think_pruned_decode_attn_ragged(const void *q, const void *k_prun
     a.Th = Th;
     a.rowoff = rowoff;
     return launch_decode_mma(G, mp.warps, mk, mv, a, mp.bytes, (int)heads, static_cast<cudaStream_t>(stream));
+}
+
+size_t think_token_mass_workspace_size(int B, int Hq, int Hkv, int64_t N, int S_obs)
+{
+    if (B < 0 || Hkv < 1 || Hq < Hkv || Hq % Hkv || N < 1 || S_obs < 1) return 0;
+    const int64_t heads = (int64_t)B * Hkv;
+    const int R = (Hq / Hkv) * S_obs;
+    const MassPlan p = plan_mass(R, heads, N);
+    return mass_ws_layout(heads, R, p.sp.splits).total;
+}
+
+think_status_t think_token_mass(const void *q_win, const void *k, const int64_t k_strides[3], int B, int Hq,
+                                int Hkv, int64_t N, int S_obs, int d, think_dtype_t dtype, float scale, float *mass,
+                                void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (B < 0 || Hq < 0 || Hkv < 0 || N < 0 || S_obs < 0 || !std::isfinite(scale)) return THINK_ERR_INVALID_ARG;
+    if (d != kD || dtype != THINK_BF16) return THINK_ERR_UNSUPPORTED;
+    if (B == 0 || Hkv == 0) return THINK_OK;
+    if (Hq < Hkv || Hq % Hkv != 0 || N < 1 || S_obs < 1) return THINK_ERR_INVALID_ARG;
+    const int R = (Hq / Hkv) * S_obs;
+    if (R > kMassRowsMax) return THINK_ERR_UNSUPPORTED;
+    if (!q_win || !k || !k_strides || !mass || !workspace) return THINK_ERR_INVALID_ARG;
+    const int64_t heads = (int64_t)B * Hkv;
+    if (heads > 65535 || N > (int64_t)INT32_MAX - kBN) return THINK_ERR_UNSUPPORTED;
+    if (!aligned16(q_win) || !aligned16(k) || !aligned16(workspace) || !strides_ok(k_strides, 2) ||
+        (reinterpret_cast<uintptr_t>(mass) & 3u))
+        return THINK_ERR_ALIGNMENT;
+    const MassPlan p = plan_mass(R, heads, N);
+    if (p.stages == 0) return THINK_ERR_UNSUPPORTED;
+    const MassWs w = mass_ws_layout(heads, R, p.sp.splits);
+    if (workspace_bytes < w.total) return THINK_ERR_WORKSPACE;
+    CUtensorMap mk;
+    // K as V is read by the decode: x = channel (two 64-channel halves), y = token
+    if (!make_map_4d(&mk, THINK_BF16, k, kD, (uint64_t)N, (uint64_t)Hkv, (uint64_t)B, k_strides[2], k_strides[1],
+                     k_strides[0], 64, kBN, true))
+        return THINK_ERR_CUDA;
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    MassArgs a;
+    a.qwin = static_cast<const __nv_bfloat16 *>(q_win);
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.S = S_obs;
+    a.G = Hq / Hkv;
+    a.R = R;
+    a.r_pad = p.r_pad;
+    a.N = N;
+    a.tiles_per_split = p.sp.tiles_per_split;
+    a.splits = p.sp.splits;
+    a.stages = p.stages;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.part = reinterpret_cast<float2 *>(ws + w.part);
+    a.stats = reinterpret_cast<float2 *>(ws + w.stats);
+    a.tickets = reinterpret_cast<unsigned *>(ws + w.tickets);
+    a.status = reinterpret_cast<unsigned *>(ws);
+    a.mass = mass;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    switch (p.ntw) {
+    case 2: return launch_mass<2>(mk, a, p, (int)heads, st);
+    case 4: return launch_mass<4>(mk, a, p, (int)heads, st);
+    case 8: return launch_mass<8>(mk, a, p, (int)heads, st);
+    default: return launch_mass<16>(mk, a, p, (int)heads, st);
+    }
+}
+
+think_status_t think_select_tokens(const float *mass, int B, int Hkv, int64_t N, int M, int32_t *kept,
+                                   void *stream)
+{
+    if (B < 0 || Hkv < 0 || N < 0) return THINK_ERR_INVALID_ARG;
+    if (B == 0 || Hkv == 0) return THINK_OK;
+    if (M < 1 || M > N || N > (int64_t)INT32_MAX) return THINK_ERR_INVALID_ARG;
+    if (!mass || !kept) return THINK_ERR_INVALID_ARG;
+    const int64_t heads = (int64_t)B * Hkv;
+    if (heads > 65535) return THINK_ERR_UNSUPPORTED;
+    if ((reinterpret_cast<uintptr_t>(mass) & 3u) || (reinterpret_cast<uintptr_t>(kept) & 3u))
+        return THINK_ERR_ALIGNMENT;
+    select_tokens_kernel<<<(unsigned)heads, 1024, 0, static_cast<cudaStream_t>(stream)>>>(mass, N, M, kept);
+    return launch_status();
+}
+
+think_status_t think_gather_tokens(const void *x, const int64_t x_strides[3], int B, int Hkv, int64_t N, int d,
+                                   think_dtype_t dtype, const int32_t *kept, int M, void *out, void *stream)
+{
+    if (B < 0 || Hkv < 0 || N < 0 || M < 0 || !dtype_ok(dtype)) return THINK_ERR_INVALID_ARG;
+    if (d != kD) return THINK_ERR_UNSUPPORTED;
+    if (B == 0 || Hkv == 0 || M == 0) return THINK_OK;
+    if (!x || !x_strides || !kept || !out) return THINK_ERR_INVALID_ARG;
+    const int64_t heads = (int64_t)B * Hkv;
+    if (heads > 65535) return THINK_ERR_UNSUPPORTED;
+    const size_t es = esize(dtype);
+    if (!aligned16(x) || !aligned16(out) || !strides_ok(x_strides, es) || (reinterpret_cast<uintptr_t>(kept) & 3u))
+        return THINK_ERR_ALIGNMENT;
+    const int rows_per_block = 256 / (kD / (int)(16 / es));
+    dim3 grid((unsigned)ceil_div(M, rows_per_block), (unsigned)heads);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dtype == THINK_BF16)
+        gather_tokens_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+            static_cast<const __nv_bfloat16 *>(x), x_strides[0], x_strides[1], x_strides[2], Hkv, M, kept, N,
+            static_cast<__nv_bfloat16 *>(out));
+    else
+        gather_tokens_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float *>(x), x_strides[0],
+                                                          x_strides[1], x_strides[2], Hkv, M, kept, N,
+                                                          static_cast<float *>(out));
+    return launch_status();
 }
 
 think_status_t think_workspace_init(void *workspace, size_t workspace_bytes, void *stream)

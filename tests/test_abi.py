@@ -188,6 +188,30 @@ def test_adaptive_validation():
     assert h(FAKE, FAKE, 64, FAKE, vs, FAKE, FAKE, FAKE, 32, 0, 4, 2, 64, 128, 0.1, FAKE, FAKE, 0, None) == qdk.THINK_OK
 
 
+def test_eviction_validation():
+    st = I64x3(128 * 64, 128 * 64, 128)
+    f = lib.think_token_mass
+    ws = qdk.think_token_mass_workspace_size(1, 4, 2, 64, 8)
+    assert ws > 256 and qdk.think_token_mass_workspace_size(1, 4, 3, 64, 8) == 0
+    # (q_win, k, strides, B, Hq, Hkv, N, S, d, dtype, scale, mass, ws, ws_bytes, stream)
+    assert f(FAKE, FAKE, st, 1, 4, 2, 64, 8, 128, 0, 0.1, FAKE, FAKE, ws, None) == qdk.THINK_ERR_UNSUPPORTED   # fp32
+    assert f(FAKE, FAKE, st, 1, 4, 2, 64, 8, 64, 1, 0.1, FAKE, FAKE, ws, None) == qdk.THINK_ERR_UNSUPPORTED    # d
+    assert f(FAKE, FAKE, st, 1, 16, 2, 64, 128, 128, 1, 0.1, FAKE, FAKE, 1 << 30, None) == qdk.THINK_ERR_UNSUPPORTED  # G*S > 512
+    assert f(FAKE, FAKE, st, 1, 4, 2, 64, 0, 128, 1, 0.1, FAKE, FAKE, ws, None) == qdk.THINK_ERR_INVALID_ARG    # S = 0
+    assert f(FAKE, FAKE, st, 1, 4, 2, 64, 8, 128, 1, 0.1, FAKE, FAKE, ws - 8, None) == qdk.THINK_ERR_WORKSPACE
+    assert f(FAKE, MISALIGNED, st, 1, 4, 2, 64, 8, 128, 1, 0.1, FAKE, FAKE, ws, None) == qdk.THINK_ERR_ALIGNMENT
+    assert f(FAKE, FAKE, st, 0, 4, 2, 64, 8, 128, 1, 0.1, FAKE, FAKE, 0, None) == qdk.THINK_OK
+    g = lib.think_select_tokens
+    assert g(FAKE, 1, 2, 64, 0, FAKE, None) == qdk.THINK_ERR_INVALID_ARG
+    assert g(FAKE, 1, 2, 64, 65, FAKE, None) == qdk.THINK_ERR_INVALID_ARG
+    assert g(None, 1, 2, 64, 8, FAKE, None) == qdk.THINK_ERR_INVALID_ARG
+    assert g(FAKE, 0, 2, 64, 8, FAKE, None) == qdk.THINK_OK
+    h = lib.think_gather_tokens
+    assert h(FAKE, st, 1, 2, 64, 96, 1, FAKE, 8, FAKE, None) == qdk.THINK_ERR_UNSUPPORTED
+    assert h(FAKE, st, 1, 2, 64, 128, 1, FAKE, 8, MISALIGNED, None) == qdk.THINK_ERR_ALIGNMENT
+    assert h(FAKE, st, 1, 2, 64, 128, 1, FAKE, 0, FAKE, None) == qdk.THINK_OK
+
+
 def test_decode_validation():
     s = I64x3(128 * 64 * 2, 128 * 64, 128)
     f = lib.think_pruned_decode_attn

@@ -293,6 +293,50 @@ def test_adaptive_width(case):
     assert qdk.think_read_device_status(cache.decode_ws) == 0
 
 
+@pytest.mark.parametrize("case", [(1, 32, 8, 5000, 32, 1000, 51), (2, 8, 2, 1000, 16, 300, 64),
+                                  (1, 4, 4, 300, 64, 300, 13), (1, 8, 1, 2049, 64, 129, 128),
+                                  (2, 16, 8, 700, 8, 1, 32), (1, 64, 8, 1500, 64, 500, 40)])
+def test_token_eviction_then_prune(case):
+    B, Hq, Hkv, N, S, M, T = case
+    q_win, k, v, q = _random_case(hash(case) & 0xFFFF, B, Hq, Hkv, N, S, torch.bfloat16, k_pad=8)
+    kd = torch.empty((B, Hkv, N + 8, 128), dtype=torch.bfloat16, device=DEV)[:, :, :N].copy_(k)
+    cache = qdk.EvictedCache(B, Hq, Hkv, N, S, M, T)
+    cache.prune(q_win.to(DEV), kd, v.to(DEV))
+    out = torch.empty((B, Hq, 128), dtype=torch.float32, device=DEV)
+    cache.decode(q.to(DEV), out)
+    torch.cuda.synchronize()
+    assert qdk.think_read_device_status(cache.mass_ws) == 0
+    # masses: fp32 sums of exp2-approximated weights against the fp64 oracle
+    ora_mass = oracle.oracle_token_mass(f64(q_win), f64(k))
+    gm = f64(cache.mass)
+    np.testing.assert_allclose(gm, ora_mass, rtol=2e-4, atol=1e-6 * (Hq // Hkv) * S)
+    # the selection on the GPU's masses is the oracle's selection on the same masses
+    kept = cache.kept.cpu().numpy()
+    assert np.array_equal(kept, oracle.oracle_select_tokens(gm, M))
+    # against the oracle's own masses it may differ only at near-ties of the cut
+    ora_kept = oracle.oracle_select_tokens(ora_mass, M)
+    for b in range(B):
+        for h in range(Hkv):
+            diff = set(kept[b, h]) ^ set(ora_kept[b, h])
+            if diff:
+                cut = np.sort(ora_mass[b, h])[::-1][M - 1]
+                assert all(abs(ora_mass[b, h, n] - cut) <= 5e-4 * cut for n in diff), (b, h, diff)
+    # gathers are exact copies; the prune and decode run on the kept tokens
+    kk = oracle.oracle_gather_tokens(f64(k), kept)
+    assert np.array_equal(f64(cache.k_kept), kk)
+    assert np.array_equal(f64(cache.v_kept), oracle.oracle_gather_tokens(f64(v), kept))
+    ora_scores, ora_idx, ora_kp = oracle.oracle_prune(f64(q_win), kk, T)
+    check_scores(cache.pruned.scores, ora_scores)
+    if idx_mismatch_heads(cache.pruned.idx.cpu().numpy(), ora_idx, ora_scores, T):
+        cache.pruned.idx.copy_(torch.from_numpy(ora_idx))
+        qdk.think_compact_keys(cache.k_kept, cache.pruned.idx, cache.pruned.k_pruned, cache.pruned.ldk)
+        cache.decode(q.to(DEV), out)
+        torch.cuda.synchronize()
+    assert np.array_equal(kp_logical(cache.pruned.k_pruned, M), ora_kp)
+    check_out(out, oracle.oracle_decode(f64(q), ora_kp, oracle.oracle_gather_tokens(f64(v), kept), ora_idx),
+              torch.bfloat16, where=str(case))
+
+
 def test_ldk_larger_than_needed_and_exact_ties():
     # duplicate channels give exact score ties: lower index must win on both sides
     B, Hq, Hkv, N, S, T = 1, 4, 2, 300, 6, 40
