@@ -23,13 +23,13 @@
 
 namespace think {
 
-constexpr int kMassWarps = 4;
+constexpr int kMassWarps = 8;
 constexpr int kMassThreads = kMassWarps * 32 + 32;  // + TMA producer warp
 constexpr int kMassRowsMax = 512;                   // G * S_obs
 
 struct MassArgs {
     const __nv_bfloat16 *qwin;  // [B][Hq][S][128]
-    int Hq, Hkv, S, G, R, r_pad;  // R = G * S rows; r_pad = R rounded up to 8 * kMassWarps
+    int Hq, Hkv, S, G, R, r_pad;  // R = G * S rows; r_pad = 8 * kMassWarps * NTW >= R
     int64_t N;
     int tiles_per_split, splits, stages;
     float scale_log2;           // scale * log2(e)
@@ -56,7 +56,8 @@ __host__ __device__ inline size_t mass_smem_bytes(int r_pad, int stages)
            (size_t)kMassWarps * kBN * 4u + (size_t)2 * stages * 8u + 16u + 1024u;
 }
 
-// NTW: 8-row query groups per warp (r_pad = 32 * NTW).
+// NTW: 8-row query groups per warp (r_pad = 64 * NTW).  With NTW <= 4 a warp
+// keeps the B fragments of its rows in registers for the whole block.
 template <int PASS, int NTW>
 __global__ void __launch_bounds__(kMassThreads)
     token_mass_kernel(const __grid_constant__ CUtensorMap tm_k, const MassArgs a)
@@ -141,9 +142,26 @@ __global__ void __launch_bounds__(kMassThreads)
     named_barrier(1, NT);
 
     const int q4 = lane & 3, r8 = lane >> 2;
+    const int mi = lane >> 3, rr = lane & 7;  // ldmatrix: matrix index, row within it
     const uint32_t qbase = smem_addr(qs);
-    // pass 1: running (max, lane-partial sum) for the warp's n-tiles (warp,
-    // warp + 4, ...), 2 columns each
+    constexpr bool kBRegs = NTW <= 4;
+    // B fragments (k = channel, n = query row) of the warp's row groups
+    // warp, warp + 8, ...: two registers per 16-channel step
+    uint32_t bq[kBRegs ? NTW : 1][8][2];
+    if (kBRegs) {
+#pragma unroll
+        for (int j = 0; j < (kBRegs ? NTW : 1); ++j) {
+            const uint32_t n = (uint32_t)(8 * (warp + kMassWarps * j) + rr);
+#pragma unroll
+            for (int kp = 0; kp < 4; ++kp) {
+                const uint32_t chunk = (uint32_t)(4 * kp + mi);
+                ldsm_x4(qbase + (chunk >> 3) * q_half + n * 128u + (((chunk & 7u) ^ (n & 7u)) << 4),
+                        bq[j][2 * kp][0], bq[j][2 * kp][1], bq[j][2 * kp + 1][0], bq[j][2 * kp + 1][1]);
+            }
+        }
+    }
+    // pass 1: this lane's running (max, sum of 2^(z - max)) over the tokens it
+    // sees, for the 2 rows of each of its row groups
     float rm[NTW][2], rl[NTW][2];
 #pragma unroll
     for (int j = 0; j < NTW; ++j)
@@ -160,10 +178,8 @@ __global__ void __launch_bounds__(kMassThreads)
         const int64_t tok0 = (tile0 + it) * kBN;
 #pragma unroll 1
         for (int mt = 0; mt < 8; ++mt) {
-            float tacc[2] = {0.f, 0.f};  // pass 2: this lane's sums for tokens 16 mt + r8, + 8
             // A fragments: tokens 16 mt .. +15, all 8 channel steps
             uint32_t af[8][4];
-            const int mi = lane >> 3, rr = lane & 7;
             const uint32_t tok = (uint32_t)(16 * mt + (mi & 1) * 8 + rr);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
@@ -172,20 +188,28 @@ __global__ void __launch_bounds__(kMassThreads)
                         af[ks][1], af[ks][2], af[ks][3]);
             }
             const bool v0 = tok0 + 16 * mt + r8 < a.N, v1 = tok0 + 16 * mt + 8 + r8 < a.N;
+            float tacc[2] = {0.f, 0.f};  // pass 2: this lane's sums for tokens 16 mt + r8, + 8
 #pragma unroll
             for (int j = 0; j < NTW; ++j) {
                 const int nt = warp + kMassWarps * j;
                 float c[4] = {0.f, 0.f, 0.f, 0.f};
-                const uint32_t n = (uint32_t)(8 * nt + rr);
+                if (kBRegs) {
 #pragma unroll
-                for (int kp = 0; kp < 4; ++kp) {
-                    uint32_t b0, b1, b2, b3;
-                    const uint32_t chunk = (uint32_t)(4 * kp + mi);
-                    ldsm_x4(qbase + (chunk >> 3) * q_half + n * 128u + (((chunk & 7u) ^ (n & 7u)) << 4), b0, b1,
-                            b2, b3);
-                    wmma16::mma_bf16(c, af[2 * kp][0], af[2 * kp][1], af[2 * kp][2], af[2 * kp][3], b0, b1);
-                    wmma16::mma_bf16(c, af[2 * kp + 1][0], af[2 * kp + 1][1], af[2 * kp + 1][2],
-                                     af[2 * kp + 1][3], b2, b3);
+                    for (int ks = 0; ks < 8; ++ks)
+                        wmma16::mma_bf16(c, af[ks][0], af[ks][1], af[ks][2], af[ks][3], bq[kBRegs ? j : 0][ks][0],
+                                         bq[kBRegs ? j : 0][ks][1]);
+                } else {
+                    const uint32_t n = (uint32_t)(8 * nt + rr);
+#pragma unroll
+                    for (int kp = 0; kp < 4; ++kp) {
+                        uint32_t b0, b1, b2, b3;
+                        const uint32_t chunk = (uint32_t)(4 * kp + mi);
+                        ldsm_x4(qbase + (chunk >> 3) * q_half + n * 128u + (((chunk & 7u) ^ (n & 7u)) << 4), b0,
+                                b1, b2, b3);
+                        wmma16::mma_bf16(c, af[2 * kp][0], af[2 * kp][1], af[2 * kp][2], af[2 * kp][3], b0, b1);
+                        wmma16::mma_bf16(c, af[2 * kp + 1][0], af[2 * kp + 1][1], af[2 * kp + 1][2],
+                                         af[2 * kp + 1][3], b2, b3);
+                    }
                 }
                 // c[0], c[1]: token 16 mt + r8, rows 8 nt + 2 q4 (+1); c[2], c[3]: token + 8
                 if (PASS == 1) {
@@ -193,17 +217,11 @@ __global__ void __launch_bounds__(kMassThreads)
                     for (int h = 0; h < 2; ++h) {
                         const float z0 = v0 ? c[h] * a.scale_log2 : -INFINITY;
                         const float z1 = v1 ? c[2 + h] * a.scale_log2 : -INFINITY;
-                        float xm = fmaxf(z0, z1);
-                        xm = fmaxf(xm, __shfl_xor_sync(0xffffffffu, xm, 4));
-                        xm = fmaxf(xm, __shfl_xor_sync(0xffffffffu, xm, 8));
-                        xm = fmaxf(xm, __shfl_xor_sync(0xffffffffu, xm, 16));
-                        const float mnew = fmaxf(rm[j][h], xm);
-                        if (mnew != -INFINITY) {
-                            const float alpha = rm[j][h] == -INFINITY ? 0.f : exp2_approx(rm[j][h] - mnew);
-                            rl[j][h] = rl[j][h] * alpha + (v0 ? exp2_approx(z0 - mnew) : 0.f) +
-                                       (v1 ? exp2_approx(z1 - mnew) : 0.f);
-                            rm[j][h] = mnew;
-                        }
+                        const float mnew = fmaxf(rm[j][h], fmaxf(z0, z1));
+                        const float mref = mnew == -INFINITY ? 0.f : mnew;
+                        rl[j][h] = rl[j][h] * exp2_approx(rm[j][h] - mref) + exp2_approx(z0 - mref) +
+                                   exp2_approx(z1 - mref);
+                        rm[j][h] = mnew;
                     }
                 } else {
                     const float2 s0 = rstat[8 * nt + 2 * q4], s1 = rstat[8 * nt + 2 * q4 + 1];
@@ -227,7 +245,7 @@ __global__ void __launch_bounds__(kMassThreads)
         __syncwarp();
         if (lane == 0) mbar_arrive(empty0 + 8 * s);
         if (PASS == 2) {
-            // the four warps' row groups in order: the tile's masses
+            // the warps' row groups in order: the tile's masses
             named_barrier(1, NT);
             if (tid < kBN && tok0 + tid < a.N) {
                 float m = 0.f;
@@ -245,13 +263,19 @@ __global__ void __launch_bounds__(kMassThreads)
     for (int j = 0; j < NTW; ++j)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            float l = rl[j][h];
-            l += __shfl_xor_sync(0xffffffffu, l, 4);
-            l += __shfl_xor_sync(0xffffffffu, l, 8);
-            l += __shfl_xor_sync(0xffffffffu, l, 16);
+            // merge the 8 lanes that saw the other tokens of these rows
+            float m = rm[j][h], l = rl[j][h];
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) {
+                const float mo = __shfl_xor_sync(0xffffffffu, m, o), lo = __shfl_xor_sync(0xffffffffu, l, o);
+                const float mm = fmaxf(m, mo);
+                const float mref = mm == -INFINITY ? 0.f : mm;
+                l = l * exp2_approx(m - mref) + lo * exp2_approx(mo - mref);
+                m = mm;
+            }
             const int r = 8 * (warp + kMassWarps * j) + 2 * q4 + h;
             if (r8 == 0 && r < a.R)
-                a.part[((int64_t)head * a.splits + split) * a.R + r] = make_float2(rm[j][h], l);
+                a.part[((int64_t)head * a.splits + split) * a.R + r] = make_float2(m, l);
         }
     __threadfence();
     named_barrier(1, NT);

@@ -517,8 +517,8 @@ struct MassPlan {
 MassPlan plan_mass(int R, int64_t heads, int64_t N)
 {
     MassPlan p;
-    p.ntw = R <= 64 ? 2 : R <= 128 ? 4 : R <= 256 ? 8 : 16;
-    p.r_pad = 32 * p.ntw;
+    p.ntw = R <= 64 ? 1 : R <= 128 ? 2 : R <= 256 ? 4 : 8;
+    p.r_pad = 8 * kMassWarps * p.ntw;
     const size_t per_block_2 = kSmemPerSM / 2 - kSmemReservedPerBlock;
     p.blocks_per_sm = mass_smem_bytes(p.r_pad, 2) <= per_block_2 ? 2 : 1;
     const size_t cap = p.blocks_per_sm == 2 ? per_block_2 : kSmemPerBlockMax;
@@ -1207,10 +1207,10 @@ think_status_t think_token_mass(const void *q_win, const void *k, const int64_t 
     a.mass = mass;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     switch (p.ntw) {
+    case 1: return launch_mass<1>(mk, a, p, (int)heads, st);
     case 2: return launch_mass<2>(mk, a, p, (int)heads, st);
     case 4: return launch_mass<4>(mk, a, p, (int)heads, st);
-    case 8: return launch_mass<8>(mk, a, p, (int)heads, st);
-    default: return launch_mass<16>(mk, a, p, (int)heads, st);
+    default: return launch_mass<8>(mk, a, p, (int)heads, st);
     }
 }
 
