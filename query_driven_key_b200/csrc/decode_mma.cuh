@@ -306,6 +306,11 @@ __global__ void __launch_bounds__(CW * 32 + 32)
     static_assert(CW == 4 || CW == 8, "32 or 16 tokens of a tile per consumer warp");
     constexpr int TPW = kBN / CW;
     constexpr int NT = CW * 32;
+    // Launched as a programmatic dependent of the previous kernel in the
+    // stream: everything it wrote is visible after this wait; let the next
+    // decode be scheduled on SMs as ours free up.
+    grid_dependency_wait();
+    grid_launch_dependents();
     extern __shared__ unsigned char smem_dyn[];
     unsigned char *smem = smem_dyn + ((1024u - (smem_addr(smem_dyn) & 1023u)) & 1023u);
 

@@ -141,6 +141,11 @@ __global__ void __launch_bounds__(CW * 32 + 32)
     constexpr int NT = CW * 32;
     constexpr int PARTS = TPW / 8;       // 8-token chunks per warp and channel row
     constexpr int RPP = 32 / PARTS;      // channel rows per pass of a warp
+    // Launched as a programmatic dependent of the previous kernel in the
+    // stream: everything it wrote is visible after this wait; let the next
+    // decode be scheduled on SMs as ours free up.
+    grid_dependency_wait();
+    grid_launch_dependents();
     extern __shared__ unsigned char smem_dyn[];
     unsigned char *smem = smem_dyn + ((1024u - (smem_addr(smem_dyn) & 1023u)) & 1023u);
 

@@ -176,6 +176,12 @@ __device__ __forceinline__ void st_release_gpu(unsigned *p, unsigned v)
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+// Programmatic dependent launch: wait until the grids this one depends on
+// have completed and their memory is visible (a no-op without them), and
+// allow the grid launched after this one to be scheduled.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
 // 2^x on the MUFU unit (flush-to-zero; relative error about 2^-22).
 __device__ __forceinline__ float exp2_approx(float x)
 {

@@ -11,6 +11,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "decode_kernels.cuh"
 #include "decode_mma.cuh"
@@ -57,6 +58,26 @@ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline think_status_t launch_status()
 {
     return cudaGetLastError() == cudaSuccess ? THINK_OK : THINK_ERR_CUDA;
+}
+
+// Launch with programmatic stream serialisation (the kernel may start while
+// the previous kernel of the stream drains; it waits in griddepcontrol.wait
+// before its first global access).  THINK_PDL=0 launches plainly.
+template <typename... KArgs, typename... Args>
+think_status_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                          Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = env_int("THINK_PDL", 1, 0, 1);
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) == cudaSuccess ? THINK_OK : THINK_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------- plans --
@@ -482,8 +503,7 @@ think_status_t launch_decode_mma_gw(const CUtensorMap &mk, const CUtensorMap &mv
         cudaSuccess)
         return THINK_ERR_CUDA;
     dim3 grid(a.splits, heads);
-    kern<<<grid, CW * 32 + 32, bytes, st>>>(mk, mv, a);
-    return launch_status();
+    return launch_pdl(kern, grid, dim3(CW * 32 + 32), bytes, st, mk, mv, a);
 }
 
 template <int G>
@@ -607,8 +627,7 @@ think_status_t launch_decode_q4_gw(const CUtensorMap &mc, const CUtensorMap &mg,
         cudaSuccess)
         return THINK_ERR_CUDA;
     dim3 grid(a.splits, heads);
-    kern<<<grid, CW * 32 + 32, bytes, st>>>(mc, mg, mv, a);
-    return launch_status();
+    return launch_pdl(kern, grid, dim3(CW * 32 + 32), bytes, st, mc, mg, mv, a);
 }
 
 template <int G>
