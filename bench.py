@@ -48,7 +48,7 @@ def parse():
     p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", default="native", choices=["native", "reference"])
-    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--e2e-steps", type=int, default=6)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-extras", action="store_true",
                    help="skip the measurements outside the step (append, 4-bit and adaptive-width decode)")
@@ -465,16 +465,17 @@ def run_native(args):
     # prune: score+select, compact; one kernel per decode
     launches_per_step = R * (2 + w.decode_steps)
 
-    def one_step(ev=None):
+    def one_step(ev=None, bufs=None):
+        qw_b, k_b, v_b, qs_b = bufs if bufs is not None else (qw_d, k_d, v_d, qs_d)
         if ev is not None:
             ev[0].record(stream)
         for r in range(R):
-            caches[r].prune(qw_d[r], k_d[r], stream=stream)
+            caches[r].prune(qw_b[r], k_b[r], stream=stream)
         if ev is not None:
             ev[1].record(stream)
         for s in range(w.decode_steps):
             for r in range(R):
-                caches[r].decode(qs_d[s], v_d[r], outs[s, r], stream=stream)
+                caches[r].decode(qs_b[s], v_b[r], outs[s, r], stream=stream)
         if ev is not None:
             ev[2].record(stream)
 
@@ -516,6 +517,12 @@ def run_native(args):
     peak, peak_kind = measured_peaks()
 
     # ---------------------------------------------- end to end (host buffers)
+    # Every step copies its inputs (window queries, K, V, the decode queries)
+    # from pinned host memory and reads its outputs (decode outputs, kept
+    # channels) back, inside the timed region.  With one resident layer the
+    # device inputs are double-buffered: a copy stream fills one set while the
+    # compute stream works on the other (events order them), as a server that
+    # prefetches the next request would.
     e2e = None
     if args.e2e_steps > 0:
         pin = lambda t: t.pin_memory()
@@ -525,33 +532,57 @@ def run_native(args):
         h2d = R * sum(t.numel() * t.element_size() for t in (h_qw, h_k, h_v)) \
             + h_qs.numel() * h_qs.element_size()
         d2h = h_out.numel() * 4 + h_idx.numel() * 4
+        sets = [(qw_d, k_d, v_d, qs_d)]
+        if R == 1:
+            with torch.cuda.stream(stream):
+                sets.append(([t.clone() for t in qw_d], [t.clone() for t in k_d], [t.clone() for t in v_d],
+                             qs_d.clone()))
+        copy_stream = torch.cuda.Stream(device=dev)
+        free = [torch.cuda.Event() for _ in sets]
+        ready = [torch.cuda.Event() for _ in sets]
+        for e in free:
+            e.record(stream)
 
-        def e2e_step():
-            for r in range(R):
-                qw_d[r].copy_(h_qw, non_blocking=True)
-                k_d[r].copy_(h_k, non_blocking=True)
-                v_d[r].copy_(h_v, non_blocking=True)
-            qs_d.copy_(h_qs, non_blocking=True)
-            one_step()
-            h_out.copy_(outs, non_blocking=True)
-            for r in range(R):
-                h_idx[r].copy_(caches[r].idx, non_blocking=True)
+        def copy_in(i):
+            qw_b, k_b, v_b, qs_b = sets[i]
+            copy_stream.wait_event(free[i])
+            with torch.cuda.stream(copy_stream):
+                for r in range(R):
+                    qw_b[r].copy_(h_qw, non_blocking=True)
+                    k_b[r].copy_(h_k, non_blocking=True)
+                    v_b[r].copy_(h_v, non_blocking=True)
+                qs_b.copy_(h_qs, non_blocking=True)
+            ready[i].record(copy_stream)
 
-        with torch.cuda.stream(stream):
-            e2e_step()
-            stream.synchronize()
-            if world > 1:
-                dist.barrier()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for _ in range(args.e2e_steps):
-                e2e_step()
-            e1.record(stream)
-            stream.synchronize()
+        def e2e_steps(n):
+            copy_in(0)
+            for j in range(n):
+                i = j % len(sets)
+                if j + 1 < n:
+                    copy_in((j + 1) % len(sets))   # the next step's inputs, while this one computes
+                stream.wait_event(ready[i])
+                with torch.cuda.stream(stream):
+                    one_step(bufs=sets[i])
+                    h_out.copy_(outs, non_blocking=True)
+                    for r in range(R):
+                        h_idx[r].copy_(caches[r].idx, non_blocking=True)
+                free[i].record(stream)
+
+        e2e_steps(2)
+        stream.synchronize()
+        copy_stream.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        copy_stream.wait_event(e0)
+        e2e_steps(args.e2e_steps)
+        e1.record(stream)
+        stream.synchronize()
         e2e_ms = max_over_ranks([e0.elapsed_time(e1) / args.e2e_steps], dev)[0]
         e2e = {"value": aggregate_gbs(world, nbytes, e2e_ms), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-               "steps": args.e2e_steps}
+               "steps": args.e2e_steps, "input_buffers": len(sets)}
 
     extras = rank == 0 and not args.no_extras
     append = measure_append(w, T, dev, stream, qw_d[0], k_d[0]) if extras else None
