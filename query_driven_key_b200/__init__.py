@@ -509,6 +509,27 @@ class PrunedCache:
                                     N=self.n, scale=scale, stream=stream)
 
     def decode(self, q, v, out, scale=None, stream=None):
-        """Attend over the current n tokens (v holds at least n token rows)."""
-        think_pruned_decode_attn(q, self.k_pruned, self.ldk, v, self.idx, out, self.decode_ws,
-                                 scale=scale, N=self.n, stream=stream)
+        """Attend over the current n tokens (v holds at least n token rows).
+
+        The arguments that do not change between decode steps (this cache's
+        buffers, V's address and strides, the scale) are marshalled once and
+        reused while V and the scale stay the same."""
+        key = (v.data_ptr(), v.stride(), tuple(v.shape), v.dtype, scale)
+        if key != getattr(self, "_dkey", None):
+            think_pruned_decode_attn(q, self.k_pruned, self.ldk, v, self.idx, out, self.decode_ws,
+                                     scale=scale, N=self.n, stream=stream)
+            d = q.shape[-1]
+            self._dconst = (self.k_pruned.data_ptr(), int(self.ldk), v.data_ptr(), _strides3(v),
+                            self.idx.data_ptr(), _dtype(q),
+                            float(1.0 / float(d) ** 0.5 if scale is None else scale),
+                            self.decode_ws.data_ptr(), self.decode_ws.numel())
+            self._dshape = (tuple(q.shape), q.dtype, tuple(out.shape))
+            self._dkey = key
+            return
+        if (tuple(q.shape), q.dtype, tuple(out.shape)) != self._dshape or not q.is_contiguous() \
+                or out.dtype != torch.float32:
+            raise ThinkError(THINK_ERR_INVALID_ARG, "PrunedCache.decode")
+        kp, ldk, vp, vs, ip, dt, sc, wp, wb = self._dconst
+        _check(lib.think_pruned_decode_attn(q.data_ptr(), kp, ldk, vp, vs, ip, self.B, self.Hq, self.Hkv, self.n,
+                                            self.d, self.T, dt, sc, out.data_ptr(), wp, wb, _stream(stream)),
+               "think_pruned_decode_attn")

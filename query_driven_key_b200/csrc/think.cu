@@ -190,11 +190,32 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
+// Encoded maps are kept in a small per-thread cache keyed by every input of
+// the encoding (a decode step re-encodes the same two maps otherwise).
+struct MapKey {
+    const void *base;
+    uint64_t dims[4], strides[3];
+    uint32_t box[2];
+    int dtype, swizzle;
+};
+
+bool map_cache_find(const MapKey &k, CUtensorMap *m);
+void map_cache_put(const MapKey &k, const CUtensorMap &m);
+
 // 4-D map over (x, y, z, w) with element strides sy, sz, sw for y, z, w; box (bx, by, 1, 1).
 bool make_map_4d(CUtensorMap *m, think_dtype_t dt, const void *base, uint64_t dx, uint64_t dy,
                  uint64_t dz, uint64_t dw, int64_t sy, int64_t sz, int64_t sw, uint32_t bx,
                  uint32_t by, bool swizzle128 = false)
 {
+    MapKey key;
+    memset(&key, 0, sizeof(key));
+    key.base = base;
+    key.dims[0] = dx, key.dims[1] = dy, key.dims[2] = dz, key.dims[3] = dw;
+    key.strides[0] = (uint64_t)sy, key.strides[1] = (uint64_t)sz, key.strides[2] = (uint64_t)sw;
+    key.box[0] = bx, key.box[1] = by;
+    key.dtype = (int)dt;
+    key.swizzle = swizzle128 ? 1 : 0;
+    if (map_cache_find(key, m)) return true;
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const size_t es = esize(dt);
@@ -208,7 +229,61 @@ bool make_map_4d(CUtensorMap *m, think_dtype_t dt, const void *base, uint64_t dx
                           CU_TENSOR_MAP_INTERLEAVE_NONE,
                           swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    if (r != CUDA_SUCCESS) return false;
+    map_cache_put(key, *m);
+    return true;
+}
+
+constexpr int kMapCacheSize = 16;
+struct MapCacheEntry {
+    MapKey key;
+    CUtensorMap map;
+    bool used;
+};
+thread_local MapCacheEntry g_map_cache[kMapCacheSize];
+thread_local int g_map_next = 0;
+
+bool map_cache_find(const MapKey &k, CUtensorMap *m)
+{
+    for (int i = 0; i < kMapCacheSize; ++i)
+        if (g_map_cache[i].used && memcmp(&g_map_cache[i].key, &k, sizeof(MapKey)) == 0) {
+            *m = g_map_cache[i].map;
+            return true;
+        }
+    return false;
+}
+
+void map_cache_put(const MapKey &k, const CUtensorMap &m)
+{
+    MapCacheEntry &e = g_map_cache[g_map_next];
+    g_map_next = (g_map_next + 1) % kMapCacheSize;
+    e.key = k;
+    e.map = m;
+    e.used = true;
+}
+
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per kernel, device
+// and size (per thread; the attribute itself is per device).
+bool ensure_smem(const void *kern, size_t bytes)
+{
+    struct Entry {
+        const void *kern;
+        int dev;
+        size_t bytes;
+    };
+    thread_local Entry seen[64];
+    thread_local int nseen = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    for (int i = 0; i < nseen; ++i)
+        if (seen[i].kern == kern && seen[i].dev == dev && seen[i].bytes >= bytes) return true;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
+        return false;
+    Entry &e = seen[nseen < 64 ? nseen++ : (int)(reinterpret_cast<uintptr_t>(kern) >> 4) % 64];
+    e.kern = kern;
+    e.dev = dev;
+    e.bytes = bytes;
+    return true;
 }
 
 // 4-D map of any element type with byte strides; box (bx, by, 1, 1), no swizzle.
@@ -216,15 +291,26 @@ bool make_map_raw_4d(CUtensorMap *m, CUtensorMapDataType dt, const void *base, u
                      uint64_t dz, uint64_t dw, uint64_t sy_bytes, uint64_t sz_bytes, uint64_t sw_bytes,
                      uint32_t bx, uint32_t by)
 {
+    MapKey key;
+    memset(&key, 0, sizeof(key));
+    key.base = base;
+    key.dims[0] = dx, key.dims[1] = dy, key.dims[2] = dz, key.dims[3] = dw;
+    key.strides[0] = sy_bytes, key.strides[1] = sz_bytes, key.strides[2] = sw_bytes;
+    key.box[0] = bx, key.box[1] = by;
+    key.dtype = 100 + (int)dt;
+    if (map_cache_find(key, m)) return true;
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[4] = {dx, dy, dz, dw};
     cuuint64_t strides[3] = {sy_bytes, sz_bytes, sw_bytes};
     cuuint32_t box[4] = {bx, by, 1, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
-    return fn(m, dt, 4, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    if (fn(m, dt, 4, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+           CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    map_cache_put(key, *m);
+    return true;
 }
 
 // ---------------------------------------------------------- validation --
@@ -242,8 +328,7 @@ think_status_t launch_decode_g(const CUtensorMap &mk, const CUtensorMap &mv, con
                                const DecodeSmem &sm, int heads, cudaStream_t st)
 {
     auto kern = pruned_decode_kernel<TIn, G>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm.bytes) !=
-        cudaSuccess)
+    if (!ensure_smem(reinterpret_cast<const void *>(kern), sm.bytes))
         return THINK_ERR_CUDA;
     dim3 grid(a.splits, heads);
     kern<<<grid, kDecodeThreads, sm.bytes, st>>>(mk, mv, a);
@@ -449,8 +534,7 @@ think_status_t launch_prune_fused(const void *q_win, const void *k, const int64_
     a.kp = static_cast<__nv_bfloat16 *>(k_pruned);
     a.ldk = ldk;
     a.N = N;
-    if (cudaFuncSetAttribute(prune_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kPfSmemBytes) != cudaSuccess)
+    if (!ensure_smem(reinterpret_cast<const void *>(prune_fused_kernel), kPfSmemBytes))
         return THINK_ERR_CUDA;
     prune_fused_kernel<<<p.grid, kPfThreads, kPfSmemBytes, st>>>(mk, a);
     return launch_status();
@@ -499,8 +583,7 @@ think_status_t launch_decode_mma_gw(const CUtensorMap &mk, const CUtensorMap &mv
                                     size_t bytes, int heads, cudaStream_t st)
 {
     auto kern = pruned_decode_mma_kernel<G, CW>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
-        cudaSuccess)
+    if (!ensure_smem(reinterpret_cast<const void *>(kern), bytes))
         return THINK_ERR_CUDA;
     dim3 grid(a.splits, heads);
     return launch_pdl(kern, grid, dim3(CW * 32 + 32), bytes, st, mk, mv, a);
@@ -573,7 +656,7 @@ think_status_t launch_mass_kernel(const CUtensorMap &mk, const MassArgs &a, cons
                                   cudaStream_t st)
 {
     auto kern = token_mass_kernel<PASS, NTW>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.bytes) != cudaSuccess)
+    if (!ensure_smem(reinterpret_cast<const void *>(kern), p.bytes))
         return THINK_ERR_CUDA;
     dim3 grid(a.splits, heads);
     kern<<<grid, kMassThreads, p.bytes, st>>>(mk, a);
@@ -623,8 +706,7 @@ think_status_t launch_decode_q4_gw(const CUtensorMap &mc, const CUtensorMap &mg,
                                    const DecodeArgs &a, size_t bytes, int heads, cudaStream_t st)
 {
     auto kern = pruned_decode_q4_kernel<G, CW>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
-        cudaSuccess)
+    if (!ensure_smem(reinterpret_cast<const void *>(kern), bytes))
         return THINK_ERR_CUDA;
     dim3 grid(a.splits, heads);
     return launch_pdl(kern, grid, dim3(CW * 32 + 32), bytes, st, mc, mg, mv, a);
@@ -686,8 +768,7 @@ think_status_t launch_decode_tc_g(const CUtensorMap &mk, const CUtensorMap &mv, 
                                   size_t bytes, int heads, cudaStream_t st)
 {
     auto kern = pruned_decode_tc_kernel<G>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
-        cudaSuccess)
+    if (!ensure_smem(reinterpret_cast<const void *>(kern), bytes))
         return THINK_ERR_CUDA;
     dim3 grid(a.splits, heads);
     kern<<<grid, kTcThreads, bytes, st>>>(mk, mv, a);
