@@ -256,44 +256,44 @@ __global__ void __launch_bounds__(kMassThreads)
             named_barrier(1, NT);
         }
     }
-    if (PASS == 2) return;
-
-    // ---- pass 1: the block's row statistics, then the last block of the head merges
+    if constexpr (PASS == 1) {
+        // ---- pass 1: the block's row statistics, then the last block of the head merges
 #pragma unroll
-    for (int j = 0; j < NTW; ++j)
+        for (int j = 0; j < NTW; ++j)
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            // merge the 8 lanes that saw the other tokens of these rows
-            float m = rm[j][h], l = rl[j][h];
+            for (int h = 0; h < 2; ++h) {
+                // merge the 8 lanes that saw the other tokens of these rows
+                float m = rm[j][h], l = rl[j][h];
 #pragma unroll
-            for (int o = 4; o < 32; o <<= 1) {
-                const float mo = __shfl_xor_sync(0xffffffffu, m, o), lo = __shfl_xor_sync(0xffffffffu, l, o);
-                const float mm = fmaxf(m, mo);
-                const float mref = mm == -INFINITY ? 0.f : mm;
-                l = l * exp2_approx(m - mref) + lo * exp2_approx(mo - mref);
-                m = mm;
+                for (int o = 4; o < 32; o <<= 1) {
+                    const float mo = __shfl_xor_sync(0xffffffffu, m, o), lo = __shfl_xor_sync(0xffffffffu, l, o);
+                    const float mm = fmaxf(m, mo);
+                    const float mref = mm == -INFINITY ? 0.f : mm;
+                    l = l * exp2_approx(m - mref) + lo * exp2_approx(mo - mref);
+                    m = mm;
+                }
+                const int r = 8 * (warp + kMassWarps * j) + 2 * q4 + h;
+                if (r8 == 0 && r < a.R)
+                    a.part[((int64_t)head * a.splits + split) * a.R + r] = make_float2(m, l);
             }
-            const int r = 8 * (warp + kMassWarps * j) + 2 * q4 + h;
-            if (r8 == 0 && r < a.R)
-                a.part[((int64_t)head * a.splits + split) * a.R + r] = make_float2(m, l);
+        __threadfence();
+        named_barrier(1, NT);
+        if (tid == 0) *flag = (atomicAdd(a.tickets + head, 1u) == (unsigned)(a.splits - 1)) ? 1u : 0u;
+        named_barrier(1, NT);
+        if (*flag == 0u) return;
+        __threadfence();
+        for (int r = tid; r < a.R; r += NT) {
+            float M = -INFINITY;
+            for (int s = 0; s < a.splits; ++s) M = fmaxf(M, __ldcg(a.part + ((int64_t)head * a.splits + s) * a.R + r).x);
+            float L = 0.f;
+            for (int s = 0; s < a.splits; ++s) {
+                const float2 p = __ldcg(a.part + ((int64_t)head * a.splits + s) * a.R + r);
+                if (p.x != -INFINITY) L = fmaf(p.y, exp2_approx(p.x - M), L);
+            }
+            a.stats[(int64_t)head * a.R + r] = make_float2(M, L > 0.f ? 1.f / L : 0.f);
         }
-    __threadfence();
-    named_barrier(1, NT);
-    if (tid == 0) *flag = (atomicAdd(a.tickets + head, 1u) == (unsigned)(a.splits - 1)) ? 1u : 0u;
-    named_barrier(1, NT);
-    if (*flag == 0u) return;
-    __threadfence();
-    for (int r = tid; r < a.R; r += NT) {
-        float M = -INFINITY;
-        for (int s = 0; s < a.splits; ++s) M = fmaxf(M, __ldcg(a.part + ((int64_t)head * a.splits + s) * a.R + r).x);
-        float L = 0.f;
-        for (int s = 0; s < a.splits; ++s) {
-            const float2 p = __ldcg(a.part + ((int64_t)head * a.splits + s) * a.R + r);
-            if (p.x != -INFINITY) L = fmaf(p.y, exp2_approx(p.x - M), L);
-        }
-        a.stats[(int64_t)head * a.R + r] = make_float2(M, L > 0.f ? 1.f / L : 0.f);
+        if (tid == 0) a.tickets[head] = 0u;
     }
-    if (tid == 0) a.tickets[head] = 0u;
 }
 
 // ---------------------------------------------------------------------------

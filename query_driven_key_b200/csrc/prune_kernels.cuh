@@ -49,6 +49,8 @@ struct ScoreArgs {
     double *scores;            // [heads][D]
     int T;                     // > 0: also select the top T into idx
     int32_t *idx;              // [heads][T]
+    unsigned *status;          // device status word (bounded waits of score_tma_kernel)
+    int stages;                // score_tma_kernel: ring stages
 };
 
 // ---------------------------------------------------------------------------
@@ -105,6 +107,100 @@ __device__ __forceinline__ void add_squares4_bf16(const uint4 (&w)[4], double *a
     }
 }
 
+// Window-query energies of the group's query heads g = split, split +
+// splits, ... (threads 0..127, one channel each): qn2[g][c] = sum_s q[s,c]^2
+// in fp64, in token order.
+template <typename TIn>
+__device__ __forceinline__ void score_window_energies(const ScoreArgs &a, int head, int split)
+{
+    const int tid = threadIdx.x;
+    if (tid >= kD) return;
+    const int b = head / a.Hkv, kv = head % a.Hkv;
+    const int G = a.Hq / a.Hkv;
+    for (int g = split; g < G; g += a.splits) {
+        const int64_t h = (int64_t)kv * G + g;
+        const TIn *qh = static_cast<const TIn *>(a.qwin) + (((int64_t)b * a.Hq + h) * a.S) * kD + tid;
+        double q2 = 0.0;
+        int s = 0;
+        for (; s + 8 <= a.S; s += 8) {  // loads issued together, added in order
+            double x[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) x[u] = (double)Elem<TIn>::to_float(qh[(int64_t)(s + u) * kD]);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) q2 = __dadd_rn(q2, __dmul_rn(x[u], x[u]));
+        }
+        for (; s < a.S; ++s) {
+            const double x = (double)Elem<TIn>::to_float(qh[(int64_t)s * kD]);
+            q2 = __dadd_rn(q2, __dmul_rn(x, x));
+        }
+        a.qn2[((int64_t)head * G + g) * kD + tid] = q2;
+    }
+}
+
+// End of a score block (called by every thread of the block; threads 0..255
+// do the work): the block partial part[head][split][c] = sum of the ROWS rows
+// of red[][c] in row order; the last block of the head to arrive (ticket
+// counter) adds the partials of all splits in a fixed order (the even and the
+// odd splits in two halves of 128 threads, each in split order, then half 0
+// plus half 1), forms
+//     s[c] = sum_g sqrt(qn2[g][c]) * sqrt(kn2[c])
+// with each operation rounded as written, resets the ticket and, for T > 0,
+// selects the top T.
+template <int ROWS>
+__device__ __forceinline__ void score_block_end(const ScoreArgs &a, int head, int split, const double *red)
+{
+    __shared__ unsigned last;
+    __shared__ unsigned long long sv[kD];
+    __shared__ double khalf[kD];
+    const int tid = threadIdx.x;
+    const int G = a.Hq / a.Hkv;
+    if (tid < kD) {
+        double s = 0.0;
+#pragma unroll 4
+        for (int rr = 0; rr < ROWS; ++rr) s += red[rr * kD + tid];
+        a.part[((int64_t)head * a.splits + split) * kD + tid] = s;
+    }
+
+    // ------------------------------------------ last block of the head
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) last = (atomicAdd(a.tickets + head, 1u) == (unsigned)(a.splits - 1)) ? 1u : 0u;
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    // channel energy: 16 loads in flight per thread
+    const int c = tid & (kD - 1), hp = tid >> 7;
+    double k0 = 0.0;
+    if (tid < 2 * kD) {
+        const double *p = a.part + (int64_t)head * a.splits * kD + c;
+        for (int s = hp; s < a.splits; s += 32) {
+            double v[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int s2 = s + 2 * u;
+                v[u] = (s2 < a.splits) ? __ldcg(p + (int64_t)s2 * kD) : 0.0;
+            }
+#pragma unroll
+            for (int u = 0; u < 16; ++u) k0 = __dadd_rn(k0, v[u]);
+        }
+    }
+    if (hp == 1) khalf[c] = k0;
+    __syncthreads();
+    if (tid < kD) {
+        k0 = __dadd_rn(k0, khalf[tid]);
+        const double knorm = sqrt(k0);
+        double sc = 0.0;
+        for (int g = 0; g < G; ++g)
+            sc = __dadd_rn(sc, __dmul_rn(sqrt(__ldcg(a.qn2 + ((int64_t)head * G + g) * kD + tid)), knorm));
+        a.scores[(int64_t)head * kD + tid] = sc;
+        sv[tid] = __double_as_longlong(sc);
+    }
+    if (tid == 0) a.tickets[head] = 0u;  // ready for the next call
+    if (a.T <= 0) return;
+    __syncthreads();
+    if (tid < 32) select_top_t_warp(sv, a.T, a.idx + (int64_t)head * a.T, tid);
+}
+
 template <typename TIn>
 __global__ void __launch_bounds__(256, 3) score_kernel(const ScoreArgs a)
 {
@@ -113,12 +209,10 @@ __global__ void __launch_bounds__(256, 3) score_kernel(const ScoreArgs a)
     constexpr int RPP = 256 / TPR;         // rows per pass
     constexpr int UNROLL = 4;              // 16-byte loads per batch (two batches in flight)
     __shared__ double red[RPP][kD];
-    __shared__ unsigned last;
 
     const int head = blockIdx.y;
     const int split = blockIdx.x;
     const int b = head / a.Hkv, kv = head % a.Hkv;
-    const int G = a.Hq / a.Hkv;
     const int tid = threadIdx.x;
     const int cg = tid % TPR;
     const int r = tid / TPR;
@@ -126,27 +220,7 @@ __global__ void __launch_bounds__(256, 3) score_kernel(const ScoreArgs a)
     const int64_t n1 = min(a.N, n0 + a.rows_per_split);
     const TIn *base = static_cast<const TIn *>(a.k) + (int64_t)b * a.sb + (int64_t)kv * a.sh + cg * VEC;
 
-    // window-query energies of the group's query heads g = split, split + splits, ...
-    if (tid < kD) {
-        for (int g = split; g < G; g += a.splits) {
-            const int64_t h = (int64_t)kv * G + g;
-            const TIn *qh = static_cast<const TIn *>(a.qwin) + (((int64_t)b * a.Hq + h) * a.S) * kD + tid;
-            double q2 = 0.0;
-            int s = 0;
-            for (; s + 8 <= a.S; s += 8) {  // loads issued together, added in order
-                double x[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) x[u] = (double)Elem<TIn>::to_float(qh[(int64_t)(s + u) * kD]);
-#pragma unroll
-                for (int u = 0; u < 8; ++u) q2 = __dadd_rn(q2, __dmul_rn(x[u], x[u]));
-            }
-            for (; s < a.S; ++s) {
-                const double x = (double)Elem<TIn>::to_float(qh[(int64_t)s * kD]);
-                q2 = __dadd_rn(q2, __dmul_rn(x, x));
-            }
-            a.qn2[((int64_t)head * G + g) * kD + tid] = q2;
-        }
-    }
+    score_window_energies<TIn>(a, head, split);
 
     double acc[VEC];
 #pragma unroll
@@ -198,54 +272,7 @@ __global__ void __launch_bounds__(256, 3) score_kernel(const ScoreArgs a)
 #pragma unroll
     for (int e = 0; e < VEC; ++e) red[r][cg * VEC + e] = acc[e];
     __syncthreads();
-    if (tid < kD) {
-        double s = 0.0;
-#pragma unroll 4
-        for (int rr = 0; rr < RPP; ++rr) s += red[rr][tid];
-        a.part[((int64_t)head * a.splits + split) * kD + tid] = s;
-    }
-
-    // ------------------------------------------ last block of the head
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) last = (atomicAdd(a.tickets + head, 1u) == (unsigned)(a.splits - 1)) ? 1u : 0u;
-    __syncthreads();
-    if (!last) return;
-    __threadfence();
-    __shared__ unsigned long long sv[kD];
-    __shared__ double khalf[kD];
-    // channel energy: the two halves of the block add the even and the odd
-    // splits (each in split order, 16 loads in flight), then half 0 adds half 1
-    const int c = tid & (kD - 1), hp = tid >> 7;
-    double k0 = 0.0;
-    {
-        const double *p = a.part + (int64_t)head * a.splits * kD + c;
-        for (int s = hp; s < a.splits; s += 32) {
-            double v[16];
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const int s2 = s + 2 * u;
-                v[u] = (s2 < a.splits) ? __ldcg(p + (int64_t)s2 * kD) : 0.0;
-            }
-#pragma unroll
-            for (int u = 0; u < 16; ++u) k0 = __dadd_rn(k0, v[u]);
-        }
-    }
-    if (hp == 1) khalf[c] = k0;
-    __syncthreads();
-    if (tid < kD) {
-        k0 = __dadd_rn(k0, khalf[tid]);
-        const double knorm = sqrt(k0);
-        double sc = 0.0;
-        for (int g = 0; g < G; ++g)
-            sc = __dadd_rn(sc, __dmul_rn(sqrt(__ldcg(a.qn2 + ((int64_t)head * G + g) * kD + tid)), knorm));
-        a.scores[(int64_t)head * kD + tid] = sc;
-        sv[tid] = __double_as_longlong(sc);
-    }
-    if (tid == 0) a.tickets[head] = 0u;  // ready for the next call
-    if (a.T <= 0) return;
-    __syncthreads();
-    if (tid < 32) select_top_t_warp(sv, a.T, a.idx + (int64_t)head * a.T, tid);
+    score_block_end<RPP>(a, head, split, &red[0][0]);
 }
 
 // ---------------------------------------------------------------------------

@@ -20,6 +20,7 @@
 #include "decode_tc.cuh"
 #include "prune_fused.cuh"
 #include "prune_kernels.cuh"
+#include "score_tma.cuh"
 #include "think.h"
 
 namespace think {
@@ -423,7 +424,21 @@ think_status_t launch_score(const void *q_win, const void *k, const int64_t k_st
     a.scores = scores;
     a.T = T;
     a.idx = idx;
+    a.status = reinterpret_cast<unsigned *>(ws + w.status);
+    a.stages = env_int("THINK_SCORE_STAGES", 4, 2, kStMaxStages);
     dim3 grid(p.splits, (unsigned)heads);
+    // bf16: key tiles staged by TMA when a tensor map can describe K
+    // (THINK_SCORE_TMA=0 selects the register-pipelined kernel, for comparison)
+    CUtensorMap mk;
+    if (dtype == THINK_BF16 && N > 0 && N <= (int64_t)INT32_MAX - kStTileRows &&
+        env_int("THINK_SCORE_TMA", 1, 0, 1) == 1 &&
+        make_map_4d(&mk, THINK_BF16, k, kD, (uint64_t)N, (uint64_t)Hkv, (uint64_t)B, k_strides[2],
+                    k_strides[1], k_strides[0], 64, kStTileRows, true)) {
+        const size_t bytes = score_tma_smem_bytes(a.stages);
+        if (!ensure_smem(reinterpret_cast<const void *>(score_tma_kernel), bytes)) return THINK_ERR_CUDA;
+        score_tma_kernel<<<grid, kStThreads, bytes, st>>>(mk, a);
+        return launch_status();
+    }
     if (dtype == THINK_BF16)
         score_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(a);
     else

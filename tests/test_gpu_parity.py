@@ -377,19 +377,26 @@ def test_fused_prune_equals_stepwise_calls():
     assert torch.equal(a.idx, b.idx)
 
 
+PRUNE_ENV_KEYS = ("THINK_PRUNE_FUSED", "THINK_PRUNE_L2_HINTS", "THINK_SCORE_TMA", "THINK_SCORE_STAGES")
+
+
 @pytest.mark.parametrize("env", [{"THINK_PRUNE_FUSED": "1"},
-                                 {"THINK_PRUNE_FUSED": "1", "THINK_PRUNE_L2_HINTS": "0"}])
+                                 {"THINK_PRUNE_FUSED": "1", "THINK_PRUNE_L2_HINTS": "0"},
+                                 {"THINK_SCORE_TMA": "0"},
+                                 {"THINK_SCORE_STAGES": "2"},
+                                 {"THINK_SCORE_STAGES": "8"}])
 def test_prune_schedules_give_identical_results(env, monkeypatch):
-    # the two-launch prune (default) and the one-kernel prune (with and without
-    # its L2 hints) must agree bit for bit: same split plan, same order of
-    # additions, pure copies
+    # the two-launch prune (default: TMA-staged score tiles) against the
+    # one-kernel prune (with and without its L2 hints), the register-pipelined
+    # score kernel and other ring depths: bit for bit the same (same split
+    # plan, same order of additions, pure copies)
     shapes = [(2, 32, 8, 5000, 64), (1, 8, 1, 70, 51), (4, 4, 4, 3000, 128), (3, 16, 8, 1, 1),
               (1, 32, 8, 40000, 51)]
     for i, (B, Hq, Hkv, N, T) in enumerate(shapes):
         q_win, k, _, _ = _random_case(100 + i, B, Hq, Hkv, N, 32, torch.bfloat16, k_pad=8)
         kd = torch.empty((B, Hkv, N + 8, 128), dtype=torch.bfloat16, device=DEV)[:, :, :N].copy_(k)
         qd = q_win.to(DEV)
-        for key in ("THINK_PRUNE_FUSED", "THINK_PRUNE_L2_HINTS"):
+        for key in PRUNE_ENV_KEYS:
             monkeypatch.delenv(key, raising=False)
         a = _prune_gpu(qd, kd, T)
         for key, val in env.items():
