@@ -284,20 +284,7 @@ __device__ __forceinline__ void pf_window_energies(const PruneFusedArgs &a, int 
     for (int g = part; g < a.G; g += a.s_items) {
         const int64_t h = (int64_t)kv * a.G + g;
         const __nv_bfloat16 *qh = a.qwin + (((int64_t)b * a.Hq + h) * a.S) * kD + tid;
-        double q2 = 0.0;
-        int s = 0;
-        for (; s + 8 <= a.S; s += 8) {
-            double x[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) x[u] = (double)Elem<__nv_bfloat16>::to_float(qh[(int64_t)(s + u) * kD]);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) q2 = __dadd_rn(q2, __dmul_rn(x[u], x[u]));
-        }
-        for (; s < a.S; ++s) {
-            const double x = (double)Elem<__nv_bfloat16>::to_float(qh[(int64_t)s * kD]);
-            q2 = __dadd_rn(q2, __dmul_rn(x, x));
-        }
-        a.qn2[((int64_t)head * a.G + g) * kD + tid] = q2;
+        a.qn2[((int64_t)head * a.G + g) * kD + tid] = window_energy<__nv_bfloat16>(qh, a.S);
     }
 }
 

@@ -36,6 +36,75 @@ __device__ __forceinline__ void select_top_t_warp(const unsigned long long *sv, 
     }
 }
 
+// The same selection (same rule, same output) by the first 256 threads of a
+// block; every thread of the block calls it.  Thread t ranks channel t/2
+// against half t%2 of the channels and the pair adds its two counts, so each
+// thread makes 64 comparisons instead of 512.
+__device__ __forceinline__ void select_top_t_block(const unsigned long long *sv, int T,
+                                                   int32_t *__restrict__ idx_out)
+{
+    __shared__ int wcnt[8];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const bool on = tid < 2 * kD;
+    const int c = (tid >> 1) & (kD - 1), h = tid & 1;
+    int rank = 0;
+    if (on) {
+        const unsigned long long mine = sv[c];
+#pragma unroll 8
+        for (int j = 0; j < kD / 2; ++j) {
+            const int c2 = h * (kD / 2) + j;
+            const unsigned long long u = sv[c2];
+            rank += (u > mine) | ((u == mine) & (c2 < c));
+        }
+    }
+    rank += __shfl_xor_sync(0xffffffffu, rank, 1);
+    const bool keep = on && h == 0 && rank < T;
+    const unsigned ball = __ballot_sync(0xffffffffu, keep);
+    if (on && lane == 0) wcnt[warp] = __popc(ball);
+    __syncthreads();
+    if (keep) {
+        int base = 0;
+        for (int w = 0; w < warp; ++w) base += wcnt[w];
+        idx_out[base + __popc(ball & ((1u << lane) - 1u))] = c;
+    }
+}
+
+// Window-query energy of one channel: sum over s of q[s][c]^2 in fp64, in row
+// order; q points at the channel's element of row 0, rows kD apart.  The loads
+// go out 32 at a time (the sum itself is sequential), so that the blocks that
+// compute these energies start streaming keys soon after the others.
+template <typename TIn>
+__device__ __forceinline__ double window_energy(const TIn *q, int S)
+{
+    double q2 = 0.0;
+    int s = 0;
+    for (; s + 32 <= S; s += 32) {
+        float x[32];
+#pragma unroll
+        for (int u = 0; u < 32; ++u) x[u] = Elem<TIn>::to_float(q[(int64_t)(s + u) * kD]);
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+            const double xd = (double)x[u];
+            q2 = __dadd_rn(q2, __dmul_rn(xd, xd));
+        }
+    }
+    for (; s + 8 <= S; s += 8) {
+        float x[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) x[u] = Elem<TIn>::to_float(q[(int64_t)(s + u) * kD]);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const double xd = (double)x[u];
+            q2 = __dadd_rn(q2, __dmul_rn(xd, xd));
+        }
+    }
+    for (; s < S; ++s) {
+        const double x = (double)Elem<TIn>::to_float(q[(int64_t)s * kD]);
+        q2 = __dadd_rn(q2, __dmul_rn(x, x));
+    }
+    return q2;
+}
+
 struct ScoreArgs {
     const void *k;
     int64_t sb, sh, sn;        // element strides of K (batch, head, token)
@@ -120,20 +189,7 @@ __device__ __forceinline__ void score_window_energies(const ScoreArgs &a, int he
     for (int g = split; g < G; g += a.splits) {
         const int64_t h = (int64_t)kv * G + g;
         const TIn *qh = static_cast<const TIn *>(a.qwin) + (((int64_t)b * a.Hq + h) * a.S) * kD + tid;
-        double q2 = 0.0;
-        int s = 0;
-        for (; s + 8 <= a.S; s += 8) {  // loads issued together, added in order
-            double x[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) x[u] = (double)Elem<TIn>::to_float(qh[(int64_t)(s + u) * kD]);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) q2 = __dadd_rn(q2, __dmul_rn(x[u], x[u]));
-        }
-        for (; s < a.S; ++s) {
-            const double x = (double)Elem<TIn>::to_float(qh[(int64_t)s * kD]);
-            q2 = __dadd_rn(q2, __dmul_rn(x, x));
-        }
-        a.qn2[((int64_t)head * G + g) * kD + tid] = q2;
+        a.qn2[((int64_t)head * G + g) * kD + tid] = window_energy<TIn>(qh, a.S);
     }
 }
 
@@ -198,7 +254,7 @@ __device__ __forceinline__ void score_block_end(const ScoreArgs &a, int head, in
     if (tid == 0) a.tickets[head] = 0u;  // ready for the next call
     if (a.T <= 0) return;
     __syncthreads();
-    if (tid < 32) select_top_t_warp(sv, a.T, a.idx + (int64_t)head * a.T, tid);
+    select_top_t_block(sv, a.T, a.idx + (int64_t)head * a.T);
 }
 
 template <typename TIn>

@@ -27,7 +27,9 @@ namespace think {
 namespace {
 
 constexpr int kTargetSMs = 148;             // B200
-constexpr int kScoreBlocksPerSM = 4;        // 256-thread score blocks resident per SM
+constexpr int kScoreBlocksPerSM = 4;        // runs per SM of the fixed score split rule
+constexpr int kScoreResidentPerSM = 3;      // score blocks resident per SM (both score kernels)
+constexpr int kScoreMaxWaves = 4;
 constexpr int kDecodeBlocksPerSM = 2;       // decode blocks the plan aims to keep per SM
 constexpr int kDecodePrefetchTiles = 0;     // tiles a decode block prefetches into L2 ahead of TMA
 constexpr int kTcBlocksPerSM = 1;           // tcgen05 decode: blocks per SM the plan aims for
@@ -83,10 +85,9 @@ think_status_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t 
 
 // ---------------------------------------------------------------- plans --
 
-// Split of each head's tokens for scoring, shared by score_kernel and the
-// fused prune kernel (so that both add the squares in the same order): runs of
-// s_tiles 64-token tiles, about kScoreBlocksPerSM runs per SM over all heads,
-// 4 to 32 tiles per run.
+// Split of each head's tokens for scoring, shared by the score kernels and
+// the fused prune kernel (so that all add the squares in the same order): runs
+// of s_tiles 64-token tiles, one score block per run.
 struct ScorePlan {
     int splits;              // runs per head
     int s_tiles;             // 64-token tiles per run
@@ -94,18 +95,60 @@ struct ScorePlan {
     int64_t tiles_per_head;
 };
 
-ScorePlan plan_score(int64_t heads, int64_t N)
+ScorePlan score_plan_from_tiles(int64_t tiles_per_head, int64_t st)
 {
     ScorePlan p;
-    p.tiles_per_head = std::max<int64_t>(1, ceil_div(N, kPfTile));
-    const int64_t total = heads * p.tiles_per_head;
-    int64_t st = total / ((int64_t)kTargetSMs * kScoreBlocksPerSM);
-    st = std::min<int64_t>(std::max<int64_t>(st, 4), 32);
-    st = std::min(st, p.tiles_per_head);
+    p.tiles_per_head = tiles_per_head;
+    st = std::min<int64_t>(std::max<int64_t>(st, 1), tiles_per_head);
     p.s_tiles = (int)st;
     p.rows_per_split = st * kPfTile;
-    p.splits = (int)ceil_div(p.tiles_per_head, st);
+    p.splits = (int)ceil_div(tiles_per_head, st);
     return p;
+}
+
+// waves = 0: about kScoreBlocksPerSM runs per SM, 4 to 32 tiles per run.
+// waves = W > 0: the shortest runs whose count fits W waves of the resident
+// block slots (148 SMs x kScoreResidentPerSM).
+ScorePlan plan_score_waves(int64_t heads, int64_t N, int waves)
+{
+    const int64_t tph = std::max<int64_t>(1, ceil_div(N, kPfTile));
+    if (waves <= 0) {
+        const int64_t st = heads * tph / ((int64_t)kTargetSMs * kScoreBlocksPerSM);
+        return score_plan_from_tiles(tph, std::min<int64_t>(std::max<int64_t>(st, 4), 32));
+    }
+    const int64_t slots = (int64_t)kTargetSMs * kScoreResidentPerSM * waves;
+    const int64_t runs_per_head = std::max<int64_t>(1, slots / std::max<int64_t>(heads, 1));
+    return score_plan_from_tiles(tph, ceil_div(tph, runs_per_head));
+}
+
+// THINK_SCORE_WAVES: 0 the fixed rule above, 1..4 that many waves; default
+// (-1): the fewest waves (up to 4) whose runs fill at least 90% of their
+// slots, else the best filled.  Whole waves leave no partly filled last wave,
+// whose blocks would stream with the rest of the GPU idle.
+ScorePlan plan_score(int64_t heads, int64_t N)
+{
+    const int mode = env_int("THINK_SCORE_WAVES", -1, -1, kScoreMaxWaves);
+    if (mode >= 0) return plan_score_waves(heads, N, mode);
+    ScorePlan best = plan_score_waves(heads, N, 1);
+    double best_fill = 0.0;
+    for (int w = 1; w <= kScoreMaxWaves; ++w) {
+        const ScorePlan p = plan_score_waves(heads, N, w);
+        const double fill = (double)(heads * p.splits) / ((double)kTargetSMs * kScoreResidentPerSM * w);
+        if (fill >= 0.9) return p;
+        if (fill > best_fill) {
+            best_fill = fill;
+            best = p;
+        }
+    }
+    return best;
+}
+
+// The most runs per head any plan above can choose (workspace size).
+int score_max_splits(int64_t heads, int64_t N)
+{
+    int m = 1;
+    for (int w = 0; w <= kScoreMaxWaves; ++w) m = std::max(m, plan_score_waves(heads, N, w).splits);
+    return m;
 }
 
 struct DecodeSplit {
@@ -376,6 +419,14 @@ ScoreWs score_ws_layout(int64_t heads, int G, const ScorePlan &p)
     return w;
 }
 
+// The layout for the largest plan, so that one workspace serves every plan.
+ScoreWs score_ws_layout_max(int64_t heads, int G, int64_t N)
+{
+    ScorePlan p = plan_score(heads, N);
+    p.splits = score_max_splits(heads, N);
+    return score_ws_layout(heads, G, p);
+}
+
 think_status_t validate_score(const void *q_win, const void *k, const int64_t k_strides[3], int B,
                               int Hq, int Hkv, int64_t N, int S_obs, int d, think_dtype_t dtype,
                               const double *scores, const void *workspace, size_t workspace_bytes)
@@ -393,7 +444,7 @@ think_status_t validate_score(const void *q_win, const void *k, const int64_t k_
     if (!aligned16(k) || !aligned16(workspace) || (q_win && !aligned16(q_win)) ||
         !strides_ok(k_strides, es) || (reinterpret_cast<uintptr_t>(scores) & 7u))
         return THINK_ERR_ALIGNMENT;
-    if (workspace_bytes < score_ws_layout(heads, Hq / Hkv, plan_score(heads, N)).total)
+    if (workspace_bytes < score_ws_layout_max(heads, Hq / Hkv, N).total)
         return THINK_ERR_WORKSPACE;
     return THINK_OK;
 }
@@ -884,7 +935,7 @@ size_t think_score_workspace_size(int B, int Hq, int Hkv, int64_t N, int d)
 {
     if (B <= 0 || Hkv <= 0 || Hq < Hkv || Hq % Hkv != 0 || N < 0 || d != kD) return 0;
     const int64_t heads = (int64_t)B * Hkv;
-    return score_ws_layout(heads, Hq / Hkv, plan_score(heads, N)).total;
+    return score_ws_layout_max(heads, Hq / Hkv, N).total;
 }
 
 think_status_t think_score_channels(const void *q_win, const void *k, const int64_t k_strides[3],
