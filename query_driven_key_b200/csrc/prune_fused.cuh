@@ -288,47 +288,6 @@ __device__ __forceinline__ void pf_window_energies(const PruneFusedArgs &a, int 
     }
 }
 
-// 4x4 transpose of 32-bit words inside each group of four lanes: lane j of
-// the group ends with word j of every lane of the group, in lane order.
-__device__ __forceinline__ void quad_transpose(uint32_t (&a)[4], int j)
-{
-    const bool o1 = j & 1, o2 = j & 2;
-    uint32_t t0 = o1 ? a[0] : a[1], t1 = o1 ? a[2] : a[3];
-    t0 = __shfl_xor_sync(0xffffffffu, t0, 1);
-    t1 = __shfl_xor_sync(0xffffffffu, t1, 1);
-    if (o1) {
-        a[0] = t0;
-        a[2] = t1;
-    } else {
-        a[1] = t0;
-        a[3] = t1;
-    }
-    uint32_t u0 = o2 ? a[0] : a[2], u1 = o2 ? a[1] : a[3];
-    u0 = __shfl_xor_sync(0xffffffffu, u0, 2);
-    u1 = __shfl_xor_sync(0xffffffffu, u1, 2);
-    if (o2) {
-        a[0] = u0;
-        a[1] = u1;
-    } else {
-        a[2] = u0;
-        a[3] = u1;
-    }
-}
-
-// 8 consecutive tokens of one K' row starting at token x (x a multiple of 8);
-// only tokens < N are written.
-__device__ __forceinline__ void pf_store_run(__nv_bfloat16 *row, int64_t x, int64_t N, const uint32_t (&v)[4])
-{
-    if (x + 8 <= N) {
-        *reinterpret_cast<uint4 *>(row + x) = make_uint4(v[0], v[1], v[2], v[3]);
-    } else if (x < N) {
-        unsigned short *r = reinterpret_cast<unsigned short *>(row + x);
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-            if (x + i < N) r[i] = (unsigned short)(v[i >> 1] >> (16 * (i & 1)));
-    }
-}
-
 __device__ __forceinline__ void pf_consume(const PruneFusedArgs &a, unsigned char *smem, uint32_t full0,
                                            uint32_t empty0, uint32_t bar, unsigned *flags)
 {
@@ -393,55 +352,17 @@ __device__ __forceinline__ void pf_consume(const PruneFusedArgs &a, unsigned cha
             }
         } else {
             if (head != cur_head) {
-                // kept-channel mask of the head (every warp builds its own)
+                // kept-channel rows of the head (every warp builds its own)
                 if (lane == 0) (void)ld_acquire_gpu(a.ready + head);
                 __syncwarp();
-                uint32_t mk[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int t = lane + 32 * i;
-                    if (t < a.T) {
-                        const int c = __ldcg(a.idx + (int64_t)head * a.T + t);
-                        if ((unsigned)c < (unsigned)kD) {
-                            const uint32_t bitv = 1u << (c & 31);
-#pragma unroll
-                            for (int wd = 0; wd < 4; ++wd) mk[wd] |= (c >> 5) == wd ? bitv : 0u;
-                        }
-                    }
-                }
-#pragma unroll
-                for (int i = 0; i < 4; ++i) mk[i] = __reduce_or_sync(0xffffffffu, mk[i]);
-                // channel 8*(cw+4k) + lane/4 lies in mask word k (k = c / 32)
-                int before = 0;
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int bit = (8 * cw + (lane >> 2)) & 31;
-                    crow[k] = ((mk[k] >> bit) & 1u)
-                                  ? (int64_t)head * a.T + before + __popc(mk[k] & ((1u << bit) - 1u))
-                                  : -1;
-                    before += __popc(mk[k]);
-                }
+                kept_rows_of_warp(a.idx + (int64_t)head * a.T, a.T, (int64_t)head * a.T, cw, lane, crow);
                 cur_head = head;
             }
-            // register m of x4 load k: channel 8*(cw+4k) + lane/4, tokens
-            // 8*(tb0+m) + 2*(lane%4) + {0,1}
             uint32_t v[4][4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint32_t chunk = (uint32_t)(cw + 4 * k);
-                const uint32_t addr = st + (chunk >> 3) * kPfHalfBytes + c_row * 128u +
-                                      (((chunk & 7u) ^ (c_row & 7u)) << 4);
-                ldsm_x4_trans(addr, v[k][0], v[k][1], v[k][2], v[k][3]);
-            }
+            compact_tile_load(st, c_row, cw, v);
             __syncwarp();
             if (lane == 0) mbar_arrive(empty0 + 8 * s);
-            // lane j of each group of four: tokens 8*(tb0+j) .. +7 of its channel
-            const int64_t x = (int64_t)tile * kPfTile + 8 * (tb0 + (lane & 3));
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                quad_transpose(v[k], lane & 3);
-                if (crow[k] >= 0) pf_store_run(a.kp + crow[k] * a.ldk, x, a.N, v[k]);
-            }
+            compact_tile_store(v, lane, crow, a.kp, a.ldk, (int64_t)tile * kPfTile + 8 * (tb0 + (lane & 3)), a.N);
         }
     }
 

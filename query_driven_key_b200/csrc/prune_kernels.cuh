@@ -507,6 +507,113 @@ template <> struct Transpose4<float> {
     }
 };
 
+// ---------------------------------------------------------------------------
+// Compaction of one 64-token K tile held in shared memory as two 64-channel
+// halves with the 128-byte swizzle (as TMA writes them), by the 8 warps of a
+// block: warp w takes the token half tb0 = 4 * (w % 2) (token blocks tb0 ..
+// tb0 + 3 of 8 tokens) and the channel chunks cw + 4k (k = 0..3, 8 channels
+// each) with cw = w / 2.  ldmatrix.trans gives each lane two tokens of one
+// channel per register; a word transpose inside each group of four lanes then
+// gives lane j of the group 8 consecutive tokens of its channel, which go to
+// the channel's K' row as one 16-byte store (64 bytes per group of four).
+// ---------------------------------------------------------------------------
+// 4x4 transpose of 32-bit words inside each group of four lanes: lane j of
+// the group ends with word j of every lane of the group, in lane order.
+__device__ __forceinline__ void quad_transpose(uint32_t (&a)[4], int j)
+{
+    const bool o1 = j & 1, o2 = j & 2;
+    uint32_t t0 = o1 ? a[0] : a[1], t1 = o1 ? a[2] : a[3];
+    t0 = __shfl_xor_sync(0xffffffffu, t0, 1);
+    t1 = __shfl_xor_sync(0xffffffffu, t1, 1);
+    if (o1) {
+        a[0] = t0;
+        a[2] = t1;
+    } else {
+        a[1] = t0;
+        a[3] = t1;
+    }
+    uint32_t u0 = o2 ? a[0] : a[2], u1 = o2 ? a[1] : a[3];
+    u0 = __shfl_xor_sync(0xffffffffu, u0, 2);
+    u1 = __shfl_xor_sync(0xffffffffu, u1, 2);
+    if (o2) {
+        a[0] = u0;
+        a[1] = u1;
+    } else {
+        a[2] = u0;
+        a[3] = u1;
+    }
+}
+
+// 8 consecutive tokens of one K' row starting at token x (x a multiple of 8);
+// only tokens < N are written.
+__device__ __forceinline__ void store_run8(__nv_bfloat16 *row, int64_t x, int64_t N, const uint32_t (&v)[4])
+{
+    if (x + 8 <= N) {
+        *reinterpret_cast<uint4 *>(row + x) = make_uint4(v[0], v[1], v[2], v[3]);
+    } else if (x < N) {
+        unsigned short *r = reinterpret_cast<unsigned short *>(row + x);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (x + i < N) r[i] = (unsigned short)(v[i >> 1] >> (16 * (i & 1)));
+    }
+}
+
+// K' rows of this warp's four channel chunks: crow[k] = row0 + rank of
+// channel 8 * (cw + 4k) + lane / 4 among the kept channels, or -1 if the
+// channel is dropped.  idx holds the T kept channels of the head.
+__device__ __forceinline__ void kept_rows_of_warp(const int32_t *idx, int T, int64_t row0, int cw, int lane,
+                                                  int64_t (&crow)[4])
+{
+    uint32_t mk[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int t = lane + 32 * i;
+        if (t < T) {
+            const int c = __ldcg(idx + t);
+            if ((unsigned)c < (unsigned)kD) {
+                const uint32_t bitv = 1u << (c & 31);
+#pragma unroll
+                for (int wd = 0; wd < 4; ++wd) mk[wd] |= (c >> 5) == wd ? bitv : 0u;
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) mk[i] = __reduce_or_sync(0xffffffffu, mk[i]);
+    // channel 8*(cw+4k) + lane/4 lies in mask word k (k = c / 32)
+    int before = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int bit = (8 * cw + (lane >> 2)) & 31;
+        crow[k] = ((mk[k] >> bit) & 1u) ? row0 + before + __popc(mk[k] & ((1u << bit) - 1u)) : -1;
+        before += __popc(mk[k]);
+    }
+}
+
+// The warp's part of the tile at shared address st into registers: register m
+// of load k holds channel 8 * (cw + 4k) + lane / 4, tokens 8 * (tb0 + m) +
+// 2 * (lane % 4) + {0, 1}; c_row = 8 * (tb0 + lane / 8) + lane % 8 is the
+// token row this lane addresses.
+__device__ __forceinline__ void compact_tile_load(uint32_t st, uint32_t c_row, int cw, uint32_t (&v)[4][4])
+{
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const uint32_t chunk = (uint32_t)(cw + 4 * k);
+        const uint32_t addr = st + (chunk >> 3) * (64u * 64u * 2u) + c_row * 128u + (((chunk & 7u) ^ (c_row & 7u)) << 4);
+        ldsm_x4_trans(addr, v[k][0], v[k][1], v[k][2], v[k][3]);
+    }
+}
+
+// Transpose and store: x = first token of this lane's run (a multiple of 8).
+__device__ __forceinline__ void compact_tile_store(uint32_t (&v)[4][4], int lane, const int64_t (&crow)[4],
+                                                   __nv_bfloat16 *kp, int64_t ldk, int64_t x, int64_t N)
+{
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        quad_transpose(v[k], lane & 3);
+        if (crow[k] >= 0) store_run8(kp + crow[k] * ldk, x, N, v[k]);
+    }
+}
+
 template <typename TIn> struct CompactTokens { static constexpr int value = 64; };
 
 template <typename TIn>

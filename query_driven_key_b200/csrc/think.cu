@@ -21,6 +21,7 @@
 #include "prune_fused.cuh"
 #include "prune_kernels.cuh"
 #include "score_tma.cuh"
+#include "compact_tma.cuh"
 #include "think.h"
 
 namespace think {
@@ -30,6 +31,7 @@ constexpr int kTargetSMs = 148;             // B200
 constexpr int kScoreBlocksPerSM = 4;        // runs per SM of the fixed score split rule
 constexpr int kScoreResidentPerSM = 3;      // score blocks resident per SM (both score kernels)
 constexpr int kScoreMaxWaves = 4;
+constexpr int kCompactWaves = 4;            // waves of compact_tma_kernel blocks the plan aims for
 constexpr int kDecodeBlocksPerSM = 2;       // decode blocks the plan aims to keep per SM
 constexpr int kDecodePrefetchTiles = 0;     // tiles a decode block prefetches into L2 ahead of TMA
 constexpr int kTcBlocksPerSM = 1;           // tcgen05 decode: blocks per SM the plan aims for
@@ -538,6 +540,51 @@ think_status_t launch_compact(const void *k, const int64_t k_strides[3], int B, 
 }
 
 
+// Tiles per block of compact_tma_kernel: runs that give about
+// kCompactWaves waves of the resident block slots, at least 4 tiles
+// (THINK_COMPACT_TILES overrides, for tuning).
+int plan_compact_tma(int64_t heads, int64_t tiles)
+{
+    const int64_t slots = (int64_t)kTargetSMs * kScoreResidentPerSM * kCompactWaves;
+    const int64_t rph = std::max<int64_t>(1, slots / std::max<int64_t>(heads, 1));
+    int64_t rt = std::max<int64_t>(4, ceil_div(tiles, rph));
+    rt = env_int("THINK_COMPACT_TILES", (int)std::min<int64_t>(rt, 1 << 20), 1, 1 << 20);
+    return (int)std::min<int64_t>(rt, tiles);
+}
+
+// The TMA compaction for bf16 keys within think_prune (its workspace holds
+// the status word).  Returns THINK_ERR_UNSUPPORTED, having launched nothing,
+// when the keys cannot be described by a tensor map, or with
+// THINK_COMPACT_TMA=0.
+think_status_t launch_compact_tma(const void *k, const int64_t k_strides[3], int B, int Hkv, int64_t N,
+                                  const int32_t *idx, int T, void *k_pruned, int64_t ldk, void *workspace,
+                                  cudaStream_t st)
+{
+    if (env_int("THINK_COMPACT_TMA", 1, 0, 1) == 0 || N > (int64_t)INT32_MAX - kCtTileRows)
+        return THINK_ERR_UNSUPPORTED;
+    const int64_t heads = (int64_t)B * Hkv;
+    CUtensorMap mk;
+    if (!make_map_4d(&mk, THINK_BF16, k, kD, (uint64_t)N, (uint64_t)Hkv, (uint64_t)B, k_strides[2],
+                     k_strides[1], k_strides[0], 64, kCtTileRows, true))
+        return THINK_ERR_UNSUPPORTED;
+    CompactTmaArgs a;
+    a.Hkv = Hkv;
+    a.T = T;
+    a.tiles = ceil_div(N, kCtTileRows);
+    a.run_tiles = plan_compact_tma(heads, a.tiles);
+    a.stages = env_int("THINK_COMPACT_STAGES", 4, 2, kCtMaxStages);
+    a.N = N;
+    a.ldk = ldk;
+    a.idx = idx;
+    a.kp = static_cast<__nv_bfloat16 *>(k_pruned);
+    a.status = reinterpret_cast<unsigned *>(static_cast<unsigned char *>(workspace));  // score workspace word 0
+    const size_t bytes = compact_tma_smem_bytes(a.stages);
+    if (!ensure_smem(reinterpret_cast<const void *>(compact_tma_kernel), bytes)) return THINK_ERR_CUDA;
+    dim3 grid((unsigned)ceil_div(a.tiles, a.run_tiles), (unsigned)heads);
+    compact_tma_kernel<<<grid, kCtThreads, bytes, st>>>(mk, a);
+    return launch_status();
+}
+
 // ---------------------------------------------------------- fused prune --
 
 struct PrunePlan {
@@ -1013,6 +1060,10 @@ think_status_t think_prune(const void *q_win, const void *k, const int64_t k_str
     }
     v = launch_score(q_win, k, k_strides, B, Hq, Hkv, N, S_obs, dtype, T, scores, idx, workspace, st);
     if (v != THINK_OK || N == 0) return v;
+    if (dtype == THINK_BF16) {
+        v = launch_compact_tma(k, k_strides, B, Hkv, N, idx, T, k_pruned, ldk, workspace, st);
+        if (v != THINK_ERR_UNSUPPORTED) return v;
+    }
     return launch_compact(k, k_strides, B, Hkv, N, dtype, idx, T, k_pruned, ldk, st);
 }
 

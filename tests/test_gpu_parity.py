@@ -377,19 +377,24 @@ def test_fused_prune_equals_stepwise_calls():
     assert torch.equal(a.idx, b.idx)
 
 
-PRUNE_ENV_KEYS = ("THINK_PRUNE_FUSED", "THINK_PRUNE_L2_HINTS", "THINK_SCORE_TMA", "THINK_SCORE_STAGES")
+PRUNE_ENV_KEYS = ("THINK_PRUNE_FUSED", "THINK_PRUNE_L2_HINTS", "THINK_SCORE_TMA", "THINK_SCORE_STAGES",
+                  "THINK_COMPACT_TMA", "THINK_COMPACT_STAGES", "THINK_COMPACT_TILES")
 
 
 @pytest.mark.parametrize("env", [{"THINK_PRUNE_FUSED": "1"},
                                  {"THINK_PRUNE_FUSED": "1", "THINK_PRUNE_L2_HINTS": "0"},
                                  {"THINK_SCORE_TMA": "0"},
                                  {"THINK_SCORE_STAGES": "2"},
-                                 {"THINK_SCORE_STAGES": "8"}])
+                                 {"THINK_SCORE_STAGES": "8"},
+                                 {"THINK_COMPACT_TMA": "0"},
+                                 {"THINK_COMPACT_STAGES": "2", "THINK_COMPACT_TILES": "1"},
+                                 {"THINK_COMPACT_STAGES": "8", "THINK_COMPACT_TILES": "37"}])
 def test_prune_schedules_give_identical_results(env, monkeypatch):
-    # the two-launch prune (default: TMA-staged score tiles) against the
-    # one-kernel prune (with and without its L2 hints), the register-pipelined
-    # score kernel and other ring depths: bit for bit the same (same split
-    # plan, same order of additions, pure copies)
+    # the two-launch prune (default: TMA-staged score and compaction tiles)
+    # against the one-kernel prune (with and without its L2 hints), the
+    # register-pipelined score and compaction kernels, other ring depths and
+    # run lengths: bit for bit the same (same split plan, same order of
+    # additions, pure copies)
     shapes = [(2, 32, 8, 5000, 64), (1, 8, 1, 70, 51), (4, 4, 4, 3000, 128), (3, 16, 8, 1, 1),
               (1, 32, 8, 40000, 51)]
     for i, (B, Hq, Hkv, N, T) in enumerate(shapes):
