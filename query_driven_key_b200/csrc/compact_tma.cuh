@@ -18,6 +18,11 @@
 // one head, so each warp finds the K' rows of its channels once.  K' is a pure
 // copy: the output is that of compact_kernel bit for bit.
 //
+// Launched with programmatic stream serialisation after the score kernel: the
+// producer streams K (not written by the score pass) while the score grid
+// drains; the consumers wait for the score grid before they read the
+// selection or write K'.
+//
 // Every wait is bounded: on expiry the kernel sets a bit in the status word,
 // the consumers stop, and the producer waits (bounded) for its loads in flight
 // before the block ends.
@@ -106,6 +111,7 @@ __global__ void __launch_bounds__(kCtThreads, 3)
     const int tb0 = 4 * (warp & 1), cw = warp >> 1;
     const uint32_t c_row = (uint32_t)(8 * (tb0 + (lane >> 3)) + (lane & 7));
     int64_t crow[4];
+    grid_dependency_wait();  // the selection (idx) is complete; K' may be written
     kept_rows_of_warp(a.idx + (int64_t)head * a.T, a.T, (int64_t)head * a.T, cw, lane, crow);
     for (int i = 0; i < ntiles; ++i) {
         const int s = i % stages;

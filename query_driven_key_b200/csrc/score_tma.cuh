@@ -70,6 +70,9 @@ __global__ void __launch_bounds__(kStThreads, 3)
         fence_barrier_init();
     }
     __syncthreads();
+    // the compaction that follows in think_prune may start its loads of K
+    // on the SMs that this grid leaves idle at its end
+    grid_launch_dependents();
 
     // consumer thread -> row group and 16-byte channel chunk, as in score_kernel
     const int cc = tid & 15, rg = tid >> 4;

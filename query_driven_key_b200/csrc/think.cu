@@ -581,8 +581,7 @@ think_status_t launch_compact_tma(const void *k, const int64_t k_strides[3], int
     const size_t bytes = compact_tma_smem_bytes(a.stages);
     if (!ensure_smem(reinterpret_cast<const void *>(compact_tma_kernel), bytes)) return THINK_ERR_CUDA;
     dim3 grid((unsigned)ceil_div(a.tiles, a.run_tiles), (unsigned)heads);
-    compact_tma_kernel<<<grid, kCtThreads, bytes, st>>>(mk, a);
-    return launch_status();
+    return launch_pdl(compact_tma_kernel, grid, dim3(kCtThreads), bytes, st, mk, a);
 }
 
 // ---------------------------------------------------------- fused prune --
