@@ -42,6 +42,7 @@ struct DecodeArgs {
     int tiles_per_split, splits, stages;
     int stages_v;           // tcgen05 kernel: V ring slots (stages = K' ring slots)
     int prefetch;           // tiles prefetched into L2 ahead of the TMA loads
+    int early;              // 1: the first tiles are prefetched into L2 before the dependency wait
     float scale_log2;       // scale * log2(e)
     uint32_t stage_bytes;   // bytes per ring stage (multiple of 1024)
     uint32_t v_off;         // offset of the V tile inside a stage

@@ -83,19 +83,48 @@ __host__ __device__ inline size_t mma_smem_bytes(int T, int G, int stages, int C
 }
 
 // q' = q[idx] of the group's query heads as [16 rows (g)][t_pad] bf16 (rows
-// g >= G and columns t >= T zero), by the consumer threads.
+// g >= G and columns t >= T zero), by the consumer threads (NT of them; every
+// one calls it).  One round of global loads: the group's G query rows (16-byte
+// loads) and the T kept channels go to scratch together (the per-warp merge
+// area, unused until the end), then q' is gathered from shared memory.
 template <int G, int NT>
 __device__ __forceinline__ void mma_stage_q(const DecodeArgs &a, unsigned char *qsm, uint32_t t_pad, int T,
-                                            const int32_t *ih, int b, int kv, int tid)
+                                            const int32_t *ih, int b, int kv, int tid, unsigned char *scratch)
 {
-    const __nv_bfloat16 *q = reinterpret_cast<const __nv_bfloat16 *>(a.q);
+    constexpr int QV = G * (kD / 8);  // 16-byte words of the group's q rows
+    static_assert(QV + kD <= 2 * NT, "at most two loads per thread");
+    uint4 *qraw = reinterpret_cast<uint4 *>(scratch);       // [G][128] bf16
+    int *is = reinterpret_cast<int *>(scratch + G * kD * 2);  // [T]
+    const uint4 *qg = reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(a.q) +
+                                                      ((int64_t)b * a.Hq + (int64_t)kv * G) * kD);
+    // both of a thread's loads are issued before either is stored
+    uint4 qv[2];
+    int iv[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const int i = tid + r * NT;
+        if (i < QV)
+            qv[r] = __ldcg(qg + i);
+        else if (i < QV + T)
+            iv[r] = __ldcg(ih + (i - QV));
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const int i = tid + r * NT;
+        if (i < QV)
+            qraw[i] = qv[r];
+        else if (i < QV + T)
+            is[i - QV] = iv[r];
+    }
+    named_barrier(1, NT);
+    const __nv_bfloat16 *qr = reinterpret_cast<const __nv_bfloat16 *>(qraw);
     __nv_bfloat16 *qs = reinterpret_cast<__nv_bfloat16 *>(qsm);
     for (int i = tid; i < 16 * (int)t_pad; i += NT) {
         const int g = i / (int)t_pad, t = i % (int)t_pad;
         __nv_bfloat16 x = __float2bfloat16(0.f);
         if (g < G && t < T) {
-            const int c = ih[t];
-            if ((unsigned)c < (unsigned)kD) x = q[((int64_t)b * a.Hq + (int64_t)kv * G + g) * kD + c];
+            const int c = is[t];
+            if ((unsigned)c < (unsigned)kD) x = qr[g * kD + c];
         }
         qs[g * t_pad + t] = x;
     }
@@ -308,7 +337,37 @@ __global__ void __launch_bounds__(CW * 32 + 32)
     constexpr int NT = CW * 32;
     // Launched as a programmatic dependent of the previous kernel in the
     // stream: everything it wrote is visible after this wait; let the next
-    // decode be scheduled on SMs as ours free up.
+    // decode be scheduled on SMs as ours free up.  Such a block becomes
+    // resident while the previous decode drains (its merge and last tiles), so
+    // before the wait the producer lane asks L2 for this block's first tiles.
+    // K' and V are inputs that no kernel which lets this one start early
+    // writes, and L2 is the point of coherence, so the prefetch cannot hand
+    // stale data to the loads made after the wait (the same holds for q and
+    // idx, which may well be written by the previous kernel: a prefetch only
+    // warms L2); only kernel parameters are read before it (a ragged cache's
+    // K' rows come from device data: V only).
+    if (a.early && threadIdx.x == CW * 32) {
+        const int kv0 = (int)blockIdx.y % a.Hkv, b0 = (int)blockIdx.y / a.Hkv;
+        const int64_t t0 = (int64_t)blockIdx.x * a.tiles_per_split;
+        const int64_t n = min((int64_t)min(a.tiles_per_split, a.stages), (a.N + kBN - 1) / kBN - t0);
+        for (int64_t it = 0; it < n; ++it) {
+            const int x = (int)((t0 + it) * kBN);
+            if (a.Th == nullptr) {
+                tma_prefetch_l2_4d(&tm_k, x, 0, kv0, b0);
+                tma_prefetch_l2_4d(&tm_k, x + 64, 0, kv0, b0);
+            }
+            tma_prefetch_l2_4d(&tm_v, 0, x, kv0, b0);
+            tma_prefetch_l2_4d(&tm_v, 64, x, kv0, b0);
+        }
+        // and the lines that the q' staging reads first (the group's q rows,
+        // the kept channels)
+        const char *qrow = reinterpret_cast<const char *>(a.q) + ((int64_t)b0 * a.Hq + (int64_t)kv0 * G) * kD * 2;
+        for (int o = 0; o < G * kD * 2; o += 128) prefetch_l2(qrow + o);
+        if (a.Th == nullptr) {
+            const char *irow = reinterpret_cast<const char *>(a.idx + (int64_t)blockIdx.y * a.T);
+            for (int o = 0; o < a.T * 4; o += 128) prefetch_l2(irow + o);
+        }
+    }
     grid_dependency_wait();
     grid_launch_dependents();
     extern __shared__ unsigned char smem_dyn[];
@@ -404,7 +463,8 @@ __global__ void __launch_bounds__(CW * 32 + 32)
             *reinterpret_cast<uint4 *>(smem + (hs >> 1) * L.stage + (hs & 1u) * L.k_half +
                                        (uint32_t)T * 128u + o * 16u) = make_uint4(0, 0, 0, 0);
         }
-        mma_stage_q<G, NT>(a, qsm, L.t_pad, T, a.idx + (ragged ? row0 : (int64_t)head * T), b, kv, tid);
+        mma_stage_q<G, NT>(a, qsm, L.t_pad, T, a.idx + (ragged ? row0 : (int64_t)head * T), b, kv, tid,
+                           reinterpret_cast<unsigned char *>(mo));
     }
     named_barrier(1, NT);  // zeroed rows and q' visible to all consumers
 

@@ -221,7 +221,8 @@ __global__ void __launch_bounds__(CW * 32 + 32)
         for (uint32_t i = tid; i < 2u * pad16; i += NT)
             *reinterpret_cast<uint4 *>(kbf + (i / pad16) * L.k_half + (uint32_t)T * 128u + (i % pad16) * 16u) =
                 make_uint4(0, 0, 0, 0);
-        mma_stage_q<G, NT>(a, qsm, L.t_pad, T, a.idx + (int64_t)head * T, b, kv, tid);
+        mma_stage_q<G, NT>(a, qsm, L.t_pad, T, a.idx + (int64_t)head * T, b, kv, tid,
+                           reinterpret_cast<unsigned char *>(mo));
     }
     named_barrier(1, NT);
 

@@ -143,6 +143,12 @@ __device__ __forceinline__ void tma_prefetch_l2_4d(const CUtensorMap *map, int c
                  : "memory");
 }
 
+// Prefetch the 128-byte line holding p into L2.
+__device__ __forceinline__ void prefetch_l2(const void *p)
+{
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p) : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

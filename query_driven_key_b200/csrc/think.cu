@@ -1165,6 +1165,7 @@ think_status_t think_pruned_decode_attn(const void *q, const void *k_pruned, int
     a.stages = use_tc ? tp.stages_k : kind == kMma ? mp.stages : sm.stages;
     a.stages_v = use_tc ? tp.stages_v : 0;
     a.prefetch = env_int("THINK_DECODE_PREFETCH", kDecodePrefetchTiles, 0, 64);
+    a.early = env_int("THINK_DECODE_EARLY_PREFETCH", 1, 0, 1);
     a.scale_log2 = scale * 1.4426950408889634f;
     a.stage_bytes = sm.stage_bytes;
     a.v_off = sm.v_off;
