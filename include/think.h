@@ -320,10 +320,17 @@ think_status_t think_token_mass(const void *q_win, const void *k, const int64_t 
                                 int Hkv, int64_t N, int S_obs, int d, think_dtype_t dtype, float scale, float *mass,
                                 void *workspace, size_t workspace_bytes, void *stream);
 /* kept [B][Hkv][M] int32 output: the M tokens of largest mass per head (ties
- * to the lower index), ascending; 1 <= M <= N.  One launch (a block per
- * head, radix select on the masses' bits). */
+ * to the lower index), ascending; 1 <= M <= N <= INT32_MAX.  mass
+ * [B][Hkv][N] fp32, contiguous, non-negative (as think_token_mass writes it).
+ * Six launches, each over the whole GPU (a block per chunk of keys and head):
+ * four 8-bit radix passes on the masses' bits for the M-th largest value,
+ * a count per chunk, then the ordered write.  workspace: device scratch of
+ * think_select_tokens_workspace_size() bytes, 16-byte aligned, zeroed once
+ * (think_workspace_init) before its first use; every call leaves its radix
+ * histograms at zero.  THINK_ERR_WORKSPACE if it is too small. */
+size_t think_select_tokens_workspace_size(int B, int Hkv, int64_t N);
 think_status_t think_select_tokens(const float *mass, int B, int Hkv, int64_t N, int M, int32_t *kept,
-                                   void *stream);
+                                   void *workspace, size_t workspace_bytes, void *stream);
 /* out[b,h,j,:] = x[b,h,kept[b,h,j],:], out contiguous [B][Hkv][M][d] (a copy;
  * an out-of-range index gives a zero row).  One launch. */
 think_status_t think_gather_tokens(const void *x, const int64_t x_strides[3], int B, int Hkv, int64_t N, int d,

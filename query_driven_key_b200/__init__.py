@@ -41,7 +41,7 @@ EXPORTED = (
     "think_pruned_decode_attn_noalloc", "think_q4_ld", "think_q4_groups_bytes",
     "think_quantize_keys_q4", "think_pruned_decode_attn_q4", "think_ragged_rows", "think_select_adaptive",
     "think_compact_keys_ragged", "think_pruned_decode_attn_ragged", "think_token_mass_workspace_size",
-    "think_token_mass", "think_select_tokens", "think_gather_tokens",
+    "think_token_mass", "think_select_tokens_workspace_size", "think_select_tokens", "think_gather_tokens",
 )
 
 
@@ -92,8 +92,10 @@ def _load() -> ctypes.CDLL:
     lib.think_token_mass_workspace_size.restype = SZ
     lib.think_token_mass.argtypes = [P, P, I64P, I, I, I, I64, I, I, I, F, P, P, SZ, P]
     lib.think_token_mass.restype = I
-    lib.think_select_tokens.argtypes = [P, I, I, I64, I, P, P]
+    lib.think_select_tokens.argtypes = [P, I, I, I64, I, P, P, SZ, P]
     lib.think_select_tokens.restype = I
+    lib.think_select_tokens_workspace_size.argtypes = [I, I, I64]
+    lib.think_select_tokens_workspace_size.restype = SZ
     lib.think_gather_tokens.argtypes = [P, I64P, I, I, I64, I, I, P, I, P, P]
     lib.think_gather_tokens.restype = I
     lib.think_decode_workspace_size.argtypes = [I, I, I, I64, I, I]
@@ -395,10 +397,18 @@ def think_token_mass(q_win: torch.Tensor, k: torch.Tensor, mass: torch.Tensor, w
                                 _stream(stream)), "think_token_mass")
 
 
-def think_select_tokens(mass: torch.Tensor, M: int, kept: torch.Tensor, stream=None) -> None:
+def think_select_tokens_workspace_size(B: int, Hkv: int, N: int) -> int:
+    return int(lib.think_select_tokens_workspace_size(B, Hkv, N))
+
+
+def think_select_tokens(mass: torch.Tensor, M: int, kept: torch.Tensor, workspace: torch.Tensor,
+                        stream=None) -> None:
     """mass [B,Hkv,N] fp32 -> kept [B,Hkv,M] int32 (largest mass, ties to the lower index, ascending)."""
     B, Hkv, N = mass.shape
-    _check(lib.think_select_tokens(_ptr(mass), B, Hkv, N, int(M), _ptr(kept), _stream(stream)),
+    if not mass.is_contiguous() or mass.dtype != torch.float32 or kept.dtype != torch.int32:
+        raise ThinkError(THINK_ERR_INVALID_ARG, "think_select_tokens")
+    _check(lib.think_select_tokens(_ptr(mass), B, Hkv, N, int(M), _ptr(kept), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream)),
            "think_select_tokens")
 
 
@@ -427,11 +437,13 @@ class EvictedCache:
         self.v_kept = torch.empty((B, Hkv, M, d), dtype=dtype, device=device)
         self.mass_ws = torch.zeros(max(256, think_token_mass_workspace_size(B, Hq, Hkv, N, S_obs)),
                                    dtype=torch.uint8, device=device)
+        self.select_ws = torch.zeros(max(256, think_select_tokens_workspace_size(B, Hkv, N)),
+                                     dtype=torch.uint8, device=device)
         self.pruned = PrunedCache(B, Hq, Hkv, M, T, d, dtype=dtype, device=device)
 
     def prune(self, q_win, k, v, stream=None):
         think_token_mass(q_win, k, self.mass, self.mass_ws, stream=stream)
-        think_select_tokens(self.mass, self.M, self.kept, stream)
+        think_select_tokens(self.mass, self.M, self.kept, self.select_ws, stream)
         think_gather_tokens(k, self.kept, self.k_kept, stream)
         think_gather_tokens(v, self.kept, self.v_kept, stream)
         self.pruned.prune(q_win, self.k_kept, stream)

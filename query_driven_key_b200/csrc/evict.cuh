@@ -297,12 +297,217 @@ __global__ void __launch_bounds__(kMassThreads)
 }
 
 // ---------------------------------------------------------------------------
-// Top-M tokens of each head by mass (one block of 1024 threads per head):
-// a radix select on the masses' bits (non-negative floats order like their
-// bits) finds the M-th largest value, then one ordered pass keeps every token
-// above it and the lowest-indexed ties, writing the kept indices ascending.
+// Top-M tokens of each head by mass: the M-th largest key K* (masses are
+// non-negative floats, whose bit patterns order like their values), then
+// every token with key > K* and the lowest-indexed `ties` tokens with key ==
+// K*, written ascending.  Spread over the whole GPU: each head's keys are cut
+// into chunks of 256 * kpt keys (a block per chunk and head, kpt consecutive
+// keys per thread), and
+//   select_hist_kernel<P> (P = 0..3): a radix pass on the 8-bit digit P from
+//     the top: each block replays passes 0..P-1 from the global histograms
+//     (the same digit choice in every block), then adds its chunk's keys that
+//     match the prefix so far into hist[P][head];
+//   select_count_kernel: replays all four passes (K*, ties) and counts each
+//     chunk's keys above K* and equal to K*;
+//   select_write_kernel: each chunk's first output position from the counts of
+//     the chunks before it, then the chunk's kept tokens in index order (two
+//     block scans).
+// Workspace: hist [4][heads][256], sel [heads][2], cnt [heads][chunks][2]
+// (int32); hist is zero between calls (pass 0 clears hist[1..3] of the
+// previous call, the write kernel clears hist[0]).
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ int block_exclusive_scan_1024(int x, int *wsum, int &total)
+constexpr int kSelThreads = 256;
+
+struct SelectArgs {
+    const float *mass;  // [heads][N]
+    int64_t N;
+    int M, kpt, chunks;
+    int *hist;          // [4][heads][256]
+    int *sel;           // [heads][2]: K* bits, ties
+    int *cnt;           // [heads][chunks][2]: keys > K*, keys == K*
+    int32_t *kept;      // [heads][M]
+    int heads;
+};
+
+// A thread's keys are handled in batches of kSelBatch consecutive keys, every
+// load of a batch issued before the first is used (kpt is a multiple of it).
+constexpr int kSelBatch = 16;
+
+__device__ __forceinline__ void select_load_batch(const uint32_t *key, int64_t n, int64_t N,
+                                                  uint32_t (&kk)[kSelBatch], unsigned &valid)
+{
+    valid = 0u;
+#pragma unroll
+    for (int e = 0; e < kSelBatch; ++e) {
+        const bool in = n + e < N;
+        kk[e] = in ? __ldcg(key + n + e) : 0u;
+        valid |= in ? (1u << e) : 0u;
+    }
+}
+
+// Radix digit choice of one pass (warp 0; h = the pass's 256-bin histogram in
+// shared memory): the largest digit dg with sum_{d >= dg} h[d] >= need (else
+// 0), and need minus the keys of the digits above dg.  Lane l holds bins
+// 255 - 8l down to 248 - 8l.
+__device__ __forceinline__ void select_pick_digit(const int *h, int lane, int &need, int &dg)
+{
+    int v[8], s = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        v[e] = h[255 - 8 * lane - e];
+        s += v[e];
+    }
+    int cum = s;  // inclusive over lanes 0..lane (the higher digits first)
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, cum, o);
+        if (lane >= o) cum += y;
+    }
+    const unsigned hit = __ballot_sync(0xffffffffu, cum >= need);
+    int d = 0, left = need;
+    if (hit) {
+        const int L = __ffs(hit) - 1;
+        const int before = __shfl_sync(0xffffffffu, cum - s, L);  // keys of the lanes before L
+        int run = before, pick = 0, rest = need - before;
+        bool found = false;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int ve = __shfl_sync(0xffffffffu, v[e], L);
+            if (!found) {
+                if (run + ve >= need) {
+                    pick = 255 - 8 * L - e;
+                    rest = need - run;
+                    found = true;
+                } else {
+                    run += ve;
+                }
+            }
+        }
+        d = pick;
+        left = rest;
+    } else {
+        // fewer matching keys than need (not reached for 1 <= M <= N): digit 0
+        // after every higher digit, as a sequential scan would end
+        d = 0;
+        left = need - (__shfl_sync(0xffffffffu, cum, 31) - h[0]);
+    }
+    dg = d;
+    need = left;
+}
+
+// Replay passes 0..P-1 of this head: prefix and mask of the digits chosen so
+// far and the keys still to take among those matching them.  Every thread
+// of the block calls it; sh: 256 shared ints; sv: 3 shared ints.
+__device__ __forceinline__ void select_replay(const SelectArgs &a, int head, int P, int *sh, int *sv,
+                                              uint32_t &prefix, uint32_t &mask, int &need)
+{
+    const int tid = threadIdx.x;
+    if (tid == 0) {
+        sv[0] = 0;
+        sv[1] = 0;
+        sv[2] = a.M;
+    }
+    __syncthreads();
+    for (int p = 0; p < P; ++p) {
+        sh[tid] = a.hist[((int64_t)p * a.heads + head) * 256 + tid];
+        __syncthreads();
+        if (tid < 32) {
+            int nd = sv[2], dg;
+            select_pick_digit(sh, tid, nd, dg);
+            if (tid == 0) {
+                const int shift = 24 - 8 * p;
+                sv[0] = (int)((uint32_t)sv[0] | ((uint32_t)dg << shift));
+                sv[1] = (int)((uint32_t)sv[1] | (255u << shift));
+                sv[2] = nd;
+            }
+        }
+        __syncthreads();
+    }
+    prefix = (uint32_t)sv[0];
+    mask = (uint32_t)sv[1];
+    need = sv[2];
+}
+
+template <int P>
+__global__ void __launch_bounds__(kSelThreads) select_hist_kernel(const SelectArgs a)
+{
+    __shared__ int sh[256];
+    __shared__ int hloc[256];
+    __shared__ int sv[3];
+    const int head = blockIdx.y, tid = threadIdx.x;
+    uint32_t prefix, mask;
+    int need;
+    select_replay(a, head, P, sh, sv, prefix, mask, need);
+    if (P == 0 && blockIdx.x == 0) {  // the previous call's passes 1..3
+        for (int p = 1; p < 4; ++p) a.hist[((int64_t)p * a.heads + head) * 256 + tid] = 0;
+    }
+    hloc[tid] = 0;
+    __syncthreads();
+    const int shift = 24 - 8 * P;
+    const uint32_t *key = reinterpret_cast<const uint32_t *>(a.mass + (int64_t)head * a.N);
+    const int64_t n0 = (int64_t)blockIdx.x * kSelThreads * a.kpt + (int64_t)tid * a.kpt;
+    for (int e0 = 0; e0 < a.kpt; e0 += kSelBatch) {
+        uint32_t kk[kSelBatch];
+        unsigned valid;
+        select_load_batch(key, n0 + e0, a.N, kk, valid);
+#pragma unroll
+        for (int e = 0; e < kSelBatch; ++e)
+            if (((valid >> e) & 1u) && (kk[e] & mask) == prefix) atomicAdd(&hloc[(kk[e] >> shift) & 255u], 1);
+    }
+    __syncthreads();
+    if (hloc[tid]) atomicAdd(a.hist + ((int64_t)P * a.heads + head) * 256 + tid, hloc[tid]);
+}
+
+__global__ void __launch_bounds__(kSelThreads) select_count_kernel(const SelectArgs a)
+{
+    __shared__ int sh[256];
+    __shared__ int sv[3];
+    __shared__ int red[2][kSelThreads / 32];
+    const int head = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint32_t kth, mask;
+    int ties;
+    select_replay(a, head, 4, sh, sv, kth, mask, ties);
+    const uint32_t *key = reinterpret_cast<const uint32_t *>(a.mass + (int64_t)head * a.N);
+    const int64_t n0 = (int64_t)blockIdx.x * kSelThreads * a.kpt + (int64_t)tid * a.kpt;
+    int gt = 0, eq = 0;
+    for (int e0 = 0; e0 < a.kpt; e0 += kSelBatch) {
+        uint32_t kk[kSelBatch];
+        unsigned valid;
+        select_load_batch(key, n0 + e0, a.N, kk, valid);
+#pragma unroll
+        for (int e = 0; e < kSelBatch; ++e) {
+            const bool in = (valid >> e) & 1u;
+            gt += in && kk[e] > kth;
+            eq += in && kk[e] == kth;
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        gt += __shfl_xor_sync(0xffffffffu, gt, o);
+        eq += __shfl_xor_sync(0xffffffffu, eq, o);
+    }
+    if (lane == 0) {
+        red[0][warp] = gt;
+        red[1][warp] = eq;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int g = 0, q = 0;
+        for (int w = 0; w < kSelThreads / 32; ++w) {
+            g += red[0][w];
+            q += red[1][w];
+        }
+        a.cnt[((int64_t)head * a.chunks + blockIdx.x) * 2] = g;
+        a.cnt[((int64_t)head * a.chunks + blockIdx.x) * 2 + 1] = q;
+        if (blockIdx.x == 0) {
+            a.sel[head * 2] = (int)kth;
+            a.sel[head * 2 + 1] = ties;
+        }
+    }
+}
+
+// Exclusive scan of one int per thread over the block (256 threads).
+__device__ __forceinline__ int select_block_scan(int x, int *wsum, int &total)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int incl = x;
@@ -313,73 +518,83 @@ __device__ __forceinline__ int block_exclusive_scan_1024(int x, int *wsum, int &
     }
     if (lane == 31) wsum[warp] = incl;
     __syncthreads();
-    if (warp == 0) {
-        int w = wsum[lane];
+    int before = 0;
+    total = 0;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, w, o);
-            if (lane >= o) w += y;
-        }
-        wsum[lane] = w;
+    for (int w = 0; w < kSelThreads / 32; ++w) {
+        const int ws = wsum[w];
+        before += w < warp ? ws : 0;
+        total += ws;
     }
     __syncthreads();
-    total = wsum[31];
-    const int excl = incl - x + (warp > 0 ? wsum[warp - 1] : 0);
-    __syncthreads();
-    return excl;
+    return before + incl - x;
 }
 
-__global__ void __launch_bounds__(1024)
-    select_tokens_kernel(const float *__restrict__ mass, int64_t N, int M, int32_t *__restrict__ kept)
+__global__ void __launch_bounds__(kSelThreads) select_write_kernel(const SelectArgs a)
 {
-    __shared__ int hist[256];
-    __shared__ int wsum[32];
-    __shared__ uint32_t s_prefix, s_mask;
-    __shared__ int s_need;
-    const int head = blockIdx.x;
-    const uint32_t *key = reinterpret_cast<const uint32_t *>(mass + (int64_t)head * N);
-    const int tid = threadIdx.x;
-    if (tid == 0) {
-        s_prefix = 0u;
-        s_mask = 0u;
-        s_need = M;
+    __shared__ int wsum[kSelThreads / 32];
+    __shared__ int red[2][kSelThreads / 32];
+    const int head = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int c = blockIdx.x;
+    const uint32_t kth = (uint32_t)a.sel[head * 2];
+    const int ties = a.sel[head * 2 + 1];
+    // keys > K* and == K* in the chunks before this one
+    int gb = 0, qb = 0;
+    for (int j = tid; j < c; j += kSelThreads) {
+        gb += a.cnt[((int64_t)head * a.chunks + j) * 2];
+        qb += a.cnt[((int64_t)head * a.chunks + j) * 2 + 1];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        gb += __shfl_xor_sync(0xffffffffu, gb, o);
+        qb += __shfl_xor_sync(0xffffffffu, qb, o);
+    }
+    if (lane == 0) {
+        red[0][warp] = gb;
+        red[1][warp] = qb;
     }
     __syncthreads();
-    // four 8-bit digits from the top: the M-th largest key
-    for (int shift = 24; shift >= 0; shift -= 8) {
-        if (tid < 256) hist[tid] = 0;
-        __syncthreads();
-        const uint32_t prefix = s_prefix, mask = s_mask;
-        for (int64_t n = tid; n < N; n += 1024) {
-            const uint32_t k = key[n];
-            if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1);
-        }
-        __syncthreads();
-        if (tid == 0) {
-            int need = s_need, dg = 255;
-            for (; dg > 0 && hist[dg] < need; --dg) need -= hist[dg];
-            s_need = need;  // how many of the keys with this digit are still to take
-            s_prefix = prefix | ((uint32_t)dg << shift);
-            s_mask = mask | (255u << shift);
-        }
-        __syncthreads();
+    gb = qb = 0;
+#pragma unroll
+    for (int w = 0; w < kSelThreads / 32; ++w) {
+        gb += red[0][w];
+        qb += red[1][w];
     }
-    const uint32_t kth = s_prefix;
-    const int ties = s_need;  // keys equal to kth that are kept: the lowest-indexed ones
-    // ordered pass: keep key > kth, and the first `ties` keys == kth
-    int written = 0, ties_seen = 0;
-    for (int64_t base = 0; base < N; base += 1024) {
-        const int64_t n = base + tid;
-        const uint32_t k = n < N ? key[n] : 0u;
-        const int eq = (n < N && k == kth) ? 1 : 0;
-        int eq_total;
-        const int eq_before = block_exclusive_scan_1024(eq, wsum, eq_total);
-        const int keep = (n < N) && (k > kth || (eq && ties_seen + eq_before < ties)) ? 1 : 0;
-        int keep_total;
-        const int pos = block_exclusive_scan_1024(keep, wsum, keep_total);
-        if (keep && written + pos < M) kept[(int64_t)head * M + written + pos] = (int32_t)n;
-        written += keep_total;
-        ties_seen += eq_total;
+    // every count-kernel block has replayed hist[0] of this head: leave it zero
+    // (passes 1..3 are cleared by the next call's pass 0)
+    if (c == 0) a.hist[(int64_t)head * 256 + tid] = 0;
+    const uint32_t *key = reinterpret_cast<const uint32_t *>(a.mass + (int64_t)head * a.N);
+    const int64_t n0 = (int64_t)c * kSelThreads * a.kpt + (int64_t)tid * a.kpt;
+    // this thread's keys equal to K*, ranked over the chunk in index order
+    // (the usual kpt = kSelBatch: one batch, loaded once and kept in registers)
+    uint32_t kk[kSelBatch];
+    unsigned valid;
+    select_load_batch(key, n0, a.N, kk, valid);
+    int myeq = 0, mygt = 0;
+    for (int e0 = 0; e0 < a.kpt; e0 += kSelBatch) {
+        if (e0 > 0) select_load_batch(key, n0 + e0, a.N, kk, valid);
+#pragma unroll
+        for (int e = 0; e < kSelBatch; ++e) {
+            const bool in = (valid >> e) & 1u;
+            myeq += in && kk[e] == kth;
+            mygt += in && kk[e] > kth;
+        }
+    }
+    int eq_tot;
+    const int eq_rank0 = qb + select_block_scan(myeq, wsum, eq_tot);
+    // kept: every key above K*, and the keys equal to K* of rank < ties
+    const int mykeep = mygt + max(0, min(ties - eq_rank0, myeq));
+    int keep_tot;
+    int pos = gb + min(qb, ties) + select_block_scan(mykeep, wsum, keep_tot);
+    int r = eq_rank0;
+    for (int e0 = 0; e0 < a.kpt; e0 += kSelBatch) {
+        if (e0 > 0 || a.kpt > kSelBatch) select_load_batch(key, n0 + e0, a.N, kk, valid);
+#pragma unroll
+        for (int e = 0; e < kSelBatch; ++e) {
+            if (!((valid >> e) & 1u)) continue;
+            const bool keep = kk[e] > kth || (kk[e] == kth && r++ < ties);
+            if (keep && pos < a.M) a.kept[(int64_t)head * a.M + pos++] = (int32_t)(n0 + e0 + e);
+        }
     }
 }
 

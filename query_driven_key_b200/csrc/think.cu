@@ -944,6 +944,28 @@ cudaError_t noalloc_scratch(void **out)
 }  // namespace
 }  // namespace think
 
+namespace think {
+namespace {
+struct SelectWs {
+    int kpt, chunks;
+    size_t hist, sel, cnt, total;
+};
+
+SelectWs select_ws_layout(int64_t heads, int64_t N)
+{
+    SelectWs w;
+    // keys per thread: a multiple of kSelBatch, at most 1024 chunks per head
+    w.kpt = (int)(kSelBatch * std::max<int64_t>(1, ceil_div(N, (int64_t)kSelThreads * 1024 * kSelBatch)));
+    w.chunks = (int)std::max<int64_t>(1, ceil_div(N, (int64_t)kSelThreads * w.kpt));
+    w.hist = 0;
+    w.sel = align_up((size_t)4 * heads * 256 * sizeof(int), 256);
+    w.cnt = w.sel + align_up((size_t)heads * 2 * sizeof(int), 256);
+    w.total = w.cnt + (size_t)heads * w.chunks * 2 * sizeof(int);
+    return w;
+}
+}  // namespace
+}  // namespace think
+
 using namespace think;
 
 extern "C" {
@@ -1431,18 +1453,46 @@ think_status_t think_token_mass(const void *q_win, const void *k, const int64_t 
     }
 }
 
+size_t think_select_tokens_workspace_size(int B, int Hkv, int64_t N)
+{
+    if (B <= 0 || Hkv <= 0 || N <= 0 || N > (int64_t)INT32_MAX) return 0;
+    return select_ws_layout((int64_t)B * Hkv, N).total;
+}
+
 think_status_t think_select_tokens(const float *mass, int B, int Hkv, int64_t N, int M, int32_t *kept,
-                                   void *stream)
+                                   void *workspace, size_t workspace_bytes, void *stream)
 {
     if (B < 0 || Hkv < 0 || N < 0) return THINK_ERR_INVALID_ARG;
     if (B == 0 || Hkv == 0) return THINK_OK;
     if (M < 1 || M > N || N > (int64_t)INT32_MAX) return THINK_ERR_INVALID_ARG;
-    if (!mass || !kept) return THINK_ERR_INVALID_ARG;
+    if (!mass || !kept || !workspace) return THINK_ERR_INVALID_ARG;
     const int64_t heads = (int64_t)B * Hkv;
     if (heads > 65535) return THINK_ERR_UNSUPPORTED;
-    if ((reinterpret_cast<uintptr_t>(mass) & 3u) || (reinterpret_cast<uintptr_t>(kept) & 3u))
+    if ((reinterpret_cast<uintptr_t>(mass) & 3u) || (reinterpret_cast<uintptr_t>(kept) & 3u) ||
+        !aligned16(workspace))
         return THINK_ERR_ALIGNMENT;
-    select_tokens_kernel<<<(unsigned)heads, 1024, 0, static_cast<cudaStream_t>(stream)>>>(mass, N, M, kept);
+    const SelectWs w = select_ws_layout(heads, N);
+    if (workspace_bytes < w.total) return THINK_ERR_WORKSPACE;
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    SelectArgs a;
+    a.mass = mass;
+    a.N = N;
+    a.M = M;
+    a.kpt = w.kpt;
+    a.chunks = w.chunks;
+    a.hist = reinterpret_cast<int *>(ws + w.hist);
+    a.sel = reinterpret_cast<int *>(ws + w.sel);
+    a.cnt = reinterpret_cast<int *>(ws + w.cnt);
+    a.kept = kept;
+    a.heads = (int)heads;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const dim3 grid((unsigned)w.chunks, (unsigned)heads);
+    select_hist_kernel<0><<<grid, kSelThreads, 0, st>>>(a);
+    select_hist_kernel<1><<<grid, kSelThreads, 0, st>>>(a);
+    select_hist_kernel<2><<<grid, kSelThreads, 0, st>>>(a);
+    select_hist_kernel<3><<<grid, kSelThreads, 0, st>>>(a);
+    select_count_kernel<<<grid, kSelThreads, 0, st>>>(a);
+    select_write_kernel<<<grid, kSelThreads, 0, st>>>(a);
     return launch_status();
 }
 

@@ -202,10 +202,16 @@ def test_eviction_validation():
     assert f(FAKE, MISALIGNED, st, 1, 4, 2, 64, 8, 128, 1, 0.1, FAKE, FAKE, ws, None) == qdk.THINK_ERR_ALIGNMENT
     assert f(FAKE, FAKE, st, 0, 4, 2, 64, 8, 128, 1, 0.1, FAKE, FAKE, 0, None) == qdk.THINK_OK
     g = lib.think_select_tokens
-    assert g(FAKE, 1, 2, 64, 0, FAKE, None) == qdk.THINK_ERR_INVALID_ARG
-    assert g(FAKE, 1, 2, 64, 65, FAKE, None) == qdk.THINK_ERR_INVALID_ARG
-    assert g(None, 1, 2, 64, 8, FAKE, None) == qdk.THINK_ERR_INVALID_ARG
-    assert g(FAKE, 0, 2, 64, 8, FAKE, None) == qdk.THINK_OK
+    sws = qdk.think_select_tokens_workspace_size(1, 2, 64)
+    assert sws > 4 * 2 * 256 * 4 and qdk.think_select_tokens_workspace_size(1, 2, 0) == 0
+    # (mass, B, Hkv, N, M, kept, ws, ws_bytes, stream)
+    assert g(FAKE, 1, 2, 64, 0, FAKE, FAKE, sws, None) == qdk.THINK_ERR_INVALID_ARG
+    assert g(FAKE, 1, 2, 64, 65, FAKE, FAKE, sws, None) == qdk.THINK_ERR_INVALID_ARG
+    assert g(None, 1, 2, 64, 8, FAKE, FAKE, sws, None) == qdk.THINK_ERR_INVALID_ARG
+    assert g(FAKE, 1, 2, 64, 8, FAKE, None, sws, None) == qdk.THINK_ERR_INVALID_ARG
+    assert g(FAKE, 1, 2, 64, 8, FAKE, FAKE, sws - 4, None) == qdk.THINK_ERR_WORKSPACE
+    assert g(FAKE, 1, 2, 64, 8, FAKE, MISALIGNED, sws, None) == qdk.THINK_ERR_ALIGNMENT
+    assert g(FAKE, 0, 2, 64, 8, FAKE, None, 0, None) == qdk.THINK_OK
     h = lib.think_gather_tokens
     assert h(FAKE, st, 1, 2, 64, 96, 1, FAKE, 8, FAKE, None) == qdk.THINK_ERR_UNSUPPORTED
     assert h(FAKE, st, 1, 2, 64, 128, 1, FAKE, 8, MISALIGNED, None) == qdk.THINK_ERR_ALIGNMENT

@@ -293,6 +293,32 @@ def test_adaptive_width(case):
     assert qdk.think_read_device_status(cache.decode_ws) == 0
 
 
+@pytest.mark.parametrize("case", [(1, 1, 1, 1, "grid"), (1, 3, 4097, 4097, "grid"), (2, 4, 131072, 32768, "grid"),
+                                  (1, 2, 70001, 1, "grid"), (1, 1, 5_000_000, 1_000_000, "grid"),
+                                  (1, 8, 20000, 6000, "cont"), (3, 2, 9000, 8999, "cont")])
+def test_select_tokens_multi_block(case):
+    # the chunked radix selection against the oracle's rule on the same masses:
+    # coarse-grid masses (many exact ties, zeros included) and continuous ones,
+    # N = M, M = 1, chunk boundaries, and more keys per thread than the default
+    # (N > 256 * 1024 * 16); a second call checks that the histograms were
+    # left at zero
+    B, Hkv, N, M, kind = case
+    g = torch.Generator().manual_seed(N + M)
+    if kind == "grid":
+        mass = torch.randint(0, 50, (B, Hkv, N), generator=g).float() * 0.125
+    else:
+        mass = torch.rand((B, Hkv, N), generator=g) * 3.0
+    want = oracle.oracle_select_tokens(mass.double().numpy(), M)
+    md = mass.to(DEV)
+    ws = torch.zeros(max(256, qdk.think_select_tokens_workspace_size(B, Hkv, N)), dtype=torch.uint8, device=DEV)
+    kept = torch.empty((B, Hkv, M), dtype=torch.int32, device=DEV)
+    for _ in range(2):
+        kept.fill_(-1)
+        qdk.think_select_tokens(md, M, kept, ws)
+        torch.cuda.synchronize()
+        assert np.array_equal(kept.cpu().numpy(), want), case
+
+
 @pytest.mark.parametrize("case", [(1, 32, 8, 5000, 32, 1000, 51), (2, 8, 2, 1000, 16, 300, 64),
                                   (1, 4, 4, 300, 64, 300, 13), (1, 8, 1, 2049, 64, 129, 128),
                                   (2, 16, 8, 700, 8, 1, 32), (1, 64, 8, 1500, 64, 500, 40)])
