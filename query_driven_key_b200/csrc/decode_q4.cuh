@@ -143,7 +143,26 @@ __global__ void __launch_bounds__(CW * 32 + 32)
     constexpr int RPP = 32 / PARTS;      // channel rows per pass of a warp
     // Launched as a programmatic dependent of the previous kernel in the
     // stream: everything it wrote is visible after this wait; let the next
-    // decode be scheduled on SMs as ours free up.
+    // decode be scheduled on SMs as ours free up.  Before the wait the
+    // producer lane asks L2 for this block's first tiles and the q and idx
+    // lines (as in pruned_decode_mma_kernel: the kernels that let a decode
+    // start early write none of codes, groups or V, and L2 is coherent).
+    if (a.early && threadIdx.x == CW * 32) {
+        const int kv0 = (int)blockIdx.y % a.Hkv, b0 = (int)blockIdx.y / a.Hkv;
+        const int64_t t0 = (int64_t)blockIdx.x * a.tiles_per_split;
+        const int64_t n = min((int64_t)min(a.tiles_per_split, a.stages), (a.N + kBN - 1) / kBN - t0);
+        for (int64_t it = 0; it < n; ++it) {
+            const int tile = (int)(t0 + it);
+            tma_prefetch_l2_4d(&tm_codes, tile * 64, 0, kv0, b0);
+            tma_prefetch_l2_4d(&tm_groups, 0, tile, kv0, b0);
+            tma_prefetch_l2_4d(&tm_v, 0, tile * kBN, kv0, b0);
+            tma_prefetch_l2_4d(&tm_v, 64, tile * kBN, kv0, b0);
+        }
+        const char *qrow = reinterpret_cast<const char *>(a.q) + ((int64_t)b0 * a.Hq + (int64_t)kv0 * G) * kD * 2;
+        for (int o = 0; o < G * kD * 2; o += 128) prefetch_l2(qrow + o);
+        const char *irow = reinterpret_cast<const char *>(a.idx + (int64_t)blockIdx.y * a.T);
+        for (int o = 0; o < a.T * 4; o += 128) prefetch_l2(irow + o);
+    }
     grid_dependency_wait();
     grid_launch_dependents();
     extern __shared__ unsigned char smem_dyn[];

@@ -1290,6 +1290,7 @@ think_status_t think_pruned_decode_attn_q4(const void *q, const uint8_t *codes, 
     a.tiles_per_split = sp.tiles_per_split;
     a.splits = sp.splits;
     a.stages = mp.stages;
+    a.early = env_int("THINK_DECODE_EARLY_PREFETCH", 1, 0, 1);
     a.scale_log2 = scale * 1.4426950408889634f;
     return launch_decode_q4(G, mp.warps, mc, mg, mv, a, mp.bytes, (int)heads, static_cast<cudaStream_t>(stream));
 }
@@ -1385,6 +1386,7 @@ think_status_t think_pruned_decode_attn_ragged(const void *q, const void *k_prun
     a.tiles_per_split = sp.tiles_per_split;
     a.splits = sp.splits;
     a.stages = mp.stages;
+    a.early = env_int("THINK_DECODE_EARLY_PREFETCH", 1, 0, 1);
     a.scale_log2 = scale * 1.4426950408889634f;
     a.Th = Th;
     a.rowoff = rowoff;
