@@ -43,6 +43,7 @@ struct DecodeArgs {
     int stages_v;           // tcgen05 kernel: V ring slots (stages = K' ring slots)
     int prefetch;           // tiles prefetched into L2 ahead of the TMA loads
     int early;              // 1: the first tiles are prefetched into L2 before the dependency wait
+    int staged_merge;       // 1: the split merge copies the partial outputs into shared memory when they fit
     float scale_log2;       // scale * log2(e)
     uint32_t stage_bytes;   // bytes per ring stage (multiple of 1024)
     uint32_t v_off;         // offset of the V tile inside a stage
@@ -144,15 +145,18 @@ template <> struct V8<float> {
 // units, sum L[g]) for (head, split); the last block of the head to arrive
 // merges every split of the head into `out`.  Called by the NT threads
 // 0 .. NT-1 of the block (NT a multiple of 128), which synchronise on named
-// barrier `bar`; `scratch` is free shared memory of at least
-// (2 * splits * G + 2 * G + (NT / 128) * G * 128) floats, `flag` one shared
-// word.  The merge issues its global loads together: one round trip for the
-// (max, sum) pairs and about one per 8 * NT / 128 splits for the outputs.
+// barrier `bar`; `scratch` is free shared memory (16-byte aligned) of
+// scratch_floats >= (2 * splits * G + 2 * G + (NT / 128) * G * 128) floats,
+// `flag` one shared word.  When scratch also holds every partial output of
+// the head (splits * G * 128 floats more), the merge copies them in with
+// asynchronous 16-byte copies issued together with the (max, sum) loads: one
+// round trip in all; otherwise it loads the outputs 8 * NT / 128 splits per
+// round trip.  Both add the splits in the same order.
 template <int G, int NT>
 __device__ __forceinline__ void finish_split(const DecodeArgs &a, int head, int split, int b, int kv,
                                              int tid, const float (&O)[G], const float (&M)[G],
                                              const float (&L)[G], float *scratch, unsigned *flag,
-                                             int bar)
+                                             int bar, size_t scratch_floats = 0)
 {
     static_assert(NT % 128 == 0, "whole channel rows per thread group");
     constexpr int P = NT / 128;            // thread groups splitting the split axis
@@ -183,6 +187,16 @@ __device__ __forceinline__ void finish_split(const DecodeArgs &a, int head, int 
     float *smax = sl + nsg;         // [G]
     float *sL = smax + G;           // [G]
     float *sp = sL + G;             // [P][G][128]  per-group output sums
+    // [splits][G][128] the head's partial outputs, when they fit
+    const size_t so_off = ((size_t)2 * nsg + 2 * G + (size_t)P * G * kD + 3) & ~(size_t)3;
+    const bool staged = so_off + (size_t)nsg * kD <= scratch_floats;
+    float *so = scratch + so_off;
+    if (staged) {
+        const uint32_t dst = smem_addr(so);
+        const float4 *src = reinterpret_cast<const float4 *>(a.part_o + (int64_t)head * S * G * kD);
+        for (int i = tid; i < nsg * (kD / 4); i += NT) cp_async_16(dst + 16u * (uint32_t)i, src + i);
+        cp_async_commit();
+    }
     const float *pml = a.part_ml + (int64_t)head * S * G * 2;
     for (int i = tid; i < nsg; i += NT) {
         const float2 ml = __ldcg(reinterpret_cast<const float2 *>(pml) + i);
@@ -212,8 +226,16 @@ __device__ __forceinline__ void finish_split(const DecodeArgs &a, int head, int 
     float acc[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) acc[g] = 0.f;
+    if (staged) {
+        cp_async_wait_all();
+        named_barrier(bar, NT);
+        for (int s2 = q; s2 < S; s2 += P) {
+#pragma unroll
+            for (int g = 0; g < G; ++g) acc[g] = fmaf(so[(s2 * G + g) * kD + d], sw[s2 * G + g], acc[g]);
+        }
+    }
     constexpr int CH = 8;
-    for (int s0 = q; s0 < S; s0 += P * CH) {
+    for (int s0 = staged ? S : q; s0 < S; s0 += P * CH) {
         float v[CH][G];
 #pragma unroll
         for (int u = 0; u < CH; ++u) {

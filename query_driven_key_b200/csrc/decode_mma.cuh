@@ -268,7 +268,7 @@ __device__ __forceinline__ void mma_tile(uint32_t kbase, uint32_t k_half, uint32
 template <int G, int CW>
 __device__ __forceinline__ void mma_merge_and_finish(const DecodeArgs &a, MmaState &S, float *mo, float *mml,
                                                      float *scratch, unsigned *flag, int head, int split,
-                                                     int b, int kv, int tid)
+                                                     int b, int kv, int tid, size_t scratch_floats)
 {
     const int warp = tid >> 5, lane = tid & 31;
     const int q4 = lane & 3, r8 = lane >> 2;
@@ -313,7 +313,7 @@ __device__ __forceinline__ void mma_merge_and_finish(const DecodeArgs &a, MmaSta
         }
     }
     named_barrier(1, CW * 32);  // the split merge below reuses stage memory
-    finish_split<G, CW * 32>(a, head, split, b, kv, tid, O, M, Lsum, scratch, flag, 1);
+    finish_split<G, CW * 32>(a, head, split, b, kv, tid, O, M, Lsum, scratch, flag, 1, scratch_floats);
 }
 
 __device__ __forceinline__ void mma_state_init(MmaState &S)
@@ -485,7 +485,8 @@ __global__ void __launch_bounds__(CW * 32 + 32)
         __syncwarp();
         if (lane == 0) mbar_arrive(empty0 + 8 * s);
     }
-    mma_merge_and_finish<G, CW>(a, S, mo, mml, reinterpret_cast<float *>(smem), flag, head, split, b, kv, tid);
+    mma_merge_and_finish<G, CW>(a, S, mo, mml, reinterpret_cast<float *>(smem), flag, head, split, b, kv, tid,
+                                a.staged_merge ? (size_t)stages * L.stage / sizeof(float) : 0);
 }
 
 }  // namespace think

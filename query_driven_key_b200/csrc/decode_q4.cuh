@@ -298,7 +298,8 @@ __global__ void __launch_bounds__(CW * 32 + 32)
         __syncwarp();
         if (lane == 0) mbar_arrive(empty0 + 8 * s);
     }
-    mma_merge_and_finish<G, CW>(a, S, mo, mml, reinterpret_cast<float *>(smem), flag, head, split, b, kv, tid);
+    mma_merge_and_finish<G, CW>(a, S, mo, mml, reinterpret_cast<float *>(smem), flag, head, split, b, kv, tid,
+                                a.staged_merge ? (size_t)stages * L.stage / sizeof(float) : 0);
 }
 
 }  // namespace think

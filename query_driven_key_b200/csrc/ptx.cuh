@@ -143,6 +143,15 @@ __device__ __forceinline__ void tma_prefetch_l2_4d(const CUtensorMap *map, int c
                  : "memory");
 }
 
+// 16-byte asynchronous copy global -> shared through L2 (no registers held),
+// and the waits for this thread's copies.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // Prefetch the 128-byte line holding p into L2.
 __device__ __forceinline__ void prefetch_l2(const void *p)
 {

@@ -1188,6 +1188,7 @@ think_status_t think_pruned_decode_attn(const void *q, const void *k_pruned, int
     a.stages_v = use_tc ? tp.stages_v : 0;
     a.prefetch = env_int("THINK_DECODE_PREFETCH", kDecodePrefetchTiles, 0, 64);
     a.early = env_int("THINK_DECODE_EARLY_PREFETCH", 1, 0, 1);
+    a.staged_merge = env_int("THINK_DECODE_STAGED_MERGE", 1, 0, 1);
     a.scale_log2 = scale * 1.4426950408889634f;
     a.stage_bytes = sm.stage_bytes;
     a.v_off = sm.v_off;
@@ -1291,6 +1292,7 @@ think_status_t think_pruned_decode_attn_q4(const void *q, const uint8_t *codes, 
     a.splits = sp.splits;
     a.stages = mp.stages;
     a.early = env_int("THINK_DECODE_EARLY_PREFETCH", 1, 0, 1);
+    a.staged_merge = env_int("THINK_DECODE_STAGED_MERGE", 1, 0, 1);
     a.scale_log2 = scale * 1.4426950408889634f;
     return launch_decode_q4(G, mp.warps, mc, mg, mv, a, mp.bytes, (int)heads, static_cast<cudaStream_t>(stream));
 }
@@ -1387,6 +1389,7 @@ think_status_t think_pruned_decode_attn_ragged(const void *q, const void *k_prun
     a.splits = sp.splits;
     a.stages = mp.stages;
     a.early = env_int("THINK_DECODE_EARLY_PREFETCH", 1, 0, 1);
+    a.staged_merge = env_int("THINK_DECODE_STAGED_MERGE", 1, 0, 1);
     a.scale_log2 = scale * 1.4426950408889634f;
     a.Th = Th;
     a.rowoff = rowoff;
