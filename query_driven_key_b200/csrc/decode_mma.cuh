@@ -335,6 +335,28 @@ __global__ void __launch_bounds__(CW * 32 + 32)
     static_assert(CW == 4 || CW == 8, "32 or 16 tokens of a tile per consumer warp");
     constexpr int TPW = kBN / CW;
     constexpr int NT = CW * 32;
+    // Shared memory layout (kernel parameters only) and the ring barriers are
+    // set up before the dependency wait: they touch no global memory.
+    extern __shared__ unsigned char smem_dyn[];
+    unsigned char *smem = smem_dyn + ((1024u - (smem_addr(smem_dyn) & 1023u)) & 1023u);
+    const int stages = a.stages;
+    const MmaLayout L = mma_layout(a.T);
+    unsigned char *qsm = smem + (size_t)stages * L.stage;                       // [16][t_pad] bf16
+    float *mo = reinterpret_cast<float *>(qsm + 32u * L.t_pad);                 // [CW][G][128]
+    float *mml = mo + CW * G * kD;                                              // [CW][G][2]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(mml + CW * G * 2);
+    unsigned *flag = reinterpret_cast<unsigned *>(bars + 2 * stages);
+    const uint32_t full0 = smem_addr(bars);
+    const uint32_t empty0 = smem_addr(bars + stages);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < stages; ++s) {
+            mbar_init(full0 + 8 * s, 1);
+            mbar_init(empty0 + 8 * s, CW);
+        }
+        fence_barrier_init();
+    }
+    __syncthreads();  // barriers initialised
+
     // Launched as a programmatic dependent of the previous kernel in the
     // stream: everything it wrote is visible after this wait; let the next
     // decode be scheduled on SMs as ours free up.  Such a block becomes
@@ -346,6 +368,10 @@ __global__ void __launch_bounds__(CW * 32 + 32)
     // idx, which may well be written by the previous kernel: a prefetch only
     // warms L2); only kernel parameters are read before it (a ragged cache's
     // K' rows come from device data: V only).
+    if (threadIdx.x == CW * 32) {
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+    }
     if (a.early && threadIdx.x == CW * 32) {
         const int kv0 = (int)blockIdx.y % a.Hkv, b0 = (int)blockIdx.y / a.Hkv;
         const int64_t t0 = (int64_t)blockIdx.x * a.tiles_per_split;
@@ -370,8 +396,6 @@ __global__ void __launch_bounds__(CW * 32 + 32)
     }
     grid_dependency_wait();
     grid_launch_dependents();
-    extern __shared__ unsigned char smem_dyn[];
-    unsigned char *smem = smem_dyn + ((1024u - (smem_addr(smem_dyn) & 1023u)) & 1023u);
 
     const int split = blockIdx.x;
     const int head = blockIdx.y;
@@ -385,36 +409,16 @@ __global__ void __launch_bounds__(CW * 32 + 32)
     // clamped (garbage in, no access outside K' or idx)
     const int64_t row_cap = (int64_t)gridDim.y * ((a.T + 15) & ~15);
     const int64_t row0 = ragged ? min(max((int64_t)a.rowoff[head], (int64_t)0), row_cap - ((T + 15) & ~15)) : 0;
-    const int stages = a.stages;
-    const MmaLayout L = mma_layout(a.T);
     const uint32_t t_rows = ragged ? (uint32_t)((T + 15) & ~15) : L.t_pad;  // K' rows used
     const int64_t tile0 = (int64_t)split * a.tiles_per_split;
     const int64_t tiles_all = (a.N + kBN - 1) / kBN;
     const int ntiles = (int)min((int64_t)a.tiles_per_split, tiles_all - tile0);
 
-    unsigned char *qsm = smem + (size_t)stages * L.stage;                       // [16][t_pad] bf16
-    float *mo = reinterpret_cast<float *>(qsm + 32u * L.t_pad);                 // [CW][G][128]
-    float *mml = mo + CW * G * kD;                                              // [CW][G][2]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(mml + CW * G * 2);
-    unsigned *flag = reinterpret_cast<unsigned *>(bars + 2 * stages);
-    const uint32_t full0 = smem_addr(bars);
-    const uint32_t empty0 = smem_addr(bars + stages);
-
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    if (tid == 0) {
-        for (int s = 0; s < stages; ++s) {
-            mbar_init(full0 + 8 * s, 1);
-            mbar_init(empty0 + 8 * s, CW);
-        }
-        fence_barrier_init();
-    }
-    __syncthreads();  // barriers initialised
 
     if (warp == CW) {
         // ------------------------------------------------------ producer
         if (lane == 0) {
-            prefetch_tensormap(&tm_k);
-            prefetch_tensormap(&tm_v);
             const uint32_t tx = ragged ? 2u * t_rows * 128u + 32768u : 2u * 64u * (uint32_t)T * 2u + 32768u;
             int issued = 0;
             bool ok = true;
