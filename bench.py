@@ -39,7 +39,7 @@ FALLBACK_HBM_GBS = 6650.0
 # default bf16 decode kernel, pruned_decode_mma_kernel<4, 4>, on the long-context
 # workload, from one ncu capture of that kernel; reported only for that
 # workload and to be reset to None whenever the kernel changes.
-DECODE_TRAFFIC_BYTES = 375_497_216 + 3_825_664
+DECODE_TRAFFIC_BYTES = 375_460_352 + 3_624_192
 
 
 def parse():
