@@ -289,6 +289,18 @@ think_status_t think_compact_keys_ragged(const void *k, const int64_t k_strides[
                                          int d, think_dtype_t dtype, const int32_t *idx, const int32_t *Th,
                                          const int32_t *rowoff, int T_max, void *k_pruned, int64_t ldk,
                                          void *stream);
+/* The whole prune with a kept width per head, as think_prune is for one T:
+ * scores (think_score_channels), the adaptive selection
+ * (think_select_adaptive) and the ragged compaction (think_compact_keys_ragged)
+ * in three launches on `stream`, with the same outputs as those three calls.
+ * Arguments as for those calls; workspace is the score workspace (its first
+ * 4 bytes are the device status word, which the compaction's bounded waits
+ * also use). */
+think_status_t think_prune_adaptive(const void *q_win, const void *k, const int64_t k_strides[3], int B, int Hq,
+                                    int Hkv, int64_t N, int S_obs, int d, think_dtype_t dtype, double tau,
+                                    int T_min, int T_max, double *scores, int32_t *Th, int32_t *rowoff,
+                                    int32_t *idx, void *k_pruned, int64_t ldk, void *workspace,
+                                    size_t workspace_bytes, void *stream);
 /* think_pruned_decode_attn for the ragged layout: query heads of KV head h
  * use its T_h kept channels; bf16 only; workspace as for
  * think_pruned_decode_attn.  One launch. */

@@ -40,7 +40,8 @@ EXPORTED = (
     "think_workspace_init", "think_read_device_status", "think_noalloc_scratch_bytes",
     "think_pruned_decode_attn_noalloc", "think_q4_ld", "think_q4_groups_bytes",
     "think_quantize_keys_q4", "think_pruned_decode_attn_q4", "think_ragged_rows", "think_select_adaptive",
-    "think_compact_keys_ragged", "think_pruned_decode_attn_ragged", "think_token_mass_workspace_size",
+    "think_compact_keys_ragged", "think_prune_adaptive", "think_pruned_decode_attn_ragged",
+    "think_token_mass_workspace_size",
     "think_token_mass", "think_select_tokens_workspace_size", "think_select_tokens", "think_gather_tokens",
 )
 
@@ -83,6 +84,8 @@ def _load() -> ctypes.CDLL:
     lib.think_ragged_rows.argtypes = [I, I, I]
     lib.think_ragged_rows.restype = I64
     lib.think_select_adaptive.argtypes = [P, I, I, I, D, I, I, P, P, P, P]
+    lib.think_prune_adaptive.argtypes = [P, P, I64P, I, I, I, I64, I, I, I, D, I, I, P, P, P, P, P, I64, P, SZ, P]
+    lib.think_prune_adaptive.restype = I
     lib.think_select_adaptive.restype = I
     lib.think_compact_keys_ragged.argtypes = [P, I64P, I, I, I64, I, I, P, P, P, I, P, I64, P]
     lib.think_compact_keys_ragged.restype = I
@@ -321,6 +324,23 @@ def think_select_adaptive(scores: torch.Tensor, tau: float, T_min: int, T_max: i
                                      _ptr(rowoff), _ptr(idx), _stream(stream)), "think_select_adaptive")
 
 
+def think_prune_adaptive(q_win: torch.Tensor, k: torch.Tensor, tau: float, T_min: int, T_max: int,
+                         scores: torch.Tensor, Th: torch.Tensor, rowoff: torch.Tensor, idx: torch.Tensor,
+                         k_pruned: torch.Tensor, ldk: int, workspace: torch.Tensor, stream=None) -> None:
+    """Scores, adaptive selection and ragged compaction (three launches): the
+    outputs of think_score_channels + think_select_adaptive +
+    think_compact_keys_ragged."""
+    B, Hq, S, d = q_win.shape
+    _, Hkv, N, _ = k.shape
+    if not q_win.is_contiguous() or scores.dtype != torch.float64 or k_pruned.dtype != k.dtype:
+        raise ThinkError(THINK_ERR_INVALID_ARG, "think_prune_adaptive")
+    _check(lib.think_prune_adaptive(_ptr(q_win), _ptr(k), _strides3(k), B, Hq, Hkv, N, S, d, _dtype(k), float(tau),
+                                    int(T_min), int(T_max), _ptr(scores), _ptr(Th), _ptr(rowoff), _ptr(idx),
+                                    _ptr(k_pruned), int(ldk), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(stream)),
+           "think_prune_adaptive")
+
+
 def think_compact_keys_ragged(k: torch.Tensor, idx: torch.Tensor, Th: torch.Tensor, rowoff: torch.Tensor,
                               T_max: int, k_pruned: torch.Tensor, ldk: int, stream=None) -> None:
     B, Hkv, N, d = k.shape
@@ -350,7 +370,8 @@ def think_pruned_decode_attn_ragged(q: torch.Tensor, k_pruned: torch.Tensor, ldk
 class AdaptiveCache:
     """Device buffers of one layer pruned with a kept width per head (ragged
     thinner K).  Allocates with torch on construction, then only calls the C
-    entry points: prune = scores, adaptive selection, ragged compaction."""
+    entry points: prune = scores, adaptive selection, ragged compaction
+    (think_prune_adaptive)."""
 
     def __init__(self, B: int, Hq: int, Hkv: int, N: int, tau: float, T_min: int, T_max: int, d: int = 128,
                  dtype: torch.dtype = torch.bfloat16, device="cuda"):
@@ -369,6 +390,11 @@ class AdaptiveCache:
                                      dtype=torch.uint8, device=device)
 
     def prune(self, q_win, k, stream=None):
+        think_prune_adaptive(q_win, k, self.tau, self.T_min, self.T_max, self.scores, self.Th, self.rowoff,
+                             self.idx, self.k_pruned, self.ldk, self.score_ws, stream)
+
+    def prune_stepwise(self, q_win, k, stream=None):
+        """The same prune through the three separate entry points."""
         think_score_channels(q_win, k, self.scores, self.score_ws, stream)
         think_select_adaptive(self.scores, self.tau, self.T_min, self.T_max, self.Th, self.rowoff, self.idx,
                               stream)

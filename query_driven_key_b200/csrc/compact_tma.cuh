@@ -16,7 +16,8 @@
 // lanes (compact_tile_load / compact_tile_store), so that each lane stores 8
 // consecutive tokens of one kept channel as one 16-byte write.  A block keeps
 // one head, so each warp finds the K' rows of its channels once.  K' is a pure
-// copy: the output is that of compact_kernel bit for bit.
+// copy: the output is that of compact_kernel bit for bit, in the uniform and
+// in the ragged layout (kept width per head, zero pad rows).
 //
 // Launched with programmatic stream serialisation after the score kernel: the
 // producer streams K (not written by the score pass) while the score grid
@@ -45,9 +46,12 @@ struct CompactTmaArgs {
     int run_tiles;           // tiles per block (block x: tiles [x * run_tiles, ...) of head y)
     int stages;
     int64_t N, tiles, ldk;   // tiles = ceil(N / 64)
-    const int32_t *idx;      // [heads][T] kept channels, ascending
-    __nv_bfloat16 *kp;       // K' [heads][T][ldk]
+    const int32_t *idx;      // [heads][T] kept channels, ascending (ragged: at rowoff[head])
+    __nv_bfloat16 *kp;       // K' [heads][T][ldk] (ragged: rows rowoff[head] ..)
     unsigned *status;        // device status word
+    const int32_t *Th;       // ragged layout: kept width per head, or null (T for every head)
+    const int32_t *rowoff;   // ragged layout: first K' row (and idx entry) of each head
+    int64_t row_cap;         // ragged layout: rows of K' (heads * roundup16(T))
 };
 
 inline size_t compact_tma_smem_bytes(int stages)
@@ -70,6 +74,19 @@ __global__ void __launch_bounds__(kCtThreads, 3)
     const int tid = threadIdx.x;
     const int64_t tile0 = (int64_t)blockIdx.x * a.run_tiles;
     const int ntiles = (int)min((int64_t)a.run_tiles, a.tiles - tile0);
+    // Ragged layout (a.Th set): this head keeps Tk = Th[head] channels at rows
+    // r0 = rowoff[head] .., then zero rows up to Tw = roundup16(Tk).  Those are
+    // device data written by the selection, so the whole block waits first; a
+    // head whose rows fall outside K' is skipped (garbage in, no access out).
+    int Tk = a.T, Tw = a.T;
+    int64_t r0 = (int64_t)head * a.T;
+    if (a.Th != nullptr) {
+        grid_dependency_wait();
+        Tk = min(max(a.Th[head], 0), a.T);
+        Tw = (Tk + 15) & ~15;
+        r0 = a.rowoff[head];
+        if (r0 < 0 || r0 + Tw > a.row_cap) return;
+    }
 
     if (tid == 0) {
         for (int s = 0; s < stages; ++s) {
@@ -112,7 +129,10 @@ __global__ void __launch_bounds__(kCtThreads, 3)
     const uint32_t c_row = (uint32_t)(8 * (tb0 + (lane >> 3)) + (lane & 7));
     int64_t crow[4];
     grid_dependency_wait();  // the selection (idx) is complete; K' may be written
-    kept_rows_of_warp(a.idx + (int64_t)head * a.T, a.T, (int64_t)head * a.T, cw, lane, crow);
+    kept_rows_of_warp(a.idx + r0, Tk, r0, cw, lane, crow);
+    // ragged: thread tid zeroes 8 tokens (run tid % 8) of pad row Tk + tid / 8
+    const int pad_row = Tk + (tid >> 3);
+    const uint32_t zero[4] = {0u, 0u, 0u, 0u};
     for (int i = 0; i < ntiles; ++i) {
         const int s = i % stages;
         if (!mbar_wait_bounded(full0 + 8 * s, (uint32_t)((i / stages) & 1), a.status, THINK_DEVICE_TIMEOUT_FULL))
@@ -121,7 +141,9 @@ __global__ void __launch_bounds__(kCtThreads, 3)
         compact_tile_load(ring + (uint32_t)s * kCtTileBytes, c_row, cw, v);
         __syncwarp();
         if (lane == 0) mbar_arrive(empty0 + 8 * s);
-        compact_tile_store(v, lane, crow, a.kp, a.ldk, (tile0 + i) * kCtTileRows + 8 * (tb0 + (lane & 3)), a.N);
+        const int64_t x0 = (tile0 + i) * kCtTileRows;
+        compact_tile_store(v, lane, crow, a.kp, a.ldk, x0 + 8 * (tb0 + (lane & 3)), a.N);
+        if (pad_row < Tw) store_run8(a.kp + (r0 + pad_row) * a.ldk, x0 + 8 * (tid & 7), a.N, zero);
     }
 }
 

@@ -558,7 +558,7 @@ int plan_compact_tma(int64_t heads, int64_t tiles)
 // THINK_COMPACT_TMA=0.
 think_status_t launch_compact_tma(const void *k, const int64_t k_strides[3], int B, int Hkv, int64_t N,
                                   const int32_t *idx, int T, void *k_pruned, int64_t ldk, void *workspace,
-                                  cudaStream_t st)
+                                  cudaStream_t st, const int32_t *Th = nullptr, const int32_t *rowoff = nullptr)
 {
     if (env_int("THINK_COMPACT_TMA", 1, 0, 1) == 0 || N > (int64_t)INT32_MAX - kCtTileRows)
         return THINK_ERR_UNSUPPORTED;
@@ -578,6 +578,9 @@ think_status_t launch_compact_tma(const void *k, const int64_t k_strides[3], int
     a.idx = idx;
     a.kp = static_cast<__nv_bfloat16 *>(k_pruned);
     a.status = reinterpret_cast<unsigned *>(static_cast<unsigned char *>(workspace));  // score workspace word 0
+    a.Th = Th;
+    a.rowoff = rowoff;
+    a.row_cap = heads * ((T + 15) & ~15);
     const size_t bytes = compact_tma_smem_bytes(a.stages);
     if (!ensure_smem(reinterpret_cast<const void *>(compact_tma_kernel), bytes)) return THINK_ERR_CUDA;
     dim3 grid((unsigned)ceil_div(a.tiles, a.run_tiles), (unsigned)heads);
@@ -1333,6 +1336,35 @@ think_status_t think_compact_keys_ragged(const void *k, const int64_t k_strides[
         return THINK_ERR_ALIGNMENT;
     return launch_compact(k, k_strides, B, Hkv, N, dtype, idx, T_max, k_pruned, ldk,
                           static_cast<cudaStream_t>(stream), 0, Th, rowoff);
+}
+
+think_status_t think_prune_adaptive(const void *q_win, const void *k, const int64_t k_strides[3], int B, int Hq,
+                                    int Hkv, int64_t N, int S_obs, int d, think_dtype_t dtype, double tau,
+                                    int T_min, int T_max, double *scores, int32_t *Th, int32_t *rowoff,
+                                    int32_t *idx, void *k_pruned, int64_t ldk, void *workspace,
+                                    size_t workspace_bytes, void *stream)
+{
+    think_status_t v = validate_score(q_win, k, k_strides, B, Hq, Hkv, N, S_obs, d, dtype, scores, workspace,
+                                      workspace_bytes);
+    if (v != THINK_OK) return v;
+    if (!(tau >= 0.0 && tau <= 1.0) || T_min < 1 || T_max < T_min || T_max > d) return THINK_ERR_INVALID_ARG;
+    v = validate_compact(k, k_strides, B, Hkv, N, d, dtype, idx, T_max, k_pruned, ldk);
+    if (v != THINK_OK || B == 0 || Hkv == 0) return v;
+    if (!Th || !rowoff) return THINK_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(Th) & 3u) || (reinterpret_cast<uintptr_t>(rowoff) & 3u))
+        return THINK_ERR_ALIGNMENT;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t heads = (int64_t)B * Hkv;
+    v = launch_score(q_win, k, k_strides, B, Hq, Hkv, N, S_obs, dtype, 0, scores, nullptr, workspace, st);
+    if (v != THINK_OK) return v;
+    select_adaptive_kernel<<<1, 1024, 0, st>>>(scores, (int)heads, tau, T_min, T_max, Th, rowoff, idx);
+    v = launch_status();
+    if (v != THINK_OK || N == 0) return v;
+    if (dtype == THINK_BF16) {
+        v = launch_compact_tma(k, k_strides, B, Hkv, N, idx, T_max, k_pruned, ldk, workspace, st, Th, rowoff);
+        if (v != THINK_ERR_UNSUPPORTED) return v;
+    }
+    return launch_compact(k, k_strides, B, Hkv, N, dtype, idx, T_max, k_pruned, ldk, st, 0, Th, rowoff);
 }
 
 think_status_t think_pruned_decode_attn_ragged(const void *q, const void *k_pruned, int64_t ldk, const void *v,

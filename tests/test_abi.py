@@ -179,6 +179,22 @@ def test_adaptive_validation():
     g = lib.think_compact_keys_ragged
     assert g(FAKE, s, 1, 2, 64, 128, 1, FAKE, None, FAKE, 10, FAKE, 64, None) == qdk.THINK_ERR_INVALID_ARG
     assert g(FAKE, s, 1, 2, 64, 128, 1, FAKE, FAKE, FAKE, 129, FAKE, 64, None) == qdk.THINK_ERR_INVALID_ARG
+    p = lib.think_prune_adaptive
+    sws = qdk.think_score_workspace_size(1, 4, 2, 64)
+    # (q_win, k, strides, B, Hq, Hkv, N, S, d, dtype, tau, T_min, T_max, scores, Th, rowoff, idx, kp, ldk,
+    #  ws, ws_bytes, stream)
+    pa = lambda **kw: (lambda a: p(a["q"], a["k"], s, a["B"], 4, 2, 64, 8, a["d"], 1, a["tau"], a["tmin"], a["tmax"],
+                                   FAKE, a["Th"], FAKE, FAKE, FAKE, 64, FAKE, a["wsb"], None))(
+        dict(dict(q=FAKE, k=FAKE, B=1, d=128, tau=0.5, tmin=1, tmax=32, Th=FAKE, wsb=sws), **kw))
+    assert pa(tau=1.5) == qdk.THINK_ERR_INVALID_ARG
+    assert pa(tmin=8, tmax=4) == qdk.THINK_ERR_INVALID_ARG
+    assert pa(tmax=129) == qdk.THINK_ERR_INVALID_ARG
+    assert pa(d=96) == qdk.THINK_ERR_UNSUPPORTED
+    assert pa(Th=None) == qdk.THINK_ERR_INVALID_ARG
+    assert pa(Th=ctypes.c_void_p(0x10002)) == qdk.THINK_ERR_ALIGNMENT
+    assert pa(k=MISALIGNED) == qdk.THINK_ERR_ALIGNMENT
+    assert pa(wsb=sws - 8) == qdk.THINK_ERR_WORKSPACE
+    assert pa(B=0, wsb=0) == qdk.THINK_OK
     h = lib.think_pruned_decode_attn_ragged
     vs = I64x3(128 * 64 * 2, 128 * 64, 128)
     ws = qdk.think_decode_workspace_size(1, 4, 2, 64)

@@ -291,6 +291,20 @@ def test_adaptive_width(case):
     check_out(out, oracle.oracle_decode_ragged(f64(q), kf, f64(v), oTh, ooff, oidx), torch.bfloat16,
               where=str(case))
     assert qdk.think_read_device_status(cache.decode_ws) == 0
+    assert qdk.think_read_device_status(cache.score_ws) == 0
+    # the one-entry prune (TMA compaction in the ragged layout) gives the
+    # outputs of the three separate calls (register compaction) bit for bit
+    step = qdk.AdaptiveCache(B, Hq, Hkv, N, tau, T_min, T_max)
+    step.k_pruned.fill_(7.0)
+    step.prune_stepwise(q_win.to(DEV), kd)
+    torch.cuda.synchronize()
+    for name in ("scores", "Th", "rowoff"):
+        assert torch.equal(getattr(step, name), getattr(cache, name)), name
+    sidx = step.idx.cpu().numpy()
+    for bh in range(B * Hkv):  # kept entries (a head's pad entries of idx are unspecified)
+        T = int(Th.ravel()[bh])
+        assert np.array_equal(sidx[rowoff[bh]:rowoff[bh] + T], gidx[rowoff[bh]:rowoff[bh] + T])
+    assert torch.equal(step.k_pruned[:, :N], cache.k_pruned[:, :N])
 
 
 @pytest.mark.parametrize("case", [(1, 1, 1, 1, "grid"), (1, 3, 4097, 4097, "grid"), (2, 4, 131072, 32768, "grid"),
