@@ -17,7 +17,8 @@
  * plus think_prune, the first three in two launches; think_append_keys,
  * which appends new tokens' keys to the thinner cache; a 4-bit thinner
  * cache (think_quantize_keys_q4, think_pruned_decode_attn_q4); a kept
- * width per head (think_select_adaptive and the _ragged calls); and token
+ * width per head (think_select_adaptive, think_prune_adaptive and the _ragged
+ * calls); and token
  * eviction to compose with it (think_token_mass, think_select_tokens,
  * think_gather_tokens).
  *
