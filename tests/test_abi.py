@@ -252,3 +252,19 @@ def test_decode_validation():
     assert call(args(wsb=64)) == qdk.THINK_ERR_WORKSPACE
     assert call(args(out=None)) == qdk.THINK_ERR_INVALID_ARG
     assert call(args(B=0)) == qdk.THINK_OK
+
+
+def test_select_tokens_workspace_layout():
+    # radix histograms [4][heads][256] + (M-th key, ties) per head + two counts
+    # per chunk and head, int32, each part padded to 256 bytes; chunks of
+    # 256 threads x kpt keys, kpt a multiple of 16 keeping chunks <= 1024
+    def want(B, Hkv, N):
+        heads = B * Hkv
+        kpt = 16 * max(1, -(-N // (256 * 1024 * 16)))
+        chunks = max(1, -(-N // (256 * kpt)))
+        pad = lambda x: -(-x // 256) * 256
+        return pad(4 * heads * 256 * 4) + pad(heads * 2 * 4) + heads * chunks * 2 * 4
+    for B, Hkv, N in [(1, 1, 1), (1, 8, 131072), (4, 8, 32768), (1, 1, 4_194_304), (1, 1, 4_194_305),
+                      (2, 3, 5_000_000), (1, 1, 2**31 - 1)]:
+        assert qdk.think_select_tokens_workspace_size(B, Hkv, N) == want(B, Hkv, N), (B, Hkv, N)
+    assert qdk.think_select_tokens_workspace_size(1, 1, 2**31) == 0
