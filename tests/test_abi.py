@@ -268,3 +268,35 @@ def test_select_tokens_workspace_layout():
                       (2, 3, 5_000_000), (1, 1, 2**31 - 1)]:
         assert qdk.think_select_tokens_workspace_size(B, Hkv, N) == want(B, Hkv, N), (B, Hkv, N)
     assert qdk.think_select_tokens_workspace_size(1, 1, 2**31) == 0
+
+
+def _score_plans(heads, N):
+    """The score pass's split plans (runs of 64-token tiles) restated: waves = 0
+    the fixed rule (about 4 runs per SM, 4..32 tiles), waves = 1..4 the
+    shortest runs whose count fits that many waves of 148 x 3 block slots."""
+    cdiv = lambda a, b: -(-a // b)
+    tph = max(1, cdiv(N, 64))
+    plans = {}
+    st = min(max(heads * tph // (148 * 4), 4), 32)
+    plans[0] = cdiv(tph, min(max(st, 1), tph))
+    for w in range(1, 5):
+        rph = max(1, 148 * 3 * w // max(heads, 1))
+        st = min(max(cdiv(tph, rph), 1), tph)
+        plans[w] = cdiv(tph, st)
+    return plans
+
+
+def test_score_workspace_covers_every_plan():
+    # header 256 B + tickets, ready flags, compact counters (256-byte aligned)
+    # + window-query energies [heads][G][128] fp64 + partials for the plan
+    # with the most runs per head; pins the plan rules on the CPU
+    pad = lambda x: -(-x // 256) * 256
+    for B, Hq, Hkv, N in [(1, 32, 8, 131072), (4, 32, 8, 32768), (1, 32, 32, 4096), (32, 32, 8, 8192),
+                          (1, 1, 1, 512), (1, 8, 1, 1), (2, 16, 8, 0), (3, 24, 8, 100_000)]:
+        heads, G = B * Hkv, Hq // Hkv
+        splits = max(_score_plans(heads, N).values())
+        want = 256 + 3 * pad(heads * 4) + pad(heads * G * 128 * 8) + heads * splits * 128 * 8
+        assert qdk.think_score_workspace_size(B, Hq, Hkv, N, 128) == want, (B, Hq, Hkv, N)
+    # the long-context layer: one wave of 432 runs of 38 tiles (the fixed rule: 76 runs of 27)
+    p = _score_plans(8, 131072)
+    assert p[1] == 54 and p[0] == 76
