@@ -51,6 +51,9 @@ MUTATIONS = {
                             "for (int n = 0; n < N; ++n) mh[n] += z[n];"),
     "adaptive_offsets_not_advanced": ("        rows += T;\n    }\n    off[B * Hkv] = rows;",
                                       "    }\n    off[B * Hkv] = rows;"),
+    "tokens_kept_list_not_reordered": ("        qsort(order, (size_t)M, sizeof(int), ascending_int);\n", ""),
+    "tokens_first_m_by_index": ("qsort(order, (size_t)N, sizeof(int), by_score_desc);",
+                                "qsort(order, (size_t)N, sizeof(int), ascending_int);"),
 }
 
 
@@ -131,6 +134,16 @@ def _pins(o: oracle.Oracle):
     mass = o.token_mass(qw, kk)
     p = torch.softmax(torch.from_numpy(qw[0].reshape(6, 8)) @ torch.from_numpy(kk[0, 0]).T / math.sqrt(8), -1)
     yield "mass_softmax", bool(np.allclose(mass[0, 0], p.sum(0).numpy(), rtol=1e-12, atol=1e-15))
+    # token selection against Python's sort (largest mass, ties to the lower
+    # index, kept indices ascending), with many exact ties
+    ms = r.integers(0, 4, size=(1, 2, 20)).astype(np.float64)
+    ok = True
+    for M in (1, 7, 20):
+        kept = o.select_tokens(ms, M)
+        for h in range(2):
+            order = sorted(range(20), key=lambda n: (-ms[0, h, n], n))
+            ok &= kept[0, h].tolist() == sorted(order[:M])
+    yield "select_tokens_sort", bool(ok)
 
 
 def _all_pass(o):
