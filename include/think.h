@@ -223,13 +223,26 @@ think_status_t think_pruned_decode_attn(const void *q, const void *k_pruned, int
  *     GPU (different streams, or different host threads without ordering)
  *     race and give wrong results.  Order them on one stream.
  *   - A problem whose workspace (think_decode_workspace_size) exceeds the
- *     array returns THINK_ERR_WORKSPACE and launches nothing. */
+ *     array returns THINK_ERR_WORKSPACE and launches nothing.
+ *   - The kernels' device status word (THINK_DEVICE_TIMEOUT_* bits) lives in
+ *     the array's first 4 bytes; each call clears it.  Read it after a call
+ *     with think_noalloc_read_device_status (a non-zero value means that
+ *     call's outputs are invalid).
+ *   - The array's device address is looked up once per device and kept for
+ *     the life of the process; after cudaDeviceReset the library must be
+ *     reloaded before this entry point is used again on that device. */
 size_t think_noalloc_scratch_bytes(void);
 think_status_t think_pruned_decode_attn_noalloc(const void *q, const void *k_pruned, int64_t ldk,
                                                 const void *v, const int64_t v_strides[3],
                                                 const int32_t *idx, int B, int Hq, int Hkv,
                                                 int64_t N, int d, int T, think_dtype_t dtype,
                                                 float scale, float *out, void *stream);
+/* The device status word of the no-allocation decode on the current device
+ * (that of the last call ordered before this one on `stream`): copies it to
+ * *status and synchronises `stream`, like think_read_device_status.  No
+ * counterpart on the pages; it allocates nothing.  THINK_ERR_INVALID_ARG for a
+ * null status, THINK_ERR_CUDA if a CUDA call fails. */
+think_status_t think_noalloc_read_device_status(uint32_t *status, void *stream);
 
 /* ---------------------------------------------------------- 4-bit K' --
  * The thinner key cache at 4 bits per element (ThinK abstract and method

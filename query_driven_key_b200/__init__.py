@@ -38,7 +38,7 @@ EXPORTED = (
     "think_compact_keys", "think_append_keys", "think_prune", "think_decode_workspace_size",
     "think_pruned_decode_attn",
     "think_workspace_init", "think_read_device_status", "think_noalloc_scratch_bytes",
-    "think_pruned_decode_attn_noalloc", "think_q4_ld", "think_q4_groups_bytes",
+    "think_pruned_decode_attn_noalloc", "think_noalloc_read_device_status", "think_q4_ld", "think_q4_groups_bytes",
     "think_quantize_keys_q4", "think_pruned_decode_attn_q4", "think_ragged_rows", "think_select_adaptive",
     "think_compact_keys_ragged", "think_prune_adaptive", "think_pruned_decode_attn_ragged",
     "think_token_mass_workspace_size",
@@ -115,6 +115,8 @@ def _load() -> ctypes.CDLL:
     lib.think_workspace_init.restype = I
     lib.think_read_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint32), P]
     lib.think_read_device_status.restype = I
+    lib.think_noalloc_read_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), P]
+    lib.think_noalloc_read_device_status.restype = I
     return lib
 
 
@@ -487,6 +489,15 @@ def think_read_device_status(workspace: torch.Tensor, stream=None) -> int:
     st = ctypes.c_uint32(0)
     _check(lib.think_read_device_status(_ptr(workspace), ctypes.byref(st), _stream(stream)),
            "think_read_device_status")
+    return st.value
+
+
+def think_noalloc_read_device_status(stream=None) -> int:
+    """Status word of the last no-allocation decode on the current device
+    (synchronises the stream)."""
+    st = ctypes.c_uint32(0)
+    _check(lib.think_noalloc_read_device_status(ctypes.byref(st), _stream(stream)),
+           "think_noalloc_read_device_status")
     return st.value
 
 

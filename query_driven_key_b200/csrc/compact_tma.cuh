@@ -139,10 +139,12 @@ __global__ void __launch_bounds__(kCtThreads, 3)
             break;
         uint32_t v[4][4];
         compact_tile_load(ring + (uint32_t)s * kCtTileBytes, c_row, cw, v);
+        compact_tile_transpose(v, lane);  // uses the loaded words: the stage has been read
+        fence_proxy_async_shared();
         __syncwarp();
         if (lane == 0) mbar_arrive(empty0 + 8 * s);
         const int64_t x0 = (tile0 + i) * kCtTileRows;
-        compact_tile_store(v, lane, crow, a.kp, a.ldk, x0 + 8 * (tb0 + (lane & 3)), a.N);
+        compact_tile_store_kept(v, crow, a.kp, a.ldk, x0 + 8 * (tb0 + (lane & 3)), a.N);
         if (pad_row < Tw) store_run8(a.kp + (r0 + pad_row) * a.ldk, x0 + 8 * (tid & 7), a.N, zero);
     }
 }

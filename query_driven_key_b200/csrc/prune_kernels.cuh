@@ -36,14 +36,24 @@ __device__ __forceinline__ void select_top_t_warp(const unsigned long long *sv, 
     }
 }
 
+// Barrier policies of the score merge: the whole block, or the 256 consumer
+// threads of a warp-specialised block whose producer warp keeps running.
+struct BlockSync {
+    __device__ __forceinline__ void operator()() const { __syncthreads(); }
+};
+struct ConsumerSync {
+    __device__ __forceinline__ void operator()() const { named_barrier(1, 256); }
+};
+
 // The same selection (same rule, same output) by the first 256 threads of a
-// block; every thread of the block calls it.  Thread t ranks channel t/2
-// against half t%2 of the channels and the pair adds its two counts, so each
-// thread makes 64 comparisons instead of 512.
+// block; every thread taking part in `sync` calls it.  Thread t ranks channel
+// t/2 against half t%2 of the channels and the pair adds its two counts, so
+// each thread makes 64 comparisons instead of 512.  wcnt: 8 ints of shared
+// memory.
+template <typename Sync>
 __device__ __forceinline__ void select_top_t_block(const unsigned long long *sv, int T,
-                                                   int32_t *__restrict__ idx_out)
+                                                   int32_t *__restrict__ idx_out, int *wcnt, Sync sync)
 {
-    __shared__ int wcnt[8];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const bool on = tid < 2 * kD;
     const int c = (tid >> 1) & (kD - 1), h = tid & 1;
@@ -61,7 +71,7 @@ __device__ __forceinline__ void select_top_t_block(const unsigned long long *sv,
     const bool keep = on && h == 0 && rank < T;
     const unsigned ball = __ballot_sync(0xffffffffu, keep);
     if (on && lane == 0) wcnt[warp] = __popc(ball);
-    __syncthreads();
+    sync();
     if (keep) {
         int base = 0;
         for (int w = 0; w < warp; ++w) base += wcnt[w];
@@ -112,9 +122,12 @@ struct ScoreArgs {
     int Hq, Hkv, S;
     int64_t N, rows_per_split;
     int splits;
-    double *part;              // [heads][splits][D]   partial channel energies
+    double *part;              // [heads][splits][D]   partial channel energies of the runs
+    double *gpart;             // [heads][groups][D]   sums of groups of kMergeGroup runs
     double *qn2;               // [heads][G][D]        window-query channel energies
-    unsigned *tickets;         // [heads], zero between calls
+    unsigned *gtickets;        // [heads][groups] runs of the group done; zero between calls
+    unsigned *tickets;         // [heads] groups of the head done; zero between calls
+    int groups;                // ceil(splits / kMergeGroup)
     double *scores;            // [heads][D]
     int T;                     // > 0: also select the top T into idx
     int32_t *idx;              // [heads][T]
@@ -193,21 +206,25 @@ __device__ __forceinline__ void score_window_energies(const ScoreArgs &a, int he
     }
 }
 
-// End of a score block (called by every thread of the block; threads 0..255
-// do the work): the block partial part[head][split][c] = sum of the ROWS rows
-// of red[][c] in row order; the last block of the head to arrive (ticket
-// counter) adds the partials of all splits in a fixed order (the even and the
-// odd splits in two halves of 128 threads, each in split order, then half 0
-// plus half 1), forms
+// Runs of a head merged by one block before the head's total is formed.
+constexpr int kMergeGroup = 16;
+
+// End of a score run (called by every thread taking part in `sync`; threads
+// 0..255 do the work).  The run's partial part[head][split][c] is the sum of
+// the ROWS rows of red[][c] in row order.  The partials are then added in a
+// fixed two-level order: the last block of each group of kMergeGroup runs
+// (group ticket) adds the group's partials in run order into gpart; the last
+// group of the head (head ticket) adds the group sums in group order, forms
 //     s[c] = sum_g sqrt(qn2[g][c]) * sqrt(kn2[c])
-// with each operation rounded as written, resets the ticket and, for T > 0,
-// selects the top T.
-template <int ROWS>
-__device__ __forceinline__ void score_block_end(const ScoreArgs &a, int head, int split, const double *red)
+// with each operation rounded as written, resets the tickets and, for T > 0,
+// selects the top T.  Every sum starts at 0 and runs in ascending order, so
+// the result depends only on the split plan.  Shared memory: flag (1 word), sv
+// (kD words), wcnt (8 ints).  Returns true (uniformly) in the block that
+// formed the head's scores.
+template <int ROWS, typename Sync>
+__device__ __forceinline__ bool score_run_end(const ScoreArgs &a, int head, int split, const double *red,
+                                              unsigned *flag, unsigned long long *sv, int *wcnt, Sync sync)
 {
-    __shared__ unsigned last;
-    __shared__ unsigned long long sv[kD];
-    __shared__ double khalf[kD];
     const int tid = threadIdx.x;
     const int G = a.Hq / a.Hkv;
     if (tid < kD) {
@@ -216,35 +233,47 @@ __device__ __forceinline__ void score_block_end(const ScoreArgs &a, int head, in
         for (int rr = 0; rr < ROWS; ++rr) s += red[rr * kD + tid];
         a.part[((int64_t)head * a.splits + split) * kD + tid] = s;
     }
+    __threadfence();
+    sync();
+    const int grp = split / kMergeGroup;
+    const int r0 = grp * kMergeGroup, r1 = min(a.splits, r0 + kMergeGroup);
+    unsigned *gt = a.gtickets + (int64_t)head * a.groups + grp;
+    if (tid == 0) *flag = (atomicAdd(gt, 1u) == (unsigned)(r1 - r0 - 1)) ? 1u : 0u;
+    sync();
+    if (!*flag) return false;
 
-    // ------------------------------------------ last block of the head
+    // ------------------------------------------ last run of the group
     __threadfence();
-    __syncthreads();
-    if (tid == 0) last = (atomicAdd(a.tickets + head, 1u) == (unsigned)(a.splits - 1)) ? 1u : 0u;
-    __syncthreads();
-    if (!last) return;
+    if (tid < kD) {
+        const double *p = a.part + ((int64_t)head * a.splits + r0) * kD + tid;
+        double v[kMergeGroup];
+#pragma unroll
+        for (int u = 0; u < kMergeGroup; ++u) v[u] = (r0 + u < r1) ? __ldcg(p + (int64_t)u * kD) : 0.0;
+        double s = 0.0;
+#pragma unroll
+        for (int u = 0; u < kMergeGroup; ++u) s = __dadd_rn(s, v[u]);  // + 0.0 past the group is exact
+        a.gpart[((int64_t)head * a.groups + grp) * kD + tid] = s;
+    }
+    if (tid == 0) *gt = 0u;  // ready for the next call
     __threadfence();
-    // channel energy: 16 loads in flight per thread
-    const int c = tid & (kD - 1), hp = tid >> 7;
-    double k0 = 0.0;
-    if (tid < 2 * kD) {
-        const double *p = a.part + (int64_t)head * a.splits * kD + c;
-        for (int s = hp; s < a.splits; s += 32) {
+    sync();
+    if (tid == 0) *flag = (atomicAdd(a.tickets + head, 1u) == (unsigned)(a.groups - 1)) ? 1u : 0u;
+    sync();
+    if (!*flag) return false;
+
+    // ------------------------------------------ last group of the head
+    __threadfence();
+    if (tid < kD) {
+        const double *p = a.gpart + (int64_t)head * a.groups * kD + tid;
+        double k2 = 0.0;
+        for (int g0 = 0; g0 < a.groups; g0 += 16) {
             double v[16];
 #pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const int s2 = s + 2 * u;
-                v[u] = (s2 < a.splits) ? __ldcg(p + (int64_t)s2 * kD) : 0.0;
-            }
+            for (int u = 0; u < 16; ++u) v[u] = (g0 + u < a.groups) ? __ldcg(p + (int64_t)(g0 + u) * kD) : 0.0;
 #pragma unroll
-            for (int u = 0; u < 16; ++u) k0 = __dadd_rn(k0, v[u]);
+            for (int u = 0; u < 16; ++u) k2 = __dadd_rn(k2, v[u]);
         }
-    }
-    if (hp == 1) khalf[c] = k0;
-    __syncthreads();
-    if (tid < kD) {
-        k0 = __dadd_rn(k0, khalf[tid]);
-        const double knorm = sqrt(k0);
+        const double knorm = sqrt(k2);
         double sc = 0.0;
         for (int g = 0; g < G; ++g)
             sc = __dadd_rn(sc, __dmul_rn(sqrt(__ldcg(a.qn2 + ((int64_t)head * G + g) * kD + tid)), knorm));
@@ -252,9 +281,21 @@ __device__ __forceinline__ void score_block_end(const ScoreArgs &a, int head, in
         sv[tid] = __double_as_longlong(sc);
     }
     if (tid == 0) a.tickets[head] = 0u;  // ready for the next call
-    if (a.T <= 0) return;
-    __syncthreads();
-    select_top_t_block(sv, a.T, a.idx + (int64_t)head * a.T);
+    if (a.T > 0) {
+        sync();
+        select_top_t_block(sv, a.T, a.idx + (int64_t)head * a.T, wcnt, sync);
+    }
+    return true;
+}
+
+// score_run_end for the score kernels (the whole block takes part).
+template <int ROWS>
+__device__ __forceinline__ void score_block_end(const ScoreArgs &a, int head, int split, const double *red)
+{
+    __shared__ unsigned flag;
+    __shared__ unsigned long long sv[kD];
+    __shared__ int wcnt[8];
+    (void)score_run_end<ROWS>(a, head, split, red, &flag, sv, wcnt, BlockSync{});
 }
 
 template <typename TIn>
@@ -603,15 +644,22 @@ __device__ __forceinline__ void compact_tile_load(uint32_t st, uint32_t c_row, i
     }
 }
 
-// Transpose and store: x = first token of this lane's run (a multiple of 8).
-__device__ __forceinline__ void compact_tile_store(uint32_t (&v)[4][4], int lane, const int64_t (&crow)[4],
-                                                   __nv_bfloat16 *kp, int64_t ldk, int64_t x, int64_t N)
+// The 4x4 word transposes of a loaded tile part: afterwards register m of
+// v[k] holds tokens 2m, 2m + 1 of this lane's 8-token run of its channel.
+__device__ __forceinline__ void compact_tile_transpose(uint32_t (&v)[4][4], int lane)
 {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        quad_transpose(v[k], lane & 3);
+    for (int k = 0; k < 4; ++k) quad_transpose(v[k], lane & 3);
+}
+
+// Store the kept channels' runs: x = first token of this lane's run (a
+// multiple of 8).
+__device__ __forceinline__ void compact_tile_store_kept(const uint32_t (&v)[4][4], const int64_t (&crow)[4],
+                                                        __nv_bfloat16 *kp, int64_t ldk, int64_t x, int64_t N)
+{
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
         if (crow[k] >= 0) store_run8(kp + crow[k] * ldk, x, N, v[k]);
-    }
 }
 
 template <typename TIn> struct CompactTokens { static constexpr int value = 64; };

@@ -134,6 +134,15 @@ __device__ __forceinline__ uint64_t l2_policy_evict_normal()
     return p;
 }
 
+// Orders this thread's earlier generic-proxy accesses of shared memory (plain
+// loads, ldmatrix) before later async-proxy accesses (TMA writes into the same
+// stage).  A ring consumer issues it, after the values it loaded from a stage
+// are in registers and used, before it releases the stage to the producer.
+__device__ __forceinline__ void fence_proxy_async_shared()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Prefetch one 4-D tile of a tensor map into L2 (no shared memory involved).
 __device__ __forceinline__ void tma_prefetch_l2_4d(const CUtensorMap *map, int c0, int c1, int c2, int c3)
 {
@@ -185,6 +194,19 @@ __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p)
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
+
+// Fetch-and-add with acquire and release semantics at GPU scope: the writes
+// this thread made before it (and those of threads that synchronised with it
+// through a block barrier) are visible to the thread that sees the new value,
+// and the writes released before the values it sees are visible to it.
+__device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned *p, unsigned v)
+{
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
 __device__ __forceinline__ void st_release_gpu(unsigned *p, unsigned v)
 {

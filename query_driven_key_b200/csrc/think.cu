@@ -14,6 +14,7 @@
 #include <utility>
 
 #include "decode_kernels.cuh"
+#include "decode_f64.cuh"
 #include "decode_mma.cuh"
 #include "decode_q4.cuh"
 #include "evict.cuh"
@@ -28,9 +29,10 @@ namespace think {
 namespace {
 
 constexpr int kTargetSMs = 148;             // B200
-constexpr int kScoreBlocksPerSM = 4;        // runs per SM of the fixed score split rule
 constexpr int kScoreResidentPerSM = 3;      // score blocks resident per SM (both score kernels)
-constexpr int kScoreMaxWaves = 4;
+constexpr int kPlanBlocks = 2 * kTargetSMs; // runs per round of the score plan
+constexpr int64_t kRoundTilesMax = 2560;    // tiles per round (40 MB of bf16 keys; L2 holds two)
+constexpr int kRunTilesMax = 64;            // tiles per run at most
 constexpr int kCompactWaves = 4;            // waves of compact_tma_kernel blocks the plan aims for
 constexpr int kDecodeBlocksPerSM = 2;       // decode blocks the plan aims to keep per SM
 constexpr int kDecodePrefetchTiles = 0;     // tiles a decode block prefetches into L2 ahead of TMA
@@ -88,69 +90,48 @@ think_status_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t 
 // ---------------------------------------------------------------- plans --
 
 // Split of each head's tokens for scoring, shared by the score kernels and
-// the fused prune kernel (so that all add the squares in the same order): runs
-// of s_tiles 64-token tiles, one score block per run.
+// the one-kernel prune (so that all add the squares in the same order): runs
+// of s_tiles 64-token tiles, one score block per run.  The heads are also
+// grouped in rounds of hpr heads for the one-kernel prune: a round holds about
+// kPlanBlocks runs and at most kRoundTilesMax tiles, so that the prune can
+// compact a round from L2 while it scores the next one.  The plan depends only
+// on the shape.
 struct ScorePlan {
     int splits;              // runs per head
     int s_tiles;             // 64-token tiles per run
     int64_t rows_per_split;  // = 64 * s_tiles
     int64_t tiles_per_head;
+    int hpr, rounds;         // heads per round, rounds
+    int groups;              // groups of kMergeGroup runs per head (the merge order)
 };
 
-ScorePlan score_plan_from_tiles(int64_t tiles_per_head, int64_t st)
-{
-    ScorePlan p;
-    p.tiles_per_head = tiles_per_head;
-    st = std::min<int64_t>(std::max<int64_t>(st, 1), tiles_per_head);
-    p.s_tiles = (int)st;
-    p.rows_per_split = st * kPfTile;
-    p.splits = (int)ceil_div(tiles_per_head, st);
-    return p;
-}
-
-// waves = 0: about kScoreBlocksPerSM runs per SM, 4 to 32 tiles per run.
-// waves = W > 0: the shortest runs whose count fits W waves of the resident
-// block slots (148 SMs x kScoreResidentPerSM).
-ScorePlan plan_score_waves(int64_t heads, int64_t N, int waves)
-{
-    const int64_t tph = std::max<int64_t>(1, ceil_div(N, kPfTile));
-    if (waves <= 0) {
-        const int64_t st = heads * tph / ((int64_t)kTargetSMs * kScoreBlocksPerSM);
-        return score_plan_from_tiles(tph, std::min<int64_t>(std::max<int64_t>(st, 4), 32));
-    }
-    const int64_t slots = (int64_t)kTargetSMs * kScoreResidentPerSM * waves;
-    const int64_t runs_per_head = std::max<int64_t>(1, slots / std::max<int64_t>(heads, 1));
-    return score_plan_from_tiles(tph, ceil_div(tph, runs_per_head));
-}
-
-// THINK_SCORE_WAVES: 0 the fixed rule above, 1..4 that many waves; default
-// (-1): the fewest waves (up to 4) whose runs fill at least 90% of their
-// slots, else the best filled.  Whole waves leave no partly filled last wave,
-// whose blocks would stream with the rest of the GPU idle.
+// Choose the run length L (tiles) that minimises rounds x runs-per-block x
+// (L + 2): the 2 tiles stand for a run's fixed cost (partial sums, tickets).
 ScorePlan plan_score(int64_t heads, int64_t N)
 {
-    const int mode = env_int("THINK_SCORE_WAVES", -1, -1, kScoreMaxWaves);
-    if (mode >= 0) return plan_score_waves(heads, N, mode);
-    ScorePlan best = plan_score_waves(heads, N, 1);
-    double best_fill = 0.0;
-    for (int w = 1; w <= kScoreMaxWaves; ++w) {
-        const ScorePlan p = plan_score_waves(heads, N, w);
-        const double fill = (double)(heads * p.splits) / ((double)kTargetSMs * kScoreResidentPerSM * w);
-        if (fill >= 0.9) return p;
-        if (fill > best_fill) {
-            best_fill = fill;
-            best = p;
+    const int64_t tph = std::max<int64_t>(1, ceil_div(N, kPfTile));
+    heads = std::max<int64_t>(heads, 1);
+    ScorePlan best{};
+    int64_t best_cost = -1;
+    for (int64_t L = 1; L <= std::min<int64_t>(kRunTilesMax, tph); ++L) {
+        const int64_t R = ceil_div(tph, L);
+        int64_t hpr = std::min<int64_t>(std::max<int64_t>(kPlanBlocks / R, 1), heads);
+        if (hpr > 1 && hpr * tph > kRoundTilesMax) hpr = std::max<int64_t>(1, kRoundTilesMax / tph);
+        const int64_t passes = ceil_div(hpr * R, kPlanBlocks);
+        const int64_t rounds = ceil_div(heads, hpr);
+        const int64_t cost = rounds * passes * (L + 2);
+        if (best_cost < 0 || cost <= best_cost) {  // ties: the longer runs
+            best_cost = cost;
+            best.s_tiles = (int)L;
+            best.splits = (int)R;
+            best.hpr = (int)hpr;
+            best.rounds = (int)rounds;
         }
     }
+    best.tiles_per_head = tph;
+    best.rows_per_split = (int64_t)best.s_tiles * kPfTile;
+    best.groups = (int)ceil_div(best.splits, kMergeGroup);
     return best;
-}
-
-// The most runs per head any plan above can choose (workspace size).
-int score_max_splits(int64_t heads, int64_t N)
-{
-    int m = 1;
-    for (int w = 0; w <= kScoreMaxWaves; ++w) m = std::max(m, plan_score_waves(heads, N, w).splits);
-    return m;
 }
 
 struct DecodeSplit {
@@ -397,36 +378,46 @@ think_status_t launch_decode(int G, const CUtensorMap &mk, const CUtensorMap &mv
 
 // ---------------------------------------------------------------- score --
 
-// Score workspace: a 256-byte header (status word at 0; the fused kernel's
-// score-queue counter at 8, front compact head at 16, block-exit counter at
-// 24), per-head arrival counters, per-head ready flags, per-head compact
-// counters, window-query energies, per-run channel energies.
+// Score workspace: a 256-byte header (status word at 0; the one-kernel
+// prune's block-exit counter at 8), per-head ready flags (one-kernel prune),
+// per-head tickets, per-(head, group) tickets, window-query energies, per-run
+// channel energies, per-group sums.
 struct ScoreWs {
-    size_t status, s_next, c_front, exits, tickets, ready, c_cnt, qn2, part, total;  // byte offsets, size
+    size_t status, exits, ready, tickets, gtickets, qn2, part, gpart, total;  // byte offsets, size
 };
 
 ScoreWs score_ws_layout(int64_t heads, int G, const ScorePlan &p)
 {
     ScoreWs w;
     w.status = 0;
-    w.s_next = 8;
-    w.c_front = 16;
-    w.exits = 24;
-    w.tickets = 256;
-    w.ready = w.tickets + align_up((size_t)heads * sizeof(unsigned), 256);
-    w.c_cnt = w.ready + align_up((size_t)heads * sizeof(unsigned), 256);
-    w.qn2 = w.c_cnt + align_up((size_t)heads * sizeof(unsigned), 256);
+    w.exits = 8;
+    w.ready = 256;
+    w.tickets = w.ready + align_up((size_t)heads * sizeof(unsigned), 256);
+    w.gtickets = w.tickets + align_up((size_t)heads * sizeof(unsigned), 256);
+    w.qn2 = w.gtickets + align_up((size_t)heads * p.groups * sizeof(unsigned), 256);
     w.part = w.qn2 + align_up((size_t)heads * G * kD * sizeof(double), 256);
-    w.total = w.part + (size_t)heads * p.splits * kD * sizeof(double);
+    w.gpart = w.part + align_up((size_t)heads * p.splits * kD * sizeof(double), 256);
+    w.total = w.gpart + (size_t)heads * p.groups * kD * sizeof(double);
     return w;
 }
 
-// The layout for the largest plan, so that one workspace serves every plan.
 ScoreWs score_ws_layout_max(int64_t heads, int G, int64_t N)
 {
-    ScorePlan p = plan_score(heads, N);
-    p.splits = score_max_splits(heads, N);
-    return score_ws_layout(heads, G, p);
+    return score_ws_layout(heads, G, plan_score(heads, N));
+}
+
+// The score fields of ScoreArgs that live in the workspace.
+void set_score_ws(ScoreArgs &a, unsigned char *ws, const ScoreWs &w, const ScorePlan &p)
+{
+    a.rows_per_split = p.rows_per_split;
+    a.splits = p.splits;
+    a.groups = p.groups;
+    a.tickets = reinterpret_cast<unsigned *>(ws + w.tickets);
+    a.gtickets = reinterpret_cast<unsigned *>(ws + w.gtickets);
+    a.qn2 = reinterpret_cast<double *>(ws + w.qn2);
+    a.part = reinterpret_cast<double *>(ws + w.part);
+    a.gpart = reinterpret_cast<double *>(ws + w.gpart);
+    a.status = reinterpret_cast<unsigned *>(ws + w.status);
 }
 
 think_status_t validate_score(const void *q_win, const void *k, const int64_t k_strides[3], int B,
@@ -469,15 +460,10 @@ think_status_t launch_score(const void *q_win, const void *k, const int64_t k_st
     a.Hkv = Hkv;
     a.S = S_obs;
     a.N = N;
-    a.rows_per_split = p.rows_per_split;
-    a.splits = p.splits;
-    a.tickets = reinterpret_cast<unsigned *>(ws + w.tickets);
-    a.qn2 = reinterpret_cast<double *>(ws + w.qn2);
-    a.part = reinterpret_cast<double *>(ws + w.part);
+    set_score_ws(a, ws, w, p);
     a.scores = scores;
     a.T = T;
     a.idx = idx;
-    a.status = reinterpret_cast<unsigned *>(ws + w.status);
     a.stages = env_int("THINK_SCORE_STAGES", 4, 2, kStMaxStages);
     dim3 grid(p.splits, (unsigned)heads);
     // bf16: key tiles staged by TMA when a tensor map can describe K
@@ -589,70 +575,92 @@ think_status_t launch_compact_tma(const void *k, const int64_t k_strides[3], int
 
 // ---------------------------------------------------------- fused prune --
 
-struct PrunePlan {
-    ScorePlan sp;
-    int c_tiles, c_items, grid;
-};
-
-// Compact items have the score items' size; one block per SM.
-PrunePlan plan_prune(int64_t heads, int64_t N)
+int device_sm_count()
 {
-    PrunePlan p;
-    p.sp = plan_score(heads, N);
-    p.c_tiles = p.sp.s_tiles;
-    p.c_items = p.sp.splits;
-    p.grid = (int)std::min<int64_t>(kTargetSMs, heads * (p.sp.splits + p.c_items));
-    return p;
+    thread_local int cached_dev = -1, cached_sms = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (dev != cached_dev) {
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        cached_dev = dev;
+        cached_sms = sms;
+    }
+    return cached_sms;
 }
 
-// The fused prune (bf16, N > 0).  Returns THINK_ERR_UNSUPPORTED, having
+// Whether the one-kernel prune serves this shape: bf16, N > 0, groups of at
+// most 8 query heads, a round of the plan (two of which must fit in L2) no
+// larger than kRoundTilesMax tiles.
+bool prune_fused_applies(think_dtype_t dtype, int64_t heads, int G, int64_t N)
+{
+    if (dtype != THINK_BF16 || N <= 0 || N > (int64_t)INT32_MAX - kPfTile || G > 8) return false;
+    if (env_int("THINK_PRUNE_FUSED", 0, 0, 1) == 0) return false;
+    const ScorePlan p = plan_score(heads, N);
+    return (int64_t)p.hpr * p.tiles_per_head <= kRoundTilesMax;
+}
+
+// The one-kernel prune (bf16, N > 0).  Returns THINK_ERR_UNSUPPORTED, having
 // launched nothing, when a tensor map cannot be built for these strides.
+// THINK_PRUNE_STAGES and THINK_PRUNE_CSTAGES set the depths of the score and
+// compaction rings (default 7 and 4 tiles), THINK_PRUNE_LAG how many rounds
+// the scoring may run ahead of the compaction; THINK_PRUNE_HINTS the L2 policies
+// (bits: 1 score loads evict-last, 2 compact loads evict-first, 4 K' stores
+// evict-first).  None of them changes the results.
 think_status_t launch_prune_fused(const void *q_win, const void *k, const int64_t k_strides[3], int B,
                                   int Hq, int Hkv, int64_t N, int S_obs, int T, double *scores,
                                   int32_t *idx, void *k_pruned, int64_t ldk, void *workspace,
                                   cudaStream_t st)
 {
     const int64_t heads = (int64_t)B * Hkv;
-    const PrunePlan p = plan_prune(heads, N);
-    const ScoreWs w = score_ws_layout(heads, Hq / Hkv, p.sp);
+    const ScorePlan p = plan_score(heads, N);
+    const ScoreWs w = score_ws_layout(heads, Hq / Hkv, p);
     CUtensorMap mk;
     if (!make_map_4d(&mk, THINK_BF16, k, kD, (uint64_t)N, (uint64_t)Hkv, (uint64_t)B, k_strides[2],
                      k_strides[1], k_strides[0], 64, kPfTile, true))
         return THINK_ERR_UNSUPPORTED;
     unsigned char *ws = static_cast<unsigned char *>(workspace);
     PruneFusedArgs a;
-    a.qwin = static_cast<const __nv_bfloat16 *>(q_win);
-    a.Hq = Hq;
-    a.Hkv = Hkv;
-    a.S = S_obs;
+    memset(&a, 0, sizeof(a));
+    a.sc.k = k;
+    a.sc.qwin = q_win;
+    a.sc.Hq = Hq;
+    a.sc.Hkv = Hkv;
+    a.sc.S = S_obs;
+    a.sc.N = N;
+    set_score_ws(a.sc, ws, w, p);
+    a.sc.scores = scores;
+    a.sc.T = T;
+    a.sc.idx = idx;
     a.G = Hq / Hkv;
     a.T = T;
     a.heads = (int)heads;
-    a.tiles_per_head = (int)p.sp.tiles_per_head;
-    a.s_tiles = p.sp.s_tiles;
-    a.s_items = p.sp.splits;
-    a.c_tiles = p.c_tiles;
-    a.c_items = p.c_items;
-    a.l2_hints = env_int("THINK_PRUNE_L2_HINTS", 1, 0, 1);
-    a.s_total = (long long)heads * p.sp.splits;
-    a.part = reinterpret_cast<double *>(ws + w.part);
-    a.qn2 = reinterpret_cast<double *>(ws + w.qn2);
-    a.tickets = reinterpret_cast<unsigned *>(ws + w.tickets);
+    a.tiles_per_head = (int)p.tiles_per_head;
+    a.s_tiles = p.s_tiles;
+    a.hpr = p.hpr;
+    a.rounds = p.rounds;
+    a.s_stages = env_int("THINK_PRUNE_STAGES", 7, 2, kPfMaxStages - 2);
+    a.c_stages = env_int("THINK_PRUNE_CSTAGES", 4, 2, kPfMaxStages - a.s_stages);
+    a.hints = env_int("THINK_PRUNE_HINTS", kPfHintScoreKeep | kPfHintCompactDrop, 0, 7);
+    a.lag = env_int("THINK_PRUNE_LAG", 2, 1, 1 << 20);
+    a.prefetch = env_int("THINK_PRUNE_PREFETCH", 0, 0, 64);
     a.ready = reinterpret_cast<unsigned *>(ws + w.ready);
-    a.status = reinterpret_cast<unsigned *>(ws + w.status);
-    a.s_next = reinterpret_cast<unsigned long long *>(ws + w.s_next);
-    a.c_front = reinterpret_cast<unsigned *>(ws + w.c_front);
-    a.c_cnt = reinterpret_cast<unsigned *>(ws + w.c_cnt);
     a.exits = reinterpret_cast<unsigned *>(ws + w.exits);
-    a.scores = scores;
-    a.idx = idx;
     a.kp = static_cast<__nv_bfloat16 *>(k_pruned);
     a.ldk = ldk;
     a.N = N;
-    if (!ensure_smem(reinterpret_cast<const void *>(prune_fused_kernel), kPfSmemBytes))
+    const size_t bytes = prune_fused_smem_bytes(a.s_stages, a.c_stages);
+    const void *kern = reinterpret_cast<const void *>(prune_fused_kernel);
+    if (!ensure_smem(kern, bytes)) return THINK_ERR_CUDA;
+    // every block must be resident at once (blocks wait for other blocks' flags)
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kPfThreads, bytes) != cudaSuccess || occ < 1)
         return THINK_ERR_CUDA;
-    prune_fused_kernel<<<p.grid, kPfThreads, kPfSmemBytes, st>>>(mk, a);
-    return launch_status();
+    const int64_t sms = device_sm_count();
+    if (sms < 1) return THINK_ERR_CUDA;
+    const int64_t runs_per_round = (int64_t)p.hpr * p.splits;
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(sms * occ, runs_per_round));
+    return launch_pdl(prune_fused_kernel, dim3(grid), dim3(kPfThreads), bytes, st, mk, a);
 }
 
 
@@ -1075,9 +1083,10 @@ think_status_t think_prune(const void *q_win, const void *k, const int64_t k_str
     v = validate_compact(k, k_strides, B, Hkv, N, d, dtype, idx, T, k_pruned, ldk);
     if (v != THINK_OK || B == 0 || Hkv == 0) return v;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    // Two launches (score + select, then compact).  THINK_PRUNE_FUSED=1 selects
-    // the one-kernel prune for bf16 (same results; not faster on B200 yet).
-    if (dtype == THINK_BF16 && N > 0 && env_flag("THINK_PRUNE_FUSED")) {
+    // Two launches (score + select, then compact); THINK_PRUNE_FUSED=1 selects
+    // for bf16 the one kernel that reads K about once (prune_fused_applies).
+    // Both give the same bits.
+    if (prune_fused_applies(dtype, (int64_t)B * Hkv, Hq / Hkv, N)) {
         v = launch_prune_fused(q_win, k, k_strides, B, Hq, Hkv, N, S_obs, T, scores, idx, k_pruned,
                                ldk, workspace, st);
         if (v != THINK_ERR_UNSUPPORTED) return v;
@@ -1099,8 +1108,48 @@ size_t think_decode_workspace_size(int B, int Hq, int Hkv, int64_t N, int d, thi
     const int G = Hq / Hkv;
     const DecodeSplit sp = plan_decode_split(heads, N);
     const size_t slots = (size_t)heads * sp.splits * G;
-    return kDecodeHeader + align_up((size_t)heads * sizeof(unsigned), 256) +
-           slots * kD * sizeof(float) + slots * 2 * sizeof(float);
+    const size_t pe = dtype == THINK_F32 ? sizeof(double) : sizeof(float);  // fp32 caches: fp64 partials
+    return kDecodeHeader + align_up((size_t)heads * sizeof(unsigned), 256) + slots * kD * pe + slots * 2 * pe;
+}
+
+// fp32 caches: the fp64 decode (decode_f64.cuh), grid (splits, heads).
+think_status_t launch_decode_f64(const void *q, const void *k_pruned, int64_t ldk, const void *v,
+                                 const int64_t v_strides[3], const int32_t *idx, int B, int Hq, int Hkv,
+                                 int64_t N, int T, float scale, float *out, void *workspace, cudaStream_t st)
+{
+    const int64_t heads = (int64_t)B * Hkv;
+    const int G = Hq / Hkv;
+    const DecodeSplit sp = plan_decode_split(heads, N);
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    const size_t slots = (size_t)heads * sp.splits * G;
+    DecodeF64Args a;
+    a.q = static_cast<const float *>(q);
+    a.kp = static_cast<const float *>(k_pruned);
+    a.v = static_cast<const float *>(v);
+    a.sb = v_strides[0];
+    a.sh = v_strides[1];
+    a.sn = v_strides[2];
+    a.idx = idx;
+    a.out = out;
+    a.tickets = reinterpret_cast<unsigned *>(ws + kDecodeHeader);
+    a.part_o = reinterpret_cast<double *>(ws + kDecodeHeader + align_up((size_t)heads * sizeof(unsigned), 256));
+    a.part_ml = a.part_o + slots * kD;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.T = T;
+    a.splits = sp.splits;
+    a.tiles_per_split = sp.tiles_per_split;
+    a.N = N;
+    a.ldk = ldk;
+    a.scale = (double)scale;
+    const dim3 grid((unsigned)sp.splits, (unsigned)heads);
+    switch (G) {
+    case 1: pruned_decode_f64_kernel<1><<<grid, 256, 0, st>>>(a); break;
+    case 2: pruned_decode_f64_kernel<2><<<grid, 256, 0, st>>>(a); break;
+    case 4: pruned_decode_f64_kernel<4><<<grid, 256, 0, st>>>(a); break;
+    default: pruned_decode_f64_kernel<8><<<grid, 256, 0, st>>>(a); break;
+    }
+    return launch_status();
 }
 
 think_status_t think_pruned_decode_attn(const void *q, const void *k_pruned, int64_t ldk,
@@ -1129,11 +1178,14 @@ think_status_t think_pruned_decode_attn(const void *q, const void *k_pruned, int
         return THINK_ERR_ALIGNMENT;
     const size_t need = think_decode_workspace_size(B, Hq, Hkv, N, d, dtype);
     if (workspace_bytes < need) return THINK_ERR_WORKSPACE;
+    if (dtype == THINK_F32)
+        return launch_decode_f64(q, k_pruned, ldk, v, v_strides, idx, B, Hq, Hkv, N, T, scale, out, workspace,
+                                 static_cast<cudaStream_t>(stream));
 
     // bf16: warp-level tensor-core kernel (mma.sync) by default;
     // THINK_DECODE_TENSOR_CORES=1 selects the tcgen05 kernel and
     // THINK_DECODE_CUDA_CORES=1 the CUDA-core kernel (same results within
-    // tolerance; for comparisons).  fp32 inputs always use the CUDA-core kernel.
+    // tolerance; for comparisons).  fp32 inputs use the fp64 decode above.
     enum { kSimt, kMma, kTc } kind = kSimt;
     if (dtype == THINK_BF16) {
         kind = kMma;
@@ -1200,8 +1252,7 @@ think_status_t think_pruned_decode_attn(const void *q, const void *k_pruned, int
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (use_tc) return launch_decode_tc(G, mk, mv, a, tp.bytes, (int)heads, st);
     if (kind == kMma) return launch_decode_mma(G, mp.warps, mk, mv, a, mp.bytes, (int)heads, st);
-    if (dtype == THINK_BF16) return launch_decode<__nv_bfloat16>(G, mk, mv, a, sm, (int)heads, st);
-    return launch_decode<float>(G, mk, mv, a, sm, (int)heads, st);
+    return launch_decode<__nv_bfloat16>(G, mk, mv, a, sm, (int)heads, st);
 }
 
 int64_t think_q4_ld(int64_t N)
@@ -1603,6 +1654,14 @@ think_status_t think_pruned_decode_attn_noalloc(const void *q, const void *k_pru
     if (cudaMemsetAsync(ws, 0, zero, st) != cudaSuccess) return THINK_ERR_CUDA;
     return think_pruned_decode_attn(q, k_pruned, ldk, v, v_strides, idx, B, Hq, Hkv, N, d, T, dtype,
                                     scale, out, ws, kNoAllocScratchBytes, stream);
+}
+
+think_status_t think_noalloc_read_device_status(uint32_t *status, void *stream)
+{
+    if (!status) return THINK_ERR_INVALID_ARG;
+    void *ws = nullptr;
+    if (noalloc_scratch(&ws) != cudaSuccess) return THINK_ERR_CUDA;
+    return think_read_device_status(ws, status, stream);  // the status word is the array's first word
 }
 
 }  // extern "C"

@@ -270,33 +270,45 @@ def test_select_tokens_workspace_layout():
     assert qdk.think_select_tokens_workspace_size(1, 1, 2**31) == 0
 
 
-def _score_plans(heads, N):
-    """The score pass's split plans (runs of 64-token tiles) restated: waves = 0
-    the fixed rule (about 4 runs per SM, 4..32 tiles), waves = 1..4 the
-    shortest runs whose count fits that many waves of 148 x 3 block slots."""
+def _score_plan(heads, N):
+    """The score pass's split plan restated: runs of L 64-token tiles per head
+    and rounds of hpr heads (about 296 runs and at most 2560 tiles per round),
+    L in 1..64 minimising rounds x ceil(runs per round / 296) x (L + 2), ties
+    to the longer run.  Returns (L, runs per head, heads per round, rounds)."""
     cdiv = lambda a, b: -(-a // b)
     tph = max(1, cdiv(N, 64))
-    plans = {}
-    st = min(max(heads * tph // (148 * 4), 4), 32)
-    plans[0] = cdiv(tph, min(max(st, 1), tph))
-    for w in range(1, 5):
-        rph = max(1, 148 * 3 * w // max(heads, 1))
-        st = min(max(cdiv(tph, rph), 1), tph)
-        plans[w] = cdiv(tph, st)
-    return plans
+    heads = max(heads, 1)
+    best = None
+    for L in range(1, min(64, tph) + 1):
+        R = cdiv(tph, L)
+        hpr = min(max(296 // R, 1), heads)
+        if hpr > 1 and hpr * tph > 2560:
+            hpr = max(1, 2560 // tph)
+        rounds = cdiv(heads, hpr)
+        cost = rounds * cdiv(hpr * R, 296) * (L + 2)
+        if best is None or cost <= best[0]:
+            best = (cost, L, R, hpr, rounds)
+    return best[1:]
 
 
-def test_score_workspace_covers_every_plan():
-    # header 256 B + tickets, ready flags, compact counters (256-byte aligned)
-    # + window-query energies [heads][G][128] fp64 + partials for the plan
-    # with the most runs per head; pins the plan rules on the CPU
+def test_score_workspace_follows_the_plan():
+    # header 256 B + ready flags, head tickets (256-byte aligned) + group
+    # tickets [heads][groups] + window-query energies [heads][G][128] fp64 +
+    # run partials [heads][runs][128] + group sums [heads][groups][128]
+    # (groups of 16 runs); pins the plan rule on the CPU
     pad = lambda x: -(-x // 256) * 256
     for B, Hq, Hkv, N in [(1, 32, 8, 131072), (4, 32, 8, 32768), (1, 32, 32, 4096), (32, 32, 8, 8192),
                           (1, 1, 1, 512), (1, 8, 1, 1), (2, 16, 8, 0), (3, 24, 8, 100_000)]:
         heads, G = B * Hkv, Hq // Hkv
-        splits = max(_score_plans(heads, N).values())
-        want = 256 + 3 * pad(heads * 4) + pad(heads * G * 128 * 8) + heads * splits * 128 * 8
+        _, R, _, _ = _score_plan(heads, N)
+        groups = -(-R // 16)
+        want = (256 + 2 * pad(heads * 4) + pad(heads * groups * 4) + pad(heads * G * 128 * 8) +
+                pad(heads * R * 128 * 8) + heads * groups * 128 * 8)
         assert qdk.think_score_workspace_size(B, Hq, Hkv, N, 128) == want, (B, Hq, Hkv, N)
-    # the long-context layer: one wave of 432 runs of 38 tiles (the fixed rule: 76 runs of 27)
-    p = _score_plans(8, 131072)
-    assert p[1] == 54 and p[0] == 76
+    # long-context layer: one head per round, 293 runs of 7 tiles; GQA batch 4
+    # at N = 32K: 4 heads per round, 74 runs of 7; the 32-batch sweep layer: 18
+    # heads per round, 16 runs of 8; the MHA layer: one round of 32 heads
+    assert _score_plan(8, 131072) == (7, 293, 1, 8)
+    assert _score_plan(32, 32768) == (7, 74, 4, 8)
+    assert _score_plan(256, 8192) == (8, 16, 18, 15)
+    assert _score_plan(32, 4096) == (8, 8, 32, 1)

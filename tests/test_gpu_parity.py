@@ -12,7 +12,8 @@ import pytest
 import torch
 
 import oracle
-from tests.helpers import TOL, check_out, check_scores, f64, idx_mismatch_heads, kp_logical
+from tests.helpers import (NEAR_TIE_REL, TOL, check_out, check_scores, f64, idx_mismatch_heads, kp_logical,
+                           width_is_near_tie)
 
 pytestmark = pytest.mark.gpu
 
@@ -254,6 +255,35 @@ def test_q4_long_context_full_size():
     _q4_check(cache, q_win, k, v, W.gen_decode_q(w, 0), T, "mistral_7b_long q4")
 
 
+def _adaptive_against_oracle_scores(ora_scores, Th, gidx, rowoff, out, q, kf, vf, tau, T_min, T_max):
+    B, Hkv = Th.shape
+    oTh, ooff, oidx = oracle.oracle_select_adaptive(ora_scores, tau, T_min, T_max)
+    agree = np.zeros((B, Hkv), dtype=bool)
+    for bh in range(B * Hkv):
+        b, h = divmod(bh, Hkv)
+        s = ora_scores[b, h]
+        kg, ko = int(Th[b, h]), int(oTh[b, h])
+        if kg != ko:
+            assert width_is_near_tie(s, tau, T_min, T_max, kg, ko), (
+                f"head {bh}: width {kg} on the GPU, {ko} from the oracle's scores, not a near-tie")
+            continue
+        gi = gidx[rowoff[bh]:rowoff[bh] + kg]
+        oi = oidx[ooff[bh]:ooff[bh] + ko]
+        if not np.array_equal(gi, oi):
+            cut = np.sort(s)[::-1][kg - 1]
+            for c in np.setxor1d(gi, oi):
+                assert abs(s[c] - cut) <= NEAR_TIE_REL * abs(cut), f"head {bh}: channel {c} not a near-tie"
+            continue
+        agree[b, h] = True
+    assert agree.any() or B * Hkv == 0
+    ora_out = oracle.oracle_decode_ragged(f64(q), kf, vf, oTh, ooff, oidx)
+    G = out.shape[1] // Hkv
+    rows = np.repeat(agree, G, axis=1)  # [B, Hq]: query heads of agreeing KV heads
+    g = f64(out)
+    if rows.any():
+        check_out(torch.from_numpy(g[rows]), ora_out[rows], torch.bfloat16, where="adaptive, oracle scores")
+
+
 @pytest.mark.parametrize("case", [(1, 32, 8, 20000, 0.9, 16, 96), (2, 8, 2, 1000, 0.5, 1, 128),
                                   (1, 16, 8, 300, 1.0, 8, 64), (2, 32, 32, 257, 0.0, 4, 40),
                                   (1, 8, 8, 2000, 0.8, 33, 33), (3, 8, 1, 129, 0.95, 1, 17)])
@@ -292,6 +322,8 @@ def test_adaptive_width(case):
               where=str(case))
     assert qdk.think_read_device_status(cache.decode_ws) == 0
     assert qdk.think_read_device_status(cache.score_ws) == 0
+    # From the inputs: the oracle's rule on the oracle's own scores.
+    _adaptive_against_oracle_scores(ora_scores, Th, gidx, rowoff, out, q, kf, f64(v), tau, T_min, T_max)
     # the one-entry prune (TMA compaction in the ragged layout) gives the
     # outputs of the three separate calls (register compaction) bit for bit
     step = qdk.AdaptiveCache(B, Hq, Hkv, N, tau, T_min, T_max)
@@ -417,12 +449,19 @@ def test_fused_prune_equals_stepwise_calls():
     assert torch.equal(a.idx, b.idx)
 
 
-PRUNE_ENV_KEYS = ("THINK_PRUNE_FUSED", "THINK_PRUNE_L2_HINTS", "THINK_SCORE_TMA", "THINK_SCORE_STAGES",
-                  "THINK_COMPACT_TMA", "THINK_COMPACT_STAGES", "THINK_COMPACT_TILES")
+PRUNE_ENV_KEYS = ("THINK_PRUNE_FUSED", "THINK_PRUNE_STAGES", "THINK_PRUNE_CSTAGES", "THINK_PRUNE_HINTS",
+                  "THINK_PRUNE_LAG", "THINK_PRUNE_PREFETCH",
+                  "THINK_SCORE_TMA", "THINK_SCORE_STAGES", "THINK_COMPACT_TMA", "THINK_COMPACT_STAGES",
+                  "THINK_COMPACT_TILES")
 
 
 @pytest.mark.parametrize("env", [{"THINK_PRUNE_FUSED": "1"},
-                                 {"THINK_PRUNE_FUSED": "1", "THINK_PRUNE_L2_HINTS": "0"},
+                                 {"THINK_PRUNE_FUSED": "1", "THINK_PRUNE_STAGES": "2", "THINK_PRUNE_CSTAGES": "2"},
+                                 {"THINK_PRUNE_FUSED": "1", "THINK_PRUNE_STAGES": "10", "THINK_PRUNE_CSTAGES": "2"},
+                                 {"THINK_PRUNE_FUSED": "1", "THINK_PRUNE_STAGES": "3", "THINK_PRUNE_CSTAGES": "5",
+                                  "THINK_PRUNE_LAG": "1"},
+                                 {"THINK_PRUNE_FUSED": "1", "THINK_PRUNE_HINTS": "0", "THINK_PRUNE_LAG": "5"},
+                                 {"THINK_PRUNE_FUSED": "1", "THINK_PRUNE_HINTS": "7", "THINK_PRUNE_PREFETCH": "8"},
                                  {"THINK_SCORE_TMA": "0"},
                                  {"THINK_SCORE_STAGES": "2"},
                                  {"THINK_SCORE_STAGES": "8"},
@@ -430,13 +469,16 @@ PRUNE_ENV_KEYS = ("THINK_PRUNE_FUSED", "THINK_PRUNE_L2_HINTS", "THINK_SCORE_TMA"
                                  {"THINK_COMPACT_STAGES": "2", "THINK_COMPACT_TILES": "1"},
                                  {"THINK_COMPACT_STAGES": "8", "THINK_COMPACT_TILES": "37"}])
 def test_prune_schedules_give_identical_results(env, monkeypatch):
-    # the two-launch prune (default: TMA-staged score and compaction tiles)
-    # against the one-kernel prune (with and without its L2 hints), the
-    # register-pipelined score and compaction kernels, other ring depths and
-    # run lengths: bit for bit the same (same split plan, same order of
-    # additions, pure copies)
+    # the default two-launch prune (TMA-staged score and compaction tiles)
+    # against the one-kernel prune (which compacts each round of heads from L2
+    # while it scores the next; several ring depths, lags, L2 hints and
+    # prefetch distances), the register-pipelined score and compaction kernels,
+    # other ring depths and run lengths: bit for bit the same (same split plan,
+    # same order of additions, pure copies).  Shapes: one round, several rounds
+    # of one and of several heads (two runs per block), a head too long for the
+    # one-kernel prune (two launches on both sides)
     shapes = [(2, 32, 8, 5000, 64), (1, 8, 1, 70, 51), (4, 4, 4, 3000, 128), (3, 16, 8, 1, 1),
-              (1, 32, 8, 40000, 51)]
+              (1, 32, 8, 40000, 51), (2, 32, 8, 60000, 51), (1, 8, 2, 200000, 40)]
     for i, (B, Hq, Hkv, N, T) in enumerate(shapes):
         q_win, k, _, _ = _random_case(100 + i, B, Hq, Hkv, N, 32, torch.bfloat16, k_pad=8)
         kd = torch.empty((B, Hkv, N + 8, 128), dtype=torch.bfloat16, device=DEV)[:, :, :N].copy_(k)
