@@ -73,6 +73,7 @@ typedef enum { THINK_F32 = 0, THINK_BF16 = 1 } think_dtype_t;
 #define THINK_DEVICE_TIMEOUT_EMPTY   0x2u   /* a stage was never released */
 #define THINK_DEVICE_TIMEOUT_READY   0x4u   /* a head's channel selection never became ready */
 #define THINK_DEVICE_TIMEOUT_BARRIER 0x8u   /* a block-internal barrier was not reached */
+#define THINK_DEVICE_OOB             0x10u  /* debug builds only: an index check failed (store skipped) */
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char *think_status_string(think_status_t status);

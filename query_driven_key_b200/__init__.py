@@ -17,7 +17,9 @@ import os
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libthink.so")
+# THINK_DEBUG_LIB=1 loads the debug build (index checks at the global stores,
+# reported as THINK_DEVICE_OOB in the device status word) instead.
+LIB_PATH = os.path.join(_PKG, "libthink_debug.so" if os.environ.get("THINK_DEBUG_LIB") == "1" else "libthink.so")
 
 THINK_OK = 0
 THINK_ERR_INVALID_ARG = 1
@@ -31,6 +33,7 @@ THINK_DEVICE_TIMEOUT_FULL = 0x1
 THINK_DEVICE_TIMEOUT_EMPTY = 0x2
 THINK_DEVICE_TIMEOUT_READY = 0x4
 THINK_DEVICE_TIMEOUT_BARRIER = 0x8
+THINK_DEVICE_OOB = 0x10
 
 EXPORTED = (
     "think_status_string", "think_t_from_lambda", "think_pruned_ld",

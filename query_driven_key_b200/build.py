@@ -11,6 +11,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libthink.so")
+DEBUG_LIB = os.path.join(PKG, "libthink_debug.so")  # -DTHINK_DEBUG: index checks at the global stores
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17",
@@ -36,18 +37,26 @@ def nvcc() -> str:
     return cand if os.path.exists(cand) else "nvcc"
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
-    """Compile csrc/*.cu into libthink.so next to this file; skip if up to date."""
-    if not force and os.path.exists(LIB):
+def _build_one(lib: str, flags, force: bool, verbose: bool) -> str:
+    if not force and os.path.exists(lib):
         newest = max(os.path.getmtime(p) for p in _deps())
-        if os.path.getmtime(LIB) >= newest:
-            return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *NVCC_FLAGS, *extra_flags, "-I", INCLUDE, "-I", CSRC, *_sources(), "-o", tmp]
+        if os.path.getmtime(lib) >= newest:
+            return lib
+    tmp = lib + f".tmp{os.getpid()}"
+    cmd = [nvcc(), *NVCC_FLAGS, *flags, "-I", INCLUDE, "-I", CSRC, *_sources(), "-o", tmp]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
+    os.replace(tmp, lib)
+    return lib
+
+
+def build(force: bool = False, verbose: bool = False, extra_flags=(), debug: bool = True) -> str:
+    """Compile csrc/*.cu into libthink.so next to this file (and the debug
+    build libthink_debug.so); skip what is up to date."""
+    _build_one(LIB, list(extra_flags), force, verbose)
+    if debug:
+        _build_one(DEBUG_LIB, ["-DTHINK_DEBUG", *extra_flags], force, verbose)
     return LIB
 
 

@@ -144,8 +144,12 @@ __global__ void __launch_bounds__(kCtThreads, 3)
         __syncwarp();
         if (lane == 0) mbar_arrive(empty0 + 8 * s);
         const int64_t x0 = (tile0 + i) * kCtTileRows;
-        compact_tile_store_kept(v, crow, a.kp, a.ldk, x0 + 8 * (tb0 + (lane & 3)), a.N);
-        if (pad_row < Tw) store_run8(a.kp + (r0 + pad_row) * a.ldk, x0 + 8 * (tid & 7), a.N, zero);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            if (crow[k] >= 0 && THINK_IN_RANGE(crow[k] < (a.Th ? a.row_cap : (int64_t)gridDim.y * a.T), a.status))
+                store_run8(a.kp + crow[k] * a.ldk, x0 + 8 * (tb0 + (lane & 3)), a.N, v[k]);
+        if (pad_row < Tw && THINK_IN_RANGE(r0 + pad_row < a.row_cap, a.status))
+            store_run8(a.kp + (r0 + pad_row) * a.ldk, x0 + 8 * (tid & 7), a.N, zero);
     }
 }
 

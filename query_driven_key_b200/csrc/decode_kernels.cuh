@@ -161,7 +161,7 @@ __device__ __forceinline__ void finish_split(const DecodeArgs &a, int head, int 
     static_assert(NT % 128 == 0, "whole channel rows per thread group");
     constexpr int P = NT / 128;            // thread groups splitting the split axis
     const int64_t slot0 = ((int64_t)head * a.splits + split) * G;
-    if (tid < 128) {
+    if (tid < 128 && THINK_IN_RANGE(split < a.splits && head < (int)gridDim.y, a.status)) {
 #pragma unroll
         for (int g = 0; g < G; ++g) {
             a.part_o[(slot0 + g) * kD + tid] = O[g];
@@ -262,7 +262,8 @@ __device__ __forceinline__ void finish_split(const DecodeArgs &a, int head, int 
             float o = sp[g * kD + d];
 #pragma unroll
             for (int q2 = 1; q2 < P; ++q2) o += sp[(q2 * G + g) * kD + d];
-            a.out[((int64_t)b * a.Hq + (int64_t)kv * G + g) * kD + d] = o / sL[g];
+            if (THINK_IN_RANGE((int64_t)b * a.Hq + (int64_t)kv * G + g < (int64_t)gridDim.y / a.Hkv * a.Hq, a.status))
+                a.out[((int64_t)b * a.Hq + (int64_t)kv * G + g) * kD + d] = o / sL[g];
         }
         if (tid == 0) a.tickets[head] = 0u;  // ready for the next call
     }

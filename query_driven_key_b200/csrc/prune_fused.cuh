@@ -22,13 +22,14 @@
 //         round r >= lag it waits until this block has compacted round
 //         r - lag, so at most `lag` rounds are scored ahead of the compaction;
 //       * eight score warps: add the squares of each tile (the thread map of
-//         score_tma_kernel) and hand each run's row-group partials to the merge
-//         warp through two shared buffers;
-//       * merge warps: window-query energies, the run partial, and the
-//         two-level merge of score_run_end (group and head tickets); the block
-//         that completes a head forms its scores, selects the top T and
-//         raises the head's ready flag.  Fences and atomics stall only this
-//         warp;
+//         score_tma_kernel), add each run's row-group partials in row order
+//         and queue the run partial (8 slots) for the merge warps, so that a
+//         merge warp busy with a group or head merge does not stall scoring;
+//       * four merge warps (one thread per channel): window-query energies,
+//         the run partial, and the two-level merge of score_run_end (group and
+//         head tickets); the block that completes a head forms its scores,
+//         selects the top T and raises the head's ready flag.  Fences and
+//         atomics stall only these warps;
 //       * compact producer (one thread): streams the block's tiles again, in
 //         the same order, through a second ring (`c_stages` x 16 KB);
 //       * eight compact warps: wait (bounded) for the head's ready flag,
@@ -57,14 +58,16 @@ constexpr int kPfMaxStages = 12;                  // score + compact stages
 constexpr uint32_t kPfHalfBytes = 64u * 64u * 2u;   // 64 tokens x 64 channels x bf16
 constexpr uint32_t kPfTileBytes = 2u * kPfHalfBytes;
 constexpr uint32_t kPfRedBytes = 16u * kD * 8u;   // [16][128] fp64 row-group partials of one run
-constexpr uint32_t kPfSvBytes = kD * 8u;          // [128] score bits
+constexpr int kPfHandSlots = 8;                   // run partials queued for the merge warps
+constexpr uint32_t kPfHandBytes = kPfHandSlots * kD * 8u;
+constexpr uint32_t kPfSvBytes = 4u * kD * 8u;     // [4][128] score bits, one row per merge warp
 constexpr uint32_t kPfMiscBytes = 128u;           // abort, compact rounds done, exit flag, merge flag,
                                                   // compact flag, wcnt[4]
 
 inline size_t prune_fused_smem_bytes(int s_stages, int c_stages)
 {
-    return (size_t)(s_stages + c_stages) * kPfTileBytes + 2u * kPfRedBytes + kPfSvBytes + kPfMiscBytes +
-           8u * (2u * (size_t)(s_stages + c_stages) + 4u) + 1024u;  // + mbarriers, alignment slack
+    return (size_t)(s_stages + c_stages) * kPfTileBytes + kPfRedBytes + kPfHandBytes + kPfSvBytes + kPfMiscBytes +
+           8u * (2u * (size_t)(s_stages + c_stages) + 2u * kPfHandSlots) + 1024u;  // + mbarriers, alignment slack
 }
 
 enum : int { kPfHintScoreKeep = 1, kPfHintCompactDrop = 2, kPfHintStoreDrop = 4 };
@@ -181,12 +184,13 @@ __device__ __forceinline__ void store_run8_hint(__nv_bfloat16 *row, int64_t x, i
 // Shared-memory layout of one block.
 struct PfSmem {
     uint32_t ring_s, ring_c;      // shared addresses of the two rings
-    double *red;                  // [2][16][128]
-    unsigned long long *sv;       // [128]
+    double *red;                  // [16][128] score warps' row-group partials
+    double *hand;                 // [kPfHandSlots][128] run partials for the merge warps
+    unsigned long long *sv;       // [4][128]
     volatile unsigned *abort, *c_done;
     unsigned *last, *mflag, *cflag;
     int *wcnt;
-    uint32_t full_s, empty_s, full_c, empty_c, red_full, red_free;  // mbarrier arrays (8 bytes apart)
+    uint32_t full_s, empty_s, full_c, empty_c, hand_full, hand_free;  // mbarrier arrays (8 bytes apart)
 };
 
 __device__ __forceinline__ PfSmem pf_smem(const PruneFusedArgs &a, unsigned char *base)
@@ -196,7 +200,9 @@ __device__ __forceinline__ PfSmem pf_smem(const PruneFusedArgs &a, unsigned char
     m.ring_c = m.ring_s + (uint32_t)a.s_stages * kPfTileBytes;
     unsigned char *p = base + (size_t)(a.s_stages + a.c_stages) * kPfTileBytes;
     m.red = reinterpret_cast<double *>(p);
-    p += 2 * kPfRedBytes;
+    p += kPfRedBytes;
+    m.hand = reinterpret_cast<double *>(p);
+    p += kPfHandBytes;
     m.sv = reinterpret_cast<unsigned long long *>(p);
     p += kPfSvBytes;
     unsigned *misc = reinterpret_cast<unsigned *>(p);
@@ -211,8 +217,8 @@ __device__ __forceinline__ PfSmem pf_smem(const PruneFusedArgs &a, unsigned char
     m.empty_s = m.full_s + 8u * (uint32_t)a.s_stages;
     m.full_c = m.empty_s + 8u * (uint32_t)a.s_stages;
     m.empty_c = m.full_c + 8u * (uint32_t)a.c_stages;
-    m.red_full = m.empty_c + 8u * (uint32_t)a.c_stages;
-    m.red_free = m.red_full + 16u;
+    m.hand_full = m.empty_c + 8u * (uint32_t)a.c_stages;
+    m.hand_free = m.hand_full + 8u * kPfHandSlots;
     return m;
 }
 
@@ -289,48 +295,74 @@ __device__ __forceinline__ void pf_score(const PruneFusedArgs &a, const PfSmem &
             double acc[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) acc[e] = 0.0;
-            for (int t = x.t0; t < x.t1; ++t, ++n) {
-                const int s = n % stages;
+            // two tiles per step: both tiles' loads are in flight together
+            for (int t = x.t0; t < x.t1; t += 2) {
+                const int nt = min(2, x.t1 - t);
+                const int n0 = n;
+                n += nt;
                 if (*m.abort) continue;
-                if (!mbar_wait_bounded(m.full_s + 8 * s, (uint32_t)((n / stages) & 1), a.sc.status,
-                                       THINK_DEVICE_TIMEOUT_FULL)) {
+                uint4 w[2][4];
+                bool ok = true;
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    if (i >= nt) break;
+                    const int s = (n0 + i) % stages;
+                    if (!mbar_wait_bounded(m.full_s + 8 * s, (uint32_t)(((n0 + i) / stages) & 1), a.sc.status,
+                                           THINK_DEVICE_TIMEOUT_FULL)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t st = m.ring_s + (uint32_t)s * kPfTileBytes + s_half;
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        const uint32_t row = (uint32_t)(rg + 16 * k4);
+                        const uint32_t addr = st + row * 128u + ((s_chunk ^ (row & 7u)) << 4);
+                        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                     : "=r"(w[i][k4].x), "=r"(w[i][k4].y), "=r"(w[i][k4].z), "=r"(w[i][k4].w)
+                                     : "r"(addr)
+                                     : "memory");
+                    }
+                }
+                if (!ok) {
                     *m.abort = 1u;
                     continue;
                 }
-                const uint32_t st = m.ring_s + (uint32_t)s * kPfTileBytes + s_half;
-                uint4 w[4];
-#pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4) {
-                    const uint32_t row = (uint32_t)(rg + 16 * k4);
-                    const uint32_t addr = st + row * 128u + ((s_chunk ^ (row & 7u)) << 4);
-                    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                                 : "=r"(w[k4].x), "=r"(w[k4].y), "=r"(w[k4].z), "=r"(w[k4].w)
-                                 : "r"(addr)
-                                 : "memory");
-                }
-                add_squares4_bf16(w, acc);  // uses the loaded words: the stage has been read
+                add_squares4_bf16(w[0], acc);  // tile order; uses the loaded words: the stages have been read
+                if (nt == 2) add_squares4_bf16(w[1], acc);
                 fence_proxy_async_shared();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(m.empty_s + 8 * s);
+                if (lane == 0) {
+                    mbar_arrive(m.empty_s + 8 * (n0 % stages));
+                    if (nt == 2) mbar_arrive(m.empty_s + 8 * ((n0 + 1) % stages));
+                }
             }
-            const int k = cnt & 1, u = cnt >> 1;
-            if (u > 0 && !*m.abort &&
-                !mbar_wait_bounded(m.red_free + 8 * k, (uint32_t)((u - 1) & 1), a.sc.status,
-                                   THINK_DEVICE_TIMEOUT_BARRIER))
-                *m.abort = 1u;
-            double *red = m.red + (size_t)k * 16 * kD;
+            // the run partial: row groups added in row order (threads 0..127,
+            // one channel each), queued for the merge warps
+            named_barrier(3, kPfGroupThreads);  // the previous run's sums have read red
 #pragma unroll
-            for (int e = 0; e < 8; ++e) red[rg * kD + cc * 8 + e] = acc[e];
-            mbar_arrive(m.red_full + 8 * k);  // every score thread (count 256)
+            for (int e = 0; e < 8; ++e) m.red[rg * kD + cc * 8 + e] = acc[e];
+            named_barrier(3, kPfGroupThreads);
+            if (tid < kD) {
+                double p = 0.0;
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr) p += m.red[rr * kD + tid];
+                const int k = cnt % kPfHandSlots, u = cnt / kPfHandSlots;
+                if (u > 0 && !*m.abort &&
+                    !mbar_wait_bounded(m.hand_free + 8 * k, (uint32_t)((u - 1) & 1), a.sc.status,
+                                       THINK_DEVICE_TIMEOUT_BARRIER))
+                    *m.abort = 1u;
+                m.hand[k * kD + tid] = p;
+                mbar_arrive(m.hand_full + 8 * k);  // threads 0..127 (count 128)
+            }
             ++cnt;
         });
     }
 }
 
 // Merge warps (128 threads, thread c = channel c): per run of the block, in
-// the score warps' order, the window-query energies (runs < G), the run
-// partial and the two-level merge of score_run_end (same additions, same
-// order), then for the block that completes a head its scores, the top T and
+// the score warps' order, the window-query energies assigned to the run, the
+// run partial (from the score warps' queue) and the two-level merge of
+// score_run_end (same additions, same order), then for the block that completes a head its scores, the top T and
 // the head's ready flag.  Only one thread per level touches a ticket, with an
 // acquire-release fetch-and-add after a merge-group barrier, so a level costs
 // about one L2 round trip for the ticket and one for its loads.
@@ -354,19 +386,16 @@ __device__ __forceinline__ void pf_merge(const PruneFusedArgs &a, const PfSmem &
                                           (((int64_t)b * sa.Hq + (int64_t)kv * G + g) * sa.S) * kD + c;
                 sa.qn2[((int64_t)head * G + g) * kD + c] = window_energy<__nv_bfloat16>(qh, sa.S);
             }
-            // the run partial: row groups added in row order
-            const int k = cnt & 1, u = cnt >> 1;
+            // the run partial from the score warps' queue
+            const int k = cnt % kPfHandSlots, u = cnt / kPfHandSlots;
             ++cnt;
-            if (!*m.abort && !mbar_wait_bounded(m.red_full + 8 * k, (uint32_t)(u & 1), sa.status,
+            if (!*m.abort && !mbar_wait_bounded(m.hand_full + 8 * k, (uint32_t)(u & 1), sa.status,
                                                 THINK_DEVICE_TIMEOUT_BARRIER))
                 *m.abort = 1u;
-            const double *red = m.red + (size_t)k * 16 * kD;
-            double p = 0.0;
-#pragma unroll
-            for (int rr = 0; rr < 16; ++rr) p += red[rr * kD + c];
-            sa.part[((int64_t)head * R + x.run) * kD + c] = p;
+            if (THINK_IN_RANGE(head < a.heads && x.run < R, sa.status))
+                sa.part[((int64_t)head * R + x.run) * kD + c] = m.hand[k * kD + c];
             __syncwarp();
-            if (lane == 0) mbar_arrive(m.red_free + 8 * k);
+            if (lane == 0) mbar_arrive(m.hand_free + 8 * k);
             sync();
             // group of kMergeGroup runs: its last run adds the group's partials
             const int grp = x.run / kMergeGroup;
@@ -462,24 +491,46 @@ __device__ __forceinline__ void pf_compact(const PruneFusedArgs &a, const PfSmem
                 cur_head = ok ? x.head : -1;
                 named_barrier(1, kPfGroupThreads);  // cflag is read before it is rewritten
             }
-            for (int t = x.t0; t < x.t1; ++t, ++n) {
-                const int s = n % stages;
+            // two tiles per step: both tiles' loads are in flight together
+            for (int t = x.t0; t < x.t1; t += 2) {
+                const int nt = min(2, x.t1 - t);
+                const int n0 = n;
+                n += nt;
                 if (*m.abort) continue;
-                if (!mbar_wait_bounded(m.full_c + 8 * s, (uint32_t)((n / stages) & 1), a.sc.status,
-                                       THINK_DEVICE_TIMEOUT_FULL)) {
+                uint32_t v[2][4][4];
+                bool ok = true;
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    if (i >= nt) break;
+                    const int s = (n0 + i) % stages;
+                    if (!mbar_wait_bounded(m.full_c + 8 * s, (uint32_t)(((n0 + i) / stages) & 1), a.sc.status,
+                                           THINK_DEVICE_TIMEOUT_FULL)) {
+                        ok = false;
+                        break;
+                    }
+                    compact_tile_load(m.ring_c + (uint32_t)s * kPfTileBytes, c_row, cw, v[i]);
+                }
+                if (!ok) {
                     *m.abort = 1u;
                     continue;
                 }
-                uint32_t v[4][4];
-                compact_tile_load(m.ring_c + (uint32_t)s * kPfTileBytes, c_row, cw, v);
-                compact_tile_transpose(v, lane);  // uses the loaded words: the stage has been read
+                compact_tile_transpose(v[0], lane);  // uses the loaded words: the stages have been read
+                if (nt == 2) compact_tile_transpose(v[1], lane);
                 fence_proxy_async_shared();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(m.empty_c + 8 * s);
-                const int64_t xo = (int64_t)t * kPfTile + 8 * (tb0 + (lane & 3));
+                if (lane == 0) {
+                    mbar_arrive(m.empty_c + 8 * (n0 % stages));
+                    if (nt == 2) mbar_arrive(m.empty_c + 8 * ((n0 + 1) % stages));
+                }
 #pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    if (crow[k] >= 0) store_run8_hint(a.kp + crow[k] * a.ldk, xo, a.N, v[k], pol_store);
+                for (int i = 0; i < 2; ++i) {
+                    if (i >= nt) break;
+                    const int64_t xo = (int64_t)(t + i) * kPfTile + 8 * (tb0 + (lane & 3));
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        if (crow[k] >= 0 && THINK_IN_RANGE(crow[k] < (int64_t)a.heads * a.T, a.sc.status))
+                            store_run8_hint(a.kp + crow[k] * a.ldk, xo, a.N, v[i][k], pol_store);
+                }
             }
         });
         // this block has compacted round r (the score producer may go on)
@@ -504,9 +555,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             mbar_init(m.full_c + 8 * s, 1);
             mbar_init(m.empty_c + 8 * s, 8);
         }
-        for (int k = 0; k < 2; ++k) {
-            mbar_init(m.red_full + 8 * k, kPfGroupThreads);
-            mbar_init(m.red_free + 8 * k, kPfMergeThreads / 32);
+        for (int k = 0; k < kPfHandSlots; ++k) {
+            mbar_init(m.hand_full + 8 * k, kD);
+            mbar_init(m.hand_free + 8 * k, kPfMergeThreads / 32);
         }
         *m.abort = 0u;
         *m.c_done = 0u;

@@ -231,7 +231,8 @@ __device__ __forceinline__ bool score_run_end(const ScoreArgs &a, int head, int 
         double s = 0.0;
 #pragma unroll 4
         for (int rr = 0; rr < ROWS; ++rr) s += red[rr * kD + tid];
-        a.part[((int64_t)head * a.splits + split) * kD + tid] = s;
+        if (THINK_IN_RANGE(split < a.splits, a.status))
+            a.part[((int64_t)head * a.splits + split) * kD + tid] = s;
     }
     __threadfence();
     sync();
@@ -252,7 +253,7 @@ __device__ __forceinline__ bool score_run_end(const ScoreArgs &a, int head, int 
         double s = 0.0;
 #pragma unroll
         for (int u = 0; u < kMergeGroup; ++u) s = __dadd_rn(s, v[u]);  // + 0.0 past the group is exact
-        a.gpart[((int64_t)head * a.groups + grp) * kD + tid] = s;
+        if (THINK_IN_RANGE(grp < a.groups, a.status)) a.gpart[((int64_t)head * a.groups + grp) * kD + tid] = s;
     }
     if (tid == 0) *gt = 0u;  // ready for the next call
     __threadfence();

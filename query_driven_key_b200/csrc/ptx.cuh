@@ -6,9 +6,21 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include "think.h"
+
 namespace think {
 
 constexpr int kD = 128;  // head width; the only one built
+
+// Debug builds (-DTHINK_DEBUG): index checks at the global stores whose
+// index is computed from device data or launch plans.  A failed check sets
+// THINK_DEVICE_OOB in the status word and the store is skipped; release
+// builds compile the check away.
+#ifdef THINK_DEBUG
+#define THINK_IN_RANGE(cond, status) ((cond) ? true : (atomicOr((status), THINK_DEVICE_OOB), false))
+#else
+#define THINK_IN_RANGE(cond, status) true
+#endif
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p)
 {

@@ -5,7 +5,7 @@ import argparse
 import pytest
 
 import bench
-from query_driven_key_b200 import workloads as W
+import workloads as W
 
 
 def _args(**kw):

@@ -28,7 +28,7 @@ def _worker(rank, world, port, q):
                             timeout=datetime.timedelta(seconds=60))
     try:
         import bench
-        from query_driven_key_b200 import workloads as W
+        import workloads as W
         # each rank times something different; every rank must agree on the max
         mx = bench.max_over_ranks([10.0 + rank, 5.0 - rank, 1.5])
         # replicas draw distinct data (layer index = rank)

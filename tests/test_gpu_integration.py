@@ -12,7 +12,7 @@ from tests.helpers import check_out, f64, idx_mismatch_heads
 pytestmark = pytest.mark.gpu
 
 qdk = pytest.importorskip("query_driven_key_b200")
-from query_driven_key_b200 import workloads as W  # noqa: E402
+import workloads as W  # noqa: E402
 
 DEV = "cuda"
 

@@ -18,7 +18,7 @@ from tests.helpers import (NEAR_TIE_REL, TOL, check_out, check_scores, f64, idx_
 pytestmark = pytest.mark.gpu
 
 qdk = pytest.importorskip("query_driven_key_b200")
-from query_driven_key_b200 import workloads as W  # noqa: E402
+import workloads as W  # noqa: E402
 
 DEV = "cuda"
 

@@ -17,7 +17,7 @@ import torch
 pytestmark = pytest.mark.gpu
 
 qdk = pytest.importorskip("query_driven_key_b200")
-from query_driven_key_b200 import workloads as W  # noqa: E402
+import workloads as W  # noqa: E402
 
 
 @pytest.mark.parametrize("name,N", [("mistral_7b_long", 20000), ("llama2_7b_mha", 4096)])

@@ -26,7 +26,7 @@ import torch
 
 @dataclasses.dataclass(frozen=True)
 class Workload:
-    name: str
+    label: str                     # the model shape it stands for; name adds the sizes
     seed: int
     B: int
     Hq: int
@@ -47,27 +47,37 @@ class Workload:
     def G(self) -> int:
         return self.Hq // self.Hkv
 
+    @property
+    def name(self) -> str:
+        """The label and the sizes the workload has now (with_ keeps them in step)."""
+        dt = {torch.bfloat16: "bf16", torch.float32: "fp32"}.get(self.dtype, str(self.dtype))
+        s = (f"{self.label}: B{self.B} Hq{self.Hq} Hkv{self.Hkv} d{self.d} N{self.N} S_obs{self.S_obs} "
+             f"lambda{self.lam} {dt}")
+        if self.layers > 1:
+            s += f", {self.layers} layers"
+        if self.k_kind == "lowrank":
+            s += ", low-rank K"
+        return s
+
     def with_(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
 
 
 # The five workloads (shapes of one decoder layer's attention, or 32 layers).
 WORKLOADS = {
-    "tiny_fp32": Workload("tiny_fp32: 1 head d128 N512 S_obs32 lambda0.5 fp32", 0,
+    "tiny_fp32": Workload("tiny single head", 0,
                           B=1, Hq=1, Hkv=1, N=512, d=128, S_obs=32, lam=0.5,
                           dtype=torch.float32, decode_steps=1),
-    "llama2_7b_mha": Workload("llama2-7b-shaped MHA: B1 H32 d128 N4096 S_obs32 lambda0.4 bf16", 1,
+    "llama2_7b_mha": Workload("llama2-7b-shaped MHA", 1,
                               B=1, Hq=32, Hkv=32, N=4096, d=128, S_obs=32, lam=0.4,
                               dtype=torch.bfloat16, decode_steps=64),
-    "llama3_8b_gqa": Workload("llama3-8b-shaped GQA: B4 Hq32 Hkv8 d128 N32768 S_obs32 lambda0.5 bf16, "
-                              "low-rank K", 2,
+    "llama3_8b_gqa": Workload("llama3-8b-shaped GQA", 2,
                               B=4, Hq=32, Hkv=8, N=32768, d=128, S_obs=32, lam=0.5,
                               dtype=torch.bfloat16, decode_steps=1, k_kind="lowrank"),
-    "mistral_7b_long": Workload("mistral-7b-shaped GQA long context: B1 Hq32 Hkv8 d128 N131072 S_obs64 "
-                                "lambda0.6 bf16", 3,
+    "mistral_7b_long": Workload("mistral-7b-shaped GQA long context", 3,
                                 B=1, Hq=32, Hkv=8, N=131072, d=128, S_obs=64, lam=0.6,
                                 dtype=torch.bfloat16, decode_steps=256, k_sigma=1.5),
-    "sweep_32l": Workload("32-layer sweep: Hq32 Hkv8 d128 N8192 S_obs32 bf16", 4,
+    "sweep_32l": Workload("32-layer sweep", 4,
                           B=1, Hq=32, Hkv=8, N=8192, d=128, S_obs=32, lam=0.4,
                           dtype=torch.bfloat16, decode_steps=1, layers=32),
 }
