@@ -139,10 +139,12 @@ __global__ void __launch_bounds__(kCtThreads, 3)
             break;
         uint32_t v[4][4];
         compact_tile_load(ring + (uint32_t)s * kCtTileBytes, c_row, cw, v);
-        compact_tile_transpose(v, lane);  // uses the loaded words: the stage has been read
+        // the loads have returned (the fence orders them before the producer's
+        // next TMA write into this stage), then release it
         fence_proxy_async_shared();
         __syncwarp();
         if (lane == 0) mbar_arrive(empty0 + 8 * s);
+        compact_tile_transpose(v, lane);
         const int64_t x0 = (tile0 + i) * kCtTileRows;
 #pragma unroll
         for (int k = 0; k < 4; ++k)

@@ -10,8 +10,8 @@
 // chosen, so K is read twice: once to score, once to compact.  This kernel
 // makes the second read an L2 hit:
 //   - The heads are taken in rounds of about 2,000 64-token tiles (about
-//     34 MB of bf16 keys), each head cut into runs of s_tiles tiles (the split
-//     plan of the score kernels, so the scores are theirs bit for bit).  Run j
+//     34 MB of bf16 keys), each head cut into runs of s_tiles tiles (the round
+//     split plan; the score kernels give the same bits on that plan).  Run j
 //     of a round belongs to block j % gridDim.x, in every round, for both its
 //     score and its compaction, so a run is compacted on the SM that scored
 //     it, about one round later, while its tiles are still in L2.

@@ -148,8 +148,9 @@ __device__ __forceinline__ uint64_t l2_policy_evict_normal()
 
 // Orders this thread's earlier generic-proxy accesses of shared memory (plain
 // loads, ldmatrix) before later async-proxy accesses (TMA writes into the same
-// stage).  A ring consumer issues it, after the values it loaded from a stage
-// are in registers and used, before it releases the stage to the producer.
+// stage).  A ring consumer issues it after its loads from a stage and before
+// it releases the stage to the producer: without it, a release that overtook
+// loads still in flight let the next TMA write overwrite the stage under them.
 __device__ __forceinline__ void fence_proxy_async_shared()
 {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -124,10 +124,12 @@ __global__ void __launch_bounds__(kStThreads, 3)
                              : "r"(addr)
                              : "memory");
             }
-            add_squares4_bf16(w, acc);  // uses the loaded words: the stage has been read
+            // the loads have returned (the fence orders them before the
+            // producer's next TMA write into this stage), then release it
             fence_proxy_async_shared();
             __syncwarp();
             if (lane == 0) mbar_arrive(empty0 + 8 * s);
+            add_squares4_bf16(w, acc);
         }
     }
     __syncthreads();  // every tile has been read: the ring is free

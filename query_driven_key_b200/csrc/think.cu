@@ -30,6 +30,7 @@ namespace {
 
 constexpr int kTargetSMs = 148;             // B200
 constexpr int kScoreResidentPerSM = 3;      // score blocks resident per SM (both score kernels)
+constexpr int kScoreMaxWaves = 4;
 constexpr int kPlanBlocks = 2 * kTargetSMs; // runs per round of the score plan
 constexpr int64_t kRoundTilesMax = 2560;    // tiles per round (40 MB of bf16 keys; L2 holds two)
 constexpr int kRunTilesMax = 64;            // tiles per run at most
@@ -105,9 +106,10 @@ struct ScorePlan {
     int groups;              // groups of kMergeGroup runs per head (the merge order)
 };
 
-// Choose the run length L (tiles) that minimises rounds x runs-per-block x
-// (L + 2): the 2 tiles stand for a run's fixed cost (partial sums, tickets).
-ScorePlan plan_score(int64_t heads, int64_t N)
+// The one-kernel prune's plan: the run length L (tiles) that minimises
+// rounds x runs-per-block x (L + 2); the 2 tiles stand for a run's fixed cost
+// (partial sums, tickets).
+ScorePlan plan_score_rounds(int64_t heads, int64_t N)
 {
     const int64_t tph = std::max<int64_t>(1, ceil_div(N, kPfTile));
     heads = std::max<int64_t>(heads, 1);
@@ -132,6 +134,68 @@ ScorePlan plan_score(int64_t heads, int64_t N)
     best.rows_per_split = (int64_t)best.s_tiles * kPfTile;
     best.groups = (int)ceil_div(best.splits, kMergeGroup);
     return best;
+}
+
+ScorePlan score_plan_from_tiles(int64_t tph, int64_t st)
+{
+    ScorePlan p{};
+    p.tiles_per_head = tph;
+    st = std::min<int64_t>(std::max<int64_t>(st, 1), tph);
+    p.s_tiles = (int)st;
+    p.rows_per_split = st * kPfTile;
+    p.splits = (int)ceil_div(tph, st);
+    p.groups = (int)ceil_div(p.splits, kMergeGroup);
+    p.hpr = p.rounds = 0;  // not a round plan
+    return p;
+}
+
+// The two-launch prune's plan (one score block per run): the shortest runs
+// whose count fits W waves of the resident score blocks (148 SMs x
+// kScoreResidentPerSM), for the fewest W (up to kScoreMaxWaves) whose runs
+// fill at least 90% of their slots, else the best filled.  Whole waves leave
+// no partly filled last wave, whose blocks would stream with the rest of the
+// GPU idle.
+ScorePlan plan_score_waves(int64_t heads, int64_t N, int waves)
+{
+    const int64_t tph = std::max<int64_t>(1, ceil_div(N, kPfTile));
+    const int64_t slots = (int64_t)kTargetSMs * kScoreResidentPerSM * waves;
+    const int64_t runs_per_head = std::max<int64_t>(1, slots / std::max<int64_t>(heads, 1));
+    return score_plan_from_tiles(tph, ceil_div(tph, runs_per_head));
+}
+
+ScorePlan plan_score_two_launch(int64_t heads, int64_t N)
+{
+    ScorePlan best = plan_score_waves(heads, N, 1);
+    double best_fill = 0.0;
+    for (int w = 1; w <= kScoreMaxWaves; ++w) {
+        const ScorePlan p = plan_score_waves(heads, N, w);
+        const double fill = (double)(heads * p.splits) / ((double)kTargetSMs * kScoreResidentPerSM * w);
+        if (fill >= 0.9) return p;
+        if (fill > best_fill) {
+            best_fill = fill;
+            best = p;
+        }
+    }
+    return best;
+}
+
+// The plan of a score pass.  The bits of the scores depend only on the plan
+// (runs, then groups of runs, in a fixed order), so every score kernel gives
+// the same bits for the same plan.  The one-kernel prune needs the round plan;
+// the two-launch passes use the wave plan unless THINK_SCORE_PLAN_ROUNDS=1
+// (for comparisons with the one-kernel prune).
+ScorePlan plan_score(int64_t heads, int64_t N, bool fused = false)
+{
+    if (fused || env_int("THINK_SCORE_PLAN_ROUNDS", 0, 0, 1)) return plan_score_rounds(heads, N);
+    return plan_score_two_launch(heads, N);
+}
+
+// The most runs per head of the plans above (workspace size).
+int score_max_splits(int64_t heads, int64_t N)
+{
+    int m = plan_score_rounds(heads, N).splits;
+    for (int w = 1; w <= kScoreMaxWaves; ++w) m = std::max(m, plan_score_waves(heads, N, w).splits);
+    return m;
 }
 
 struct DecodeSplit {
@@ -403,7 +467,10 @@ ScoreWs score_ws_layout(int64_t heads, int G, const ScorePlan &p)
 
 ScoreWs score_ws_layout_max(int64_t heads, int G, int64_t N)
 {
-    return score_ws_layout(heads, G, plan_score(heads, N));
+    ScorePlan p = plan_score_rounds(heads, N);
+    p.splits = score_max_splits(heads, N);
+    p.groups = (int)ceil_div(p.splits, kMergeGroup);
+    return score_ws_layout(heads, G, p);
 }
 
 // The score fields of ScoreArgs that live in the workspace.
@@ -596,7 +663,7 @@ bool prune_fused_applies(think_dtype_t dtype, int64_t heads, int G, int64_t N)
 {
     if (dtype != THINK_BF16 || N <= 0 || N > (int64_t)INT32_MAX - kPfTile || G > 8) return false;
     if (env_int("THINK_PRUNE_FUSED", 0, 0, 1) == 0) return false;
-    const ScorePlan p = plan_score(heads, N);
+    const ScorePlan p = plan_score(heads, N, true);
     return (int64_t)p.hpr * p.tiles_per_head <= kRoundTilesMax;
 }
 
@@ -613,7 +680,7 @@ think_status_t launch_prune_fused(const void *q_win, const void *k, const int64_
                                   cudaStream_t st)
 {
     const int64_t heads = (int64_t)B * Hkv;
-    const ScorePlan p = plan_score(heads, N);
+    const ScorePlan p = plan_score(heads, N, true);
     const ScoreWs w = score_ws_layout(heads, Hq / Hkv, p);
     CUtensorMap mk;
     if (!make_map_4d(&mk, THINK_BF16, k, kD, (uint64_t)N, (uint64_t)Hkv, (uint64_t)B, k_strides[2],

@@ -270,11 +270,12 @@ def test_select_tokens_workspace_layout():
     assert qdk.think_select_tokens_workspace_size(1, 1, 2**31) == 0
 
 
-def _score_plan(heads, N):
-    """The score pass's split plan restated: runs of L 64-token tiles per head
-    and rounds of hpr heads (about 296 runs and at most 2560 tiles per round),
-    L in 1..64 minimising rounds x ceil(runs per round / 296) x (L + 2), ties
-    to the longer run.  Returns (L, runs per head, heads per round, rounds)."""
+def _round_plan(heads, N):
+    """The one-kernel prune's split plan restated: runs of L 64-token tiles per
+    head and rounds of hpr heads (about 296 runs and at most 2560 tiles per
+    round), L in 1..64 minimising rounds x ceil(runs per round / 296) x (L + 2),
+    ties to the longer run.  Returns (L, runs per head, heads per round,
+    rounds)."""
     cdiv = lambda a, b: -(-a // b)
     tph = max(1, cdiv(N, 64))
     heads = max(heads, 1)
@@ -291,16 +292,32 @@ def _score_plan(heads, N):
     return best[1:]
 
 
-def test_score_workspace_follows_the_plan():
+def _wave_plans(heads, N):
+    """The two-launch score pass's split plans restated: for W = 1..4 waves of
+    148 x 3 resident blocks, the shortest runs whose count fits them.  Returns
+    {W: runs per head}; the pass takes the fewest W filling >= 90% of the
+    slots (else the best filled)."""
+    cdiv = lambda a, b: -(-a // b)
+    tph = max(1, cdiv(N, 64))
+    plans = {}
+    for w in range(1, 5):
+        rph = max(1, 148 * 3 * w // max(heads, 1))
+        st = min(max(cdiv(tph, rph), 1), tph)
+        plans[w] = cdiv(tph, st)
+    return plans
+
+
+def test_score_workspace_follows_the_plans():
     # header 256 B + ready flags, head tickets (256-byte aligned) + group
     # tickets [heads][groups] + window-query energies [heads][G][128] fp64 +
     # run partials [heads][runs][128] + group sums [heads][groups][128]
-    # (groups of 16 runs); pins the plan rule on the CPU
+    # (groups of 16 runs), for the plan with the most runs per head; pins the
+    # plan rules on the CPU
     pad = lambda x: -(-x // 256) * 256
     for B, Hq, Hkv, N in [(1, 32, 8, 131072), (4, 32, 8, 32768), (1, 32, 32, 4096), (32, 32, 8, 8192),
                           (1, 1, 1, 512), (1, 8, 1, 1), (2, 16, 8, 0), (3, 24, 8, 100_000)]:
         heads, G = B * Hkv, Hq // Hkv
-        _, R, _, _ = _score_plan(heads, N)
+        R = max(_round_plan(heads, N)[1], max(_wave_plans(heads, N).values()))
         groups = -(-R // 16)
         want = (256 + 2 * pad(heads * 4) + pad(heads * groups * 4) + pad(heads * G * 128 * 8) +
                 pad(heads * R * 128 * 8) + heads * groups * 128 * 8)
@@ -308,7 +325,9 @@ def test_score_workspace_follows_the_plan():
     # long-context layer: one head per round, 293 runs of 7 tiles; GQA batch 4
     # at N = 32K: 4 heads per round, 74 runs of 7; the 32-batch sweep layer: 18
     # heads per round, 16 runs of 8; the MHA layer: one round of 32 heads
-    assert _score_plan(8, 131072) == (7, 293, 1, 8)
-    assert _score_plan(32, 32768) == (7, 74, 4, 8)
-    assert _score_plan(256, 8192) == (8, 16, 18, 15)
-    assert _score_plan(32, 4096) == (8, 8, 32, 1)
+    assert _round_plan(8, 131072) == (7, 293, 1, 8)
+    assert _round_plan(32, 32768) == (7, 74, 4, 8)
+    assert _round_plan(256, 8192) == (8, 16, 18, 15)
+    assert _round_plan(32, 4096) == (8, 8, 32, 1)
+    # the two-launch pass on the long-context layer: one wave of 432 runs of 38 tiles
+    assert _wave_plans(8, 131072)[1] == 54

@@ -450,18 +450,21 @@ def test_fused_prune_equals_stepwise_calls():
 
 
 PRUNE_ENV_KEYS = ("THINK_PRUNE_FUSED", "THINK_PRUNE_STAGES", "THINK_PRUNE_CSTAGES", "THINK_PRUNE_HINTS",
-                  "THINK_PRUNE_LAG", "THINK_PRUNE_PREFETCH",
+                  "THINK_PRUNE_LAG", "THINK_PRUNE_PREFETCH", "THINK_SCORE_PLAN_ROUNDS",
                   "THINK_SCORE_TMA", "THINK_SCORE_STAGES", "THINK_COMPACT_TMA", "THINK_COMPACT_STAGES",
                   "THINK_COMPACT_TILES")
 
 
-@pytest.mark.parametrize("env", [{"THINK_PRUNE_FUSED": "1"},
-                                 {"THINK_PRUNE_FUSED": "1", "THINK_PRUNE_STAGES": "2", "THINK_PRUNE_CSTAGES": "2"},
-                                 {"THINK_PRUNE_FUSED": "1", "THINK_PRUNE_STAGES": "10", "THINK_PRUNE_CSTAGES": "2"},
-                                 {"THINK_PRUNE_FUSED": "1", "THINK_PRUNE_STAGES": "3", "THINK_PRUNE_CSTAGES": "5",
-                                  "THINK_PRUNE_LAG": "1"},
-                                 {"THINK_PRUNE_FUSED": "1", "THINK_PRUNE_HINTS": "0", "THINK_PRUNE_LAG": "5"},
-                                 {"THINK_PRUNE_FUSED": "1", "THINK_PRUNE_HINTS": "7", "THINK_PRUNE_PREFETCH": "8"},
+FUSED = {"THINK_PRUNE_FUSED": "1", "THINK_SCORE_PLAN_ROUNDS": "1"}
+
+
+@pytest.mark.parametrize("env", [FUSED,
+                                 dict(FUSED, THINK_PRUNE_STAGES="2", THINK_PRUNE_CSTAGES="2"),
+                                 dict(FUSED, THINK_PRUNE_STAGES="10", THINK_PRUNE_CSTAGES="2"),
+                                 dict(FUSED, THINK_PRUNE_STAGES="3", THINK_PRUNE_CSTAGES="5", THINK_PRUNE_LAG="1"),
+                                 dict(FUSED, THINK_PRUNE_HINTS="0", THINK_PRUNE_LAG="5"),
+                                 dict(FUSED, THINK_PRUNE_HINTS="7", THINK_PRUNE_PREFETCH="8"),
+                                 {"THINK_SCORE_PLAN_ROUNDS": "1", "THINK_SCORE_TMA": "0"},
                                  {"THINK_SCORE_TMA": "0"},
                                  {"THINK_SCORE_STAGES": "2"},
                                  {"THINK_SCORE_STAGES": "8"},
@@ -470,13 +473,14 @@ PRUNE_ENV_KEYS = ("THINK_PRUNE_FUSED", "THINK_PRUNE_STAGES", "THINK_PRUNE_CSTAGE
                                  {"THINK_COMPACT_STAGES": "8", "THINK_COMPACT_TILES": "37"}])
 def test_prune_schedules_give_identical_results(env, monkeypatch):
     # the default two-launch prune (TMA-staged score and compaction tiles)
-    # against the one-kernel prune (which compacts each round of heads from L2
-    # while it scores the next; several ring depths, lags, L2 hints and
-    # prefetch distances), the register-pipelined score and compaction kernels,
-    # other ring depths and run lengths: bit for bit the same (same split plan,
-    # same order of additions, pure copies).  Shapes: one round, several rounds
-    # of one and of several heads (two runs per block), a head too long for the
-    # one-kernel prune (two launches on both sides)
+    # against the register-pipelined score and compaction kernels, other ring
+    # depths and run lengths, and -- on the round split plan, which the
+    # one-kernel prune needs -- the one-kernel prune (which compacts each round
+    # of heads from L2 while it scores the next; several ring depths, lags, L2
+    # hints and prefetch distances): bit for bit the same for the same split
+    # plan (same order of additions, pure copies).  Shapes: one round, several
+    # rounds of one and of several heads (two runs per block), a head too long
+    # for the one-kernel prune (two launches on both sides)
     shapes = [(2, 32, 8, 5000, 64), (1, 8, 1, 70, 51), (4, 4, 4, 3000, 128), (3, 16, 8, 1, 1),
               (1, 32, 8, 40000, 51), (2, 32, 8, 60000, 51), (1, 8, 2, 200000, 40)]
     for i, (B, Hq, Hkv, N, T) in enumerate(shapes):
@@ -485,6 +489,8 @@ def test_prune_schedules_give_identical_results(env, monkeypatch):
         qd = q_win.to(DEV)
         for key in PRUNE_ENV_KEYS:
             monkeypatch.delenv(key, raising=False)
+        if "THINK_SCORE_PLAN_ROUNDS" in env:  # the reference uses the same split plan
+            monkeypatch.setenv("THINK_SCORE_PLAN_ROUNDS", env["THINK_SCORE_PLAN_ROUNDS"])
         a = _prune_gpu(qd, kd, T)
         for key, val in env.items():
             monkeypatch.setenv(key, val)
