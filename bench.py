@@ -37,9 +37,11 @@ NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the
 # default bf16 decode kernel, pruned_decode_mma_kernel<4, 4>, on the long-context
-# workload, from one ncu capture of that kernel; reported only for that
-# workload and to be reset to None whenever the kernel changes.
-DECODE_TRAFFIC_BYTES = 375_460_352 + 3_624_192
+# workload: the capture of the 101st launch in a step's back-to-back loop with
+# ncu's cache control off (profiles/pruned_decode_mma_kernel_mistral7b_long.md,
+# "In the back-to-back loop"); reported only for that workload and to be reset
+# to None whenever the kernel changes.
+DECODE_TRAFFIC_BYTES = 375_458_048 + 9_862_144
 
 
 def parse():
