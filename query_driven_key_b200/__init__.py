@@ -157,6 +157,9 @@ def _stream(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(stream.cuda_stream)
 
 
+_raw_stream = torch._C._cuda_getCurrentRawStream  # device index -> current stream handle
+
+
 def _strides3(t: torch.Tensor):
     if t.dim() != 4 or t.stride(3) != 1:
         raise ThinkError(THINK_ERR_INVALID_ARG, "expected a [B,H,N,d] tensor with contiguous channels")
@@ -252,7 +255,9 @@ def think_pruned_decode_attn(q: torch.Tensor, k_pruned: torch.Tensor, ldk: int, 
     T = idx.shape[-1]
     if scale is None:
         scale = 1.0 / float(d) ** 0.5
-    if not q.is_contiguous() or out.dtype != torch.float32 or idx.dtype != torch.int32:
+    if not q.is_contiguous() or out.dtype != torch.float32 or idx.dtype != torch.int32 \
+            or not out.is_contiguous() or tuple(out.shape) != (B, Hq, d) \
+            or not (q.is_cuda and k_pruned.is_cuda and v.is_cuda and idx.is_cuda and out.is_cuda):
         raise ThinkError(THINK_ERR_INVALID_ARG, "think_pruned_decode_attn")
     _check(lib.think_pruned_decode_attn(_ptr(q), _ptr(k_pruned), int(ldk), _ptr(v), _strides3(v),
                                         _ptr(idx), B, Hq, Hkv, N, d, T, _dtype(q), float(scale),
@@ -563,25 +568,28 @@ class PrunedCache:
     def decode(self, q, v, out, scale=None, stream=None):
         """Attend over the current n tokens (v holds at least n token rows).
 
-        The arguments that do not change between decode steps (this cache's
-        buffers, V's address and strides, the scale) are marshalled once and
-        reused while V and the scale stay the same."""
-        key = (v.data_ptr(), v.stride(), tuple(v.shape), v.dtype, scale)
-        if key != getattr(self, "_dkey", None):
-            think_pruned_decode_attn(q, self.k_pruned, self.ldk, v, self.idx, out, self.decode_ws,
-                                     scale=scale, N=self.n, stream=stream)
-            d = q.shape[-1]
-            self._dconst = (self.k_pruned.data_ptr(), int(self.ldk), v.data_ptr(), _strides3(v),
-                            self.idx.data_ptr(), _dtype(q),
-                            float(1.0 / float(d) ** 0.5 if scale is None else scale),
-                            self.decode_ws.data_ptr(), self.decode_ws.numel())
-            self._dshape = (tuple(q.shape), q.dtype, tuple(out.shape))
-            self._dkey = key
+        Decode steps are short (a few microseconds on the device for short
+        caches), so the host path matters: the arguments that do not change
+        between steps (this cache's buffers, V's address, shape and strides,
+        the scale, the shapes of q and out) are checked and marshalled on the
+        first call, and later calls with the same V tensor and scale only check
+        q and out against them and pass their addresses."""
+        f = getattr(self, "_dfast", None)
+        if f is not None and v is f[0] and scale == f[1] and v.data_ptr() == f[2] and v.shape == f[3] \
+                and q.shape == f[4] and out.shape == f[4] and q.dtype == self.dtype \
+                and out.dtype == torch.float32 and q.is_contiguous() and out.is_contiguous() \
+                and q.is_cuda and out.is_cuda:
+            rc = lib.think_pruned_decode_attn(
+                q.data_ptr(), f[5], f[6], f[2], f[7], f[8], self.B, self.Hq, self.Hkv, self.n, self.d, self.T,
+                f[9], f[10], out.data_ptr(), f[11], f[12],
+                _raw_stream(f[13]) if stream is None else stream.cuda_stream)
+            if rc != THINK_OK:
+                raise ThinkError(rc, "think_pruned_decode_attn")
             return
-        if (tuple(q.shape), q.dtype, tuple(out.shape)) != self._dshape or not q.is_contiguous() \
-                or out.dtype != torch.float32:
-            raise ThinkError(THINK_ERR_INVALID_ARG, "PrunedCache.decode")
-        kp, ldk, vp, vs, ip, dt, sc, wp, wb = self._dconst
-        _check(lib.think_pruned_decode_attn(q.data_ptr(), kp, ldk, vp, vs, ip, self.B, self.Hq, self.Hkv, self.n,
-                                            self.d, self.T, dt, sc, out.data_ptr(), wp, wb, _stream(stream)),
-               "think_pruned_decode_attn")
+        think_pruned_decode_attn(q, self.k_pruned, self.ldk, v, self.idx, out, self.decode_ws,
+                                 scale=scale, N=self.n, stream=stream)
+        d = q.shape[-1]
+        self._dfast = (v, scale, v.data_ptr(), v.shape, q.shape, self.k_pruned.data_ptr(), int(self.ldk),
+                       _strides3(v), self.idx.data_ptr(), _dtype(q),
+                       float(1.0 / float(d) ** 0.5 if scale is None else scale),
+                       self.decode_ws.data_ptr(), self.decode_ws.numel(), self.k_pruned.device.index)

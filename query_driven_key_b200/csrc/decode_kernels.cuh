@@ -44,6 +44,8 @@ struct DecodeArgs {
     int prefetch;           // tiles prefetched into L2 ahead of the TMA loads
     int early;              // 1: the first tiles are prefetched into L2 before the dependency wait
     int staged_merge;       // 1: the split merge copies the partial outputs into shared memory when they fit
+    int cluster;            // warp-MMA decode: > 0 when the splits of a head form one thread-block
+                            // cluster of that many blocks and merge through distributed shared memory
     float scale_log2;       // scale * log2(e)
     uint32_t stage_bytes;   // bytes per ring stage (multiple of 1024)
     uint32_t v_off;         // offset of the V tile inside a stage

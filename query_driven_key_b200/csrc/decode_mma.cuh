@@ -263,8 +263,67 @@ __device__ __forceinline__ void mma_tile(uint32_t kbase, uint32_t k_half, uint32
     (void)q4;
 }
 
+// The split merge of a head whose splits form one thread-block cluster (the
+// producer warp calls it too, with tid >= NT, for the cluster barriers): each
+// block puts its (O, max, sum) in its own shared memory (`scratch`); after a
+// cluster barrier, block r of S merges output channels [r * 128 / S, ...) of
+// every query head of the group from all S blocks' shared memory, in split
+// order, and writes them; a second barrier keeps every block's shared memory
+// alive until the reads are done.  No global partials, no ticket.
+template <int G, int NT>
+__device__ __forceinline__ void cluster_finish(const DecodeArgs &a, const float (&O)[G], const float (&M)[G],
+                                               const float (&L)[G], float *scratch, int b, int kv, int tid)
+{
+    float *co = scratch;            // [G][128]
+    float *cml = scratch + G * kD;  // [G][2]
+    if (tid < kD) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) co[g * kD + tid] = O[g];
+        if (tid == 0) {
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                cml[2 * g] = M[g];
+                cml[2 * g + 1] = L[g];
+            }
+        }
+    }
+    cluster_sync_all();
+    const int S = a.cluster;
+    const int per = kD / S;  // S divides 128
+    const uint32_t r = cluster_rank();
+    for (int i = tid; i < G * per && tid < NT; i += NT) {
+        const int g = i / per, c = (int)r * per + i % per;
+        float ms[16], ls[16], os[16];  // all loads first, so that their latencies overlap
+#pragma unroll
+        for (int s2 = 0; s2 < 16; ++s2) {
+            if (s2 < S) {
+                ms[s2] = ld_dsmem_f32(cml + 2 * g, (uint32_t)s2);
+                ls[s2] = ld_dsmem_f32(cml + 2 * g + 1, (uint32_t)s2);
+                os[s2] = ld_dsmem_f32(co + g * kD + c, (uint32_t)s2);
+            }
+        }
+        float Mx = -INFINITY;
+#pragma unroll
+        for (int s2 = 0; s2 < 16; ++s2)
+            if (s2 < S) Mx = fmaxf(Mx, ms[s2]);
+        float o = 0.f, l = 0.f;
+#pragma unroll
+        for (int s2 = 0; s2 < 16; ++s2) {
+            if (s2 < S && ms[s2] != -INFINITY) {  // an empty split holds (0, -inf, 0)
+                const float w = exp2_approx(ms[s2] - Mx);
+                o = fmaf(os[s2], w, o);
+                l = fmaf(ls[s2], w, l);
+            }
+        }
+        const int64_t hq = (int64_t)b * a.Hq + (int64_t)kv * G + g;
+        if (THINK_IN_RANGE(hq < (int64_t)gridDim.y / a.Hkv * a.Hq, a.status)) a.out[hq * kD + c] = o / l;
+    }
+    cluster_sync_all();
+}
+
 // Merge the CW consumer warps of the block (through mo/mml in shared
-// memory), then the split merge (finish_split, which reuses `scratch`).
+// memory), then the split merge (finish_split, which reuses `scratch`, or
+// cluster_finish when the head's splits form a cluster).
 template <int G, int CW>
 __device__ __forceinline__ void mma_merge_and_finish(const DecodeArgs &a, MmaState &S, float *mo, float *mml,
                                                      float *scratch, unsigned *flag, int head, int split,
@@ -313,6 +372,10 @@ __device__ __forceinline__ void mma_merge_and_finish(const DecodeArgs &a, MmaSta
         }
     }
     named_barrier(1, CW * 32);  // the split merge below reuses stage memory
+    if (a.cluster > 0) {
+        cluster_finish<G, CW * 32>(a, O, M, Lsum, scratch, b, kv, tid);
+        return;
+    }
     finish_split<G, CW * 32>(a, head, split, b, kv, tid, O, M, Lsum, scratch, flag, 1, scratch_floats);
 }
 
@@ -452,6 +515,11 @@ __global__ void __launch_bounds__(CW * 32 + 32)
                     mbar_wait_bounded(full0 + 8 * (it % stages), (it / stages) & 1, a.status,
                                       THINK_DEVICE_TIMEOUT_FULL);
             }
+        }
+        __syncwarp();
+        if (a.cluster > 0) {  // the cluster barriers count every thread of every block
+            const float z[G] = {};
+            cluster_finish<G, NT>(a, z, z, z, reinterpret_cast<float *>(smem), b, kv, tid);
         }
         return;
     }

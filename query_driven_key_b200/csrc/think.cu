@@ -71,21 +71,41 @@ inline think_status_t launch_status()
 // Launch with programmatic stream serialisation (the kernel may start while
 // the previous kernel of the stream drains; it waits in griddepcontrol.wait
 // before its first global access).  THINK_PDL=0 launches plainly.
+// With cluster > 0, blocks (x, y) .. (x + cluster - 1, y), x a multiple of
+// cluster, form one thread-block cluster.
 template <typename... KArgs, typename... Args>
-think_status_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
-                          Args &&...args)
+think_status_t launch_pdl_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                  int cluster, Args &&...args)
 {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    if (cluster > 0) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = (unsigned)cluster;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    if (env_int("THINK_PDL", 1, 0, 1)) {
+        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = env_int("THINK_PDL", 1, 0, 1);
+    cfg.numAttrs = n;
     return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) == cudaSuccess ? THINK_OK : THINK_ERR_CUDA;
+}
+
+template <typename... KArgs, typename... Args>
+think_status_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                          Args &&...args)
+{
+    return launch_pdl_cluster(kern, grid, block, smem, st, 0, std::forward<Args>(args)...);
 }
 
 // ---------------------------------------------------------------- plans --
@@ -768,15 +788,97 @@ MmaPlan plan_decode_mma(int T, int G, int64_t heads, int64_t N)
     return p;
 }
 
+// Clusters of `cluster` blocks of `kern` (threads, bytes of shared memory)
+// that can be resident at once on this device; 0 if the launch cannot form
+// them.  Cached per kernel, device, cluster size and shared-memory size.
+int max_active_clusters(const void *kern, int cluster, int threads, size_t bytes)
+{
+    struct Entry {
+        const void *kern;
+        int dev, cluster;
+        size_t bytes;
+        int n;
+    };
+    thread_local Entry seen[32];
+    thread_local int nseen = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    for (int i = 0; i < nseen; ++i)
+        if (seen[i].kern == kern && seen[i].dev == dev && seen[i].cluster == cluster && seen[i].bytes == bytes)
+            return seen[i].n;
+    int n = 0;
+    if (cluster <= 8 ||
+        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)cluster, 1, 1);
+        cfg.blockDim = dim3((unsigned)threads, 1, 1);
+        cfg.dynamicSmemBytes = bytes;
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeClusterDimension;
+        attr.val.clusterDim.x = (unsigned)cluster;
+        attr.val.clusterDim.y = 1;
+        attr.val.clusterDim.z = 1;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) n = 0;
+    }
+    (void)cudaGetLastError();  // a refused size is an answer (0), not an error of the next launch
+    Entry &e = seen[nseen < 32 ? nseen++ : (cluster * 7 + (int)bytes) % 32];
+    e.kern = kern;
+    e.dev = dev;
+    e.cluster = cluster;
+    e.bytes = bytes;
+    e.n = n;
+    return n;
+}
+
+// The split merge through a thread-block cluster serves short heads: each
+// head becomes one cluster of S blocks (S a power of two, 2..16) that merges
+// its split partials in distributed shared memory (no global partials, no
+// ticket), when
+//   - a split reads at most kClusterTilesMax tiles (longer heads keep the
+//     global merge, whose cost is small beside their stream),
+//   - all heads' clusters are resident at once, and
+//   - the busiest SM streams no more tiles than under the global merge's
+//     split (tiles per block x blocks per SM, blocks spread evenly), so that
+//     the coarser split costs no bandwidth.
+// The largest such S below twice the head's tiles is taken (a split may be
+// empty).  THINK_DECODE_CLUSTER caps S (0: never; tuning and tests).
+constexpr int kClusterTilesMax = 8;
+
+int plan_decode_cluster(const void *kern, int threads, size_t bytes, int64_t heads, int64_t N,
+                        int global_splits, int global_tps)
+{
+    const int cap = env_int("THINK_DECODE_CLUSTER", 16, 0, 16);
+    const int64_t tiles = ceil_div(N, kBN);
+    const int64_t sms = device_sm_count();
+    if (sms < 1) return 0;
+    const int64_t global_load = (int64_t)global_tps * ceil_div(heads * global_splits, sms);
+    for (int S = 16; S >= 2; S /= 2) {
+        if (S > cap || S >= 2 * tiles) continue;  // no cluster of one tile; S < 2 x tiles
+        const int64_t tps = ceil_div(tiles, S);
+        if (tps > kClusterTilesMax || tps * ceil_div(heads * S, sms) > global_load) continue;
+        if ((int64_t)max_active_clusters(kern, S, threads, bytes) >= heads) return S;
+    }
+    return 0;
+}
+
 template <int G, int CW>
-think_status_t launch_decode_mma_gw(const CUtensorMap &mk, const CUtensorMap &mv, const DecodeArgs &a,
+think_status_t launch_decode_mma_gw(const CUtensorMap &mk, const CUtensorMap &mv, DecodeArgs a,
                                     size_t bytes, int heads, cudaStream_t st)
 {
     auto kern = pruned_decode_mma_kernel<G, CW>;
     if (!ensure_smem(reinterpret_cast<const void *>(kern), bytes))
         return THINK_ERR_CUDA;
+    const int S = plan_decode_cluster(reinterpret_cast<const void *>(kern), CW * 32 + 32, bytes, heads, a.N,
+                                      a.splits, a.tiles_per_split);
+    if (S > 0) {  // one cluster of S splits per head (a split may be empty)
+        a.cluster = S;
+        a.splits = S;
+        a.tiles_per_split = (int)ceil_div(ceil_div(a.N, kBN), S);
+    }
     dim3 grid(a.splits, heads);
-    return launch_pdl(kern, grid, dim3(CW * 32 + 32), bytes, st, mk, mv, a);
+    return launch_pdl_cluster(kern, grid, dim3(CW * 32 + 32), bytes, st, S, mk, mv, a);
 }
 
 template <int G>

@@ -1,6 +1,6 @@
 """GPU parity: the CUDA path (through the C ABI) against the fp64 CPU oracle.
 
-Every input comes from the seeded generators in query_driven_key_b200.workloads;
+Every input comes from the seeded generators in workloads.py;
 every expected value comes from the oracle on the same (bf16-rounded) inputs.
 Kept channels and the thinner key cache must match bit for bit (near-ties at the
 cut excepted, see tests/helpers.py); decode outputs within the stated
@@ -526,6 +526,58 @@ def test_every_bf16_decode_kernel(kernel, monkeypatch):
         wg = w.with_(Hq=Hq, N=3000)
         q_win, k, v = W.gen_layer(wg)
         _full_path_check(wg, q_win, k, v, steps=[0])
+
+
+# (B, Hq, Hkv, N): the 32-layer sweep's layer (8 heads of 64 tiles), the
+# llama2-shaped MHA layer (32 heads of 32 tiles), 9 tiles (clusters of up to
+# 16 with empty splits), 3 tiles with a ragged tail (16 heads: clusters of 4,
+# which are always resident).  Whether the first three use clusters depends
+# on how many clusters of a size the device keeps resident.
+CLUSTER_SHAPES = [(1, 32, 8, 8192), (1, 32, 32, 4096), (1, 64, 8, 1100), (2, 16, 8, 300)]
+
+
+@pytest.mark.parametrize("warps", ["4", "8"])
+@pytest.mark.parametrize("shape", CLUSTER_SHAPES)
+def test_cluster_split_merge(shape, warps, monkeypatch):
+    # The warp-MMA decode merges a short head's splits inside a thread-block
+    # cluster (distributed shared memory): every cluster size cap gives the
+    # oracle's output within tolerance, and the capped-off global merge (cap 0)
+    # too.  With clusters on, the workspace's split partials stay untouched.
+    for key in ("THINK_DECODE_TENSOR_CORES", "THINK_DECODE_CUDA_CORES"):
+        monkeypatch.delenv(key, raising=False)
+    monkeypatch.setenv("THINK_DECODE_WARPS", warps)
+    B, Hq, Hkv, N = shape
+    w = W.WORKLOADS["sweep_32l"].with_(B=B, Hq=Hq, Hkv=Hkv, N=N, layers=1)
+    q_win, k, v = W.gen_layer(w)
+    T = qdk.think_t_from_lambda(w.d, w.lam)
+    ora_scores, ora_idx, ora_kp = oracle.oracle_prune(f64(q_win), f64(k), T)
+    cache = _prune_gpu(q_win.to(DEV), k.to(DEV), T)
+    cache.idx.copy_(torch.from_numpy(ora_idx))
+    qdk.think_compact_keys(k.to(DEV), cache.idx, cache.k_pruned, cache.ldk)
+    q = W.gen_decode_q(w, 0)
+    ora = oracle.oracle_decode(f64(q), ora_kp, f64(v), ora_idx)
+    vd, qd = v.to(DEV), q.to(DEV)
+    heads = B * Hkv
+    part0 = 256 + (heads * 4 + 255) // 256 * 256  # status header, tickets, then the partials
+    outs = {}
+    for cap in ["0", "2", "4", "8", "16"]:
+        monkeypatch.setenv("THINK_DECODE_CLUSTER", cap)
+        ws = torch.empty(qdk.think_decode_workspace_size(B, Hq, Hkv, N), dtype=torch.uint8, device=DEV)
+        qdk.think_workspace_init(ws)
+        ws[part0:].fill_(0xA5)
+        out = torch.full((B, Hq, w.d), float("nan"), dtype=torch.float32, device=DEV)
+        for _ in range(2):  # the same workspace twice
+            qdk.think_pruned_decode_attn(qd, cache.k_pruned, cache.ldk, vd, cache.idx, out, ws)
+        torch.cuda.synchronize()
+        assert qdk.think_read_device_status(ws) == 0
+        check_out(out, ora, w.dtype, where=f"cluster cap {cap}")
+        untouched = bool(torch.all(ws[part0:] == 0xA5))
+        if cap == "0":
+            assert not untouched, "the global merge writes split partials"
+        elif cap in ("4", "16") and shape == (2, 16, 8, 300):
+            assert untouched, "a clustered decode writes no split partials"
+        outs[cap] = out.clone()
+    monkeypatch.delenv("THINK_DECODE_CLUSTER")
 
 
 def test_scores_are_deterministic():
