@@ -43,6 +43,13 @@
  *   - Inputs must be finite; selection on NaN/Inf keys is unspecified.
  *   - Calls on different streams with disjoint buffers may run concurrently;
  *     calls that share a workspace must be stream-ordered.
+ *   - Workspaces hold arrival counters that every call leaves at zero; where
+ *     they sit depends on the call's shape (and, in a score workspace, on the
+ *     split plan).  One workspace may serve calls of any shape it is large
+ *     enough for: the library remembers, per workspace address, where the
+ *     counters of the last call on it were, and when a call's counters sit
+ *     elsewhere it zeroes them first (a memset on the call's stream).  The
+ *     first call on an address relies on think_workspace_init.
  */
 #ifndef THINK_H_
 #define THINK_H_
@@ -107,8 +114,8 @@ int64_t think_pruned_ld(int64_t N, think_dtype_t dtype);
  *   scores    [B][Hkv][d] fp64 output, contiguous.
  *   workspace device scratch of at least think_score_workspace_size() bytes,
  *             16-byte aligned, zeroed once by think_workspace_init before its
- *             first use (it starts with per-head arrival counters that every
- *             call leaves at zero; the rest is scratch).
+ *             first use (it holds arrival counters that every call leaves at
+ *             zero, see the workspace rule above; the rest is scratch).
  * One kernel launch.  Bit-for-bit deterministic for a given shape (fixed
  * summation order).  N == 0 or S_obs == 0 gives all-zero scores. */
 size_t think_score_workspace_size(int B, int Hq, int Hkv, int64_t N, int d);
@@ -363,7 +370,8 @@ think_status_t think_select_tokens(const float *mass, int B, int Hkv, int64_t N,
 think_status_t think_gather_tokens(const void *x, const int64_t x_strides[3], int B, int Hkv, int64_t N, int d,
                                    think_dtype_t dtype, const int32_t *kept, int M, void *out, void *stream);
 
-/* Zero a score or decode workspace (stream-ordered memset). */
+/* Zero a score or decode workspace (stream-ordered memset); the library
+ * forgets the counter place it remembered for this address. */
 think_status_t think_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
 
 /* Copy the device status bits of a decode or score workspace (its first 4

@@ -565,8 +565,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         fence_barrier_init();
     }
     __syncthreads();
-    // everything the previous kernel of the stream wrote is visible
-    grid_dependency_wait();
 
     if (warp < 8) {
         pf_score(a, m);

@@ -11,6 +11,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <unordered_map>
 #include <utility>
 
 #include "decode_kernels.cuh"
@@ -66,6 +67,43 @@ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline think_status_t launch_status()
 {
     return cudaGetLastError() == cudaSuccess ? THINK_OK : THINK_ERR_CUDA;
+}
+
+// Arrival counters.  Several kernels count arrivals (blocks of a head, runs of
+// a group) in counters that live in the caller's workspace and that every
+// call leaves at zero.  Where they sit depends on the call's shape (B x Hkv,
+// N) and, in a score workspace, on its split plan; a workspace reused for a
+// call whose counters sit elsewhere may hold the earlier call's scratch
+// values there.  So the library remembers, per workspace address, the byte
+// range of the counters of the last call made on it, and zeroes the new range
+// first (a memset in stream order) when it differs.  The first call on an
+// address relies on think_workspace_init, which also forgets the address.
+std::mutex g_counters_mu;
+std::unordered_map<const void *, std::pair<size_t, size_t>> g_counters;
+
+think_status_t ready_counters(void *ws, size_t begin, size_t end, cudaStream_t st)
+{
+    if (end <= begin) return THINK_OK;
+    {
+        std::lock_guard<std::mutex> lock(g_counters_mu);
+        auto it = g_counters.find(ws);
+        if (it == g_counters.end()) {
+            if (g_counters.size() >= 65536) g_counters.clear();
+            g_counters.emplace(ws, std::make_pair(begin, end));
+            return THINK_OK;
+        }
+        if (it->second == std::make_pair(begin, end)) return THINK_OK;
+        it->second = std::make_pair(begin, end);
+    }
+    return cudaMemsetAsync(static_cast<unsigned char *>(ws) + begin, 0, end - begin, st) == cudaSuccess
+               ? THINK_OK
+               : THINK_ERR_CUDA;
+}
+
+void forget_counters(const void *ws)
+{
+    std::lock_guard<std::mutex> lock(g_counters_mu);
+    g_counters.erase(ws);
 }
 
 // Launch with programmatic stream serialisation (the kernel may start while
@@ -548,6 +586,7 @@ think_status_t launch_score(const void *q_win, const void *k, const int64_t k_st
     a.S = S_obs;
     a.N = N;
     set_score_ws(a, ws, w, p);
+    if (ready_counters(ws, w.ready, w.qn2, st) != THINK_OK) return THINK_ERR_CUDA;
     a.scores = scores;
     a.T = T;
     a.idx = idx;
@@ -716,6 +755,7 @@ think_status_t launch_prune_fused(const void *q_win, const void *k, const int64_
     a.sc.S = S_obs;
     a.sc.N = N;
     set_score_ws(a.sc, ws, w, p);
+    if (ready_counters(ws, w.ready, w.qn2, st) != THINK_OK) return THINK_ERR_CUDA;
     a.sc.scores = scores;
     a.sc.T = T;
     a.sc.idx = idx;
@@ -747,7 +787,20 @@ think_status_t launch_prune_fused(const void *q_win, const void *k, const int64_
     if (sms < 1) return THINK_ERR_CUDA;
     const int64_t runs_per_round = (int64_t)p.hpr * p.splits;
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(sms * occ, runs_per_round));
-    return launch_pdl(prune_fused_kernel, dim3(grid), dim3(kPfThreads), bytes, st, mk, a);
+    // A cooperative launch: the runtime starts the grid only when every block
+    // can be resident at once (else the launch fails), so that no block waits
+    // on a flag of a block that has not been scheduled.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kPfThreads);
+    cfg.dynamicSmemBytes = bytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, prune_fused_kernel, mk, a) == cudaSuccess ? THINK_OK : THINK_ERR_CUDA;
 }
 
 
@@ -1301,6 +1354,9 @@ think_status_t launch_decode_f64(const void *q, const void *k_pruned, int64_t ld
     a.idx = idx;
     a.out = out;
     a.tickets = reinterpret_cast<unsigned *>(ws + kDecodeHeader);
+    if (ready_counters(ws, kDecodeHeader, kDecodeHeader + align_up((size_t)heads * sizeof(unsigned), 256),
+                       st) != THINK_OK)
+        return THINK_ERR_CUDA;
     a.part_o = reinterpret_cast<double *>(ws + kDecodeHeader + align_up((size_t)heads * sizeof(unsigned), 256));
     a.part_ml = a.part_o + slots * kD;
     a.Hq = Hq;
@@ -1398,6 +1454,9 @@ think_status_t think_pruned_decode_attn(const void *q, const void *k_pruned, int
     a.idx = idx;
     a.status = reinterpret_cast<unsigned *>(ws);
     a.tickets = reinterpret_cast<unsigned *>(ws + kDecodeHeader);
+    if (ready_counters(ws, kDecodeHeader, kDecodeHeader + align_up((size_t)heads * sizeof(unsigned), 256),
+                       static_cast<cudaStream_t>(stream)) != THINK_OK)
+        return THINK_ERR_CUDA;
     a.part_o = reinterpret_cast<float *>(ws + kDecodeHeader +
                                          align_up((size_t)heads * sizeof(unsigned), 256));
     a.out = out;
@@ -1504,6 +1563,9 @@ think_status_t think_pruned_decode_attn_q4(const void *q, const uint8_t *codes, 
     a.idx = idx;
     a.status = reinterpret_cast<unsigned *>(ws);
     a.tickets = reinterpret_cast<unsigned *>(ws + kDecodeHeader);
+    if (ready_counters(ws, kDecodeHeader, kDecodeHeader + align_up((size_t)heads * sizeof(unsigned), 256),
+                       static_cast<cudaStream_t>(stream)) != THINK_OK)
+        return THINK_ERR_CUDA;
     a.part_o = reinterpret_cast<float *>(ws + kDecodeHeader + align_up((size_t)heads * sizeof(unsigned), 256));
     a.out = out;
     a.part_ml = a.part_o + slots * kD;
@@ -1630,6 +1692,9 @@ think_status_t think_pruned_decode_attn_ragged(const void *q, const void *k_prun
     a.idx = idx;
     a.status = reinterpret_cast<unsigned *>(ws);
     a.tickets = reinterpret_cast<unsigned *>(ws + kDecodeHeader);
+    if (ready_counters(ws, kDecodeHeader, kDecodeHeader + align_up((size_t)heads * sizeof(unsigned), 256),
+                       static_cast<cudaStream_t>(stream)) != THINK_OK)
+        return THINK_ERR_CUDA;
     a.part_o = reinterpret_cast<float *>(ws + kDecodeHeader + align_up((size_t)heads * sizeof(unsigned), 256));
     a.out = out;
     a.part_ml = a.part_o + slots * kD;
@@ -1702,6 +1767,7 @@ think_status_t think_token_mass(const void *q_win, const void *k, const int64_t 
     a.status = reinterpret_cast<unsigned *>(ws);
     a.mass = mass;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (ready_counters(ws, w.tickets, w.part, st) != THINK_OK) return THINK_ERR_CUDA;
     switch (p.ntw) {
     case 1: return launch_mass<1>(mk, a, p, (int)heads, st);
     case 2: return launch_mass<2>(mk, a, p, (int)heads, st);
@@ -1743,6 +1809,7 @@ think_status_t think_select_tokens(const float *mass, int B, int Hkv, int64_t N,
     a.kept = kept;
     a.heads = (int)heads;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (ready_counters(ws, w.hist, w.sel, st) != THINK_OK) return THINK_ERR_CUDA;
     const dim3 grid((unsigned)w.chunks, (unsigned)heads);
     select_hist_kernel<0><<<grid, kSelThreads, 0, st>>>(a);
     select_hist_kernel<1><<<grid, kSelThreads, 0, st>>>(a);
@@ -1783,6 +1850,7 @@ think_status_t think_workspace_init(void *workspace, size_t workspace_bytes, voi
 {
     if (!workspace) return THINK_ERR_INVALID_ARG;
     if (workspace_bytes == 0) return THINK_OK;
+    forget_counters(workspace);
     return cudaMemsetAsync(workspace, 0, workspace_bytes, static_cast<cudaStream_t>(stream)) ==
                    cudaSuccess
                ? THINK_OK

@@ -507,6 +507,42 @@ def test_prune_schedules_give_identical_results(env, monkeypatch):
         assert np.array_equal(kp_logical(a.k_pruned, N), ora_kp)
 
 
+def test_one_workspace_serves_every_shape(monkeypatch):
+    # One score workspace and one decode workspace, sized for the largest
+    # shape, serve prunes (both prune paths, whose split plans differ) and
+    # decodes of several shapes in turn.  The arrival counters of each call sit
+    # where the previous call left scratch values; every call must still give
+    # the results of a fresh workspace, with a clear status.
+    shapes = [(1, 32, 8, 40000, 51), (2, 16, 8, 3000, 64), (1, 8, 2, 60000, 40), (1, 32, 8, 40000, 51)]
+    s_bytes = max(qdk.think_score_workspace_size(B, Hq, Hkv, N) for B, Hq, Hkv, N, _ in shapes)
+    d_bytes = max(qdk.think_decode_workspace_size(B, Hq, Hkv, N) for B, Hq, Hkv, N, _ in shapes)
+    sws = torch.empty(s_bytes, dtype=torch.uint8, device=DEV)
+    dws = torch.empty(d_bytes, dtype=torch.uint8, device=DEV)
+    qdk.think_workspace_init(sws)
+    qdk.think_workspace_init(dws)
+    for i, (B, Hq, Hkv, N, T) in enumerate(shapes):
+        q_win, k, v, q = _random_case(300 + i, B, Hq, Hkv, N, 32, torch.bfloat16)
+        qd, kd, vd, qq = q_win.to(DEV), k.to(DEV), v.to(DEV), q.to(DEV)
+        for fused in ("0", "1"):
+            monkeypatch.setenv("THINK_PRUNE_FUSED", fused)
+            fresh = _prune_gpu(qd, kd, T)
+            ref = torch.empty((B, Hq, 128), dtype=torch.float32, device=DEV)
+            fresh.decode(qq, vd, ref)
+            scores = torch.empty_like(fresh.scores)
+            idx = torch.empty_like(fresh.idx)
+            kp = torch.empty_like(fresh.k_pruned)
+            qdk.think_prune(qd, kd, T, scores, idx, kp, fresh.ldk, sws)
+            out = torch.empty_like(ref)
+            qdk.think_pruned_decode_attn(qq, kp, fresh.ldk, vd, idx, out, dws)
+            torch.cuda.synchronize()
+            assert qdk.think_read_device_status(sws) == 0 and qdk.think_read_device_status(dws) == 0
+            where = (B, Hq, Hkv, N, T, fused)
+            assert torch.equal(scores, fresh.scores) and torch.equal(idx, fresh.idx), where
+            assert torch.equal(kp[..., :N], fresh.k_pruned[..., :N]), where
+            assert torch.equal(out, ref), where
+    monkeypatch.delenv("THINK_PRUNE_FUSED")
+
+
 @pytest.mark.parametrize("kernel", ["warp_mma", "warp_mma_8_warps", "cuda_cores", "tensor_cores"])
 def test_every_bf16_decode_kernel(kernel, monkeypatch):
     # the bf16 decode kernels on the same inputs: warp-level mma (default; four
