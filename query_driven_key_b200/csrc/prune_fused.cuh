@@ -38,7 +38,9 @@
 //         as 16-byte writes.
 //     The ready flag of round r depends only on score work of round r, which
 //     no block delays behind its compaction of round r or later, and every
-//     block of the grid is resident (grid <= SMs), so every wait ends.
+//     block of the grid is resident (the grid is launched cooperatively, so
+//     the runtime starts it only when all its blocks fit at once), so every
+//     wait ends.
 // Every wait is bounded; after the first one that runs out the block stops
 // waiting (abort flag), still passes every barrier, and the producers let
 // their loads in flight land before the block ends.
