@@ -1018,9 +1018,12 @@ think_status_t launch_mass(const CUtensorMap &mk, const MassArgs &a, const MassP
 
 // ------------------------------------------------------------ 4-bit K' --
 
-// Two blocks per SM (eight consumer warps) first: the dequantisation makes
-// the consumers' latency, not the stream, the limit with four warps per SM
-// (long-context workload: 64 us at two blocks per SM, 94 us at one).
+// Two blocks per SM of four consumer warps (32 tokens each) first: with one
+// block per SM the dequantisation makes the consumers' latency, not the
+// stream, the limit; at two blocks per SM four consumer warps beat eight of 16
+// tokens, whose per-warp softmax and MMA set-up is paid twice per tile
+// (long-context workload: 54.5 us against 56.7 us with eight warps, 66-71 us
+// at one block per SM).
 MmaPlan plan_decode_q4(int T, int G, int64_t heads, int64_t N)
 {
     MmaPlan p;
@@ -1029,7 +1032,7 @@ MmaPlan plan_decode_q4(int T, int G, int64_t heads, int64_t N)
     const size_t per_block_2 = kSmemPerSM / 2 - kSmemReservedPerBlock;
     const int max_bps = env_int("THINK_DECODE_BLOCKS_PER_SM", 2, 1, 2);
     const int max_st = env_int("THINK_DECODE_STAGES", 6, 2, 6);
-    p.warps = consumer_warps(8);
+    p.warps = consumer_warps(4);
     for (int bps = max_bps; bps >= 1; --bps)
         for (int st = max_st; st >= 2; --st) {
             const size_t bytes = q4_smem_bytes(T, G, st, p.warps);
