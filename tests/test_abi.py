@@ -331,3 +331,23 @@ def test_score_workspace_follows_the_plans():
     assert _round_plan(32, 4096) == (8, 8, 32, 1)
     # the two-launch pass on the long-context layer: one wave of 432 runs of 38 tiles
     assert _wave_plans(8, 131072)[1] == 54
+
+
+def test_python_decode_checks_before_any_call():
+    # The binding rejects a decode whose output is not a contiguous [B, Hq, d]
+    # fp32 tensor, or whose tensors are not on the GPU, before it calls the
+    # library (CPU tensors here: nothing reaches the C entry point).
+    import torch
+    B, Hq, Hkv, N, T, d = 1, 4, 2, 64, 10, 128
+    q = torch.zeros((B, Hq, d), dtype=torch.bfloat16)
+    kp = torch.zeros((B, Hkv, T, 64), dtype=torch.bfloat16)
+    v = torch.zeros((B, Hkv, N, d), dtype=torch.bfloat16)
+    idx = torch.zeros((B, Hkv, T), dtype=torch.int32)
+    ws = torch.zeros(4096, dtype=torch.uint8)
+    bad_outs = [torch.zeros((B, Hq, d), dtype=torch.float32),                 # host memory
+                torch.zeros((B, Hq, 2 * d), dtype=torch.float32)[..., ::2],  # not contiguous
+                torch.zeros((B, Hq + 1, d), dtype=torch.float32),            # wrong shape
+                torch.zeros((B, Hq, d), dtype=torch.bfloat16)]               # wrong dtype
+    for out in bad_outs:
+        with pytest.raises(qdk.ThinkError):
+            qdk.think_pruned_decode_attn(q, kp, 64, v, idx, out, ws)
