@@ -860,8 +860,10 @@ int max_active_clusters(const void *kern, int cluster, int threads, size_t bytes
         if (seen[i].kern == kern && seen[i].dev == dev && seen[i].cluster == cluster && seen[i].bytes == bytes)
             return seen[i].n;
     int n = 0;
-    if (cluster <= 8 ||
-        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+    bool refused = false;
+    if (cluster > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+        refused = true;
+    if (!refused) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)cluster, 1, 1);
         cfg.blockDim = dim3((unsigned)threads, 1, 1);
@@ -873,9 +875,14 @@ int max_active_clusters(const void *kern, int cluster, int threads, size_t bytes
         attr.val.clusterDim.z = 1;
         cfg.attrs = &attr;
         cfg.numAttrs = 1;
-        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+            n = 0;
+            refused = true;
+        }
     }
-    (void)cudaGetLastError();  // a refused size is an answer (0), not an error of the next launch
+    // a refused size is an answer (0), not an error for the caller's next
+    // check: clear the error state that the refusing call left, and only then
+    if (refused) (void)cudaGetLastError();
     Entry &e = seen[nseen < 32 ? nseen++ : (cluster * 7 + (int)bytes) % 32];
     e.kern = kern;
     e.dev = dev;
