@@ -191,9 +191,13 @@ think_status_t think_prune(const void *q_win, const void *k, const int64_t k_str
  *     out    = sum_n softmax(z)[n] * V[b,h_kv,n,:]
  * Pass scale = 1/sqrt(d) (the full head width, not T) for the unpruned
  * model's temperature.  Split-N flash decoding in one kernel launch: tiles of
- * K' and V are staged in shared memory by TMA, each block writes a partial
- * (max, sum, weighted V) for its split to the workspace, and the last block
- * of each KV head to finish merges that head's partials into `out`.
+ * K' and V are staged in shared memory by TMA, each block forms a partial
+ * (max, sum, weighted V) for its split, and the partials of a KV head are
+ * merged into `out`: through the workspace by the head's last block to
+ * finish, or, for bf16 heads short enough that their splits form one
+ * thread-block cluster, through the blocks' shared memory (the workspace's
+ * partials are then not used).  fp32 caches are decoded with fp64 arithmetic
+ * after the loads (one rounding to fp32 at the end).
  *   q         [B][Hq][d] contiguous, dtype.
  *   k_pruned  thinner key cache with pitch ldk, as written by think_compact_keys.
  *   v         element (b,h,n,c) at v[b*v_strides[0] + h*v_strides[1] + n*v_strides[2] + c].
