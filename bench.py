@@ -207,6 +207,28 @@ def step_bytes(w, T):
     return W.prune_bytes(w, T) + w.decode_steps * W.decode_bytes(w, T)
 
 
+def measure_read_probe(dev, stream, gib=4, reps=10):
+    """Context for the decode's fraction of the copy peak: the read bandwidth
+    of a plain read-only stream (torch's max reduction, a library kernel, over
+    a buffer larger than L2), next to the driver's read+write copy peak."""
+    import torch
+    buf = torch.ones((gib << 30) // 4, dtype=torch.int32, device=dev)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            torch.amax(buf)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            torch.amax(buf)
+        e1.record(stream)
+    stream.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / reps
+    nbytes = buf.numel() * 4
+    del buf
+    return {"gbs": nbytes / (us * 1e-6) / 1e9, "bytes": nbytes,
+            "kernel": "torch.amax over a 4 GiB int32 buffer (read-only stream, library kernel; context only)"}
+
+
 def measure_append(w, T, dev, stream, qw_d, k_d, chunk=4096, reps=50):
     """Growing cache, outside the timed step: device time of appending one new
     token's keys (all heads) and a chunk of new tokens' keys to a pruned cache
@@ -627,6 +649,8 @@ def run_native(args):
                 if extras and w.dtype == torch.bfloat16 else None)
     evict = (measure_evict(w, T, dev, stream, qw_d[0], k_d[0], v_d[0], qs_d, outs[:, 0], peak)
              if extras and w.dtype == torch.bfloat16 else None)
+    read_probe = measure_read_probe(dev, stream) if extras else None
+    prune_1read, prune_2read = W.prune_bytes(w, T), W.prune_bytes(w, T, k_reads=2)
 
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -644,7 +668,10 @@ def run_native(args):
         "decode_pct_of_8tbs": achieved / NOMINAL_HBM_GBS * 100.0,
         "decode_us_per_step": dec_us,
         "prune_us_per_layer": prune_us,
-        "prune_gbs_1read": W.prune_bytes(w, T) / (prune_us * 1e-6) / 1e9,
+        "prune_gbs_1read": prune_1read / (prune_us * 1e-6) / 1e9,
+        "prune_frac_1read": prune_1read / (prune_us * 1e-6) / 1e9 / peak,
+        "prune_gbs_2read": prune_2read / (prune_us * 1e-6) / 1e9,
+        "prune_frac_2read": prune_2read / (prune_us * 1e-6) / 1e9 / peak,
         "roofline": {"kernel": f"{decode_kernel_name(w)} (think_pruned_decode_attn, one launch), "
                                f"CUDA events around each step's {w.decode_steps * R} decode calls",
                      "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
@@ -655,6 +682,7 @@ def run_native(args):
         "q4": q4,
         "adaptive": adaptive,
         "evict": evict,
+        "read_probe": read_probe,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
         "e2e": e2e,
