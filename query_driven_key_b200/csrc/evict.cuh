@@ -56,6 +56,31 @@ __host__ __device__ inline size_t mass_smem_bytes(int r_pad, int stages)
            (size_t)kMassWarps * kBN * 4u + (size_t)2 * stages * 8u + 16u + 1024u;
 }
 
+// Pass 1's end: the block's per-row (max, sum) partials are in a.part; the
+// head's last block (ticket) merges the splits in split order into
+// (max, 1 / sum) per row.  NT threads (tid < NT) take part, barrier 1.
+template <int NT>
+__device__ __forceinline__ void mass_merge_splits(const MassArgs &a, int head, int tid, unsigned *flag)
+{
+    __threadfence();
+    named_barrier(1, NT);
+    if (tid == 0) *flag = (atomicAdd(a.tickets + head, 1u) == (unsigned)(a.splits - 1)) ? 1u : 0u;
+    named_barrier(1, NT);
+    if (*flag == 0u) return;
+    __threadfence();
+    for (int r = tid; r < a.R; r += NT) {
+        float M = -INFINITY;
+        for (int s = 0; s < a.splits; ++s) M = fmaxf(M, __ldcg(a.part + ((int64_t)head * a.splits + s) * a.R + r).x);
+        float L = 0.f;
+        for (int s = 0; s < a.splits; ++s) {
+            const float2 p = __ldcg(a.part + ((int64_t)head * a.splits + s) * a.R + r);
+            if (p.x != -INFINITY) L = fmaf(p.y, exp2_approx(p.x - M), L);
+        }
+        a.stats[(int64_t)head * a.R + r] = make_float2(M, L > 0.f ? 1.f / L : 0.f);
+    }
+    if (tid == 0) a.tickets[head] = 0u;
+}
+
 // NTW: 8-row query groups per warp (r_pad = 64 * NTW).  With NTW <= 4 a warp
 // keeps the B fragments of its rows in registers for the whole block.
 template <int PASS, int NTW>
@@ -276,23 +301,7 @@ __global__ void __launch_bounds__(kMassThreads)
                 if (r8 == 0 && r < a.R)
                     a.part[((int64_t)head * a.splits + split) * a.R + r] = make_float2(m, l);
             }
-        __threadfence();
-        named_barrier(1, NT);
-        if (tid == 0) *flag = (atomicAdd(a.tickets + head, 1u) == (unsigned)(a.splits - 1)) ? 1u : 0u;
-        named_barrier(1, NT);
-        if (*flag == 0u) return;
-        __threadfence();
-        for (int r = tid; r < a.R; r += NT) {
-            float M = -INFINITY;
-            for (int s = 0; s < a.splits; ++s) M = fmaxf(M, __ldcg(a.part + ((int64_t)head * a.splits + s) * a.R + r).x);
-            float L = 0.f;
-            for (int s = 0; s < a.splits; ++s) {
-                const float2 p = __ldcg(a.part + ((int64_t)head * a.splits + s) * a.R + r);
-                if (p.x != -INFINITY) L = fmaf(p.y, exp2_approx(p.x - M), L);
-            }
-            a.stats[(int64_t)head * a.R + r] = make_float2(M, L > 0.f ? 1.f / L : 0.f);
-        }
-        if (tid == 0) a.tickets[head] = 0u;
+        mass_merge_splits<NT>(a, head, tid, flag);
     }
 }
 

@@ -19,6 +19,7 @@
 #include "decode_mma.cuh"
 #include "decode_q4.cuh"
 #include "evict.cuh"
+#include "mass_tc.cuh"
 #include "decode_tc.cuh"
 #include "prune_fused.cuh"
 #include "prune_kernels.cuh"
@@ -1023,6 +1024,52 @@ think_status_t launch_mass(const CUtensorMap &mk, const MassArgs &a, const MassP
     return launch_mass_kernel<2, NTW>(mk, a, p, heads, st);
 }
 
+// The token mass on tcgen05 (mass_tc.cuh): R <= 256 window rows in MB = 1 or
+// 2 blocks of 128, one block per SM, the deepest K ring (2..4 stages) that
+// fits.  stages == 0: it does not apply (THINK_MASS_TC=0 also turns it off).
+struct MassTcPlan {
+    int mb, stages;
+    size_t bytes;
+    DecodeSplit sp;
+};
+
+MassTcPlan plan_mass_tc(int R, int64_t heads, int64_t N)
+{
+    MassTcPlan p{};
+    if (R > 256 || env_int("THINK_MASS_TC", 1, 0, 1) == 0) return p;
+    p.mb = R <= 128 ? 1 : 2;
+    for (int st = 4; st >= 2; --st) {
+        const size_t bytes = p.mb == 1 ? mass_tc_smem_bytes<1>(st) : mass_tc_smem_bytes<2>(st);
+        if (bytes <= kSmemPerBlockMax) {
+            p.stages = st;
+            p.bytes = bytes;
+            break;
+        }
+    }
+    p.sp = plan_decode_split(heads, N, 1);
+    return p;
+}
+
+template <int PASS, int MB>
+think_status_t launch_mass_tc_kernel(const CUtensorMap &mk, const MassArgs &a, size_t bytes, int heads,
+                                     cudaStream_t st)
+{
+    auto kern = token_mass_tc_kernel<PASS, MB>;
+    if (!ensure_smem(reinterpret_cast<const void *>(kern), bytes))
+        return THINK_ERR_CUDA;
+    dim3 grid(a.splits, heads);
+    kern<<<grid, MassTc<MB>::kThreads, bytes, st>>>(mk, a);
+    return launch_status();
+}
+
+template <int MB>
+think_status_t launch_mass_tc(const CUtensorMap &mk, const MassArgs &a, size_t bytes, int heads, cudaStream_t st)
+{
+    const think_status_t v = launch_mass_tc_kernel<1, MB>(mk, a, bytes, heads, st);
+    if (v != THINK_OK) return v;
+    return launch_mass_tc_kernel<2, MB>(mk, a, bytes, heads, st);
+}
+
 // ------------------------------------------------------------ 4-bit K' --
 
 // Two blocks per SM of four consumer warps (32 tokens each) first: with one
@@ -1750,7 +1797,13 @@ think_status_t think_token_mass(const void *q_win, const void *k, const int64_t 
         return THINK_ERR_ALIGNMENT;
     const MassPlan p = plan_mass(R, heads, N);
     if (p.stages == 0) return THINK_ERR_UNSUPPORTED;
-    const MassWs w = mass_ws_layout(heads, R, p.sp.splits);
+    if (workspace_bytes < mass_ws_layout(heads, R, p.sp.splits).total) return THINK_ERR_WORKSPACE;
+    // tcgen05 kernels when they apply (their one block per SM never needs more
+    // splits, so the workspace sized for plan_mass holds their partials)
+    const MassTcPlan tp = plan_mass_tc(R, heads, N);
+    const bool use_tc = tp.stages > 0;
+    const DecodeSplit sp = use_tc ? tp.sp : p.sp;
+    const MassWs w = mass_ws_layout(heads, R, sp.splits);
     if (workspace_bytes < w.total) return THINK_ERR_WORKSPACE;
     CUtensorMap mk;
     // K as V is read by the decode: x = channel (two 64-channel halves), y = token
@@ -1767,9 +1820,9 @@ think_status_t think_token_mass(const void *q_win, const void *k, const int64_t 
     a.R = R;
     a.r_pad = p.r_pad;
     a.N = N;
-    a.tiles_per_split = p.sp.tiles_per_split;
-    a.splits = p.sp.splits;
-    a.stages = p.stages;
+    a.tiles_per_split = sp.tiles_per_split;
+    a.splits = sp.splits;
+    a.stages = use_tc ? tp.stages : p.stages;
     a.scale_log2 = scale * 1.4426950408889634f;
     a.part = reinterpret_cast<float2 *>(ws + w.part);
     a.stats = reinterpret_cast<float2 *>(ws + w.stats);
@@ -1778,6 +1831,9 @@ think_status_t think_token_mass(const void *q_win, const void *k, const int64_t 
     a.mass = mass;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (ready_counters(ws, w.tickets, w.part, st) != THINK_OK) return THINK_ERR_CUDA;
+    if (use_tc)
+        return tp.mb == 1 ? launch_mass_tc<1>(mk, a, tp.bytes, (int)heads, st)
+                          : launch_mass_tc<2>(mk, a, tp.bytes, (int)heads, st);
     switch (p.ntw) {
     case 1: return launch_mass<1>(mk, a, p, (int)heads, st);
     case 2: return launch_mass<2>(mk, a, p, (int)heads, st);
