@@ -22,7 +22,7 @@
 //           tokens (the sum rescaled only when the maximum grows), the two
 //           halves of a row merged at the end, then the head's last block
 //           merges the splits into (max, 1 / sum);
-//   pass 2: per row the weights 2^(z - max) / sum; the weights of a token are
+//   pass 2: per row the weights 2^(z - max - log2(sum)); the weights of a token are
 //           summed over rows by a butterfly reduce-scatter across the 32 lanes
 //           of a warp (lane L ends with tokens 2L, 2L + 1 of its half, summed
 //           over its warp's 32 rows), then over the warps in a fixed order.
@@ -201,7 +201,10 @@ __global__ void __launch_bounds__(MassTc<MB>::kThreads, 1)
         const int row = 128 * m + 32 * wq + lane;
         const uint32_t lane_addr = tmem + ((uint32_t)(wq * 32) << 16) + 64u * (uint32_t)hh;
         const float sl = a.scale_log2;
-        const float2 st = PASS == 2 ? rstat[row] : make_float2(0.f, 0.f);  // (max, 1 / sum); 0 for rows >= R
+        // pass 2: 2^(z - max) / sum = 2^(z - off) with off = max + log2(sum)
+        // (+inf for rows >= R, whose 1 / sum is 0: their weights are 0)
+        const float2 st = PASS == 2 ? rstat[row] : make_float2(0.f, 1.f);
+        const float off = st.x - log2f(st.y);
         // Every softmax warp runs every tile's iteration, so that the named
         // barriers of pass 2 always match; after an abort (tc_wait then
         // returns false at once) the iterations only pass the barriers.
@@ -258,10 +261,10 @@ __global__ void __launch_bounds__(MassTc<MB>::kThreads, 1)
             } else {
                 if (nvalid == 64) {
 #pragma unroll
-                    for (int c = 0; c < 64; ++c) v[c] = exp2_approx(v[c] * sl - st.x) * st.y;
+                    for (int c = 0; c < 64; ++c) v[c] = exp2_approx(fmaf(v[c], sl, -off));
                 } else {
 #pragma unroll
-                    for (int c = 0; c < 64; ++c) v[c] = c < nvalid ? exp2_approx(v[c] * sl - st.x) * st.y : 0.f;
+                    for (int c = 0; c < 64; ++c) v[c] = c < nvalid ? exp2_approx(fmaf(v[c], sl, -off)) : 0.f;
                 }
                 // butterfly reduce-scatter over the warp's rows: after the step
                 // with lane offset o, this lane keeps the columns whose bit for o
