@@ -339,6 +339,27 @@ def test_adaptive_width(case):
     assert torch.equal(step.k_pruned[:, :N], cache.k_pruned[:, :N])
 
 
+@pytest.mark.parametrize("tc", ["1", "0"])
+@pytest.mark.parametrize("case", [(1, 32, 8, 3000, 64), (1, 32, 8, 1300, 50), (2, 16, 8, 777, 48),
+                                  (1, 8, 2, 129, 16)])
+def test_token_mass_both_kernels(case, tc, monkeypatch):
+    # the window attention masses from the tcgen05 kernel (default up to 256
+    # window rows: here 256, 200 with padding rows, 96 and 64 rows) and from
+    # the mma.sync kernel, against the fp64 oracle; ragged last tiles
+    monkeypatch.setenv("THINK_MASS_TC", tc)
+    B, Hq, Hkv, N, S = case
+    q_win, k, _, _ = _random_case(hash(case) & 0xFFFF, B, Hq, Hkv, N, S, torch.bfloat16)
+    mass = torch.full((B, Hkv, N), float("nan"), dtype=torch.float32, device=DEV)
+    ws = torch.zeros(qdk.think_token_mass_workspace_size(B, Hq, Hkv, N, S), dtype=torch.uint8, device=DEV)
+    for _ in range(2):  # twice on the same workspace
+        qdk.think_token_mass(q_win.to(DEV), k.to(DEV), mass, ws)
+    torch.cuda.synchronize()
+    assert qdk.think_read_device_status(ws) == 0
+    ora = oracle.oracle_token_mass(f64(q_win), f64(k))
+    np.testing.assert_allclose(f64(mass), ora, rtol=2e-4, atol=1e-6 * (Hq // Hkv) * S)
+    np.testing.assert_allclose(f64(mass).sum(axis=-1), (Hq // Hkv) * S, rtol=1e-5)
+
+
 @pytest.mark.parametrize("case", [(1, 1, 1, 1, "grid"), (1, 3, 4097, 4097, "grid"), (2, 4, 131072, 32768, "grid"),
                                   (1, 2, 70001, 1, "grid"), (1, 1, 5_000_000, 1_000_000, "grid"),
                                   (1, 8, 20000, 6000, "cont"), (3, 2, 9000, 8999, "cont")])
