@@ -15,17 +15,19 @@
 // block with the 128-byte swizzle (rows >= R zero), each K tile by TMA with
 // the same swizzle (two 64-channel halves), accumulators in tensor memory in
 // two buffers of MB x 128 fp32 columns, so the MMA of tile i + 1 runs while
-// the softmax warps work on tile i.  Two softmax warpgroups per row block m
-// read its TMEM lanes: thread t of warpgroup 2 m + hh holds row 128 m + t and
-// the tile's tokens 64 hh .. 64 hh + 63 (the column half).
+// the softmax warps work on tile i.  Pass 1: two softmax warpgroups per row
+// block m read its TMEM lanes: thread t of warpgroup 2 m + hh holds row
+// 128 m + t and the tile's tokens 64 hh .. 64 hh + 63 (the column half).
 //   pass 1: per row, the maximum z and the sum of 2^(z - max) over the block's
 //           tokens (the sum rescaled only when the maximum grows), the two
 //           halves of a row merged at the end, then the head's last block
 //           merges the splits into (max, 1 / sum);
-//   pass 2: per row the weights 2^(z - max - log2(sum)); the weights of a token are
-//           summed over rows by a butterfly reduce-scatter across the 32 lanes
-//           of a warp (lane L ends with tokens 2L, 2L + 1 of its half, summed
-//           over its warp's 32 rows), then over the warps in a fixed order.
+//   pass 2: the product transposed, D[token][row] (M = 128 tokens, N = 128 MB
+//           rows), with one extra K step that adds -off_r / sl to every row
+//           (off_r = max_r + log2(sum_r), its bf16 parts against channels of
+//           ones), so that a token's weights 2^(sl D) lie in one TMEM lane:
+//           each thread sums 64 rows of its token, then the four (MB = 1: two)
+//           row groups are added in order.
 // Warps: 8 MB softmax warps, one TMA producer warp, one MMA warp (which also
 // owns the tensor memory).  Every wait is bounded; a wait that runs out sets
 // the status bit and a block abort flag, and every warp still reaches the
@@ -48,16 +50,18 @@ struct MassTc {
     static constexpr uint32_t kCols = 2u * MB * 128u;  // two accumulator buffers
 };
 
-// shared memory: K ring (stages x 32 KB), Q (MB x 32 KB), per-warp token sums
-// [softmax warps][64] fp32, row statistics [MB * 128] float2, the upper
-// column halves' pass-1 row partials [MB * 128] float2, mbarriers
+// shared memory: K ring (stages x 32 KB), Q (MB x 32 KB), pass 2's extra K
+// step operands (4 KB + MB x 4 KB), per-warp token sums [softmax warps][64]
+// fp32, the upper column halves' pass-1 row partials [MB * 128] float2,
+// mbarriers
 // (K full/empty per stage, accumulator full/empty per buffer), TMEM address,
 // abort flag, a flag, alignment slack
 template <int MB>
 __host__ __device__ inline size_t mass_tc_smem_bytes(int stages)
 {
-    return (size_t)stages * 32768u + (size_t)MB * 32768u + (size_t)MassTc<MB>::kSoftWarps * 64u * 4u +
-           (size_t)MB * 128u * 8u + (size_t)MB * 128u * 8u + (size_t)(2 * stages + 4) * 8u + 16u + 1024u;
+    return (size_t)stages * 32768u + (size_t)MB * 32768u + 4096u + (size_t)MB * 4096u +
+           (size_t)MassTc<MB>::kSoftWarps * 64u * 4u + (size_t)MB * 128u * 8u + (size_t)(2 * stages + 4) * 8u +
+           16u + 1024u;
 }
 
 template <int PASS, int MB>
@@ -76,10 +80,11 @@ __global__ void __launch_bounds__(MassTc<MB>::kThreads, 1)
     const int64_t tiles_all = (a.N + kBN - 1) / kBN;
     const int ntiles = (int)max((int64_t)0, min((int64_t)a.tiles_per_split, tiles_all - tile0));
 
-    unsigned char *qs = smem + (size_t)stages * 32768u;                         // [MB][2 halves][128 rows][128 B]
-    float *tsum = reinterpret_cast<float *>(qs + (size_t)MB * 32768u);          // [softmax warps][64]
-    float2 *rstat = reinterpret_cast<float2 *>(tsum + C::kSoftWarps * 64);      // [MB * 128]
-    float2 *rhalf = rstat + MB * 128;                                           // [MB * 128] pass 1, upper half
+    unsigned char *qs = smem + (size_t)stages * 32768u;                         // [2 halves][MB * 128 rows][128 B]
+    unsigned char *xa = qs + (size_t)MB * 32768u;                               // pass 2: [128 tokens][16] bf16
+    unsigned char *xb = xa + 4096u;                                             // pass 2: [MB * 128 rows][16] bf16
+    float *tsum = reinterpret_cast<float *>(xb + (size_t)MB * 4096u);           // [softmax warps][64]
+    float2 *rhalf = reinterpret_cast<float2 *>(tsum + C::kSoftWarps * 64);      // [MB * 128] pass 1, upper half
     uint64_t *bars = reinterpret_cast<uint64_t *>(rhalf + MB * 128);
     const uint32_t kfull0 = smem_addr(bars);
     const uint32_t kempty0 = kfull0 + 8u * (uint32_t)stages;
@@ -107,7 +112,8 @@ __global__ void __launch_bounds__(MassTc<MB>::kThreads, 1)
         tc05::tmem_relinquish();
     }
     // the window rows r = g * S + s of the group (rows >= R zero), K-major with
-    // the 128-byte swizzle: row block m, channel half h at qs + (2 m + h) * 16 KB
+    // the 128-byte swizzle: channel half h at qs + h * MB * 16 KB, row r at
+    // + 128 r (rows of both row blocks contiguous, 8-row atoms 1 KB apart)
     for (int i = tid; i < MB * 128 * 16; i += C::kThreads) {
         const int r = i >> 4, c16 = i & 15;
         uint4 v = make_uint4(0, 0, 0, 0);
@@ -116,13 +122,40 @@ __global__ void __launch_bounds__(MassTc<MB>::kThreads, 1)
             v = *reinterpret_cast<const uint4 *>(
                 a.qwin + (((int64_t)b * a.Hq + (int64_t)kv * a.G + g) * a.S + s) * kD + 8 * c16);
         }
-        const int m = r >> 7, rr = r & 127;
-        *reinterpret_cast<uint4 *>(qs + (size_t)(2 * m + (c16 >> 3)) * 16384u + (uint32_t)rr * 128u +
-                                   ((((uint32_t)c16 & 7u) ^ ((uint32_t)rr & 7u)) << 4)) = v;
+        *reinterpret_cast<uint4 *>(qs + (size_t)(c16 >> 3) * (MB * 16384u) + (uint32_t)r * 128u +
+                                   ((((uint32_t)c16 & 7u) ^ ((uint32_t)r & 7u)) << 4)) = v;
     }
-    if (PASS == 2)
-        for (int r = tid; r < MB * 128; r += C::kThreads)
-            rstat[r] = r < a.R ? __ldcg(a.stats + (int64_t)head * a.R + r) : make_float2(0.f, 0.f);
+    if (PASS == 2) {
+        // The extra K step of pass 2's product: token t's 16 extra channels
+        // are (1, 1, 1, 0, ...), row r's are the bf16 parts of -off_r / sl,
+        // off_r = max_r + log2(sum_r), so that the accumulator holds
+        // z - off_r / sl and the weight is 2^(sl * that).  Rows >= R get a
+        // large finite negative value (weight 0).  K-major, no swizzle (core
+        // matrices of 8 rows x 8 channels, 128 B; the two along K 128 B apart,
+        // row groups 256 B apart).
+        const float sl = a.scale_log2;
+        for (int i = tid; i < 128 * 16; i += C::kThreads) {
+            const int t = i >> 4, c = i & 15;
+            *reinterpret_cast<__nv_bfloat16 *>(xa + kmajor_off((uint32_t)t, (uint32_t)c, 256u)) =
+                __float2bfloat16_rn(c < 3 ? 1.f : 0.f);
+        }
+        for (int r = tid; r < MB * 128; r += C::kThreads) {
+            float x = -1.0e30f;
+            if (r < a.R) {
+                const float2 st = __ldcg(a.stats + (int64_t)head * a.R + r);  // (max, 1 / sum)
+                x = -(st.x - log2f(st.y)) / sl;
+            }
+            const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+            const float r1 = x - __bfloat162float(hi);
+            const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+            const __nv_bfloat16 z = __float2bfloat16_rn(0.f);
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+                *reinterpret_cast<__nv_bfloat16 *>(xb + kmajor_off((uint32_t)r, (uint32_t)c, 256u)) =
+                    c == 0 ? hi : c == 1 ? mid : c == 2 ? lo : z;
+        }
+    }
     tc05::fence_proxy_async_smem();  // Q written by threads -> read by the tensor core
     tc05::fence_before_sync();
     __syncthreads();
@@ -157,7 +190,10 @@ __global__ void __launch_bounds__(MassTc<MB>::kThreads, 1)
     } else if (warp == C::kMmaWarp) {
         // -------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc = tc05::idesc_bf16_f32<128, 128, false>();
+            // pass 1: D[row][token], one MMA per row block (M = 128 rows, N = 128 tokens);
+            // pass 2: D[token][row] (M = 128 tokens, N = MB * 128 rows) plus the extra K step
+            constexpr uint32_t idesc = PASS == 1 ? tc05::idesc_bf16_f32<128, 128, false>()
+                                                 : tc05::idesc_bf16_f32<128, 128 * MB, false>();
             const uint32_t q_addr = smem_addr(qs);
             int last = -1;
             for (int it = 0; it < ntiles; ++it) {
@@ -169,17 +205,34 @@ __global__ void __launch_bounds__(MassTc<MB>::kThreads, 1)
                     break;
                 tc05::fence_after_sync();
                 const uint32_t kb = smem_addr(smem + (size_t)s * 32768u);
+                if constexpr (PASS == 1) {
 #pragma unroll
-                for (int m = 0; m < MB; ++m) {
+                    for (int m = 0; m < MB; ++m) {
+#pragma unroll
+                        for (int ks = 0; ks < 8; ++ks) {
+                            // 16 channels: half ks / 4, 32 bytes into each 128-byte row
+                            const uint32_t ko = (uint32_t)(ks & 3) * 32u;
+                            const uint64_t ad = tc05::smem_desc(q_addr + (uint32_t)(ks >> 2) * (MB * 16384u) +
+                                                                    (uint32_t)m * 16384u + ko,
+                                                                16u, 1024u, tc05::kLayoutSwizzle128B);
+                            const uint64_t bd = tc05::smem_desc(kb + (uint32_t)(ks >> 2) * 16384u + ko, 16u, 1024u,
+                                                                tc05::kLayoutSwizzle128B);
+                            tc05::mma_bf16(tmem + (uint32_t)(buf * MB + m) * 128u, ad, bd, idesc, ks > 0);
+                        }
+                    }
+                } else {
+                    const uint32_t d = tmem + (uint32_t)buf * (MB * 128u);
 #pragma unroll
                     for (int ks = 0; ks < 8; ++ks) {
-                        // 16 channels: half ks / 4, 32 bytes into each 128-byte row
-                        const uint32_t koff = (uint32_t)(ks >> 2) * 16384u + (uint32_t)(ks & 3) * 32u;
-                        const uint64_t ad = tc05::smem_desc(q_addr + (uint32_t)(2 * m) * 16384u + koff, 16u, 1024u,
+                        const uint32_t ko = (uint32_t)(ks & 3) * 32u;
+                        const uint64_t ad = tc05::smem_desc(kb + (uint32_t)(ks >> 2) * 16384u + ko, 16u, 1024u,
                                                             tc05::kLayoutSwizzle128B);
-                        const uint64_t bd = tc05::smem_desc(kb + koff, 16u, 1024u, tc05::kLayoutSwizzle128B);
-                        tc05::mma_bf16(tmem + (uint32_t)(buf * MB + m) * 128u, ad, bd, idesc, ks > 0);
+                        const uint64_t bd = tc05::smem_desc(q_addr + (uint32_t)(ks >> 2) * (MB * 16384u) + ko, 16u,
+                                                            1024u, tc05::kLayoutSwizzle128B);
+                        tc05::mma_bf16(d, ad, bd, idesc, ks > 0);
                     }
+                    tc05::mma_bf16(d, tc05::smem_desc(smem_addr(xa), 128u, 256u, tc05::kLayoutInterleave),
+                                   tc05::smem_desc(smem_addr(xb), 128u, 256u, tc05::kLayoutInterleave), idesc, true);
                 }
                 tc05::commit(dfull0 + 8 * buf);
                 tc05::commit(kempty0 + 8 * s);
@@ -195,19 +248,18 @@ __global__ void __launch_bounds__(MassTc<MB>::kThreads, 1)
         __syncwarp();
     } else {
         // ----------------------------------------------------- softmax warps
-        // warp w = 8 m + 4 hh + wq: row block m, column half hh (tokens 64 hh ..
-        // 64 hh + 63 of the tile), TMEM lane quarter wq (rows 32 wq .. + 31)
-        const int m = warp >> 3, hh = (warp >> 2) & 1, wq = warp & 3;
-        const int row = 128 * m + 32 * wq + lane;
-        const uint32_t lane_addr = tmem + ((uint32_t)(wq * 32) << 16) + 64u * (uint32_t)hh;
-        const float sl = a.scale_log2;
-        // pass 2: 2^(z - max) / sum = 2^(z - off) with off = max + log2(sum)
-        // (+inf for rows >= R, whose 1 / sum is 0: their weights are 0)
-        const float2 st = PASS == 2 ? rstat[row] : make_float2(0.f, 1.f);
-        const float off = st.x - log2f(st.y);
         // Every softmax warp runs every tile's iteration, so that the named
         // barriers of pass 2 always match; after an abort (tc_wait then
         // returns false at once) the iterations only pass the barriers.
+        // pass 1: warp w = 8 m + 4 hh + wq holds rows 128 m + 32 wq + lane and
+        //         the tile's tokens 64 hh .. 64 hh + 63;
+        // pass 2: warp w = 4 cg + wq holds token 32 wq + lane of the tile and
+        //         the rows 64 cg .. 64 cg + 63.
+        const int wq = warp & 3, hi = warp >> 2;  // hi: 2 m + hh (pass 1), cg (pass 2)
+        const int m = hi >> 1, hh = hi & 1;
+        const int row = 128 * m + 32 * wq + lane;
+        const uint32_t lane_addr = tmem + ((uint32_t)(wq * 32) << 16);
+        const float sl = a.scale_log2;
         for (int it = 0; it < ntiles; ++it) {
             const int buf = it & 1;
             float v[64];
@@ -216,7 +268,8 @@ __global__ void __launch_bounds__(MassTc<MB>::kThreads, 1)
             if (ok) {
                 tc05::fence_after_sync();
                 uint32_t r[4][16];
-                const uint32_t col = lane_addr + (uint32_t)(buf * MB + m) * 128u;
+                const uint32_t col = PASS == 1 ? lane_addr + (uint32_t)(buf * MB + m) * 128u + 64u * (uint32_t)hh
+                                               : lane_addr + (uint32_t)buf * (MB * 128u) + 64u * (uint32_t)hi;
 #pragma unroll
                 for (int j = 0; j < 4; ++j) tc05::tmem_ld16_issue(col + 16u * j, r[j]);
 #pragma unroll
@@ -233,9 +286,9 @@ __global__ void __launch_bounds__(MassTc<MB>::kThreads, 1)
                 for (int c = 0; c < 64; ++c) v[c] = 0.f;
             }
             const int64_t tok0 = (tile0 + it) * kBN;
-            // valid columns of this thread's half
-            const int nvalid = ok ? (int)max((int64_t)0, min((int64_t)64, a.N - tok0 - 64 * hh)) : 0;
-            if (PASS == 1) {
+            if constexpr (PASS == 1) {
+                // valid columns of this thread's half
+                const int nvalid = ok ? (int)max((int64_t)0, min((int64_t)64, a.N - tok0 - 64 * hh)) : 0;
                 float tmax = -INFINITY, l = 0.f;
                 if (nvalid == 64) {
 #pragma unroll
@@ -259,38 +312,22 @@ __global__ void __launch_bounds__(MassTc<MB>::kThreads, 1)
                 }
                 row_l += l;
             } else {
-                if (nvalid == 64) {
+                // the token's weights over these 64 rows (the accumulator
+                // holds z - off / sl; rows >= R give 0), summed in row order
+                const int tok = 32 * wq + lane;
+                float x = 0.f;
+                if (ok && tok0 + tok < a.N) {
 #pragma unroll
-                    for (int c = 0; c < 64; ++c) v[c] = exp2_approx(fmaf(v[c], sl, -off));
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 64; ++c) v[c] = c < nvalid ? exp2_approx(fmaf(v[c], sl, -off)) : 0.f;
+                    for (int c = 0; c < 64; ++c) x += exp2_approx(v[c] * sl);
                 }
-                // butterfly reduce-scatter over the warp's rows: after the step
-                // with lane offset o, this lane keeps the columns whose bit for o
-                // matches its own; lane L ends with columns 2L, 2L + 1 of the half
-#pragma unroll
-                for (int o = 16, w = 32; o >= 1; o >>= 1, w >>= 1) {
-                    const bool up = (lane & o) != 0;
-#pragma unroll
-                    for (int j = 0; j < w; ++j) {
-                        const float send = up ? v[j] : v[w + j];
-                        const float keep = up ? v[w + j] : v[j];
-                        v[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-                    }
-                }
-                *reinterpret_cast<float2 *>(tsum + warp * 64 + 2 * lane) = make_float2(v[0], v[1]);
+                tsum[hi * kBN + tok] = x;
                 named_barrier(1, NT);
-                // column c of the tile: half c / 64, summed over the row blocks and
-                // lane quarters in order
+                // token t: its row groups' sums in order
                 if (tid < kBN && tok0 + tid < a.N && !*abort_flag) {
-                    const int h2 = tid >> 6, c2 = tid & 63;
-                    float x = 0.f;
+                    float y = 0.f;
 #pragma unroll
-                    for (int m2 = 0; m2 < MB; ++m2)
-#pragma unroll
-                        for (int q2 = 0; q2 < 4; ++q2) x += tsum[(8 * m2 + 4 * h2 + q2) * 64 + c2];
-                    a.mass[(int64_t)head * a.N + tok0 + tid] = x;
+                    for (int g2 = 0; g2 < 2 * MB; ++g2) y += tsum[g2 * kBN + tid];
+                    a.mass[(int64_t)head * a.N + tok0 + tid] = y;
                 }
                 named_barrier(1, NT);  // tsum is read before the next tile rewrites it
             }
