@@ -104,7 +104,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
 }
 
 // 4-D tiled TMA load global -> shared, completion counted on `bar` (bytes).
-// No multicast: every CTA loads its own tiles.
+// Every CTA loads its own tiles into its own shared memory.
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map, int c0, int c1,
                                             int c2, int c3, uint32_t bar)
 {
