@@ -53,9 +53,8 @@ struct MassTc {
 // shared memory: K ring (stages x 32 KB), Q (MB x 32 KB), pass 2's extra K
 // step operands (4 KB + MB x 4 KB), per-warp token sums [softmax warps][64]
 // fp32, the upper column halves' pass-1 row partials [MB * 128] float2,
-// mbarriers
-// (K full/empty per stage, accumulator full/empty per buffer), TMEM address,
-// abort flag, a flag, alignment slack
+// mbarriers (K full/empty per stage, accumulator full/empty per buffer), the
+// TMEM address, an abort flag, a flag, alignment slack
 template <int MB>
 __host__ __device__ inline size_t mass_tc_smem_bytes(int stages)
 {
